@@ -1,0 +1,535 @@
+#!/usr/bin/env python
+"""Benchmark of the B200 BitNet b1.58 BitLinear forward.
+
+Workload (one "step"): the decode forward (RMSNorm + absmax int8 quant,
+ternary matmul, dequant) of the BitNet-3B-shaped problems
+K=3200->N=3200, 3200->8640 and 8640->3200 at M = 1, 4 and 16 tokens each
+(nine problems), bf16 activations with 0.1% x20 outlier channels, bf16
+output, inputs resident in HBM.  Weights rotate over several distinct copies
+so that a step never reads weights that are still in L2.
+
+Prints one JSON line (rank 0).  `--impl reference` times the CPU oracle on
+the same metric instead.  Under torchrun each rank runs an independent
+replica (no data-path collective); timing is the max over ranks.
+"""
+import argparse
+import ctypes
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "BitLinear fwd: decode HBM GB/s & tok/s, prefill int8 TOPS (% of B200 peak)"
+WORKLOAD = "decode_bitnet3b"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+# DRAM traffic per GEMV launch from an ncu capture of this workload (bytes,
+# averaged over the nine problems), valid only for the kernel source it was
+# measured on (sha256 of csrc/gemv.cuh); None until measured.
+GEMV_TRAFFIC = {"src_sha256": None, "bytes_per_launch": None}
+
+
+# ------------------------------------------------------------------ helpers
+
+def env_rank():
+    return (int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")),
+            int(os.environ.get("LOCAL_RANK", "0")))
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    except (OSError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def forward_bytes(M, N, K, x_bytes=2, y_bytes=2):
+    """Algorithmic HBM bytes of one forward: x read, x_q written and read back,
+    scales/row sums, packed weights, y written."""
+    return M * K * x_bytes + 2 * M * K + 16 * M + 4 + N * K // 4 + M * N * y_bytes
+
+
+def gemv_bytes(M, N, K, y_bytes=2):
+    """Algorithmic bytes of the matmul kernel: packed weights, quantized
+    activations, scales and row sums, s_w, y."""
+    return N * K // 4 + M * K + 8 * M + 4 + M * N * y_bytes
+
+
+def quant_bytes(M, K, x_bytes=2):
+    return M * K * x_bytes + M * K + 8 * M
+
+
+def problems():
+    from ternary_quantized_linear_b200 import workloads
+    case = workloads.CASE_BY_NAME[WORKLOAD]
+    return case, list(workloads.all_problems(case))
+
+
+def step_bytes(probs):
+    return sum(forward_bytes(M, N, K) for _, K, N, M in probs)
+
+
+def step_tokens(probs):
+    return sum(M for _, _, _, M in probs)
+
+
+def max_over_ranks(value, world, device=None):
+    """Max of a float over all ranks (identity for one rank)."""
+    if world <= 1:
+        return float(value)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(value)], dtype=torch.float64,
+                     device=device if device is not None else "cpu")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(bytes_per_step_per_rank, steps, world, max_ms):
+    """Whole-job GB/s: the bytes all ranks processed over the slowest rank's time."""
+    return bytes_per_step_per_rank * steps * world / (max_ms * 1e-3) / 1e9
+
+
+def file_sha256(path):
+    import hashlib
+    with open(path, "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()
+
+
+class ClockSampler:
+    """Polls SM clock and clock-event reasons through NVML while running."""
+
+    REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+               0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+               0x100: "display_clock_setting"}
+
+    def __init__(self, index, period_s=0.002):
+        self.index, self.period = index, period_s
+        self.samples, self.reasons = [], 0
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._t = None
+        self.ok = False
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self._nv = pynvml
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:
+            self.ok = False
+
+    def _run(self):
+        nv = self._nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
+                self.reasons |= int(nv.nvmlDeviceGetCurrentClocksEventReasons(self._h))
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.ok:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        return self
+
+    def __exit__(self, *exc):
+        if self._t is not None:
+            self._stop.set()
+            self._t.join()
+
+    def summary(self):
+        if not self.ok:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0,
+                    "source": "nvml unavailable"}
+        names = [n for bit, n in self.REASONS.items() if self.reasons & bit and n != "gpu_idle"]
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+                "sm_max_mhz": self.max_mhz, "reasons": names, "samples": len(self.samples),
+                "source": "nvml"}
+
+
+# --------------------------------------------------------------- CPU oracle
+
+def time_oracle(probs, budget_s, max_steps=None, per_problem=False):
+    """Run the CPU oracle over the workload: whole steps (or single problems,
+    cycling, when per_problem) until budget_s is spent.  Returns
+    (bytes, seconds, units, threads)."""
+    import oracle
+    from ternary_quantized_linear_b200 import workloads
+    threads = oracle.set_threads(1)
+    case = workloads.CASE_BY_NAME[WORKLOAD]
+    prepared = []
+    wcache = {}
+    for si, K, N, M in probs:
+        if si not in wcache:
+            W = workloads.weights(case, si)
+            s_w, _ = oracle.weight_scale(W)
+            W_p, _ = oracle.quantize_pack(W, s_w)
+            wcache[si] = (W_p, s_w)
+        prepared.append((workloads.activations(case, si, M), wcache[si], K, N, M))
+    total_b, total_s, units = 0, 0.0, 0
+    t_start = time.perf_counter()
+    i = 0
+    while True:
+        batch = [prepared[i % len(prepared)]] if per_problem else prepared
+        t0 = time.perf_counter()
+        for x, (W_p, s_w), K, N, M in batch:
+            oracle.linear_forward(x, None, workloads.DEFAULT_EPS, W_p, s_w, K)
+            total_b += forward_bytes(M, N, K)
+        total_s += time.perf_counter() - t0
+        units += 1
+        i += 1
+        if max_steps is not None and units >= max_steps:
+            break
+        if max_steps is None and time.perf_counter() - t_start >= budget_s:
+            break
+    return total_b, total_s, units, threads
+
+
+def run_reference(args):
+    rank, world, _ = env_rank()
+    if rank != 0:
+        return 0
+    case, probs = problems()
+    # warm-up steps (untimed), then exactly `steps` timed steps; one step here is
+    # one problem of the workload (cycling through the nine), so the run stays short
+    time_oracle(probs, 0, max_steps=max(args.warmup, 0) or 1, per_problem=True)
+    b, s, units, threads = time_oracle(probs, 0, max_steps=args.steps, per_problem=True)
+    gbs = b / s / 1e9
+    line = {
+        "metric": METRIC, "value": gbs, "unit": "GB/s", "n_gpus": args.gpus, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": 1e3 * s / units, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "i8", "data": "synthetic",
+        "impl": "reference",
+        "config": {"workload": WORKLOAD + ": " + case.description, "x_dtype": "bf16",
+                   "y_dtype": "bf16"},
+        "cpu_baseline": {"value": gbs, "unit": "GB/s", "cores": threads, "kind": "oracle",
+                         "sample": f"{units} single-problem steps cycling through the nine "
+                                   "decode problems, plain C oracle, 1 thread"},
+        "e2e": {"value": gbs, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# -------------------------------------------------------------- GPU path
+
+def run_ours(args):
+    import numpy as np
+    import torch
+
+    rank, world, local_rank = env_rank()
+    torch.cuda.set_device(local_rank)
+    device = torch.device("cuda", local_rank)
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=device)
+
+    import ternary_quantized_linear_b200 as tql
+    from ternary_quantized_linear_b200 import build as tql_build
+    from ternary_quantized_linear_b200 import workloads
+
+    tql_build.build()
+    lib = tql.load_library()
+    case, probs = problems()
+    R = args.rotations
+    eps = workloads.DEFAULT_EPS
+
+    # ---- inputs resident in HBM: R rotation sets x 9 problems
+    packed = {}
+    for si in range(len(case.shapes)):
+        W = torch.from_numpy(workloads.weights(case, si)).to(device)
+        packed[si] = tql.bitnet_quantize_pack_weights(W)
+        del W
+    sets = []
+    for r in range(R):
+        entries = []
+        for si, K, N, M in probs:
+            W_p, s_w = packed[si]
+            xh = workloads.activations(case, si, M)
+            x = torch.from_numpy(xh.view(np.int16).copy()).view(torch.bfloat16).to(device)
+            y = torch.empty((M, N), dtype=torch.bfloat16, device=device)
+            ws = torch.zeros(tql.bitnet_linear_forward_workspace_bytes(M, N, K),
+                             dtype=torch.uint8, device=device)
+            entries.append({"x": x, "W_p": W_p.clone(), "s_w": s_w, "y": y, "ws": ws,
+                            "M": M, "N": N, "K": K})
+        sets.append(entries)
+    torch.cuda.synchronize()
+    weight_mb_per_set = sum(e["W_p"].numel() for e in sets[0]) / 1e6
+
+    stream = torch.cuda.Stream(device=device)
+    P = ctypes.c_void_p
+
+    def fwd(e, sp):
+        return lib.bitnet_linear_forward(
+            P(e["x"].data_ptr()), tql.BITNET_BF16, None, ctypes.c_float(eps),
+            P(e["W_p"].data_ptr()), P(e["s_w"].data_ptr()), e["M"], e["N"], e["K"],
+            P(e["y"].data_ptr()), tql.BITNET_BF16, P(e["ws"].data_ptr()), e["ws"].numel(), sp)
+
+    def launch_step(r, sp):
+        for e in sets[r]:
+            rc = fwd(e, sp)
+            if rc != 0:
+                raise RuntimeError(f"bitnet_linear_forward: {tql.bitnet_status_string(rc)}")
+
+    # ---- one CUDA graph per rotation set
+    graphs = []
+    with torch.cuda.stream(stream):
+        launch_step(0, P(stream.cuda_stream))  # first call sets up the device state
+        stream.synchronize()
+        for r in range(R):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream):
+                launch_step(r, P(torch.cuda.current_stream().cuda_stream))
+            graphs.append(g)
+    torch.cuda.synchronize()
+
+    def barrier():
+        if world > 1:
+            import torch.distributed as dist
+            dist.barrier(device_ids=[local_rank])
+
+    # ---- warm-up, then exactly K timed steps (graph replays)
+    with torch.cuda.stream(stream):
+        for i in range(args.warmup):
+            graphs[i % R].replay()
+    stream.synchronize()
+    barrier()
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local_rank) as clocks:
+        with torch.cuda.stream(stream):
+            e0.record(stream)
+            for i in range(args.steps):
+                graphs[i % R].replay()
+            e1.record(stream)
+        stream.synchronize()
+    torch.cuda.synchronize()
+    barrier()
+    local_ms = e0.elapsed_time(e1)
+    max_ms = max_over_ranks(local_ms, world, device)
+    sb = step_bytes(probs)
+    value = job_throughput(sb, args.steps, world, max_ms)
+    ms_per_step = max_ms / args.steps
+    launches = 2 * len(probs) * args.steps
+
+    # ---- per-kernel durations with CUDA events (the roofline of the matmul kernel)
+    ev = [[[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in probs]
+          for _ in range(R)]
+    q_ms, m_ms = {}, {}
+    with torch.cuda.stream(stream):
+        sp = P(stream.cuda_stream)
+        for i in range(args.steps + args.warmup):
+            r = i % R
+            torch.cuda._sleep(2_000_000)  # queue the step while the GPU is busy
+            for j, e in enumerate(sets[r]):
+                ev[r][j][0].record(stream)
+                tql.bitnet_linear_quantize_input(e["x"], None, eps, e["N"], e["ws"],
+                                                 stream=stream)
+                ev[r][j][1].record(stream)
+                tql.bitnet_linear_matmul(e["W_p"], e["s_w"], e["M"], e["K"], e["ws"], y=e["y"],
+                                         stream=stream)
+                ev[r][j][2].record(stream)
+            stream.synchronize()
+            if i < args.warmup:
+                continue
+            for j, e in enumerate(sets[r]):
+                q_ms.setdefault(j, []).append(ev[r][j][0].elapsed_time(ev[r][j][1]))
+                m_ms.setdefault(j, []).append(ev[r][j][1].elapsed_time(ev[r][j][2]))
+    per_problem = []
+    tot_b, tot_ms = 0, 0.0
+    for j, (si, K, N, M) in enumerate(probs):
+        t = statistics.mean(m_ms[j])
+        b = gemv_bytes(M, N, K)
+        tot_b += b
+        tot_ms += t
+        per_problem.append({"K": K, "N": N, "M": M, "matmul_us": round(1e3 * t, 3),
+                            "matmul_gbs": round(b / (t * 1e-3) / 1e9, 1),
+                            "quant_us": round(1e3 * statistics.mean(q_ms[j]), 3)})
+    peaks, peak_src = load_peaks()
+    hbm_peak = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+    achieved = tot_b / (tot_ms * 1e-3) / 1e9
+    sha = file_sha256(os.path.join(ROOT, "ternary_quantized_linear_b200", "csrc", "gemv.cuh"))
+    traffic = GEMV_TRAFFIC["bytes_per_launch"] if GEMV_TRAFFIC["src_sha256"] == sha else None
+    roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm_peak,
+                "unit": "GB/s", "frac": round(achieved / hbm_peak, 4), "traffic": traffic,
+                "kernel": "ternary_gemv_kernel (decode matmul + fused dequant)",
+                "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)",
+                "algorithmic_bytes_per_launch": round(tot_b / len(probs)),
+                "avg_launch_us": round(1e3 * tot_ms / len(probs), 3),
+                "per_problem": per_problem}
+
+    # ---- end to end through the public call with host buffers
+    e2e = None
+    if not args.no_e2e:
+        hx = [[e["x"].cpu().pin_memory() for e in s] for s in sets]
+        hy = [[torch.empty(e["y"].shape, dtype=e["y"].dtype).pin_memory() for e in s]
+              for s in sets]
+        h2d = sum(e["x"].numel() * 2 for e in sets[0])
+        d2h = sum(e["y"].numel() * 2 for e in sets[0])
+        with torch.cuda.stream(stream):
+            sp = P(stream.cuda_stream)
+
+            def e2e_step(r):
+                for j, e in enumerate(sets[r]):
+                    e["x"].copy_(hx[r][j], non_blocking=True)
+                    rc = fwd(e, sp)
+                    if rc != 0:
+                        raise RuntimeError(tql.bitnet_status_string(rc))
+                    hy[r][j].copy_(e["y"], non_blocking=True)
+
+            for i in range(args.warmup):
+                e2e_step(i % R)
+            stream.synchronize()
+            barrier()
+            a0 = torch.cuda.Event(enable_timing=True)
+            a1 = torch.cuda.Event(enable_timing=True)
+            a0.record(stream)
+            for i in range(args.steps):
+                e2e_step(i % R)
+            a1.record(stream)
+            stream.synchronize()
+        e2e_ms = max_over_ranks(a0.elapsed_time(a1), world, device)
+        e2e = {"value": job_throughput(sb, args.steps, world, e2e_ms), "unit": "GB/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+               "ms_per_step": e2e_ms / args.steps,
+               "how": "per problem: pinned-host x -> device copy, bitnet_linear_forward "
+                      "(C ABI, eager launches), y -> pinned host; device-timed"}
+
+    # ---- prefill extra: tcgen05 GEMM TOPS on the Llama-3-8B FFN shapes
+    prefill = None
+    if not args.no_prefill:
+        prefill = measure_prefill(args, device, stream, peaks, peak_src)
+
+    # ---- CPU baseline (rank 0, one GPU only)
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        b, s, units, threads = time_oracle(probs, args.cpu_budget)
+        cpu = {"value": b / s / 1e9, "unit": "GB/s", "cores": threads, "kind": "oracle",
+               "sample": f"{units} full decode step(s) (all nine problems) of the plain C "
+                         f"oracle, {threads} thread(s), {s:.1f} s"}
+
+    if world > 1:
+        import torch.distributed as dist
+        for g in graphs:
+            del g
+        graphs.clear()
+        dist.barrier(device_ids=[local_rank])
+        dist.destroy_process_group()
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "i8",
+            "data": "synthetic",
+            "config": {"workload": WORKLOAD + ": " + case.description,
+                       "problems": [[K, N, M] for _, K, N, M in probs],
+                       "x_dtype": "bf16", "y_dtype": "bf16",
+                       "l2": f"inputs larger than L2: {R} rotating weight/activation sets, "
+                             f"{R * weight_mb_per_set:.0f} MB of packed weights",
+                       "launch": "one CUDA graph per rotation set (2 kernels per problem, "
+                                 "programmatic dependent launch between them)",
+                       "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
+            "tok_s": round(world * step_tokens(probs) * args.steps / (max_ms * 1e-3), 1),
+            "roofline": roofline,
+            "cpu_baseline": cpu,
+            "e2e": e2e,
+            "gpu_launches": launches,
+            "clocks": clocks.summary(),
+            "prefill": prefill,
+        }
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+def measure_prefill(args, device, stream, peaks, peak_src):
+    """Tensor-core path on the Llama-3-8B FFN shapes at M = 2048 (not the
+    headline number): TOPS of the GEMM kernel alone and of the whole forward."""
+    import numpy as np
+    import torch
+
+    import ternary_quantized_linear_b200 as tql
+    from ternary_quantized_linear_b200 import workloads
+
+    case = workloads.CASE_BY_NAME["prefill_llama3_8b"]
+    M = 2048
+    out = []
+    i8_peak = 2.0 * float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    for si, (K, N) in enumerate(case.shapes):
+        W = torch.from_numpy(workloads.weights(case, si)).to(device)
+        W_p, s_w = tql.bitnet_quantize_pack_weights(W)
+        del W
+        xh = workloads.activations(case, si, M)
+        R = 6
+        xs = [torch.from_numpy(xh.view(np.int16).copy()).view(torch.bfloat16).to(device)
+              for _ in range(R)]
+        wps = [W_p.clone() for _ in range(R)]
+        y = torch.empty((M, N), dtype=torch.bfloat16, device=device)
+        ws = torch.zeros(tql.bitnet_linear_forward_workspace_bytes(M, N, K), dtype=torch.uint8,
+                         device=device)
+        iters = 20
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(iters)]
+        with torch.cuda.stream(stream):
+            for i in range(3):
+                tql.bitnet_linear_forward(xs[i % R], None, 1e-5, wps[i % R], s_w, y=y,
+                                          workspace=ws, stream=stream)
+            for i in range(iters):
+                evs[i][0].record(stream)
+                tql.bitnet_linear_quantize_input(xs[i % R], None, 1e-5, N, ws, stream=stream)
+                evs[i][1].record(stream)
+                tql.bitnet_linear_matmul(wps[i % R], s_w, M, K, ws, y=y, stream=stream)
+                evs[i][2].record(stream)
+            stream.synchronize()
+        gemm_ms = statistics.median(e[1].elapsed_time(e[2]) for e in evs)
+        fwd_ms = statistics.median(e[0].elapsed_time(e[2]) for e in evs)
+        ops = 2.0 * M * N * K
+        out.append({"K": K, "N": N, "M": M, "gemm_us": round(1e3 * gemm_ms, 2),
+                    "gemm_tops": round(ops / (gemm_ms * 1e-3) / 1e12, 1),
+                    "forward_tops": round(ops / (fwd_ms * 1e-3) / 1e12, 1)})
+    tops = [o["gemm_tops"] for o in out]
+    return {"workload": "prefill_llama3_8b at M=2048 (K=4096->N=14336, K=14336->N=4096)",
+            "shapes": out, "gemm_tops_mean": round(statistics.mean(tops), 1),
+            "frac_of_int8_peak": round(statistics.mean(tops) / i8_peak, 4),
+            "int8_peak_tops": i8_peak,
+            "int8_peak_source": f"{peak_src} bf16 burst x 2 (dense int8 = 2x bf16 rate)",
+            "frac_of_4500_tops_spec": round(statistics.mean(tops) / 4500.0, 4)}
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--rotations", type=int, default=6)
+    ap.add_argument("--cpu-budget", type=float, default=10.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-prefill", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3 and args.impl == "ours":
+        args.warmup = 3
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,242 @@
+/*
+ * bitnet_b200.h -- C ABI of the B200 (sm_100a) BitNet b1.58 BitLinear forward.
+ *
+ * The forward pass, as the pages define it:
+ *   1. RMSNorm of each token row, then per-token absmax quantization of the
+ *      activations to int8 in [-128, 127]
+ *      ("LLM を 1.58 ビットにファインチューニング：BitNet による極端な量子化",
+ *       section 量子化の仕組み, activations bullet; "[論文レビュー] The Era of
+ *       1-bit LLMs", section 提案手法, RMSNorm);
+ *   2. ternary weights from a per-tensor absmean scale, four 2-bit codes per
+ *      byte (same first page, 量子化の仕組み weights bullet and 主な発見
+ *      packing; The Era of 1-bit LLMs review, 提案手法 absmean);
+ *   3. an integer matmul with int32 accumulation (first page, 計算パラダイム);
+ *   4. the rescale y = acc / (s_x * s_w) (first page, 量子化の仕組み; the
+ *      bitnet.cpp article, section 数学的基礎 item 3).
+ *
+ * Exact arithmetic of every step (all of it reproduced bit for bit by the
+ * kernels):
+ *   r      = 1 / sqrt(ss / K + eps), ss = sum of x^2 over the row, reduced in a
+ *            fixed order: element k goes to partial (k/8) mod 256 (fp32,
+ *            fused multiply-add, increasing k), then partial i absorbs
+ *            partial i+s for s = 128, 64, ..., 1; division and sqrt correctly
+ *            rounded.  A row with ss/K + eps == 0 normalises to all zeros.
+ *   x_n    = (x * r) * gamma                  (two rounded fp32 products)
+ *   s_x    = 127 / max(max|x_n|, 1e-5)
+ *   x_q    = clamp(rint(x_n * s_x), -128, 127)          (ties to even)
+ *   S      = sum |W| in fp64: per row, element k to partial (k/4) mod 256,
+ *            same tree; then row sums to partial n mod 256, same tree.
+ *   s_w    = 1 / max((float)(S / (N*K)), 1e-5)
+ *   t      = clamp(rint(W * s_w), -1, 1)  stored as code t+1 in 2 bits;
+ *            weight k of row n sits in bits [2(k%4), 2(k%4)+1] of byte
+ *            W_packed[n*(K/4) + k/4].  Code 3 is never written.
+ *   acc    = sum_k x_q[m,k] * t[n,k]   (int32, exact)
+ *   y      = (float)acc / (s_x[m] * s_w)  (product rounded to fp32 first);
+ *            bf16 output = round-to-nearest-even of that fp32 value.
+ *
+ * Layouts: row-major, x [M][K], W [N][K] (y = x W^T as in a linear layer),
+ * W_packed [N][K/4] bytes, x_q [M][K] int8, acc and y [M][N].
+ *
+ * Conventions for every entry point:
+ *   - All tensor pointers are DEVICE pointers owned by the caller; the
+ *     library allocates nothing and never synchronises (except the two
+ *     status calls that say so).  Work is queued on `stream` (a
+ *     cudaStream_t; NULL = the legacy default stream) and runs
+ *     asynchronously.
+ *   - Shapes: M >= 0 (M == 0 queues nothing and returns BITNET_OK), N >= 1,
+ *     64 <= K <= BITNET_MAX_K and K % 64 == 0.
+ *   - Every tensor pointer must be 16-byte aligned (workspace: 256-byte).
+ *   - Invalid arguments return a status and queue nothing.
+ *   - Errors of the CUDA launch itself return BITNET_ERR_CUDA.
+ *   - Kernels that wait on on-chip barriers give up after a bounded time,
+ *     record BITNET_ERR_TIMEOUT in a device status word and exit cleanly;
+ *     bitnet_device_status() reads it.
+ */
+#ifndef BITNET_B200_H
+#define BITNET_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define BITNET_API __attribute__((visibility("default")))
+#else
+#define BITNET_API
+#endif
+
+/* cudaStream_t without pulling in the CUDA headers. */
+typedef struct CUstream_st *bitnet_stream_t;
+
+typedef enum {
+    BITNET_OK = 0,
+    BITNET_ERR_INVALID_ARG = 1,       /* null pointer, negative size, bad dtype, eps < 0 */
+    BITNET_ERR_UNSUPPORTED_SHAPE = 2, /* K % 64 != 0, K out of range, N < 1 */
+    BITNET_ERR_MISALIGNED = 3,        /* a pointer is not 16-byte (workspace 256-byte) aligned */
+    BITNET_ERR_CUDA = 4,              /* a CUDA launch or query failed */
+    BITNET_ERR_TIMEOUT = 5,           /* a bounded on-device wait gave up */
+    BITNET_ERR_WORKSPACE = 6          /* workspace missing or too small */
+} bitnet_status;
+
+typedef enum { BITNET_F32 = 0, BITNET_BF16 = 1 } bitnet_dtype;
+
+/* Matmul path selection for the debug entry point (results never depend on it). */
+typedef enum {
+    BITNET_PATH_AUTO = 0,  /* decode GEMV for M <= 16, tensor-core GEMM above */
+    BITNET_PATH_GEMV = 1,  /* tensor-core (mma.sync) streaming GEMV; needs M <= 16 */
+    BITNET_PATH_GEMM = 2   /* tcgen05 + TMA GEMM with TMEM accumulators */
+} bitnet_path;
+
+#define BITNET_MAX_K (1 << 20)
+
+/* Human-readable name of a status code (static string, never NULL). */
+BITNET_API const char *bitnet_status_string(int status);
+
+/* Library version as 10000*major + 100*minor + patch. */
+BITNET_API int bitnet_version(void);
+
+/* ------------------------------------------------------------------------
+ * bitnet_quantize_pack_weights -- absmean ternary quantization + packing.
+ * (first page, 量子化の仕組み weights bullet; The Era of 1-bit LLMs review,
+ *  提案手法; packing: first page, 主な発見.)
+ *
+ *   W          [N][K] fp32 in.
+ *   W_packed   [N][K/4] bytes out (layout above).
+ *   s_w        one fp32 out (device memory): the per-tensor scale 1/mean|W|.
+ *   workspace  >= bitnet_quantize_pack_weights_workspace_bytes(N, K) bytes of
+ *              device scratch (fp64 row sums); contents on entry don't matter.
+ * Deterministic: the same W gives the same bytes and s_w on every call.
+ * ---------------------------------------------------------------------- */
+BITNET_API size_t bitnet_quantize_pack_weights_workspace_bytes(int64_t N, int64_t K);
+BITNET_API bitnet_status bitnet_quantize_pack_weights(const float *W, int64_t N, int64_t K,
+                                                      uint8_t *W_packed, float *s_w,
+                                                      void *workspace, size_t workspace_bytes,
+                                                      bitnet_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * bitnet_rmsnorm_quant_act -- fused RMSNorm + per-token absmax int8 quant.
+ * (first page, 量子化の仕組み activations bullet; The Era of 1-bit LLMs
+ *  review, 提案手法 RMSNorm; bitnet.cpp article, 数学的基礎 item 2.)
+ *
+ *   x        [M][K], fp32 or bf16 per x_dtype.
+ *   gamma    [K] fp32 RMSNorm gain, or NULL for all ones.
+ *   eps      >= 0, added to the mean square.
+ *   x_q      [M][K] int8 out (natural k order).
+ *   s_x      [M] fp32 out, 127 / max|x_n| per token.
+ * ---------------------------------------------------------------------- */
+BITNET_API bitnet_status bitnet_rmsnorm_quant_act(const void *x, int x_dtype, const float *gamma,
+                                                  float eps, int64_t M, int64_t K, int8_t *x_q,
+                                                  float *s_x, bitnet_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * bitnet_linear_forward -- the whole BitLinear forward, y = dequant(
+ *   quant(rmsnorm(x)) * ternary(W)^T ).  Picks the decode GEMV for M <= 16
+ *   and the tcgen05 GEMM above; both give identical bits.
+ *
+ *   x, x_dtype, gamma, eps   as bitnet_rmsnorm_quant_act.
+ *   W_packed, s_w            as produced by bitnet_quantize_pack_weights
+ *                            (s_w is read on the device).
+ *   y                        [M][N] out, fp32 or bf16 per y_dtype.
+ *   workspace                >= bitnet_linear_forward_workspace_bytes(M,N,K)
+ *                            bytes, 256-byte aligned.  It MUST be zero-filled
+ *                            before its first use: for M <= 16 it holds int32
+ *                            split-K partial sums and arrival counters that
+ *                            must start at zero, and every successful call
+ *                            returns that region to zero, so a buffer zeroed
+ *                            once can be reused by any number of calls that
+ *                            do not overlap in time (its other bytes are
+ *                            rewritten by each call).  After a failed call,
+ *                            zero it again.
+ * ---------------------------------------------------------------------- */
+BITNET_API size_t bitnet_linear_forward_workspace_bytes(int64_t M, int64_t N, int64_t K);
+BITNET_API bitnet_status bitnet_linear_forward(const void *x, int x_dtype, const float *gamma,
+                                               float eps, const uint8_t *W_packed,
+                                               const float *s_w, int64_t M, int64_t N, int64_t K,
+                                               void *y, int y_dtype, void *workspace,
+                                               size_t workspace_bytes, bitnet_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * The forward in two phases, for callers that reuse one quantized input for
+ * several weight matrices (e.g. the q, k and v projections of one token
+ * batch) or time the phases separately.  bitnet_linear_forward(...) queues
+ * exactly bitnet_linear_quantize_input(...) followed by
+ * bitnet_linear_matmul(...).
+ *
+ * bitnet_linear_quantize_input -- RMSNorm + absmax int8 quant of x into the
+ *   workspace (the kernels' internal layout: x_q k-interleaved inside
+ *   16-element groups, s_x, per-token sums of x_q).  Arguments as
+ *   bitnet_linear_forward; N is the largest output width the workspace will
+ *   serve (it only sizes the workspace).
+ * bitnet_linear_matmul -- integer matmul of the workspace's quantized input
+ *   with W_packed and the fused dequant into y.  M and K must equal those of
+ *   the preceding bitnet_linear_quantize_input on the same workspace, and
+ *   workspace_bytes must cover (M, N, K).  Any number of matmuls may follow
+ *   one quantize call, in stream order.
+ * ---------------------------------------------------------------------- */
+BITNET_API bitnet_status bitnet_linear_quantize_input(const void *x, int x_dtype,
+                                                      const float *gamma, float eps, int64_t M,
+                                                      int64_t N, int64_t K, void *workspace,
+                                                      size_t workspace_bytes,
+                                                      bitnet_stream_t stream);
+BITNET_API bitnet_status bitnet_linear_matmul(const uint8_t *W_packed, const float *s_w,
+                                              int64_t M, int64_t N, int64_t K, void *y,
+                                              int y_dtype, void *workspace,
+                                              size_t workspace_bytes, bitnet_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * bitnet_linear_forward_debug -- bitnet_linear_forward that also exports the
+ * intermediate results, and can force a matmul path.
+ *
+ *   x_q_out  [M][K] int8 (natural k order) or NULL.
+ *   s_x_out  [M] fp32 or NULL.
+ *   acc_out  [M][N] int32 accumulators (before dequant) or NULL.
+ *   y        may be NULL (then only the debug outputs are written).
+ *   path     a bitnet_path value.
+ * ---------------------------------------------------------------------- */
+BITNET_API bitnet_status bitnet_linear_forward_debug(
+    const void *x, int x_dtype, const float *gamma, float eps, const uint8_t *W_packed,
+    const float *s_w, int64_t M, int64_t N, int64_t K, void *y, int y_dtype, void *workspace,
+    size_t workspace_bytes, int8_t *x_q_out, float *s_x_out, int32_t *acc_out, int path,
+    bitnet_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * bitnet_ternary_matmul_i32 -- debug: acc = x_q * t^T on the integer path
+ * alone (first page, 計算パラダイム).
+ *
+ *   x_q       [M][K] int8 (natural k order, any values in [-128, 127]).
+ *   W_packed  [N][K/4].
+ *   acc       [M][N] int32 out.
+ *   workspace >= bitnet_linear_forward_workspace_bytes(M,N,K), zero-filled
+ *             before first use (same contract as the forward).
+ *   path      a bitnet_path value.
+ * ---------------------------------------------------------------------- */
+BITNET_API bitnet_status bitnet_ternary_matmul_i32(const int8_t *x_q, const uint8_t *W_packed,
+                                                   int64_t M, int64_t N, int64_t K, int32_t *acc,
+                                                   void *workspace, size_t workspace_bytes,
+                                                   int path, bitnet_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * Device status word.  bitnet_device_status synchronises `stream`, returns
+ * BITNET_OK or the first BITNET_ERR_TIMEOUT recorded by a kernel since the
+ * last reset, stores the kernel-side detail code in *detail (may be NULL),
+ * and clears the word when reset != 0.  It is per device and per process.
+ * ---------------------------------------------------------------------- */
+BITNET_API bitnet_status bitnet_device_status(bitnet_stream_t stream, int reset, int *detail);
+
+/* ------------------------------------------------------------------------
+ * bitnet_selftest_bounded_wait -- runs one tiny kernel that waits on an
+ * on-chip barrier nothing ever completes, with the given limit in
+ * nanoseconds (1e3..1e9), so callers can check that bounded waits end and
+ * report BITNET_ERR_TIMEOUT through bitnet_device_status.  It does not touch
+ * any tensor.  Queues on `stream`.
+ * ---------------------------------------------------------------------- */
+BITNET_API bitnet_status bitnet_selftest_bounded_wait(uint64_t limit_ns, bitnet_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* BITNET_B200_H */

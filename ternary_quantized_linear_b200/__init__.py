@@ -1,0 +1,311 @@
+"""B200 (sm_100a) BitNet b1.58 BitLinear forward -- Python binding.
+
+Thin ctypes marshalling over libbitnet_b200.so: the functions below carry the
+names of the C entry points declared in include/bitnet_b200.h, take torch
+CUDA tensors, check dtypes/shapes, and pass raw device pointers plus the
+current CUDA stream.  Every step of the computation runs in the library's
+CUDA kernels; PyTorch only provides device memory and streams.  There is no
+CPU fallback: if the library is missing or a call fails, an exception is
+raised.
+"""
+import ctypes
+import os
+import threading
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libbitnet_b200.so")
+
+BITNET_OK = 0
+BITNET_ERR_INVALID_ARG = 1
+BITNET_ERR_UNSUPPORTED_SHAPE = 2
+BITNET_ERR_MISALIGNED = 3
+BITNET_ERR_CUDA = 4
+BITNET_ERR_TIMEOUT = 5
+BITNET_ERR_WORKSPACE = 6
+
+BITNET_F32 = 0
+BITNET_BF16 = 1
+
+BITNET_PATH_AUTO = 0
+BITNET_PATH_GEMV = 1
+BITNET_PATH_GEMM = 2
+
+# Every entry point the header declares (checked by the tests).
+EXPORTED = (
+    "bitnet_status_string", "bitnet_version",
+    "bitnet_quantize_pack_weights_workspace_bytes", "bitnet_quantize_pack_weights",
+    "bitnet_rmsnorm_quant_act", "bitnet_linear_forward_workspace_bytes",
+    "bitnet_linear_forward", "bitnet_linear_quantize_input", "bitnet_linear_matmul",
+    "bitnet_linear_forward_debug", "bitnet_ternary_matmul_i32",
+    "bitnet_device_status", "bitnet_selftest_bounded_wait",
+)
+
+
+class BitnetError(RuntimeError):
+    def __init__(self, fn, code, msg):
+        super().__init__(f"{fn} failed: {msg} (status {code})")
+        self.code = code
+
+
+_lib = None
+_lib_lock = threading.Lock()
+
+
+def load_library(path: str = LIB_PATH):
+    """Load (once) and return the ctypes handle of libbitnet_b200.so."""
+    global _lib
+    with _lib_lock:
+        if _lib is not None:
+            return _lib
+        if not os.path.exists(path):
+            raise ImportError(
+                f"{path} is missing; build it with `python ternary_quantized_linear_b200/build.py`"
+                " (there is no CPU fallback)")
+        lib = ctypes.CDLL(path)
+        P, I64, SZ, I = ctypes.c_void_p, ctypes.c_int64, ctypes.c_size_t, ctypes.c_int
+        F = ctypes.c_float
+        sig = {
+            "bitnet_status_string": ([I], ctypes.c_char_p),
+            "bitnet_version": ([], I),
+            "bitnet_quantize_pack_weights_workspace_bytes": ([I64, I64], SZ),
+            "bitnet_quantize_pack_weights": ([P, I64, I64, P, P, P, SZ, P], I),
+            "bitnet_rmsnorm_quant_act": ([P, I, P, F, I64, I64, P, P, P], I),
+            "bitnet_linear_forward_workspace_bytes": ([I64, I64, I64], SZ),
+            "bitnet_linear_forward": ([P, I, P, F, P, P, I64, I64, I64, P, I, P, SZ, P], I),
+            "bitnet_linear_quantize_input": ([P, I, P, F, I64, I64, I64, P, SZ, P], I),
+            "bitnet_linear_matmul": ([P, P, I64, I64, I64, P, I, P, SZ, P], I),
+            "bitnet_linear_forward_debug": (
+                [P, I, P, F, P, P, I64, I64, I64, P, I, P, SZ, P, P, P, I, P], I),
+            "bitnet_ternary_matmul_i32": ([P, P, I64, I64, I64, P, P, SZ, I, P], I),
+            "bitnet_device_status": ([P, I, ctypes.POINTER(I)], I),
+            "bitnet_selftest_bounded_wait": ([ctypes.c_uint64, P], I),
+        }
+        for name, (argtypes, restype) in sig.items():
+            fn = getattr(lib, name)
+            fn.argtypes = argtypes
+            fn.restype = restype
+        _lib = lib
+        return lib
+
+
+def _check(fn_name, code):
+    if code != BITNET_OK:
+        msg = load_library().bitnet_status_string(code).decode()
+        raise BitnetError(fn_name, code, msg)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _dtype_code(dt):
+    if dt == torch.float32:
+        return BITNET_F32
+    if dt == torch.bfloat16:
+        return BITNET_BF16
+    raise TypeError(f"unsupported dtype {dt} (float32 or bfloat16)")
+
+
+def _need_cuda(*ts):
+    for t in ts:
+        if t is not None and (not t.is_cuda or not t.is_contiguous()):
+            raise ValueError("tensors must be contiguous CUDA tensors")
+
+
+class Workspace:
+    """Zero-initialised device scratch reused across calls on one stream.
+
+    The forward's split-K partials and counters must start at zero; the
+    kernels leave them zeroed after every successful call, so one buffer
+    allocated with zeros serves any number of stream-ordered calls."""
+
+    def __init__(self):
+        self._buf = {}
+
+    def get(self, nbytes, device, stream=None):
+        key = (device.index if isinstance(device, torch.device) else int(device),
+               0 if stream is None else stream.cuda_stream)
+        buf = self._buf.get(key)
+        if buf is None or buf.numel() < nbytes:
+            buf = torch.zeros(max(int(nbytes), 256), dtype=torch.uint8, device=device)
+            self._buf[key] = buf
+        return buf
+
+
+_default_ws = Workspace()
+
+
+def bitnet_version() -> int:
+    return int(load_library().bitnet_version())
+
+
+def bitnet_status_string(code: int) -> str:
+    return load_library().bitnet_status_string(int(code)).decode()
+
+
+def bitnet_quantize_pack_weights_workspace_bytes(N: int, K: int) -> int:
+    return int(load_library().bitnet_quantize_pack_weights_workspace_bytes(N, K))
+
+
+def bitnet_linear_forward_workspace_bytes(M: int, N: int, K: int) -> int:
+    return int(load_library().bitnet_linear_forward_workspace_bytes(M, N, K))
+
+
+def bitnet_quantize_pack_weights(W, W_packed=None, s_w=None, workspace=None, stream=None):
+    """W fp32 [N,K] -> (W_packed uint8 [N,K/4], s_w fp32 [1]) on W's device."""
+    if W.dtype != torch.float32 or W.dim() != 2:
+        raise TypeError("W must be a 2-D float32 tensor")
+    _need_cuda(W)
+    N, K = W.shape
+    if W_packed is None:
+        W_packed = torch.empty((N, K // 4), dtype=torch.uint8, device=W.device)
+    if s_w is None:
+        s_w = torch.empty((1,), dtype=torch.float32, device=W.device)
+    nb = bitnet_quantize_pack_weights_workspace_bytes(N, K)
+    if workspace is None:
+        workspace = torch.empty(max(nb, 256), dtype=torch.uint8, device=W.device)
+    _need_cuda(W_packed, s_w, workspace)
+    _check("bitnet_quantize_pack_weights", load_library().bitnet_quantize_pack_weights(
+        _ptr(W), N, K, _ptr(W_packed), _ptr(s_w), _ptr(workspace), workspace.numel(),
+        _stream(stream)))
+    return W_packed, s_w
+
+
+def bitnet_rmsnorm_quant_act(x, gamma=None, eps=1e-5, x_q=None, s_x=None, stream=None):
+    """x [M,K] fp32/bf16 -> (x_q int8 [M,K], s_x fp32 [M])."""
+    if x.dim() != 2:
+        raise ValueError("x must be 2-D")
+    _need_cuda(x, gamma)
+    M, K = x.shape
+    if x_q is None:
+        x_q = torch.empty((M, K), dtype=torch.int8, device=x.device)
+    if s_x is None:
+        s_x = torch.empty((M,), dtype=torch.float32, device=x.device)
+    _need_cuda(x_q, s_x)
+    _check("bitnet_rmsnorm_quant_act", load_library().bitnet_rmsnorm_quant_act(
+        _ptr(x), _dtype_code(x.dtype), _ptr(gamma), float(eps), M, K, _ptr(x_q), _ptr(s_x),
+        _stream(stream)))
+    return x_q, s_x
+
+
+def _ws_for(M, N, K, device, workspace, stream):
+    nb = bitnet_linear_forward_workspace_bytes(M, N, K)
+    if workspace is None:
+        workspace = _default_ws.get(nb, device, stream)
+    _need_cuda(workspace)
+    return workspace
+
+
+def bitnet_linear_forward(x, gamma, eps, W_packed, s_w, y_dtype=torch.bfloat16, y=None,
+                          workspace=None, stream=None):
+    """y = BitLinear(x) with packed ternary weights; y [M,N] in y_dtype."""
+    _need_cuda(x, gamma, W_packed, s_w)
+    M, K = x.shape
+    N = W_packed.shape[0]
+    if W_packed.shape[1] * 4 != K:
+        raise ValueError("W_packed must be [N, K/4]")
+    if y is None:
+        y = torch.empty((M, N), dtype=y_dtype, device=x.device)
+    _need_cuda(y)
+    ws = _ws_for(M, N, K, x.device, workspace, stream)
+    _check("bitnet_linear_forward", load_library().bitnet_linear_forward(
+        _ptr(x), _dtype_code(x.dtype), _ptr(gamma), float(eps), _ptr(W_packed), _ptr(s_w),
+        M, N, K, _ptr(y), _dtype_code(y.dtype), _ptr(ws), ws.numel(), _stream(stream)))
+    return y
+
+
+def bitnet_linear_quantize_input(x, gamma, eps, N, workspace, stream=None):
+    """Phase 1 of the forward: quantize x [M,K] into `workspace` (sized for (M,N,K))."""
+    _need_cuda(x, gamma, workspace)
+    M, K = x.shape
+    _check("bitnet_linear_quantize_input", load_library().bitnet_linear_quantize_input(
+        _ptr(x), _dtype_code(x.dtype), _ptr(gamma), float(eps), M, int(N), K, _ptr(workspace),
+        workspace.numel(), _stream(stream)))
+    return workspace
+
+
+def bitnet_linear_matmul(W_packed, s_w, M, K, workspace, y_dtype=torch.bfloat16, y=None,
+                         stream=None):
+    """Phase 2: y [M,N] = dequant(quantized input in `workspace` x ternary(W)^T)."""
+    _need_cuda(W_packed, s_w, workspace)
+    N = W_packed.shape[0]
+    if y is None:
+        y = torch.empty((M, N), dtype=y_dtype, device=W_packed.device)
+    _need_cuda(y)
+    _check("bitnet_linear_matmul", load_library().bitnet_linear_matmul(
+        _ptr(W_packed), _ptr(s_w), int(M), N, int(K), _ptr(y), _dtype_code(y.dtype),
+        _ptr(workspace), workspace.numel(), _stream(stream)))
+    return y
+
+
+def bitnet_linear_forward_debug(x, gamma, eps, W_packed, s_w, y_dtype=torch.float32,
+                                path=BITNET_PATH_AUTO, want_y=True, workspace=None,
+                                stream=None):
+    """Forward that also returns x_q (natural order), s_x and the int32 accumulators."""
+    _need_cuda(x, gamma, W_packed, s_w)
+    M, K = x.shape
+    N = W_packed.shape[0]
+    dev = x.device
+    y = torch.empty((M, N), dtype=y_dtype, device=dev) if want_y else None
+    x_q = torch.empty((M, K), dtype=torch.int8, device=dev)
+    s_x = torch.empty((M,), dtype=torch.float32, device=dev)
+    acc = torch.empty((M, N), dtype=torch.int32, device=dev)
+    ws = _ws_for(M, N, K, dev, workspace, stream)
+    _check("bitnet_linear_forward_debug", load_library().bitnet_linear_forward_debug(
+        _ptr(x), _dtype_code(x.dtype), _ptr(gamma), float(eps), _ptr(W_packed), _ptr(s_w),
+        M, N, K, _ptr(y), _dtype_code(y_dtype), _ptr(ws), ws.numel(), _ptr(x_q), _ptr(s_x),
+        _ptr(acc), int(path), _stream(stream)))
+    return {"y": y, "x_q": x_q, "s_x": s_x, "acc": acc}
+
+
+def bitnet_ternary_matmul_i32(x_q, W_packed, path=BITNET_PATH_AUTO, acc=None, workspace=None,
+                              stream=None):
+    """acc int32 [M,N] = x_q (int8 [M,K]) times the ternary weights transposed."""
+    _need_cuda(x_q, W_packed)
+    if x_q.dtype != torch.int8:
+        raise TypeError("x_q must be int8")
+    M, K = x_q.shape
+    N = W_packed.shape[0]
+    if acc is None:
+        acc = torch.empty((M, N), dtype=torch.int32, device=x_q.device)
+    ws = _ws_for(M, N, K, x_q.device, workspace, stream)
+    _check("bitnet_ternary_matmul_i32", load_library().bitnet_ternary_matmul_i32(
+        _ptr(x_q), _ptr(W_packed), M, N, K, _ptr(acc), _ptr(ws), ws.numel(), int(path),
+        _stream(stream)))
+    return acc
+
+
+def bitnet_device_status(reset=True, stream=None):
+    """(status, detail) of the device status word; synchronises the stream."""
+    detail = ctypes.c_int(0)
+    code = load_library().bitnet_device_status(_stream(stream), 1 if reset else 0,
+                                               ctypes.byref(detail))
+    return int(code), int(detail.value)
+
+
+def bitnet_selftest_bounded_wait(limit_ns: int, stream=None):
+    _check("bitnet_selftest_bounded_wait",
+           load_library().bitnet_selftest_bounded_wait(int(limit_ns), _stream(stream)))
+
+
+class BitLinear:
+    """A linear layer y = x W^T with ternary weights, packed once on creation.
+
+    Holds W_packed (uint8 [N, K/4]), s_w (fp32 [1]) and the RMSNorm gain."""
+
+    def __init__(self, W, gamma=None, eps=1e-5):
+        self.W_packed, self.s_w = bitnet_quantize_pack_weights(W.contiguous())
+        self.gamma = gamma
+        self.eps = float(eps)
+        self.out_features, self.in_features = W.shape
+
+    def __call__(self, x, y_dtype=torch.bfloat16, y=None, stream=None):
+        return bitnet_linear_forward(x, self.gamma, self.eps, self.W_packed, self.s_w,
+                                     y_dtype=y_dtype, y=y, stream=stream)

@@ -1,0 +1,266 @@
+// act_quant.cuh -- fused RMSNorm + per-token absmax int8 activation
+// quantization, one CTA of 256 threads per token row.
+//
+// Method: "LLM を 1.58 ビットにファインチューニング：BitNet による極端な量子化",
+// section 量子化の仕組み (activations: per-token absmax to 8 bits in
+// [-128, 127] after a normalisation); "[論文レビュー] The Era of 1-bit LLMs",
+// section 提案手法 (RMSNorm); bitnet.cpp article (unite.ai), section 数学的基礎
+// item 2 (infinity-norm scale; its epsilon has no value on the page, read here
+// as a 1e-5 floor on max|x_n|).
+//
+// Bit-exactness: the row's sum of squares uses a fixed order -- element k
+// feeds partial (k/8) mod 256 through a fused multiply-add in increasing k
+// (thread t owns the 8-element chunks t, t+256, ...), then partial i absorbs
+// partial i+s for s = 128, ..., 1 -- and every other step is one correctly
+// rounded IEEE operation (explicit _rn intrinsics; no fast-math).  The max
+// and the integer row sum do not depend on order.
+//
+// Outputs: x_q in natural k order, or "k-interleaved" for the matmul kernels:
+// inside every 16-element group G the byte at 16G + 4r + i holds x_q at
+// k = 16G + 4i + r.  That matches how the matmul kernels unpack 2-bit codes
+// (mask-and-shift of a 32-bit word of 16 codes yields four words holding the
+// codes with k = 4i + r for a fixed r), so integer dot products pair the same
+// k on both sides.  rowsum[m] = sum_k x_q[m,k] lets the matmul use the raw
+// codes t+1 in {0,1,2} and subtract rowsum afterwards.
+#pragma once
+
+#include "common.cuh"
+
+namespace bitnet {
+
+constexpr int kActThreads = 256;
+
+template <bool kBF16>
+__device__ __forceinline__ void load_chunk8(const void* x, int64_t elem, float (&v)[8]) {
+  if (kBF16) {
+    const uint4 u = __ldg(reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(x) + elem));
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      v[2 * j] = __uint_as_float(w[j] << 16);
+      v[2 * j + 1] = __uint_as_float(w[j] & 0xFFFF0000u);
+    }
+  } else {
+    const float4* p = reinterpret_cast<const float4*>(static_cast<const float*>(x) + elem);
+    const float4 a = __ldg(p), b = __ldg(p + 1);
+    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+    v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+  }
+}
+
+__device__ __forceinline__ void load_gamma8(const float* gamma, int64_t k, float (&g)[8]) {
+  if (gamma) {
+    const float4* p = reinterpret_cast<const float4*>(gamma + k);
+    const float4 a = __ldg(p), b = __ldg(p + 1);
+    g[0] = a.x; g[1] = a.y; g[2] = a.z; g[3] = a.w;
+    g[4] = b.x; g[5] = b.y; g[6] = b.z; g[7] = b.w;
+  } else {
+#pragma unroll
+    for (int j = 0; j < 8; ++j) g[j] = 1.0f;
+  }
+}
+
+// Quantized bytes of one 8-element chunk packed little-endian into two words.
+struct Chunk8 {
+  uint32_t lo, hi;  // bytes k+0..3, k+4..7
+};
+
+// Store one chunk of quantized values.  In interleaved mode the two threads
+// (lanes l and l^1) holding the halves of a 16-element group swap four bytes
+// each so that every lane writes 8 contiguous output bytes.  All 32 lanes of
+// the warp must call this (valid or not).
+template <bool kInterleave>
+__device__ __forceinline__ void store_chunk8(int8_t* xq_row, int64_t k, Chunk8 c, bool valid) {
+  if (!kInterleave) {
+    if (valid) *reinterpret_cast<uint2*>(xq_row + k) = make_uint2(c.lo, c.hi);
+    return;
+  }
+  const int h = static_cast<int>((k >> 3) & 1);   // which half of the 16-group
+  // A = bytes (q0, q4, q1, q5), B = (q2, q6, q3, q7) of this half.
+  const uint32_t A = __byte_perm(c.lo, c.hi, 0x5140);
+  const uint32_t B = __byte_perm(c.lo, c.hi, 0x7362);
+  const uint32_t send = h ? A : B;
+  const uint32_t recv = __shfl_xor_sync(0xFFFFFFFFu, send, 1);
+  const uint32_t lo = h ? recv : A;   // half 0 contribution
+  const uint32_t hi = h ? B : recv;   // half 1 contribution
+  const uint32_t w0 = __byte_perm(lo, hi, 0x5410);
+  const uint32_t w1 = __byte_perm(lo, hi, 0x7632);
+  // half h writes bytes [8h, 8h+8) of the group, which start at element k
+  if (valid) *reinterpret_cast<uint2*>(xq_row + k) = make_uint2(w0, w1);
+}
+
+__device__ __forceinline__ int8_t quant_one(float xn, float sx) {
+  float q = rintf(__fmul_rn(xn, sx));
+  q = fminf(fmaxf(q, -128.0f), 127.0f);
+  return static_cast<int8_t>(static_cast<int>(q));
+}
+
+__device__ __forceinline__ uint32_t pack4(int8_t a, int8_t b, int8_t c, int8_t d) {
+  return (static_cast<uint32_t>(static_cast<uint8_t>(a))) |
+         (static_cast<uint32_t>(static_cast<uint8_t>(b)) << 8) |
+         (static_cast<uint32_t>(static_cast<uint8_t>(c)) << 16) |
+         (static_cast<uint32_t>(static_cast<uint8_t>(d)) << 24);
+}
+
+// Block-wide sum of squares in the canonical tree order; result valid in
+// all threads.
+__device__ __forceinline__ float block_tree_sum_f32(float p, float* red) {
+  const int tid = threadIdx.x;
+  red[tid] = p;
+  __syncthreads();
+#pragma unroll
+  for (int s = 128; s >= 32; s >>= 1) {
+    if (tid < s) red[tid] = __fadd_rn(red[tid], red[tid + s]);
+    __syncthreads();
+  }
+  if (tid < 32) {
+    float v = red[tid];
+#pragma unroll
+    for (int s = 16; s >= 1; s >>= 1) v = __fadd_rn(v, __shfl_down_sync(0xFFFFFFFFu, v, s));
+    if (tid == 0) red[0] = v;
+  }
+  __syncthreads();
+  const float r = red[0];
+  __syncthreads();
+  return r;
+}
+
+__device__ __forceinline__ float block_max_f32(float v, float* red) {
+  const int tid = threadIdx.x;
+#pragma unroll
+  for (int s = 16; s >= 1; s >>= 1) v = fmaxf(v, __shfl_xor_sync(0xFFFFFFFFu, v, s));
+  if ((tid & 31) == 0) red[tid >> 5] = v;
+  __syncthreads();
+  if (tid < 32) {
+    float w = (tid < kActThreads / 32) ? red[tid] : 0.0f;
+#pragma unroll
+    for (int s = 16; s >= 1; s >>= 1) w = fmaxf(w, __shfl_xor_sync(0xFFFFFFFFu, w, s));
+    if (tid == 0) red[0] = w;
+  }
+  __syncthreads();
+  const float r = red[0];
+  __syncthreads();
+  return r;
+}
+
+__device__ __forceinline__ int block_sum_i32(int v, int* red) {
+  const int tid = threadIdx.x;
+#pragma unroll
+  for (int s = 16; s >= 1; s >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, s);
+  if ((tid & 31) == 0) red[tid >> 5] = v;
+  __syncthreads();
+  int r = 0;
+#pragma unroll
+  for (int i = 0; i < kActThreads / 32; ++i) r += red[i];
+  __syncthreads();
+  return r;
+}
+
+// One CTA per row.  x: [M][K] (fp32 or bf16 bits), gamma: [K] or null.
+template <bool kBF16, bool kInterleave>
+__global__ void __launch_bounds__(kActThreads)
+rmsnorm_quant_kernel(const void* __restrict__ x, const float* __restrict__ gamma, float eps,
+                     int64_t K, int8_t* __restrict__ x_q, float* __restrict__ s_x,
+                     int32_t* __restrict__ rowsum, int trigger_dependents) {
+  __shared__ float redf[kActThreads];
+  __shared__ int redi[kActThreads / 32];
+  if (trigger_dependents) pdl_launch_dependents();
+
+  const int tid = threadIdx.x;
+  const int64_t m = blockIdx.x;
+  const int64_t nchunk = K >> 3;
+  const int iters = static_cast<int>((nchunk + kActThreads - 1) / kActThreads);
+  const int64_t row = m * K;
+
+  // Pass 1: sum of squares, partial = this thread's chunks in increasing k.
+  float p = 0.0f;
+  for (int it = 0; it < iters; ++it) {
+    const int64_t c = tid + static_cast<int64_t>(kActThreads) * it;
+    if (c < nchunk) {
+      float v[8];
+      load_chunk8<kBF16>(x, row + 8 * c, v);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) p = __fmaf_rn(v[j], v[j], p);
+    }
+  }
+  const float ss = block_tree_sum_f32(p, redf);
+  const float ms = __fdiv_rn(ss, static_cast<float>(K));
+  const float d = __fadd_rn(ms, eps);
+  const bool zero_row = (d == 0.0f);
+  const float r = zero_row ? 0.0f : __fdiv_rn(1.0f, __fsqrt_rn(d));
+
+  // Pass 2: max |x_n|.
+  float amax = 0.0f;
+  for (int it = 0; it < iters; ++it) {
+    const int64_t c = tid + static_cast<int64_t>(kActThreads) * it;
+    if (c < nchunk && !zero_row) {
+      float v[8], g[8];
+      load_chunk8<kBF16>(x, row + 8 * c, v);
+      load_gamma8(gamma, 8 * c, g);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) amax = fmaxf(amax, fabsf(__fmul_rn(__fmul_rn(v[j], r), g[j])));
+    }
+  }
+  amax = block_max_f32(amax, redf);
+  amax = fmaxf(amax, 1e-5f);
+  const float sx = __fdiv_rn(127.0f, amax);
+
+  // Pass 3: quantize, store, row sum.
+  int sum = 0;
+  int8_t* xq_row = x_q + row;
+  for (int it = 0; it < iters; ++it) {
+    const int64_t c = tid + static_cast<int64_t>(kActThreads) * it;
+    const bool valid = c < nchunk;
+    int8_t q[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+    if (valid && !zero_row) {
+      float v[8], g[8];
+      load_chunk8<kBF16>(x, row + 8 * c, v);
+      load_gamma8(gamma, 8 * c, g);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        q[j] = quant_one(__fmul_rn(__fmul_rn(v[j], r), g[j]), sx);
+        sum += q[j];
+      }
+    }
+    Chunk8 ch{pack4(q[0], q[1], q[2], q[3]), pack4(q[4], q[5], q[6], q[7])};
+    store_chunk8<kInterleave>(xq_row, 8 * c, ch, valid);
+  }
+  sum = block_sum_i32(sum, redi);
+  if (tid == 0) {
+    if (s_x) s_x[m] = sx;
+    if (rowsum) rowsum[m] = sum;
+  }
+}
+
+// Natural-order x_q -> k-interleaved copy plus per-row sums (used when the
+// caller hands in already-quantized activations).
+__global__ void __launch_bounds__(kActThreads)
+interleave_rowsum_kernel(const int8_t* __restrict__ x_q, int64_t K, int8_t* __restrict__ xi,
+                         int32_t* __restrict__ rowsum) {
+  __shared__ int redi[kActThreads / 32];
+  const int tid = threadIdx.x;
+  const int64_t m = blockIdx.x;
+  const int64_t nchunk = K >> 3;
+  const int iters = static_cast<int>((nchunk + kActThreads - 1) / kActThreads);
+  int sum = 0;
+  for (int it = 0; it < iters; ++it) {
+    const int64_t c = tid + static_cast<int64_t>(kActThreads) * it;
+    const bool valid = c < nchunk;
+    Chunk8 ch{0u, 0u};
+    if (valid) {
+      const uint2 u = __ldg(reinterpret_cast<const uint2*>(x_q + m * K + 8 * c));
+      ch.lo = u.x;
+      ch.hi = u.y;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        sum += static_cast<int8_t>((u.x >> (8 * j)) & 0xFF);
+        sum += static_cast<int8_t>((u.y >> (8 * j)) & 0xFF);
+      }
+    }
+    store_chunk8<true>(xi + m * K, 8 * c, ch, valid);
+  }
+  sum = block_sum_i32(sum, redi);
+  if (tid == 0) rowsum[m] = sum;
+}
+
+}  // namespace bitnet

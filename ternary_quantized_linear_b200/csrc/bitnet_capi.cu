@@ -1,0 +1,542 @@
+// bitnet_capi.cu -- the extern "C" boundary of libbitnet_b200.so: argument
+// validation, workspace layout, launch planning and kernel launches for the
+// BitNet b1.58 BitLinear forward.  The operations and their citations are
+// documented in include/bitnet_b200.h; the kernels are in the .cuh files
+// included below (one translation unit, so the device status word is a
+// single symbol).
+#include "bitnet_b200.h"
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cstdint>
+#include <mutex>
+
+#include "act_quant.cuh"
+#include "common.cuh"
+#include "gemm_tc.cuh"
+#include "gemv.cuh"
+#include "weight_quant.cuh"
+
+namespace bitnet {
+
+// First failure recorded by a kernel's bounded wait (per device).
+__device__ int g_device_status;
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+size_t align256(size_t v) { return (v + 255) & ~static_cast<size_t>(255); }
+
+cudaStream_t as_stream(bitnet_stream_t s) { return reinterpret_cast<cudaStream_t>(s); }
+
+bitnet_status launch_status() {
+  return cudaGetLastError() == cudaSuccess ? BITNET_OK : BITNET_ERR_CUDA;
+}
+
+// ------------------------------------------------------------ per-device state
+
+struct DeviceState {
+  std::once_flag once;
+  bool ok = false;
+  int* status = nullptr;  // device address of g_device_status
+  int num_sms = 148;
+};
+DeviceState g_dev[kMaxDevices];
+
+template <typename K>
+bool set_smem(K kernel, int bytes) {
+  return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) ==
+         cudaSuccess;
+}
+
+// Set up the current device once: status-word address, SM count, and the
+// shared-memory opt-in of every kernel instance.
+DeviceState* device_state() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  DeviceState& st = g_dev[dev];
+  std::call_once(st.once, [&st, dev]() {
+    bool ok = cudaGetSymbolAddress(reinterpret_cast<void**>(&st.status), g_device_status) ==
+              cudaSuccess;
+    ok = ok && cudaDeviceGetAttribute(&st.num_sms, cudaDevAttrMultiProcessorCount, dev) ==
+                   cudaSuccess;
+    ok = ok && set_smem(ternary_gemv_kernel<2, 1>, 8 * 1 * (16 * 256 + 16));
+    ok = ok && set_smem(ternary_gemv_kernel<2, 2>, 8 * 2 * (16 * 256 + 16));
+    ok = ok && set_smem(ternary_gemm_tc_kernel<64>, GemmCfg<64>::SMEM_DYN);
+    ok = ok && set_smem(ternary_gemm_tc_kernel<128>, GemmCfg<128>::SMEM_DYN);
+    ok = ok && set_smem(ternary_gemm_tc_kernel<256>, GemmCfg<256>::SMEM_DYN);
+    st.ok = ok;
+  });
+  return st.ok ? &st : nullptr;
+}
+
+// --------------------------------------------------------------- TMA maps
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, []() {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault,
+                                         &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// 2-D uint8 tensor [rows][inner] with the given row stride (bytes), boxes
+// of box_rows x box_inner; out-of-range elements read as zero.
+bool make_tmap_u8(CUtensorMap* map, const void* base, uint64_t inner, uint64_t rows,
+                  uint64_t row_stride, uint32_t box_inner, uint32_t box_rows,
+                  CUtensorMapSwizzle swz) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {inner, rows};
+  cuuint64_t strides[1] = {row_stride};
+  cuuint32_t box[2] = {box_inner, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box,
+             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// -------------------------------------------------------- workspace layout
+
+struct FwdWorkspace {
+  size_t xq, sx, rs, acc, cnt, total;
+};
+
+constexpr int64_t kGemvMaxM = 16;
+
+FwdWorkspace fwd_layout(int64_t M, int64_t N, int64_t K) {
+  FwdWorkspace w{};
+  size_t o = 0;
+  w.xq = o;
+  o = align256(o + static_cast<size_t>(M * K));
+  w.sx = o;
+  o = align256(o + 4 * static_cast<size_t>(M));
+  w.rs = o;
+  o = align256(o + 4 * static_cast<size_t>(M));
+  const bool gemv_capable = M <= kGemvMaxM;
+  w.acc = o;
+  o = align256(o + (gemv_capable ? 4 * static_cast<size_t>(M * N) : 0));
+  w.cnt = o;
+  o = align256(o + (gemv_capable ? 4 * static_cast<size_t>((N + 15) / 16) : 0));
+  w.total = o;
+  return w;
+}
+
+// ---------------------------------------------------------------- checks
+
+bitnet_status check_shape(int64_t M, int64_t N, int64_t K) {
+  if (M < 0 || N < 0 || K < 0) return BITNET_ERR_INVALID_ARG;
+  if (N < 1 || N > (1 << 24) || M > (1 << 24)) return BITNET_ERR_UNSUPPORTED_SHAPE;
+  if (K < 64 || K > BITNET_MAX_K || (K % 64) != 0) return BITNET_ERR_UNSUPPORTED_SHAPE;
+  return BITNET_OK;
+}
+
+bool ok_dtype(int d) { return d == BITNET_F32 || d == BITNET_BF16; }
+
+// ------------------------------------------------------------ launchers
+
+struct GemvPlan {
+  int NT, rb, ksplit, ips, warps;
+  size_t smem;
+};
+
+GemvPlan plan_gemv(int64_t M, int64_t N, int64_t K, int num_sms) {
+  GemvPlan pl{};
+  constexpr int kRows = 32;  // RG = 2
+  pl.NT = M <= 8 ? 1 : 2;
+  pl.rb = static_cast<int>((N + kRows - 1) / kRows);
+  const int iters = static_cast<int>((K + 255) / 256);
+  const int ks_min = (iters + 15) / 16;  // at most 16 steps (4096 k) staged per CTA
+  const int target = 4 * num_sms;
+  int ks = std::min(iters, (target + pl.rb - 1) / pl.rb);
+  ks = std::max(ks, ks_min);
+  pl.ips = (iters + ks - 1) / ks;
+  pl.ksplit = (iters + pl.ips - 1) / pl.ips;
+  pl.warps = std::min(8, pl.ips);
+  pl.smem = static_cast<size_t>(8 * pl.NT) * (pl.ips * 256 + 16);
+  return pl;
+}
+
+bitnet_status launch_gemv(const DeviceState& ds, const uint8_t* Wp, const int8_t* xi,
+                          const int32_t* rowsum, const float* s_x, const float* s_w, int64_t M,
+                          int64_t N, int64_t K, uint8_t* ws, const FwdWorkspace& L, void* y,
+                          int y_dtype, int32_t* acc_out, bool pdl, bool early_weights,
+                          cudaStream_t stream) {
+  const GemvPlan pl = plan_gemv(M, N, K, ds.num_sms);
+  GemvParams p{};
+  p.Wp = Wp;
+  p.xi = xi;
+  p.rowsum = rowsum;
+  p.s_x = s_x;
+  p.s_w = s_w;
+  p.M = static_cast<int>(M);
+  p.N = static_cast<int>(N);
+  p.K = static_cast<int>(K);
+  p.iters_per_split = pl.ips;
+  p.ws_acc = reinterpret_cast<int32_t*>(ws + L.acc);
+  p.ws_cnt = reinterpret_cast<unsigned*>(ws + L.cnt);
+  p.y = y;
+  p.y_bf16 = (y_dtype == BITNET_BF16) ? 1 : 0;
+  p.acc_out = acc_out;
+  p.use_pdl = pdl ? 1 : 0;
+  p.early_weights = (pdl && early_weights) ? 1 : 0;
+
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(static_cast<unsigned>(pl.rb), static_cast<unsigned>(pl.ksplit), 1);
+  cfg.blockDim = dim3(32 * pl.warps, 1, 1);
+  cfg.dynamicSmemBytes = pl.smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  cudaError_t e = (pl.NT == 1) ? cudaLaunchKernelEx(&cfg, ternary_gemv_kernel<2, 1>, p)
+                               : cudaLaunchKernelEx(&cfg, ternary_gemv_kernel<2, 2>, p);
+  return e == cudaSuccess ? BITNET_OK : BITNET_ERR_CUDA;
+}
+
+template <int BN>
+bitnet_status launch_gemm_bn(const DeviceState& ds, const CUtensorMap& tx, const CUtensorMap& tw,
+                             const GemmParams& p, int64_t M, int64_t N, cudaStream_t stream) {
+  (void)ds;
+  dim3 grid(static_cast<unsigned>((N + 127) / 128), static_cast<unsigned>((M + BN - 1) / BN), 1);
+  ternary_gemm_tc_kernel<BN><<<grid, 256, GemmCfg<BN>::SMEM_DYN, stream>>>(tx, tw, p);
+  return launch_status();
+}
+
+bitnet_status launch_gemm(const DeviceState& ds, const uint8_t* Wp, const int8_t* xi,
+                          const int32_t* rowsum, const float* s_x, const float* s_w, int64_t M,
+                          int64_t N, int64_t K, void* y, int y_dtype, int32_t* acc_out,
+                          cudaStream_t stream) {
+  const int BN = M <= 64 ? 64 : (M <= 128 ? 128 : 256);
+  CUtensorMap tx, tw;
+  if (!make_tmap_u8(&tx, xi, static_cast<uint64_t>(K), static_cast<uint64_t>(M),
+                    static_cast<uint64_t>(K), 128, static_cast<uint32_t>(BN),
+                    CU_TENSOR_MAP_SWIZZLE_128B))
+    return BITNET_ERR_CUDA;
+  if (!make_tmap_u8(&tw, Wp, static_cast<uint64_t>(K / 4), static_cast<uint64_t>(N),
+                    static_cast<uint64_t>(K / 4), 32, 128, CU_TENSOR_MAP_SWIZZLE_NONE))
+    return BITNET_ERR_CUDA;
+  GemmParams p{};
+  p.rowsum = rowsum;
+  p.s_x = s_x;
+  p.s_w = s_w;
+  p.M = static_cast<int>(M);
+  p.N = static_cast<int>(N);
+  p.K = static_cast<int>(K);
+  p.y = y;
+  p.y_bf16 = (y_dtype == BITNET_BF16) ? 1 : 0;
+  p.acc_out = acc_out;
+  p.status = ds.status;
+  p.wait_limit_ns = kWaitLimitNs;
+  switch (BN) {
+    case 64: return launch_gemm_bn<64>(ds, tx, tw, p, M, N, stream);
+    case 128: return launch_gemm_bn<128>(ds, tx, tw, p, M, N, stream);
+    default: return launch_gemm_bn<256>(ds, tx, tw, p, M, N, stream);
+  }
+}
+
+bitnet_status launch_act_quant(const void* x, int x_dtype, const float* gamma, float eps,
+                               int64_t M, int64_t K, int8_t* x_q, float* s_x, int32_t* rowsum,
+                               bool interleave, bool trigger, cudaStream_t stream) {
+  dim3 grid(static_cast<unsigned>(M)), block(kActThreads);
+  const int trig = trigger ? 1 : 0;
+  if (x_dtype == BITNET_BF16) {
+    if (interleave)
+      rmsnorm_quant_kernel<true, true><<<grid, block, 0, stream>>>(x, gamma, eps, K, x_q, s_x,
+                                                                   rowsum, trig);
+    else
+      rmsnorm_quant_kernel<true, false><<<grid, block, 0, stream>>>(x, gamma, eps, K, x_q, s_x,
+                                                                    rowsum, trig);
+  } else {
+    if (interleave)
+      rmsnorm_quant_kernel<false, true><<<grid, block, 0, stream>>>(x, gamma, eps, K, x_q, s_x,
+                                                                    rowsum, trig);
+    else
+      rmsnorm_quant_kernel<false, false><<<grid, block, 0, stream>>>(x, gamma, eps, K, x_q, s_x,
+                                                                     rowsum, trig);
+  }
+  return launch_status();
+}
+
+// Matmul + fused dequant on already-prepared interleaved activations.
+bitnet_status run_matmul(const DeviceState& ds, int path, const uint8_t* Wp, uint8_t* ws,
+                         const FwdWorkspace& L, const float* s_x, const float* s_w, int64_t M,
+                         int64_t N, int64_t K, void* y, int y_dtype, int32_t* acc_out, bool pdl,
+                         bool early_weights, cudaStream_t stream) {
+  const int8_t* xi = reinterpret_cast<const int8_t*>(ws + L.xq);
+  const int32_t* rs = reinterpret_cast<const int32_t*>(ws + L.rs);
+  if (path == BITNET_PATH_GEMV)
+    return launch_gemv(ds, Wp, xi, rs, s_x, s_w, M, N, K, ws, L, y, y_dtype, acc_out, pdl,
+                       early_weights, stream);
+  return launch_gemm(ds, Wp, xi, rs, s_x, s_w, M, N, K, y, y_dtype, acc_out, stream);
+}
+
+int resolve_path(int path, int64_t M) {
+  if (path == BITNET_PATH_AUTO) return M <= kGemvMaxM ? BITNET_PATH_GEMV : BITNET_PATH_GEMM;
+  return path;
+}
+
+bitnet_status forward_impl(const void* x, int x_dtype, const float* gamma, float eps,
+                           const uint8_t* W_packed, const float* s_w, int64_t M, int64_t N,
+                           int64_t K, void* y, int y_dtype, void* workspace,
+                           size_t workspace_bytes, int8_t* x_q_out, float* s_x_out,
+                           int32_t* acc_out, int path, cudaStream_t stream) {
+  bitnet_status st = check_shape(M, N, K);
+  if (st != BITNET_OK) return st;
+  if (!x || !W_packed || !s_w || !ok_dtype(x_dtype) || !(eps >= 0.0f) || eps > 3.0e38f)
+    return BITNET_ERR_INVALID_ARG;
+  if (y && !ok_dtype(y_dtype)) return BITNET_ERR_INVALID_ARG;
+  if (path < BITNET_PATH_AUTO || path > BITNET_PATH_GEMM) return BITNET_ERR_INVALID_ARG;
+  path = resolve_path(path, M);
+  if (path == BITNET_PATH_GEMV && M > kGemvMaxM) return BITNET_ERR_INVALID_ARG;
+  if (!aligned(x, 16) || (gamma && !aligned(gamma, 16)) || !aligned(W_packed, 16) ||
+      !aligned(s_w, 4) || (y && !aligned(y, 16)) || (x_q_out && !aligned(x_q_out, 16)) ||
+      (s_x_out && !aligned(s_x_out, 4)) || (acc_out && !aligned(acc_out, 16)))
+    return BITNET_ERR_MISALIGNED;
+  if (M == 0) return BITNET_OK;
+  const FwdWorkspace L = fwd_layout(M, N, K);
+  if (!workspace || workspace_bytes < L.total) return BITNET_ERR_WORKSPACE;
+  if (!aligned(workspace, 256)) return BITNET_ERR_MISALIGNED;
+  DeviceState* ds = device_state();
+  if (!ds) return BITNET_ERR_CUDA;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+
+  if (x_q_out || s_x_out) {
+    // Debug export in natural k order (same arithmetic as the fused pass).
+    int8_t* xq_nat = x_q_out ? x_q_out : reinterpret_cast<int8_t*>(ws + L.xq);
+    st = launch_act_quant(x, x_dtype, gamma, eps, M, K, xq_nat, s_x_out, nullptr, false, false,
+                          stream);
+    if (st != BITNET_OK) return st;
+  }
+  const bool pdl = (path == BITNET_PATH_GEMV);
+  float* sx = reinterpret_cast<float*>(ws + L.sx);
+  st = launch_act_quant(x, x_dtype, gamma, eps, M, K, reinterpret_cast<int8_t*>(ws + L.xq), sx,
+                        reinterpret_cast<int32_t*>(ws + L.rs), true, pdl, stream);
+  if (st != BITNET_OK) return st;
+  // The activation-quant kernel just queued started after every earlier
+  // write to W_packed, so the GEMV may fetch weights before waiting on it.
+  return run_matmul(*ds, path, W_packed, ws, L, sx, s_w, M, N, K, y, y_dtype, acc_out, pdl,
+                    pdl, stream);
+}
+
+}  // namespace
+}  // namespace bitnet
+
+using namespace bitnet;
+
+extern "C" {
+
+BITNET_API const char* bitnet_status_string(int status) {
+  switch (status) {
+    case BITNET_OK: return "ok";
+    case BITNET_ERR_INVALID_ARG: return "invalid argument";
+    case BITNET_ERR_UNSUPPORTED_SHAPE: return "unsupported shape (need N >= 1, 64 <= K <= 2^20, K % 64 == 0)";
+    case BITNET_ERR_MISALIGNED: return "misaligned pointer (tensors 16-byte, workspace 256-byte)";
+    case BITNET_ERR_CUDA: return "CUDA error";
+    case BITNET_ERR_TIMEOUT: return "bounded on-device wait timed out";
+    case BITNET_ERR_WORKSPACE: return "workspace missing or too small";
+    default: return "unknown status";
+  }
+}
+
+BITNET_API int bitnet_version(void) { return 100; }
+
+BITNET_API size_t bitnet_quantize_pack_weights_workspace_bytes(int64_t N, int64_t K) {
+  (void)K;
+  return N > 0 ? align256(8 * static_cast<size_t>(N)) : 0;
+}
+
+BITNET_API bitnet_status bitnet_quantize_pack_weights(const float* W, int64_t N, int64_t K,
+                                                      uint8_t* W_packed, float* s_w,
+                                                      void* workspace, size_t workspace_bytes,
+                                                      bitnet_stream_t stream) {
+  bitnet_status st = check_shape(0, N, K);
+  if (st != BITNET_OK) return st;
+  if (!W || !W_packed || !s_w) return BITNET_ERR_INVALID_ARG;
+  if (!aligned(W, 16) || !aligned(W_packed, 16) || !aligned(s_w, 4)) return BITNET_ERR_MISALIGNED;
+  if (!workspace || workspace_bytes < bitnet_quantize_pack_weights_workspace_bytes(N, K))
+    return BITNET_ERR_WORKSPACE;
+  if (!aligned(workspace, 256)) return BITNET_ERR_MISALIGNED;
+  DeviceState* ds = device_state();
+  if (!ds) return BITNET_ERR_CUDA;
+  cudaStream_t s = as_stream(stream);
+  double* R = static_cast<double*>(workspace);
+  row_abs_sum_kernel<<<static_cast<unsigned>(N), kWqThreads, 0, s>>>(W, K, R);
+  abs_total_kernel<<<1, kWqThreads, 0, s>>>(R, N, K, s_w);
+  const int64_t nwords = N * K / 16;
+  const int64_t blocks = std::min<int64_t>((nwords + kWqThreads - 1) / kWqThreads,
+                                           static_cast<int64_t>(ds->num_sms) * 16);
+  pack_kernel<<<static_cast<unsigned>(blocks), kWqThreads, 0, s>>>(
+      W, nwords, s_w, reinterpret_cast<uint32_t*>(W_packed));
+  return launch_status();
+}
+
+BITNET_API bitnet_status bitnet_rmsnorm_quant_act(const void* x, int x_dtype, const float* gamma,
+                                                  float eps, int64_t M, int64_t K, int8_t* x_q,
+                                                  float* s_x, bitnet_stream_t stream) {
+  bitnet_status st = check_shape(M, 1, K);
+  if (st != BITNET_OK) return st;
+  if (!x || !x_q || !s_x || !ok_dtype(x_dtype) || !(eps >= 0.0f) || eps > 3.0e38f)
+    return BITNET_ERR_INVALID_ARG;
+  if (!aligned(x, 16) || (gamma && !aligned(gamma, 16)) || !aligned(x_q, 16) || !aligned(s_x, 4))
+    return BITNET_ERR_MISALIGNED;
+  if (M == 0) return BITNET_OK;
+  if (!device_state()) return BITNET_ERR_CUDA;
+  return launch_act_quant(x, x_dtype, gamma, eps, M, K, x_q, s_x, nullptr, false, false,
+                          as_stream(stream));
+}
+
+BITNET_API size_t bitnet_linear_forward_workspace_bytes(int64_t M, int64_t N, int64_t K) {
+  if (M < 0 || N < 0 || K < 0) return 0;
+  return fwd_layout(M, N, K).total;
+}
+
+BITNET_API bitnet_status bitnet_linear_forward(const void* x, int x_dtype, const float* gamma,
+                                               float eps, const uint8_t* W_packed,
+                                               const float* s_w, int64_t M, int64_t N, int64_t K,
+                                               void* y, int y_dtype, void* workspace,
+                                               size_t workspace_bytes, bitnet_stream_t stream) {
+  if (!y) return BITNET_ERR_INVALID_ARG;
+  return forward_impl(x, x_dtype, gamma, eps, W_packed, s_w, M, N, K, y, y_dtype, workspace,
+                      workspace_bytes, nullptr, nullptr, nullptr, BITNET_PATH_AUTO,
+                      as_stream(stream));
+}
+
+BITNET_API bitnet_status bitnet_linear_quantize_input(const void* x, int x_dtype,
+                                                      const float* gamma, float eps, int64_t M,
+                                                      int64_t N, int64_t K, void* workspace,
+                                                      size_t workspace_bytes,
+                                                      bitnet_stream_t stream) {
+  bitnet_status st = check_shape(M, N, K);
+  if (st != BITNET_OK) return st;
+  if (!x || !ok_dtype(x_dtype) || !(eps >= 0.0f) || eps > 3.0e38f) return BITNET_ERR_INVALID_ARG;
+  if (!aligned(x, 16) || (gamma && !aligned(gamma, 16))) return BITNET_ERR_MISALIGNED;
+  if (M == 0) return BITNET_OK;
+  const FwdWorkspace L = fwd_layout(M, N, K);
+  if (!workspace || workspace_bytes < L.total) return BITNET_ERR_WORKSPACE;
+  if (!aligned(workspace, 256)) return BITNET_ERR_MISALIGNED;
+  if (!device_state()) return BITNET_ERR_CUDA;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  return launch_act_quant(x, x_dtype, gamma, eps, M, K, reinterpret_cast<int8_t*>(ws + L.xq),
+                          reinterpret_cast<float*>(ws + L.sx),
+                          reinterpret_cast<int32_t*>(ws + L.rs), true, M <= kGemvMaxM,
+                          as_stream(stream));
+}
+
+BITNET_API bitnet_status bitnet_linear_matmul(const uint8_t* W_packed, const float* s_w,
+                                              int64_t M, int64_t N, int64_t K, void* y,
+                                              int y_dtype, void* workspace,
+                                              size_t workspace_bytes, bitnet_stream_t stream) {
+  bitnet_status st = check_shape(M, N, K);
+  if (st != BITNET_OK) return st;
+  if (!W_packed || !s_w || !y || !ok_dtype(y_dtype)) return BITNET_ERR_INVALID_ARG;
+  if (!aligned(W_packed, 16) || !aligned(s_w, 4) || !aligned(y, 16)) return BITNET_ERR_MISALIGNED;
+  if (M == 0) return BITNET_OK;
+  const FwdWorkspace L = fwd_layout(M, N, K);
+  if (!workspace || workspace_bytes < L.total) return BITNET_ERR_WORKSPACE;
+  if (!aligned(workspace, 256)) return BITNET_ERR_MISALIGNED;
+  DeviceState* ds = device_state();
+  if (!ds) return BITNET_ERR_CUDA;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  const int path = resolve_path(BITNET_PATH_AUTO, M);
+  return run_matmul(*ds, path, W_packed, ws, L, reinterpret_cast<const float*>(ws + L.sx), s_w,
+                    M, N, K, y, y_dtype, nullptr, path == BITNET_PATH_GEMV, false,
+                    as_stream(stream));
+}
+
+BITNET_API bitnet_status bitnet_linear_forward_debug(
+    const void* x, int x_dtype, const float* gamma, float eps, const uint8_t* W_packed,
+    const float* s_w, int64_t M, int64_t N, int64_t K, void* y, int y_dtype, void* workspace,
+    size_t workspace_bytes, int8_t* x_q_out, float* s_x_out, int32_t* acc_out, int path,
+    bitnet_stream_t stream) {
+  return forward_impl(x, x_dtype, gamma, eps, W_packed, s_w, M, N, K, y, y_dtype, workspace,
+                      workspace_bytes, x_q_out, s_x_out, acc_out, path, as_stream(stream));
+}
+
+BITNET_API bitnet_status bitnet_ternary_matmul_i32(const int8_t* x_q, const uint8_t* W_packed,
+                                                   int64_t M, int64_t N, int64_t K, int32_t* acc,
+                                                   void* workspace, size_t workspace_bytes,
+                                                   int path, bitnet_stream_t stream) {
+  bitnet_status st = check_shape(M, N, K);
+  if (st != BITNET_OK) return st;
+  if (!x_q || !W_packed || !acc) return BITNET_ERR_INVALID_ARG;
+  if (path < BITNET_PATH_AUTO || path > BITNET_PATH_GEMM) return BITNET_ERR_INVALID_ARG;
+  path = resolve_path(path, M);
+  if (path == BITNET_PATH_GEMV && M > kGemvMaxM) return BITNET_ERR_INVALID_ARG;
+  if (!aligned(x_q, 16) || !aligned(W_packed, 16) || !aligned(acc, 16))
+    return BITNET_ERR_MISALIGNED;
+  if (M == 0) return BITNET_OK;
+  const FwdWorkspace L = fwd_layout(M, N, K);
+  if (!workspace || workspace_bytes < L.total) return BITNET_ERR_WORKSPACE;
+  if (!aligned(workspace, 256)) return BITNET_ERR_MISALIGNED;
+  DeviceState* ds = device_state();
+  if (!ds) return BITNET_ERR_CUDA;
+  cudaStream_t s = as_stream(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  interleave_rowsum_kernel<<<static_cast<unsigned>(M), kActThreads, 0, s>>>(
+      x_q, K, reinterpret_cast<int8_t*>(ws + L.xq), reinterpret_cast<int32_t*>(ws + L.rs));
+  st = launch_status();
+  if (st != BITNET_OK) return st;
+  return run_matmul(*ds, path, W_packed, ws, L, nullptr, nullptr, M, N, K, nullptr, BITNET_F32,
+                    acc, false, false, s);
+}
+
+BITNET_API bitnet_status bitnet_device_status(bitnet_stream_t stream, int reset, int* detail) {
+  DeviceState* ds = device_state();
+  if (!ds) return BITNET_ERR_CUDA;
+  cudaStream_t s = as_stream(stream);
+  int v = 0;
+  if (cudaMemcpyAsync(&v, ds->status, sizeof(int), cudaMemcpyDeviceToHost, s) != cudaSuccess)
+    return BITNET_ERR_CUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return BITNET_ERR_CUDA;
+  if (detail) *detail = v;
+  if (reset && v != 0) {
+    if (cudaMemsetAsync(ds->status, 0, sizeof(int), s) != cudaSuccess) return BITNET_ERR_CUDA;
+    if (cudaStreamSynchronize(s) != cudaSuccess) return BITNET_ERR_CUDA;
+  }
+  return v == 0 ? BITNET_OK : BITNET_ERR_TIMEOUT;
+}
+
+}  // extern "C"
+
+namespace bitnet {
+namespace {
+__global__ void bounded_wait_selftest_kernel(int* status, uint64_t limit_ns) {
+  __shared__ uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);  // nothing ever arrives on it
+    fence_mbarrier_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0 && !mbar_wait_bounded(&bar, 0u, nullptr, limit_ns))
+    record_failure(status, DEV_TIMEOUT_SELFTEST);
+}
+}  // namespace
+}  // namespace bitnet
+
+extern "C" BITNET_API bitnet_status bitnet_selftest_bounded_wait(uint64_t limit_ns,
+                                                                 bitnet_stream_t stream) {
+  if (limit_ns < 1000ull || limit_ns > 1000000000ull) return BITNET_ERR_INVALID_ARG;
+  DeviceState* ds = device_state();
+  if (!ds) return BITNET_ERR_CUDA;
+  bounded_wait_selftest_kernel<<<1, 32, 0, as_stream(stream)>>>(ds->status, limit_ns);
+  return launch_status();
+}

@@ -1,0 +1,121 @@
+"""Host-side checks of the C ABI that need no GPU: the library loads, exports
+every entry point include/bitnet_b200.h declares, sizes its workspaces, and
+rejects bad arguments before touching the device (the invalid calls below use
+fake pointer values that are never dereferenced)."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+import ternary_quantized_linear_b200 as tql
+from ternary_quantized_linear_b200 import build as tql_build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "bitnet_b200.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    tql_build.build()
+    return tql.load_library()
+
+
+def _declared():
+    src = open(HEADER).read()
+    return sorted(set(re.findall(r"BITNET_API[^;{]*?\b(bitnet_\w+)\s*\(", src, re.S)))
+
+
+def test_header_declares_the_three_core_calls():
+    names = _declared()
+    for n in ("bitnet_quantize_pack_weights", "bitnet_rmsnorm_quant_act",
+              "bitnet_linear_forward", "bitnet_linear_forward_debug",
+              "bitnet_ternary_matmul_i32"):
+        assert n in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    out = subprocess.run(["nm", "-D", "--defined-only", tql.LIB_PATH], capture_output=True,
+                         text=True, check=True).stdout
+    exported = set(re.findall(r"\s[TW]\s+(bitnet_\w+)$", out, re.M))
+    declared = set(_declared())
+    assert declared <= exported, declared - exported
+    assert declared == set(tql.EXPORTED)
+    # nothing else leaks out of the library
+    assert exported == declared
+
+
+def test_status_strings(lib):
+    for code in range(0, 7):
+        assert tql.bitnet_status_string(code)
+    assert tql.bitnet_status_string(99) == "unknown status"
+    assert tql.bitnet_version() >= 100
+
+
+def test_workspace_sizes(lib):
+    assert tql.bitnet_quantize_pack_weights_workspace_bytes(1000, 4096) >= 8000
+    small = tql.bitnet_linear_forward_workspace_bytes(16, 3200, 3200)
+    # x_q + scales + row sums + split-K int32 partials + counters
+    assert small >= 16 * 3200 + 16 * 3200 * 4
+    assert small % 256 == 0
+    big = tql.bitnet_linear_forward_workspace_bytes(2048, 14336, 4096)
+    assert big >= 2048 * 4096 and big < 2048 * 4096 + 64 * 1024
+    assert tql.bitnet_linear_forward_workspace_bytes(-1, 1, 64) == 0
+
+
+FAKE = 0x10000  # 64 KiB-aligned fake device address, never dereferenced
+
+
+def _fwd(lib, x=FAKE, xd=1, gamma=None, eps=1e-5, wp=FAKE, sw=FAKE, M=4, N=64, K=256,
+         y=FAKE, yd=1, ws=FAKE, wsb=1 << 30):
+    P = ctypes.c_void_p
+    return lib.bitnet_linear_forward(P(x), xd, P(gamma) if gamma else None, ctypes.c_float(eps),
+                                     P(wp), P(sw), M, N, K, P(y), yd, P(ws), wsb, None)
+
+
+def test_forward_rejects_bad_arguments(lib):
+    assert _fwd(lib, K=100) == tql.BITNET_ERR_UNSUPPORTED_SHAPE
+    assert _fwd(lib, K=0) == tql.BITNET_ERR_UNSUPPORTED_SHAPE
+    assert _fwd(lib, K=32) == tql.BITNET_ERR_UNSUPPORTED_SHAPE
+    assert _fwd(lib, N=0) == tql.BITNET_ERR_UNSUPPORTED_SHAPE
+    assert _fwd(lib, M=-1) == tql.BITNET_ERR_INVALID_ARG
+    assert _fwd(lib, x=0) == tql.BITNET_ERR_INVALID_ARG
+    assert _fwd(lib, y=0) == tql.BITNET_ERR_INVALID_ARG
+    assert _fwd(lib, xd=7) == tql.BITNET_ERR_INVALID_ARG
+    assert _fwd(lib, eps=-1.0) == tql.BITNET_ERR_INVALID_ARG
+    assert _fwd(lib, eps=float("nan")) == tql.BITNET_ERR_INVALID_ARG
+    assert _fwd(lib, x=FAKE + 8) == tql.BITNET_ERR_MISALIGNED
+    assert _fwd(lib, wp=FAKE + 4) == tql.BITNET_ERR_MISALIGNED
+    assert _fwd(lib, ws=FAKE + 128) == tql.BITNET_ERR_MISALIGNED
+    assert _fwd(lib, wsb=16) == tql.BITNET_ERR_WORKSPACE
+    assert _fwd(lib, ws=0) == tql.BITNET_ERR_WORKSPACE
+    # empty batch: valid, queues nothing, touches no pointer
+    assert _fwd(lib, M=0) == tql.BITNET_OK
+
+
+def test_other_entry_points_reject_bad_arguments(lib):
+    P = ctypes.c_void_p
+    assert lib.bitnet_quantize_pack_weights(P(FAKE), 64, 100, P(FAKE), P(FAKE), P(FAKE), 1 << 20,
+                                            None) == tql.BITNET_ERR_UNSUPPORTED_SHAPE
+    assert lib.bitnet_quantize_pack_weights(P(FAKE), 64, 128, P(FAKE), P(FAKE), P(FAKE), 8,
+                                            None) == tql.BITNET_ERR_WORKSPACE
+    assert lib.bitnet_quantize_pack_weights(P(FAKE + 4), 64, 128, P(FAKE), P(FAKE), P(FAKE),
+                                            1 << 20, None) == tql.BITNET_ERR_MISALIGNED
+    assert lib.bitnet_rmsnorm_quant_act(P(FAKE), 0, None, ctypes.c_float(1e-5), 2, 96, P(FAKE),
+                                        P(FAKE), None) == tql.BITNET_ERR_UNSUPPORTED_SHAPE
+    assert lib.bitnet_rmsnorm_quant_act(P(FAKE), 0, None, ctypes.c_float(1e-5), 0, 128, P(FAKE),
+                                        P(FAKE), None) == tql.BITNET_OK
+    # the GEMV path is only for M <= 16
+    assert lib.bitnet_ternary_matmul_i32(P(FAKE), P(FAKE), 17, 64, 128, P(FAKE), P(FAKE), 1 << 30,
+                                         tql.BITNET_PATH_GEMV, None) == tql.BITNET_ERR_INVALID_ARG
+    assert lib.bitnet_ternary_matmul_i32(P(FAKE), P(FAKE), 4, 64, 128, P(FAKE), P(FAKE), 1 << 30,
+                                         9, None) == tql.BITNET_ERR_INVALID_ARG
+    assert lib.bitnet_selftest_bounded_wait(10, None) == tql.BITNET_ERR_INVALID_ARG
+
+
+def test_binding_refuses_cpu_tensors(lib):
+    import torch
+    W = torch.zeros(64, 128)
+    with pytest.raises(ValueError):
+        tql.bitnet_quantize_pack_weights(W)
