@@ -141,15 +141,10 @@ BITNET_API bitnet_status bitnet_rmsnorm_quant_act(const void *x, int x_dtype, co
  *                            (s_w is read on the device).
  *   y                        [M][N] out, fp32 or bf16 per y_dtype.
  *   workspace                >= bitnet_linear_forward_workspace_bytes(M,N,K)
- *                            bytes, 256-byte aligned.  It MUST be zero-filled
- *                            before its first use: for M <= 16 it holds int32
- *                            split-K partial sums and arrival counters that
- *                            must start at zero, and every successful call
- *                            returns that region to zero, so a buffer zeroed
- *                            once can be reused by any number of calls that
- *                            do not overlap in time (its other bytes are
- *                            rewritten by each call).  After a failed call,
- *                            zero it again.
+ *                            bytes, 256-byte aligned; its contents on entry
+ *                            do not matter (the call clears what must start
+ *                            at zero).  Calls that share a workspace must not
+ *                            overlap in time (use one per stream).
  * ---------------------------------------------------------------------- */
 BITNET_API size_t bitnet_linear_forward_workspace_bytes(int64_t M, int64_t N, int64_t K);
 BITNET_API bitnet_status bitnet_linear_forward(const void *x, int x_dtype, const float *gamma,
@@ -172,9 +167,9 @@ BITNET_API bitnet_status bitnet_linear_forward(const void *x, int x_dtype, const
  *   serve (it only sizes the workspace).
  * bitnet_linear_matmul -- integer matmul of the workspace's quantized input
  *   with W_packed and the fused dequant into y.  M and K must equal those of
- *   the preceding bitnet_linear_quantize_input on the same workspace, and
- *   workspace_bytes must cover (M, N, K).  Any number of matmuls may follow
- *   one quantize call, in stream order.
+ *   the preceding bitnet_linear_quantize_input on the same workspace, N must
+ *   not exceed the N given to it, and workspace_bytes must cover (M, N, K).
+ *   Any number of matmuls may follow one quantize call, in stream order.
  * ---------------------------------------------------------------------- */
 BITNET_API bitnet_status bitnet_linear_quantize_input(const void *x, int x_dtype,
                                                       const float *gamma, float eps, int64_t M,
@@ -209,8 +204,8 @@ BITNET_API bitnet_status bitnet_linear_forward_debug(
  *   x_q       [M][K] int8 (natural k order, any values in [-128, 127]).
  *   W_packed  [N][K/4].
  *   acc       [M][N] int32 out.
- *   workspace >= bitnet_linear_forward_workspace_bytes(M,N,K), zero-filled
- *             before first use (same contract as the forward).
+ *   workspace >= bitnet_linear_forward_workspace_bytes(M,N,K) (same contract
+ *             as the forward).
  *   path      a bitnet_path value.
  * ---------------------------------------------------------------------- */
 BITNET_API bitnet_status bitnet_ternary_matmul_i32(const int8_t *x_q, const uint8_t *W_packed,

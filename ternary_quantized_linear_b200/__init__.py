@@ -120,11 +120,8 @@ def _need_cuda(*ts):
 
 
 class Workspace:
-    """Zero-initialised device scratch reused across calls on one stream.
-
-    The forward's split-K partials and counters must start at zero; the
-    kernels leave them zeroed after every successful call, so one buffer
-    allocated with zeros serves any number of stream-ordered calls."""
+    """Device scratch reused across stream-ordered calls (one buffer per
+    device and stream, grown on demand; the library clears what it needs)."""
 
     def __init__(self):
         self._buf = {}
@@ -134,7 +131,7 @@ class Workspace:
                0 if stream is None else stream.cuda_stream)
         buf = self._buf.get(key)
         if buf is None or buf.numel() < nbytes:
-            buf = torch.zeros(max(int(nbytes), 256), dtype=torch.uint8, device=device)
+            buf = torch.empty(max(int(nbytes), 256), dtype=torch.uint8, device=device)
             self._buf[key] = buf
         return buf
 

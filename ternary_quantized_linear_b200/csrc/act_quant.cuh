@@ -156,15 +156,32 @@ __device__ __forceinline__ int block_sum_i32(int v, int* red) {
   return r;
 }
 
-// One CTA per row.  x: [M][K] (fp32 or bf16 bits), gamma: [K] or null.
+// Blocks past the M row blocks clear a byte range of the workspace (the
+// matmul's split-K partials and counters, which must start at zero) so that
+// no separate memset launch is needed.  n16 = number of 16-byte words.
+__device__ __forceinline__ void zero_fill_blocks(uint4* __restrict__ dst, int64_t n16,
+                                                 int64_t first_block) {
+  const int64_t nb = static_cast<int64_t>(gridDim.x) - first_block;
+  const int64_t start = (static_cast<int64_t>(blockIdx.x) - first_block) * kActThreads +
+                        threadIdx.x;
+  for (int64_t i = start; i < n16; i += nb * kActThreads) dst[i] = make_uint4(0u, 0u, 0u, 0u);
+}
+
+// One CTA per row (blocks >= M zero `zero16` instead).  x: [M][K] (fp32 or
+// bf16 bits), gamma: [K] or null.
 template <bool kBF16, bool kInterleave>
 __global__ void __launch_bounds__(kActThreads)
 rmsnorm_quant_kernel(const void* __restrict__ x, const float* __restrict__ gamma, float eps,
-                     int64_t K, int8_t* __restrict__ x_q, float* __restrict__ s_x,
-                     int32_t* __restrict__ rowsum, int trigger_dependents) {
+                     int64_t M, int64_t K, int8_t* __restrict__ x_q, float* __restrict__ s_x,
+                     int32_t* __restrict__ rowsum, uint4* __restrict__ zero16, int64_t n_zero16,
+                     int trigger_dependents) {
   __shared__ float redf[kActThreads];
   __shared__ int redi[kActThreads / 32];
   if (trigger_dependents) pdl_launch_dependents();
+  if (static_cast<int64_t>(blockIdx.x) >= M) {
+    zero_fill_blocks(zero16, n_zero16, M);
+    return;
+  }
 
   const int tid = threadIdx.x;
   const int64_t m = blockIdx.x;
@@ -235,9 +252,14 @@ rmsnorm_quant_kernel(const void* __restrict__ x, const float* __restrict__ gamma
 // Natural-order x_q -> k-interleaved copy plus per-row sums (used when the
 // caller hands in already-quantized activations).
 __global__ void __launch_bounds__(kActThreads)
-interleave_rowsum_kernel(const int8_t* __restrict__ x_q, int64_t K, int8_t* __restrict__ xi,
-                         int32_t* __restrict__ rowsum) {
+interleave_rowsum_kernel(const int8_t* __restrict__ x_q, int64_t M, int64_t K,
+                         int8_t* __restrict__ xi, int32_t* __restrict__ rowsum,
+                         uint4* __restrict__ zero16, int64_t n_zero16) {
   __shared__ int redi[kActThreads / 32];
+  if (static_cast<int64_t>(blockIdx.x) >= M) {
+    zero_fill_blocks(zero16, n_zero16, M);
+    return;
+  }
   const int tid = threadIdx.x;
   const int64_t m = blockIdx.x;
   const int64_t nchunk = K >> 3;

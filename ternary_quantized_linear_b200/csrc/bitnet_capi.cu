@@ -253,27 +253,47 @@ bitnet_status launch_gemm(const DeviceState& ds, const uint8_t* Wp, const int8_t
   }
 }
 
+// Extra blocks appended to a row-per-block kernel to clear `bytes` bytes.
+int64_t zero_blocks(size_t bytes) {
+  if (bytes == 0) return 0;
+  const int64_t per_block = 16 * kActThreads * 4;  // four 16-byte stores per thread
+  return std::min<int64_t>(256, (static_cast<int64_t>(bytes) + per_block - 1) / per_block);
+}
+
+// zero/zero_bytes: a 16-byte aligned range (multiple of 16 bytes) cleared by
+// extra blocks of the same launch, or null/0.
 bitnet_status launch_act_quant(const void* x, int x_dtype, const float* gamma, float eps,
                                int64_t M, int64_t K, int8_t* x_q, float* s_x, int32_t* rowsum,
-                               bool interleave, bool trigger, cudaStream_t stream) {
-  dim3 grid(static_cast<unsigned>(M)), block(kActThreads);
+                               bool interleave, bool trigger, void* zero, size_t zero_bytes,
+                               cudaStream_t stream) {
+  const int64_t zb = zero ? zero_blocks(zero_bytes) : 0;
+  dim3 grid(static_cast<unsigned>(M + zb)), block(kActThreads);
   const int trig = trigger ? 1 : 0;
+  uint4* z = static_cast<uint4*>(zero);
+  const int64_t n16 = zero ? static_cast<int64_t>(zero_bytes / 16) : 0;
   if (x_dtype == BITNET_BF16) {
     if (interleave)
-      rmsnorm_quant_kernel<true, true><<<grid, block, 0, stream>>>(x, gamma, eps, K, x_q, s_x,
-                                                                   rowsum, trig);
+      rmsnorm_quant_kernel<true, true><<<grid, block, 0, stream>>>(x, gamma, eps, M, K, x_q,
+                                                                   s_x, rowsum, z, n16, trig);
     else
-      rmsnorm_quant_kernel<true, false><<<grid, block, 0, stream>>>(x, gamma, eps, K, x_q, s_x,
-                                                                    rowsum, trig);
+      rmsnorm_quant_kernel<true, false><<<grid, block, 0, stream>>>(x, gamma, eps, M, K, x_q,
+                                                                    s_x, rowsum, z, n16, trig);
   } else {
     if (interleave)
-      rmsnorm_quant_kernel<false, true><<<grid, block, 0, stream>>>(x, gamma, eps, K, x_q, s_x,
-                                                                    rowsum, trig);
+      rmsnorm_quant_kernel<false, true><<<grid, block, 0, stream>>>(x, gamma, eps, M, K, x_q,
+                                                                    s_x, rowsum, z, n16, trig);
     else
-      rmsnorm_quant_kernel<false, false><<<grid, block, 0, stream>>>(x, gamma, eps, K, x_q, s_x,
-                                                                     rowsum, trig);
+      rmsnorm_quant_kernel<false, false><<<grid, block, 0, stream>>>(x, gamma, eps, M, K, x_q,
+                                                                     s_x, rowsum, z, n16, trig);
   }
   return launch_status();
+}
+
+// The split-K partials + counters of a layout (zero bytes when the layout
+// has no GEMV region).
+void* splitk_region(uint8_t* ws, const FwdWorkspace& L, size_t* bytes) {
+  *bytes = L.total - L.acc;
+  return *bytes ? ws + L.acc : nullptr;
 }
 
 // Matmul + fused dequant on already-prepared interleaved activations.
@@ -301,6 +321,7 @@ bitnet_status forward_impl(const void* x, int x_dtype, const float* gamma, float
                            int32_t* acc_out, int path, cudaStream_t stream) {
   bitnet_status st = check_shape(M, N, K);
   if (st != BITNET_OK) return st;
+  if (M == 0) return BITNET_OK;  // empty batch: nothing to read or write
   if (!x || !W_packed || !s_w || !ok_dtype(x_dtype) || !(eps >= 0.0f) || eps > 3.0e38f)
     return BITNET_ERR_INVALID_ARG;
   if (y && !ok_dtype(y_dtype)) return BITNET_ERR_INVALID_ARG;
@@ -311,7 +332,6 @@ bitnet_status forward_impl(const void* x, int x_dtype, const float* gamma, float
       !aligned(s_w, 4) || (y && !aligned(y, 16)) || (x_q_out && !aligned(x_q_out, 16)) ||
       (s_x_out && !aligned(s_x_out, 4)) || (acc_out && !aligned(acc_out, 16)))
     return BITNET_ERR_MISALIGNED;
-  if (M == 0) return BITNET_OK;
   const FwdWorkspace L = fwd_layout(M, N, K);
   if (!workspace || workspace_bytes < L.total) return BITNET_ERR_WORKSPACE;
   if (!aligned(workspace, 256)) return BITNET_ERR_MISALIGNED;
@@ -323,13 +343,15 @@ bitnet_status forward_impl(const void* x, int x_dtype, const float* gamma, float
     // Debug export in natural k order (same arithmetic as the fused pass).
     int8_t* xq_nat = x_q_out ? x_q_out : reinterpret_cast<int8_t*>(ws + L.xq);
     st = launch_act_quant(x, x_dtype, gamma, eps, M, K, xq_nat, s_x_out, nullptr, false, false,
-                          stream);
+                          nullptr, 0, stream);
     if (st != BITNET_OK) return st;
   }
   const bool pdl = (path == BITNET_PATH_GEMV);
   float* sx = reinterpret_cast<float*>(ws + L.sx);
+  size_t zbytes = 0;
+  void* zero = (path == BITNET_PATH_GEMV) ? splitk_region(ws, L, &zbytes) : nullptr;
   st = launch_act_quant(x, x_dtype, gamma, eps, M, K, reinterpret_cast<int8_t*>(ws + L.xq), sx,
-                        reinterpret_cast<int32_t*>(ws + L.rs), true, pdl, stream);
+                        reinterpret_cast<int32_t*>(ws + L.rs), true, pdl, zero, zbytes, stream);
   if (st != BITNET_OK) return st;
   // The activation-quant kernel just queued started after every earlier
   // write to W_packed, so the GEMV may fetch weights before waiting on it.
@@ -394,14 +416,14 @@ BITNET_API bitnet_status bitnet_rmsnorm_quant_act(const void* x, int x_dtype, co
                                                   float* s_x, bitnet_stream_t stream) {
   bitnet_status st = check_shape(M, 1, K);
   if (st != BITNET_OK) return st;
+  if (M == 0) return BITNET_OK;
   if (!x || !x_q || !s_x || !ok_dtype(x_dtype) || !(eps >= 0.0f) || eps > 3.0e38f)
     return BITNET_ERR_INVALID_ARG;
   if (!aligned(x, 16) || (gamma && !aligned(gamma, 16)) || !aligned(x_q, 16) || !aligned(s_x, 4))
     return BITNET_ERR_MISALIGNED;
-  if (M == 0) return BITNET_OK;
   if (!device_state()) return BITNET_ERR_CUDA;
   return launch_act_quant(x, x_dtype, gamma, eps, M, K, x_q, s_x, nullptr, false, false,
-                          as_stream(stream));
+                          nullptr, 0, as_stream(stream));
 }
 
 BITNET_API size_t bitnet_linear_forward_workspace_bytes(int64_t M, int64_t N, int64_t K) {
@@ -414,7 +436,7 @@ BITNET_API bitnet_status bitnet_linear_forward(const void* x, int x_dtype, const
                                                const float* s_w, int64_t M, int64_t N, int64_t K,
                                                void* y, int y_dtype, void* workspace,
                                                size_t workspace_bytes, bitnet_stream_t stream) {
-  if (!y) return BITNET_ERR_INVALID_ARG;
+  if (!y && M != 0) return BITNET_ERR_INVALID_ARG;
   return forward_impl(x, x_dtype, gamma, eps, W_packed, s_w, M, N, K, y, y_dtype, workspace,
                       workspace_bytes, nullptr, nullptr, nullptr, BITNET_PATH_AUTO,
                       as_stream(stream));
@@ -427,18 +449,20 @@ BITNET_API bitnet_status bitnet_linear_quantize_input(const void* x, int x_dtype
                                                       bitnet_stream_t stream) {
   bitnet_status st = check_shape(M, N, K);
   if (st != BITNET_OK) return st;
+  if (M == 0) return BITNET_OK;
   if (!x || !ok_dtype(x_dtype) || !(eps >= 0.0f) || eps > 3.0e38f) return BITNET_ERR_INVALID_ARG;
   if (!aligned(x, 16) || (gamma && !aligned(gamma, 16))) return BITNET_ERR_MISALIGNED;
-  if (M == 0) return BITNET_OK;
   const FwdWorkspace L = fwd_layout(M, N, K);
   if (!workspace || workspace_bytes < L.total) return BITNET_ERR_WORKSPACE;
   if (!aligned(workspace, 256)) return BITNET_ERR_MISALIGNED;
   if (!device_state()) return BITNET_ERR_CUDA;
   uint8_t* ws = static_cast<uint8_t*>(workspace);
+  size_t zbytes = 0;
+  void* zero = (M <= kGemvMaxM) ? splitk_region(ws, L, &zbytes) : nullptr;
   return launch_act_quant(x, x_dtype, gamma, eps, M, K, reinterpret_cast<int8_t*>(ws + L.xq),
                           reinterpret_cast<float*>(ws + L.sx),
-                          reinterpret_cast<int32_t*>(ws + L.rs), true, M <= kGemvMaxM,
-                          as_stream(stream));
+                          reinterpret_cast<int32_t*>(ws + L.rs), true, M <= kGemvMaxM, zero,
+                          zbytes, as_stream(stream));
 }
 
 BITNET_API bitnet_status bitnet_linear_matmul(const uint8_t* W_packed, const float* s_w,
@@ -447,9 +471,9 @@ BITNET_API bitnet_status bitnet_linear_matmul(const uint8_t* W_packed, const flo
                                               size_t workspace_bytes, bitnet_stream_t stream) {
   bitnet_status st = check_shape(M, N, K);
   if (st != BITNET_OK) return st;
+  if (M == 0) return BITNET_OK;
   if (!W_packed || !s_w || !y || !ok_dtype(y_dtype)) return BITNET_ERR_INVALID_ARG;
   if (!aligned(W_packed, 16) || !aligned(s_w, 4) || !aligned(y, 16)) return BITNET_ERR_MISALIGNED;
-  if (M == 0) return BITNET_OK;
   const FwdWorkspace L = fwd_layout(M, N, K);
   if (!workspace || workspace_bytes < L.total) return BITNET_ERR_WORKSPACE;
   if (!aligned(workspace, 256)) return BITNET_ERR_MISALIGNED;
@@ -477,13 +501,13 @@ BITNET_API bitnet_status bitnet_ternary_matmul_i32(const int8_t* x_q, const uint
                                                    int path, bitnet_stream_t stream) {
   bitnet_status st = check_shape(M, N, K);
   if (st != BITNET_OK) return st;
+  if (M == 0) return BITNET_OK;
   if (!x_q || !W_packed || !acc) return BITNET_ERR_INVALID_ARG;
   if (path < BITNET_PATH_AUTO || path > BITNET_PATH_GEMM) return BITNET_ERR_INVALID_ARG;
   path = resolve_path(path, M);
   if (path == BITNET_PATH_GEMV && M > kGemvMaxM) return BITNET_ERR_INVALID_ARG;
   if (!aligned(x_q, 16) || !aligned(W_packed, 16) || !aligned(acc, 16))
     return BITNET_ERR_MISALIGNED;
-  if (M == 0) return BITNET_OK;
   const FwdWorkspace L = fwd_layout(M, N, K);
   if (!workspace || workspace_bytes < L.total) return BITNET_ERR_WORKSPACE;
   if (!aligned(workspace, 256)) return BITNET_ERR_MISALIGNED;
@@ -491,8 +515,12 @@ BITNET_API bitnet_status bitnet_ternary_matmul_i32(const int8_t* x_q, const uint
   if (!ds) return BITNET_ERR_CUDA;
   cudaStream_t s = as_stream(stream);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
-  interleave_rowsum_kernel<<<static_cast<unsigned>(M), kActThreads, 0, s>>>(
-      x_q, K, reinterpret_cast<int8_t*>(ws + L.xq), reinterpret_cast<int32_t*>(ws + L.rs));
+  size_t zbytes = 0;
+  void* zero = (path == BITNET_PATH_GEMV) ? splitk_region(ws, L, &zbytes) : nullptr;
+  const int64_t zb = zero ? zero_blocks(zbytes) : 0;
+  interleave_rowsum_kernel<<<static_cast<unsigned>(M + zb), kActThreads, 0, s>>>(
+      x_q, M, K, reinterpret_cast<int8_t*>(ws + L.xq), reinterpret_cast<int32_t*>(ws + L.rs),
+      static_cast<uint4*>(zero), zero ? static_cast<int64_t>(zbytes / 16) : 0);
   st = launch_status();
   if (st != BITNET_OK) return st;
   return run_matmul(*ds, path, W_packed, ws, L, nullptr, nullptr, M, N, K, nullptr, BITNET_F32,
