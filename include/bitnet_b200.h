@@ -78,7 +78,8 @@ typedef enum {
     BITNET_ERR_MISALIGNED = 3,        /* a pointer is not 16-byte (workspace 256-byte) aligned */
     BITNET_ERR_CUDA = 4,              /* a CUDA launch or query failed */
     BITNET_ERR_TIMEOUT = 5,           /* a bounded on-device wait gave up */
-    BITNET_ERR_WORKSPACE = 6          /* workspace missing or too small */
+    BITNET_ERR_WORKSPACE = 6,         /* workspace missing or too small */
+    BITNET_ERR_SCRATCH_LIMIT = 7      /* N above BITNET_STATIC_SCRATCH_MAX_N (static-scratch call) */
 } bitnet_status;
 
 typedef enum { BITNET_F32 = 0, BITNET_BF16 = 1 } bitnet_dtype;
@@ -115,6 +116,39 @@ BITNET_API bitnet_status bitnet_quantize_pack_weights(const float *W, int64_t N,
                                                       uint8_t *W_packed, float *s_w,
                                                       void *workspace, size_t workspace_bytes,
                                                       bitnet_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * bitnet_quantize_pack_weights_static -- the same quantization and packing
+ * as bitnet_quantize_pack_weights (identical bytes and s_w), but it needs no
+ * workspace and allocates nothing.  The pages have no counterpart: this only
+ * changes where the kernels' scratch lives.
+ *
+ * Why: some callers cannot call cudaMalloc -- plugins run by an inference
+ * engine that owns the whole device-memory budget and hands its plugins only
+ * their input and output tensors; code that must not risk the device-wide
+ * synchronisation that cudaMalloc/cudaFree may cause; processes whose memory
+ * is reserved up front by a capped pool.  Such callers still pass W,
+ * W_packed and s_w (their own buffers).
+ *
+ * Scratch: a file-scope device array of BITNET_STATIC_SCRATCH_MAX_N fp64
+ * row sums (512 KiB) inside the library, which every GPU that loads the
+ * library holds until the process exits.  Limit: N <= 65536 rows; a larger N
+ * returns BITNET_ERR_SCRATCH_LIMIT and queues nothing.  Every row sum is
+ * written before it is read, so nothing in the array needs clearing between
+ * calls, but all calls on a device share the one array: calls whose kernels
+ * overlap on the GPU (different streams without ordering between them) race
+ * and may produce wrong scales.  Order such calls on one stream.
+ *
+ * Set-up: the first call on each device looks up the array's device address
+ * (with that device current) and keeps it for the process; make that first
+ * call before any stream capture on the device.
+ * Other arguments, layouts and errors as bitnet_quantize_pack_weights.
+ * ---------------------------------------------------------------------- */
+#define BITNET_STATIC_SCRATCH_MAX_N 65536
+BITNET_API bitnet_status bitnet_quantize_pack_weights_static(const float *W, int64_t N,
+                                                             int64_t K, uint8_t *W_packed,
+                                                             float *s_w,
+                                                             bitnet_stream_t stream);
 
 /* ------------------------------------------------------------------------
  * bitnet_rmsnorm_quant_act -- fused RMSNorm + per-token absmax int8 quant.

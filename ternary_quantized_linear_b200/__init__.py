@@ -24,6 +24,8 @@ BITNET_ERR_MISALIGNED = 3
 BITNET_ERR_CUDA = 4
 BITNET_ERR_TIMEOUT = 5
 BITNET_ERR_WORKSPACE = 6
+BITNET_ERR_SCRATCH_LIMIT = 7
+BITNET_STATIC_SCRATCH_MAX_N = 65536
 
 BITNET_F32 = 0
 BITNET_BF16 = 1
@@ -40,6 +42,7 @@ EXPORTED = (
     "bitnet_linear_forward", "bitnet_linear_quantize_input", "bitnet_linear_matmul",
     "bitnet_linear_forward_debug", "bitnet_ternary_matmul_i32",
     "bitnet_device_status", "bitnet_selftest_bounded_wait",
+    "bitnet_quantize_pack_weights_static",
 )
 
 
@@ -81,6 +84,7 @@ def load_library(path: str = LIB_PATH):
             "bitnet_ternary_matmul_i32": ([P, P, I64, I64, I64, P, P, SZ, I, P], I),
             "bitnet_device_status": ([P, I, ctypes.POINTER(I)], I),
             "bitnet_selftest_bounded_wait": ([ctypes.c_uint64, P], I),
+            "bitnet_quantize_pack_weights_static": ([P, I64, I64, P, P, P], I),
         }
         for name, (argtypes, restype) in sig.items():
             fn = getattr(lib, name)
@@ -172,6 +176,23 @@ def bitnet_quantize_pack_weights(W, W_packed=None, s_w=None, workspace=None, str
     _check("bitnet_quantize_pack_weights", load_library().bitnet_quantize_pack_weights(
         _ptr(W), N, K, _ptr(W_packed), _ptr(s_w), _ptr(workspace), workspace.numel(),
         _stream(stream)))
+    return W_packed, s_w
+
+
+def bitnet_quantize_pack_weights_static(W, W_packed, s_w, stream=None):
+    """Weight quantization + packing that allocates nothing: for callers that
+    cannot allocate device memory (e.g. plugins of an engine that owns the
+    memory budget).  The caller provides W, W_packed [N,K/4] and s_w [1]; the
+    library's own static scratch (N <= 65536 rows) replaces the workspace.
+    Calls on one device share that scratch, so calls that overlap on the GPU
+    race."""
+    if W.dtype != torch.float32 or W.dim() != 2:
+        raise TypeError("W must be a 2-D float32 tensor")
+    _need_cuda(W, W_packed, s_w)
+    N, K = W.shape
+    _check("bitnet_quantize_pack_weights_static",
+           load_library().bitnet_quantize_pack_weights_static(
+               _ptr(W), N, K, _ptr(W_packed), _ptr(s_w), _stream(stream)))
     return W_packed, s_w
 
 

@@ -375,6 +375,8 @@ BITNET_API const char* bitnet_status_string(int status) {
     case BITNET_ERR_CUDA: return "CUDA error";
     case BITNET_ERR_TIMEOUT: return "bounded on-device wait timed out";
     case BITNET_ERR_WORKSPACE: return "workspace missing or too small";
+    case BITNET_ERR_SCRATCH_LIMIT:
+      return "N exceeds the static scratch of the allocation-free call (65536 rows)";
     default: return "unknown status";
   }
 }
@@ -566,5 +568,62 @@ extern "C" BITNET_API bitnet_status bitnet_selftest_bounded_wait(uint64_t limit_
   DeviceState* ds = device_state();
   if (!ds) return BITNET_ERR_CUDA;
   bounded_wait_selftest_kernel<<<1, 32, 0, as_stream(stream)>>>(ds->status, limit_ns);
+  return launch_status();
+}
+
+// ---------------------------------------------------------------------------
+// Allocation-free weight quantization: the fp64 per-row |W| sums live in a
+// file-scope device array instead of a caller workspace, for callers that
+// cannot allocate device memory.  The array is per device (one copy in every
+// context that loads this library) and lives until the process exits.
+
+namespace bitnet {
+namespace {
+
+static __device__ __align__(256) double g_static_row_sums[BITNET_STATIC_SCRATCH_MAX_N];
+
+struct StaticScratch {
+  std::once_flag once;
+  double* ptr = nullptr;  // device address of g_static_row_sums on this device
+};
+StaticScratch g_static_scratch[kMaxDevices];
+
+// In host code the array's name is only a host-side handle; the kernels need
+// its device address, looked up once per device with that device current.
+double* static_row_sums() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  StaticScratch& sc = g_static_scratch[dev];
+  std::call_once(sc.once, [&sc]() {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_static_row_sums) == cudaSuccess)
+      sc.ptr = static_cast<double*>(p);
+  });
+  return sc.ptr;
+}
+
+}  // namespace
+}  // namespace bitnet
+
+extern "C" BITNET_API bitnet_status bitnet_quantize_pack_weights_static(
+    const float* W, int64_t N, int64_t K, uint8_t* W_packed, float* s_w,
+    bitnet_stream_t stream) {
+  bitnet_status st = check_shape(0, N, K);
+  if (st != BITNET_OK) return st;
+  if (N > BITNET_STATIC_SCRATCH_MAX_N) return BITNET_ERR_SCRATCH_LIMIT;
+  if (!W || !W_packed || !s_w) return BITNET_ERR_INVALID_ARG;
+  if (!aligned(W, 16) || !aligned(W_packed, 16) || !aligned(s_w, 4)) return BITNET_ERR_MISALIGNED;
+  DeviceState* ds = device_state();
+  if (!ds) return BITNET_ERR_CUDA;
+  double* R = static_row_sums();
+  if (!R) return BITNET_ERR_CUDA;
+  cudaStream_t s = as_stream(stream);
+  row_abs_sum_kernel<<<static_cast<unsigned>(N), kWqThreads, 0, s>>>(W, K, R);
+  abs_total_kernel<<<1, kWqThreads, 0, s>>>(R, N, K, s_w);
+  const int64_t nwords = N * K / 16;
+  const int64_t blocks = std::min<int64_t>((nwords + kWqThreads - 1) / kWqThreads,
+                                           static_cast<int64_t>(ds->num_sms) * 16);
+  pack_kernel<<<static_cast<unsigned>(blocks), kWqThreads, 0, s>>>(
+      W, nwords, s_w, reinterpret_cast<uint32_t*>(W_packed));
   return launch_status();
 }

@@ -47,7 +47,7 @@ def test_every_declared_symbol_is_exported(lib):
 
 
 def test_status_strings(lib):
-    for code in range(0, 7):
+    for code in range(0, 8):
         assert tql.bitnet_status_string(code)
     assert tql.bitnet_status_string(99) == "unknown status"
     assert tql.bitnet_version() >= 100
