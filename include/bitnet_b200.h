@@ -216,6 +216,52 @@ BITNET_API bitnet_status bitnet_linear_matmul(const uint8_t *W_packed, const flo
                                               size_t workspace_bytes, bitnet_stream_t stream);
 
 /* ------------------------------------------------------------------------
+ * bitnet_linear_forward_grouped -- several independent BitLinear forwards in
+ * one call: the result is exactly that of calling bitnet_linear_forward on
+ * each problem in order, but the decode problems (M <= 16) share one
+ * activation-quant launch and one matmul launch, so their weight streams
+ * overlap instead of paying one launch latency each.  Typical use: the
+ * projections of one decode step (q, k, v, o, gate, up, down).  Problems
+ * with M > 16 run afterwards on the tensor-core GEMM, one at a time.
+ *
+ *   count      0 <= count <= BITNET_MAX_GROUP.
+ *   problems   host array of `count` problem descriptions (each field as in
+ *              bitnet_linear_forward).  No problem's y may overlap another
+ *              problem's inputs or output.
+ *   workspace  >= bitnet_linear_forward_grouped_workspace_bytes(count,
+ *              problems), 256-byte aligned, contents on entry irrelevant.
+ *   phases     BITNET_PHASE_ALL, or one phase at a time: BITNET_PHASE_QUANTIZE
+ *              (activation quant of the decode problems into the workspace)
+ *              then, later on the same stream with the same problems and
+ *              workspace, BITNET_PHASE_MATMUL (their matmuls, then every
+ *              M > 16 problem in full).  Splitting lets a caller time the
+ *              phases or reuse one quantization; the results are identical.
+ * Any invalid problem rejects the whole call before anything is queued.
+ * ---------------------------------------------------------------------- */
+#define BITNET_MAX_GROUP 16
+#define BITNET_PHASE_QUANTIZE 1
+#define BITNET_PHASE_MATMUL 2
+#define BITNET_PHASE_ALL 3
+typedef struct {
+    const void *x;            /* [M][K] */
+    int x_dtype;              /* bitnet_dtype */
+    const float *gamma;       /* [K] or NULL */
+    float eps;
+    const uint8_t *W_packed;  /* [N][K/4] */
+    const float *s_w;         /* [1] */
+    int64_t M, N, K;
+    void *y;                  /* [M][N] */
+    int y_dtype;              /* bitnet_dtype */
+} bitnet_linear_problem;
+
+BITNET_API size_t bitnet_linear_forward_grouped_workspace_bytes(
+    int count, const bitnet_linear_problem *problems);
+BITNET_API bitnet_status bitnet_linear_forward_grouped(int count,
+                                                       const bitnet_linear_problem *problems,
+                                                       void *workspace, size_t workspace_bytes,
+                                                       int phases, bitnet_stream_t stream);
+
+/* ------------------------------------------------------------------------
  * bitnet_linear_forward_debug -- bitnet_linear_forward that also exports the
  * intermediate results, and can force a matmul path.
  *

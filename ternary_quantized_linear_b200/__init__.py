@@ -43,7 +43,22 @@ EXPORTED = (
     "bitnet_linear_forward_debug", "bitnet_ternary_matmul_i32",
     "bitnet_device_status", "bitnet_selftest_bounded_wait",
     "bitnet_quantize_pack_weights_static",
+    "bitnet_linear_forward_grouped_workspace_bytes", "bitnet_linear_forward_grouped",
 )
+
+BITNET_MAX_GROUP = 16
+BITNET_PHASE_QUANTIZE = 1
+BITNET_PHASE_MATMUL = 2
+BITNET_PHASE_ALL = 3
+
+
+class LinearProblem(ctypes.Structure):
+    """Mirror of bitnet_linear_problem (include/bitnet_b200.h)."""
+    _fields_ = [("x", ctypes.c_void_p), ("x_dtype", ctypes.c_int),
+                ("gamma", ctypes.c_void_p), ("eps", ctypes.c_float),
+                ("W_packed", ctypes.c_void_p), ("s_w", ctypes.c_void_p),
+                ("M", ctypes.c_int64), ("N", ctypes.c_int64), ("K", ctypes.c_int64),
+                ("y", ctypes.c_void_p), ("y_dtype", ctypes.c_int)]
 
 
 class BitnetError(RuntimeError):
@@ -85,6 +100,8 @@ def load_library(path: str = LIB_PATH):
             "bitnet_device_status": ([P, I, ctypes.POINTER(I)], I),
             "bitnet_selftest_bounded_wait": ([ctypes.c_uint64, P], I),
             "bitnet_quantize_pack_weights_static": ([P, I64, I64, P, P, P], I),
+            "bitnet_linear_forward_grouped_workspace_bytes": ([I, P], SZ),
+            "bitnet_linear_forward_grouped": ([I, P, P, SZ, I, P], I),
         }
         for name, (argtypes, restype) in sig.items():
             fn = getattr(lib, name)
@@ -261,6 +278,41 @@ def bitnet_linear_matmul(W_packed, s_w, M, K, workspace, y_dtype=torch.bfloat16,
         _ptr(W_packed), _ptr(s_w), int(M), N, int(K), _ptr(y), _dtype_code(y.dtype),
         _ptr(workspace), workspace.numel(), _stream(stream)))
     return y
+
+
+def grouped_problems(items):
+    """items: iterable of (x, gamma, eps, W_packed, s_w, y) -> ctypes array of
+    LinearProblem (keep the tensors alive while it is used)."""
+    items = list(items)
+    arr = (LinearProblem * max(1, len(items)))()
+    for i, (x, gamma, eps, W_packed, s_w, y) in enumerate(items):
+        _need_cuda(x, gamma, W_packed, s_w, y)
+        M, K = x.shape
+        arr[i] = LinearProblem(x.data_ptr(), _dtype_code(x.dtype),
+                               None if gamma is None else gamma.data_ptr(), float(eps),
+                               W_packed.data_ptr(), s_w.data_ptr(), M, W_packed.shape[0], K,
+                               y.data_ptr(), _dtype_code(y.dtype))
+    return arr, len(items)
+
+
+def bitnet_linear_forward_grouped_workspace_bytes(problems, count):
+    return int(load_library().bitnet_linear_forward_grouped_workspace_bytes(
+        count, ctypes.cast(problems, ctypes.c_void_p)))
+
+
+def bitnet_linear_forward_grouped(items, workspace=None, phases=BITNET_PHASE_ALL, stream=None):
+    """Run several independent forwards in one call.  items: list of
+    (x, gamma, eps, W_packed, s_w, y) with y preallocated [M, N]."""
+    items = list(items)
+    arr, count = grouped_problems(items)
+    nb = bitnet_linear_forward_grouped_workspace_bytes(arr, count)
+    if workspace is None:
+        workspace = _default_ws.get(nb, items[0][0].device if items else 0, stream)
+    _need_cuda(workspace)
+    _check("bitnet_linear_forward_grouped", load_library().bitnet_linear_forward_grouped(
+        count, ctypes.cast(arr, ctypes.c_void_p), _ptr(workspace), workspace.numel(),
+        int(phases), _stream(stream)))
+    return [it[5] for it in items]
 
 
 def bitnet_linear_forward_debug(x, gamma, eps, W_packed, s_w, y_dtype=torch.float32,

@@ -30,24 +30,6 @@ namespace bitnet {
 
 constexpr int kActThreads = 256;
 
-template <bool kBF16>
-__device__ __forceinline__ void load_chunk8(const void* x, int64_t elem, float (&v)[8]) {
-  if (kBF16) {
-    const uint4 u = __ldg(reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(x) + elem));
-    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      v[2 * j] = __uint_as_float(w[j] << 16);
-      v[2 * j + 1] = __uint_as_float(w[j] & 0xFFFF0000u);
-    }
-  } else {
-    const float4* p = reinterpret_cast<const float4*>(static_cast<const float*>(x) + elem);
-    const float4 a = __ldg(p), b = __ldg(p + 1);
-    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
-    v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
-  }
-}
-
 __device__ __forceinline__ void load_gamma8(const float* gamma, int64_t k, float (&g)[8]) {
   if (gamma) {
     const float4* p = reinterpret_cast<const float4*>(gamma + k);
@@ -156,15 +138,171 @@ __device__ __forceinline__ int block_sum_i32(int v, int* red) {
   return r;
 }
 
-// Blocks past the M row blocks clear a byte range of the workspace (the
-// matmul's split-K partials and counters, which must start at zero) so that
-// no separate memset launch is needed.  n16 = number of 16-byte words.
+// Clear n16 16-byte words at dst using `nblocks` CTAs; this CTA is number
+// `block` among them.  Used by blocks appended to a row-per-block launch to
+// zero the matmul's split-K partials and counters without a memset launch.
 __device__ __forceinline__ void zero_fill_blocks(uint4* __restrict__ dst, int64_t n16,
-                                                 int64_t first_block) {
-  const int64_t nb = static_cast<int64_t>(gridDim.x) - first_block;
-  const int64_t start = (static_cast<int64_t>(blockIdx.x) - first_block) * kActThreads +
-                        threadIdx.x;
-  for (int64_t i = start; i < n16; i += nb * kActThreads) dst[i] = make_uint4(0u, 0u, 0u, 0u);
+                                                 int64_t block, int64_t nblocks) {
+  for (int64_t i = block * kActThreads + threadIdx.x; i < n16; i += nblocks * kActThreads)
+    dst[i] = make_uint4(0u, 0u, 0u, 0u);
+}
+
+// Raw bytes of one 8-element chunk (bf16: one 16-byte word; fp32: two).
+template <bool kBF16>
+struct RawChunk {
+  uint4 w[kBF16 ? 1 : 2];
+};
+
+template <bool kBF16>
+__device__ __forceinline__ RawChunk<kBF16> load_raw8(const void* x, int64_t elem) {
+  RawChunk<kBF16> r;
+  if (kBF16) {
+    r.w[0] = __ldg(reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(x) + elem));
+  } else {
+    const uint4* p = reinterpret_cast<const uint4*>(static_cast<const float*>(x) + elem);
+    r.w[0] = __ldg(p);
+    r.w[kBF16 ? 0 : 1] = __ldg(p + 1);
+  }
+  return r;
+}
+
+template <bool kBF16>
+__device__ __forceinline__ void widen8(const RawChunk<kBF16>& r, float (&v)[8]) {
+  if (kBF16) {
+    const uint32_t w[4] = {r.w[0].x, r.w[0].y, r.w[0].z, r.w[0].w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      v[2 * j] = __uint_as_float(w[j] << 16);
+      v[2 * j + 1] = __uint_as_float(w[j] & 0xFFFF0000u);
+    }
+  } else {
+    const uint4 a = r.w[0], b = r.w[kBF16 ? 0 : 1];
+    v[0] = __uint_as_float(a.x); v[1] = __uint_as_float(a.y);
+    v[2] = __uint_as_float(a.z); v[3] = __uint_as_float(a.w);
+    v[4] = __uint_as_float(b.x); v[5] = __uint_as_float(b.y);
+    v[6] = __uint_as_float(b.z); v[7] = __uint_as_float(b.w);
+  }
+}
+
+// RMSNorm + absmax quantization of row m of x [M][K] by the whole CTA.
+// Thread t owns the 8-element chunks t, t+256, ...; with CACHE > 0 (and at
+// most CACHE chunks per thread) the row is loaded once into registers with
+// all loads in flight together, otherwise each pass re-reads it (L1 hits).
+template <bool kBF16, bool kInterleave, int CACHE>
+__device__ __forceinline__ void quant_row(const void* __restrict__ x,
+                                          const float* __restrict__ gamma, float eps, int64_t m,
+                                          int64_t K, int8_t* __restrict__ x_q,
+                                          float* __restrict__ s_x, int32_t* __restrict__ rowsum,
+                                          float* redf, int* redi) {
+  const int tid = threadIdx.x;
+  const int64_t nchunk = K >> 3;
+  const int iters = static_cast<int>((nchunk + kActThreads - 1) / kActThreads);
+  const int64_t row = m * K;
+  constexpr int CN = CACHE > 0 ? CACHE : 1;
+  RawChunk<kBF16> cache[CN];
+  if (CACHE > 0) {
+#pragma unroll
+    for (int it = 0; it < CN; ++it) {
+      const int64_t c = tid + static_cast<int64_t>(kActThreads) * it;
+      if (it < iters && c < nchunk) cache[it] = load_raw8<kBF16>(x, row + 8 * c);
+    }
+  }
+  auto chunk = [&](int it, int64_t c, float (&v)[8]) {
+    if (CACHE > 0) {
+#pragma unroll
+      for (int u = 0; u < CN; ++u)
+        if (u == it) widen8<kBF16>(cache[u], v);
+    } else {
+      widen8<kBF16>(load_raw8<kBF16>(x, row + 8 * c), v);
+    }
+  };
+
+  // Pass 1: sum of squares, partial = this thread's chunks in increasing k.
+  float p = 0.0f;
+#pragma unroll
+  for (int it = 0; it < (CACHE > 0 ? CN : 1); ++it) {
+    for (int it2 = it; it2 < (CACHE > 0 ? it + 1 : iters); ++it2) {
+      const int64_t c = tid + static_cast<int64_t>(kActThreads) * it2;
+      if (it2 < iters && c < nchunk) {
+        float v[8];
+        chunk(it2, c, v);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) p = __fmaf_rn(v[j], v[j], p);
+      }
+    }
+  }
+  const float ss = block_tree_sum_f32(p, redf);
+  const float ms = __fdiv_rn(ss, static_cast<float>(K));
+  const float d = __fadd_rn(ms, eps);
+  const bool zero_row = (d == 0.0f);
+  const float r = zero_row ? 0.0f : __fdiv_rn(1.0f, __fsqrt_rn(d));
+
+  // Pass 2: max |x_n|.
+  float amax = 0.0f;
+#pragma unroll
+  for (int it = 0; it < (CACHE > 0 ? CN : 1); ++it) {
+    for (int it2 = it; it2 < (CACHE > 0 ? it + 1 : iters); ++it2) {
+      const int64_t c = tid + static_cast<int64_t>(kActThreads) * it2;
+      if (it2 < iters && c < nchunk && !zero_row) {
+        float v[8], g[8];
+        chunk(it2, c, v);
+        load_gamma8(gamma, 8 * c, g);
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+          amax = fmaxf(amax, fabsf(__fmul_rn(__fmul_rn(v[j], r), g[j])));
+      }
+    }
+  }
+  amax = block_max_f32(amax, redf);
+  amax = fmaxf(amax, 1e-5f);
+  const float sx = __fdiv_rn(127.0f, amax);
+
+  // Pass 3: quantize, store, row sum (every lane runs every iteration: the
+  // interleaved store exchanges bytes between lane pairs).
+  int sum = 0;
+  int8_t* xq_row = x_q + row;
+#pragma unroll
+  for (int it = 0; it < (CACHE > 0 ? CN : 1); ++it) {
+    for (int it2 = it; it2 < (CACHE > 0 ? it + 1 : iters); ++it2) {
+      if (it2 >= iters) continue;  // uniform: iters is the same for the whole CTA
+      const int64_t c = tid + static_cast<int64_t>(kActThreads) * it2;
+      const bool valid = c < nchunk;
+      int8_t q[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+      if (valid && !zero_row) {
+        float v[8], g[8];
+        chunk(it2, c, v);
+        load_gamma8(gamma, 8 * c, g);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          q[j] = quant_one(__fmul_rn(__fmul_rn(v[j], r), g[j]), sx);
+          sum += q[j];
+        }
+      }
+      Chunk8 ch{pack4(q[0], q[1], q[2], q[3]), pack4(q[4], q[5], q[6], q[7])};
+      store_chunk8<kInterleave>(xq_row, 8 * c, ch, valid);
+    }
+  }
+  sum = block_sum_i32(sum, redi);
+  if (tid == 0) {
+    if (s_x) s_x[m] = sx;
+    if (rowsum) rowsum[m] = sum;
+  }
+}
+
+// Chunks per thread held in registers: 16 for bf16 rows (K <= 32768), 4 for
+// fp32 rows (K <= 8192); longer rows re-read.
+template <bool kBF16>
+__host__ __device__ constexpr int quant_cache_chunks() { return kBF16 ? 16 : 4; }
+
+template <bool kBF16, bool kInterleave>
+__device__ __forceinline__ void quant_row_any(const void* x, const float* gamma, float eps,
+                                              int64_t m, int64_t K, int8_t* x_q, float* s_x,
+                                              int32_t* rowsum, float* redf, int* redi) {
+  constexpr int C = quant_cache_chunks<kBF16>();
+  if ((K >> 3) <= static_cast<int64_t>(C) * kActThreads)
+    quant_row<kBF16, kInterleave, C>(x, gamma, eps, m, K, x_q, s_x, rowsum, redf, redi);
+  else
+    quant_row<kBF16, kInterleave, 0>(x, gamma, eps, m, K, x_q, s_x, rowsum, redf, redi);
 }
 
 // One CTA per row (blocks >= M zero `zero16` instead).  x: [M][K] (fp32 or
@@ -179,74 +317,57 @@ rmsnorm_quant_kernel(const void* __restrict__ x, const float* __restrict__ gamma
   __shared__ int redi[kActThreads / 32];
   if (trigger_dependents) pdl_launch_dependents();
   if (static_cast<int64_t>(blockIdx.x) >= M) {
-    zero_fill_blocks(zero16, n_zero16, M);
+    zero_fill_blocks(zero16, n_zero16, static_cast<int64_t>(blockIdx.x) - M,
+                     static_cast<int64_t>(gridDim.x) - M);
     return;
   }
+  quant_row_any<kBF16, kInterleave>(x, gamma, eps, blockIdx.x, K, x_q, s_x, rowsum, redf, redi);
+}
 
-  const int tid = threadIdx.x;
-  const int64_t m = blockIdx.x;
-  const int64_t nchunk = K >> 3;
-  const int iters = static_cast<int>((nchunk + kActThreads - 1) / kActThreads);
-  const int64_t row = m * K;
+constexpr int kQuantMaxGroup = 16;
 
-  // Pass 1: sum of squares, partial = this thread's chunks in increasing k.
-  float p = 0.0f;
-  for (int it = 0; it < iters; ++it) {
-    const int64_t c = tid + static_cast<int64_t>(kActThreads) * it;
-    if (c < nchunk) {
-      float v[8];
-      load_chunk8<kBF16>(x, row + 8 * c, v);
-#pragma unroll
-      for (int j = 0; j < 8; ++j) p = __fmaf_rn(v[j], v[j], p);
-    }
-  }
-  const float ss = block_tree_sum_f32(p, redf);
-  const float ms = __fdiv_rn(ss, static_cast<float>(K));
-  const float d = __fadd_rn(ms, eps);
-  const bool zero_row = (d == 0.0f);
-  const float r = zero_row ? 0.0f : __fdiv_rn(1.0f, __fsqrt_rn(d));
+struct QuantProblem {
+  const void* x;          // [M][K] fp32 or bf16
+  const float* gamma;     // [K] or null
+  int8_t* xi;             // [M][K] k-interleaved out
+  float* s_x;             // [M]
+  int32_t* rowsum;        // [M]
+  uint4* zero16;          // region to clear (null: none)
+  int64_t n_zero16;
+  float eps;
+  int M, K;
+  int x_bf16;
+  int block_begin;        // first block of this problem
+  int zero_blocks;        // blocks after the M row blocks that clear zero16
+};
 
-  // Pass 2: max |x_n|.
-  float amax = 0.0f;
-  for (int it = 0; it < iters; ++it) {
-    const int64_t c = tid + static_cast<int64_t>(kActThreads) * it;
-    if (c < nchunk && !zero_row) {
-      float v[8], g[8];
-      load_chunk8<kBF16>(x, row + 8 * c, v);
-      load_gamma8(gamma, 8 * c, g);
-#pragma unroll
-      for (int j = 0; j < 8; ++j) amax = fmaxf(amax, fabsf(__fmul_rn(__fmul_rn(v[j], r), g[j])));
-    }
-  }
-  amax = block_max_f32(amax, redf);
-  amax = fmaxf(amax, 1e-5f);
-  const float sx = __fdiv_rn(127.0f, amax);
+struct QuantLaunch {
+  int count;
+  int trigger_dependents;
+  QuantProblem prob[kQuantMaxGroup];
+};
 
-  // Pass 3: quantize, store, row sum.
-  int sum = 0;
-  int8_t* xq_row = x_q + row;
-  for (int it = 0; it < iters; ++it) {
-    const int64_t c = tid + static_cast<int64_t>(kActThreads) * it;
-    const bool valid = c < nchunk;
-    int8_t q[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-    if (valid && !zero_row) {
-      float v[8], g[8];
-      load_chunk8<kBF16>(x, row + 8 * c, v);
-      load_gamma8(gamma, 8 * c, g);
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        q[j] = quant_one(__fmul_rn(__fmul_rn(v[j], r), g[j]), sx);
-        sum += q[j];
-      }
-    }
-    Chunk8 ch{pack4(q[0], q[1], q[2], q[3]), pack4(q[4], q[5], q[6], q[7])};
-    store_chunk8<kInterleave>(xq_row, 8 * c, ch, valid);
+// Several independent problems in one launch: rows of every problem, then
+// each problem's zero-fill blocks, laid out by block_begin.
+__global__ void __launch_bounds__(kActThreads)
+rmsnorm_quant_grouped_kernel(const __grid_constant__ QuantLaunch L) {
+  __shared__ float redf[kActThreads];
+  __shared__ int redi[kActThreads / 32];
+  if (L.trigger_dependents) pdl_launch_dependents();
+  int pi = 0;
+  for (int i = 1; i < L.count; ++i)
+    if (static_cast<int>(blockIdx.x) >= L.prob[i].block_begin) pi = i;
+  const QuantProblem& q = L.prob[pi];
+  const int local = static_cast<int>(blockIdx.x) - q.block_begin;
+  if (local >= q.M) {
+    zero_fill_blocks(q.zero16, q.n_zero16, local - q.M, q.zero_blocks);
+    return;
   }
-  sum = block_sum_i32(sum, redi);
-  if (tid == 0) {
-    if (s_x) s_x[m] = sx;
-    if (rowsum) rowsum[m] = sum;
-  }
+  if (q.x_bf16)
+    quant_row_any<true, true>(q.x, q.gamma, q.eps, local, q.K, q.xi, q.s_x, q.rowsum, redf, redi);
+  else
+    quant_row_any<false, true>(q.x, q.gamma, q.eps, local, q.K, q.xi, q.s_x, q.rowsum, redf,
+                               redi);
 }
 
 // Natural-order x_q -> k-interleaved copy plus per-row sums (used when the
@@ -257,7 +378,8 @@ interleave_rowsum_kernel(const int8_t* __restrict__ x_q, int64_t M, int64_t K,
                          uint4* __restrict__ zero16, int64_t n_zero16) {
   __shared__ int redi[kActThreads / 32];
   if (static_cast<int64_t>(blockIdx.x) >= M) {
-    zero_fill_blocks(zero16, n_zero16, M);
+    zero_fill_blocks(zero16, n_zero16, static_cast<int64_t>(blockIdx.x) - M,
+                     static_cast<int64_t>(gridDim.x) - M);
     return;
   }
   const int tid = threadIdx.x;

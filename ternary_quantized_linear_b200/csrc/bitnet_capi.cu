@@ -65,8 +65,9 @@ DeviceState* device_state() {
               cudaSuccess;
     ok = ok && cudaDeviceGetAttribute(&st.num_sms, cudaDevAttrMultiProcessorCount, dev) ==
                    cudaSuccess;
-    ok = ok && set_smem(ternary_gemv_kernel<2, 1>, 8 * 1 * (16 * 256 + 16));
-    ok = ok && set_smem(ternary_gemv_kernel<2, 2>, 8 * 2 * (16 * 256 + 16));
+    ok = ok && set_smem(ternary_gemv_kernel, kGemvRows * gemv_row_stride(kGemvMaxIps));
+    ok = ok && set_smem(ternary_gemm_tc_kernel<16>, GemmCfg<16>::SMEM_DYN);
+    ok = ok && set_smem(ternary_gemm_tc_kernel<32>, GemmCfg<32>::SMEM_DYN);
     ok = ok && set_smem(ternary_gemm_tc_kernel<64>, GemmCfg<64>::SMEM_DYN);
     ok = ok && set_smem(ternary_gemm_tc_kernel<128>, GemmCfg<128>::SMEM_DYN);
     ok = ok && set_smem(ternary_gemm_tc_kernel<256>, GemmCfg<256>::SMEM_DYN);
@@ -152,87 +153,130 @@ bool ok_dtype(int d) { return d == BITNET_F32 || d == BITNET_BF16; }
 // ------------------------------------------------------------ launchers
 
 struct GemvPlan {
-  int NT, rb, ksplit, ips, warps;
+  int rb, ksplit, ips, blocks;
   size_t smem;
 };
 
-GemvPlan plan_gemv(int64_t M, int64_t N, int64_t K, int num_sms) {
+// Row blocks of 16 weight rows; K is split across CTAs only when a slice
+// would not fit (more than kGemvMaxIps 256-k steps) or when there are too few
+// row blocks to give every SM a CTA.
+GemvPlan plan_gemv(int64_t N, int64_t K, int num_sms) {
   GemvPlan pl{};
-  constexpr int kRows = 32;  // RG = 2
-  pl.NT = M <= 8 ? 1 : 2;
-  pl.rb = static_cast<int>((N + kRows - 1) / kRows);
+  pl.rb = static_cast<int>((N + kGemvRows - 1) / kGemvRows);
   const int iters = static_cast<int>((K + 255) / 256);
-  const int ks_min = (iters + 15) / 16;  // at most 16 steps (4096 k) staged per CTA
-  const int target = 4 * num_sms;
-  int ks = std::min(iters, (target + pl.rb - 1) / pl.rb);
-  ks = std::max(ks, ks_min);
+  int ks = (iters + kGemvMaxIps - 1) / kGemvMaxIps;
+  if (pl.rb * ks < num_sms) ks = std::max(ks, std::min(iters, (num_sms + pl.rb - 1) / pl.rb));
   pl.ips = (iters + ks - 1) / ks;
   pl.ksplit = (iters + pl.ips - 1) / pl.ips;
-  pl.warps = std::min(8, pl.ips);
-  pl.smem = static_cast<size_t>(8 * pl.NT) * (pl.ips * 256 + 16);
+  pl.blocks = pl.rb * pl.ksplit;
+  pl.smem = static_cast<size_t>(kGemvRows) * gemv_row_stride(pl.ips);
   return pl;
 }
 
-bitnet_status launch_gemv(const DeviceState& ds, const uint8_t* Wp, const int8_t* xi,
-                          const int32_t* rowsum, const float* s_x, const float* s_w, int64_t M,
-                          int64_t N, int64_t K, uint8_t* ws, const FwdWorkspace& L, void* y,
-                          int y_dtype, int32_t* acc_out, bool pdl, bool early_weights,
-                          cudaStream_t stream) {
-  const GemvPlan pl = plan_gemv(M, N, K, ds.num_sms);
-  GemvParams p{};
-  p.Wp = Wp;
-  p.xi = xi;
-  p.rowsum = rowsum;
-  p.s_x = s_x;
-  p.s_w = s_w;
-  p.M = static_cast<int>(M);
-  p.N = static_cast<int>(N);
-  p.K = static_cast<int>(K);
-  p.iters_per_split = pl.ips;
-  p.ws_acc = reinterpret_cast<int32_t*>(ws + L.acc);
-  p.ws_cnt = reinterpret_cast<unsigned*>(ws + L.cnt);
-  p.y = y;
-  p.y_bf16 = (y_dtype == BITNET_BF16) ? 1 : 0;
-  p.acc_out = acc_out;
-  p.use_pdl = pdl ? 1 : 0;
-  p.early_weights = (pdl && early_weights) ? 1 : 0;
+void fill_gemv_problem(GemvProblem& q, const GemvPlan& pl, const uint8_t* Wp, uint8_t* ws,
+                       const FwdWorkspace& L, const float* s_x, const float* s_w, int64_t M,
+                       int64_t N, int64_t K, void* y, int y_dtype, int32_t* acc_out,
+                       int block_begin) {
+  q.Wp = Wp;
+  q.xi = reinterpret_cast<const int8_t*>(ws + L.xq);
+  q.rowsum = reinterpret_cast<const int32_t*>(ws + L.rs);
+  q.s_x = s_x;
+  q.s_w = s_w;
+  q.y = y;
+  q.acc_out = acc_out;
+  q.ws_acc = reinterpret_cast<int32_t*>(ws + L.acc);
+  q.ws_cnt = reinterpret_cast<unsigned*>(ws + L.cnt);
+  q.M = static_cast<int>(M);
+  q.N = static_cast<int>(N);
+  q.K = static_cast<int>(K);
+  q.y_bf16 = (y_dtype == BITNET_BF16) ? 1 : 0;
+  q.rb = pl.rb;
+  q.ksplit = pl.ksplit;
+  q.ips = pl.ips;
+  q.block_begin = block_begin;
+}
 
+bitnet_status launch_gemv_group(const DeviceState& ds, GemvLaunch& L, int blocks, size_t smem,
+                                bool pdl, bool early_weights, cudaStream_t stream) {
+  L.use_pdl = pdl ? 1 : 0;
+  L.early_weights = (pdl && early_weights) ? 1 : 0;
+  L.status = ds.status;
+  L.wait_limit_ns = kWaitLimitNs;
   cudaLaunchConfig_t cfg{};
-  cfg.gridDim = dim3(static_cast<unsigned>(pl.rb), static_cast<unsigned>(pl.ksplit), 1);
-  cfg.blockDim = dim3(32 * pl.warps, 1, 1);
-  cfg.dynamicSmemBytes = pl.smem;
+  cfg.gridDim = dim3(static_cast<unsigned>(blocks), 1, 1);
+  cfg.blockDim = dim3(kGemvWarps * 32, 1, 1);
+  cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = pdl ? 1 : 0;
-  cudaError_t e = (pl.NT == 1) ? cudaLaunchKernelEx(&cfg, ternary_gemv_kernel<2, 1>, p)
-                               : cudaLaunchKernelEx(&cfg, ternary_gemv_kernel<2, 2>, p);
-  return e == cudaSuccess ? BITNET_OK : BITNET_ERR_CUDA;
+  return cudaLaunchKernelEx(&cfg, ternary_gemv_kernel, L) == cudaSuccess ? BITNET_OK
+                                                                         : BITNET_ERR_CUDA;
+}
+
+bitnet_status launch_gemv(const DeviceState& ds, const uint8_t* Wp, const float* s_x,
+                          const float* s_w, int64_t M, int64_t N, int64_t K, uint8_t* ws,
+                          const FwdWorkspace& Lw, void* y, int y_dtype, int32_t* acc_out,
+                          bool pdl, bool early_weights, cudaStream_t stream) {
+  const GemvPlan pl = plan_gemv(N, K, ds.num_sms);
+  GemvLaunch L{};
+  L.count = 1;
+  fill_gemv_problem(L.prob[0], pl, Wp, ws, Lw, s_x, s_w, M, N, K, y, y_dtype, acc_out, 0);
+  return launch_gemv_group(ds, L, pl.blocks, pl.smem, pdl, early_weights, stream);
+}
+
+struct GemmPlan {
+  int BN, rb, tb, ksplit, steps_per_split;
+};
+
+// Token tile BN from M; K is split across CTAs only for small M (then the
+// int32 partials go through the workspace), to give every SM work.
+GemmPlan plan_gemm(int64_t M, int64_t N, int64_t K, int num_sms) {
+  GemmPlan pl{};
+  pl.BN = M <= 16 ? 16 : (M <= 32 ? 32 : (M <= 64 ? 64 : (M <= 128 ? 128 : 256)));
+  pl.rb = static_cast<int>((N + 127) / 128);
+  pl.tb = static_cast<int>((M + pl.BN - 1) / pl.BN);
+  const int kstep = pl.BN <= 64 ? 512 : 128;  // GemmCfg<BN>::KSTEP
+  const int steps = static_cast<int>((K + kstep - 1) / kstep);
+  int ks = 1;
+  if (M <= kGemvMaxM) {
+    const int target = num_sms;  // one CTA per SM (each owns all of TMEM)
+    const int tiles = pl.rb * pl.tb;
+    ks = std::max(1, std::min(steps, (target + tiles - 1) / tiles));
+  }
+  pl.steps_per_split = (steps + ks - 1) / ks;
+  pl.ksplit = (steps + pl.steps_per_split - 1) / pl.steps_per_split;
+  return pl;
 }
 
 template <int BN>
-bitnet_status launch_gemm_bn(const DeviceState& ds, const CUtensorMap& tx, const CUtensorMap& tw,
-                             const GemmParams& p, int64_t M, int64_t N, cudaStream_t stream) {
-  (void)ds;
-  dim3 grid(static_cast<unsigned>((N + 127) / 128), static_cast<unsigned>((M + BN - 1) / BN), 1);
-  ternary_gemm_tc_kernel<BN><<<grid, 256, GemmCfg<BN>::SMEM_DYN, stream>>>(tx, tw, p);
+bitnet_status launch_gemm_bn(const CUtensorMap& tx, const CUtensorMap& tw, const GemmParams& p,
+                             const GemmPlan& pl, cudaStream_t stream) {
+  dim3 grid(static_cast<unsigned>(pl.rb), static_cast<unsigned>(pl.tb),
+            static_cast<unsigned>(pl.ksplit));
+  ternary_gemm_tc_kernel<BN><<<grid, GemmCfg<BN>::THREADS, GemmCfg<BN>::SMEM_DYN, stream>>>(
+      tx, tw, p);
   return launch_status();
 }
 
 bitnet_status launch_gemm(const DeviceState& ds, const uint8_t* Wp, const int8_t* xi,
                           const int32_t* rowsum, const float* s_x, const float* s_w, int64_t M,
-                          int64_t N, int64_t K, void* y, int y_dtype, int32_t* acc_out,
-                          cudaStream_t stream) {
-  const int BN = M <= 64 ? 64 : (M <= 128 ? 128 : 256);
+                          int64_t N, int64_t K, uint8_t* ws, const FwdWorkspace& Lw, void* y,
+                          int y_dtype, int32_t* acc_out, cudaStream_t stream) {
+  const GemmPlan pl = plan_gemm(M, N, K, ds.num_sms);
   CUtensorMap tx, tw;
   if (!make_tmap_u8(&tx, xi, static_cast<uint64_t>(K), static_cast<uint64_t>(M),
-                    static_cast<uint64_t>(K), 128, static_cast<uint32_t>(BN),
+                    static_cast<uint64_t>(K), 128, static_cast<uint32_t>(pl.BN),
                     CU_TENSOR_MAP_SWIZZLE_128B))
     return BITNET_ERR_CUDA;
+  // GemmCfg<BN>::WP_ROW bytes per row, swizzled so the unpack reads are
+  // bank-conflict free.
+  const uint32_t wp_row = pl.BN <= 64 ? 128 : 32;
   if (!make_tmap_u8(&tw, Wp, static_cast<uint64_t>(K / 4), static_cast<uint64_t>(N),
-                    static_cast<uint64_t>(K / 4), 32, 128, CU_TENSOR_MAP_SWIZZLE_NONE))
+                    static_cast<uint64_t>(K / 4), wp_row, 128,
+                    wp_row == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_32B))
     return BITNET_ERR_CUDA;
   GemmParams p{};
   p.rowsum = rowsum;
@@ -244,13 +288,27 @@ bitnet_status launch_gemm(const DeviceState& ds, const uint8_t* Wp, const int8_t
   p.y = y;
   p.y_bf16 = (y_dtype == BITNET_BF16) ? 1 : 0;
   p.acc_out = acc_out;
+  p.ksplit = pl.ksplit;
+  p.steps_per_split = pl.steps_per_split;
+  p.ws_acc = reinterpret_cast<int32_t*>(ws + Lw.acc);
+  p.ws_cnt = reinterpret_cast<unsigned*>(ws + Lw.cnt);
   p.status = ds.status;
   p.wait_limit_ns = kWaitLimitNs;
-  switch (BN) {
-    case 64: return launch_gemm_bn<64>(ds, tx, tw, p, M, N, stream);
-    case 128: return launch_gemm_bn<128>(ds, tx, tw, p, M, N, stream);
-    default: return launch_gemm_bn<256>(ds, tx, tw, p, M, N, stream);
+  switch (pl.BN) {
+    case 16: return launch_gemm_bn<16>(tx, tw, p, pl, stream);
+    case 32: return launch_gemm_bn<32>(tx, tw, p, pl, stream);
+    case 64: return launch_gemm_bn<64>(tx, tw, p, pl, stream);
+    case 128: return launch_gemm_bn<128>(tx, tw, p, pl, stream);
+    default: return launch_gemm_bn<256>(tx, tw, p, pl, stream);
   }
+}
+
+// Whether the matmul chosen for (path, M, N, K) accumulates split-K partials
+// in the workspace (which must then start at zero).
+bool needs_zeroed_partials(const DeviceState& ds, int path, int64_t M, int64_t N, int64_t K) {
+  if (M > kGemvMaxM) return false;
+  if (path == BITNET_PATH_GEMV) return plan_gemv(N, K, ds.num_sms).ksplit > 1;
+  return plan_gemm(M, N, K, ds.num_sms).ksplit > 1;
 }
 
 // Extra blocks appended to a row-per-block kernel to clear `bytes` bytes.
@@ -301,12 +359,12 @@ bitnet_status run_matmul(const DeviceState& ds, int path, const uint8_t* Wp, uin
                          const FwdWorkspace& L, const float* s_x, const float* s_w, int64_t M,
                          int64_t N, int64_t K, void* y, int y_dtype, int32_t* acc_out, bool pdl,
                          bool early_weights, cudaStream_t stream) {
+  if (path == BITNET_PATH_GEMV)
+    return launch_gemv(ds, Wp, s_x, s_w, M, N, K, ws, L, y, y_dtype, acc_out, pdl,
+                       early_weights, stream);
   const int8_t* xi = reinterpret_cast<const int8_t*>(ws + L.xq);
   const int32_t* rs = reinterpret_cast<const int32_t*>(ws + L.rs);
-  if (path == BITNET_PATH_GEMV)
-    return launch_gemv(ds, Wp, xi, rs, s_x, s_w, M, N, K, ws, L, y, y_dtype, acc_out, pdl,
-                       early_weights, stream);
-  return launch_gemm(ds, Wp, xi, rs, s_x, s_w, M, N, K, y, y_dtype, acc_out, stream);
+  return launch_gemm(ds, Wp, xi, rs, s_x, s_w, M, N, K, ws, L, y, y_dtype, acc_out, stream);
 }
 
 int resolve_path(int path, int64_t M) {
@@ -349,7 +407,8 @@ bitnet_status forward_impl(const void* x, int x_dtype, const float* gamma, float
   const bool pdl = (path == BITNET_PATH_GEMV);
   float* sx = reinterpret_cast<float*>(ws + L.sx);
   size_t zbytes = 0;
-  void* zero = (path == BITNET_PATH_GEMV) ? splitk_region(ws, L, &zbytes) : nullptr;
+  void* zero = needs_zeroed_partials(*ds, path, M, N, K) ? splitk_region(ws, L, &zbytes)
+                                                          : nullptr;
   st = launch_act_quant(x, x_dtype, gamma, eps, M, K, reinterpret_cast<int8_t*>(ws + L.xq), sx,
                         reinterpret_cast<int32_t*>(ws + L.rs), true, pdl, zero, zbytes, stream);
   if (st != BITNET_OK) return st;
@@ -357,6 +416,121 @@ bitnet_status forward_impl(const void* x, int x_dtype, const float* gamma, float
   // write to W_packed, so the GEMV may fetch weights before waiting on it.
   return run_matmul(*ds, path, W_packed, ws, L, sx, s_w, M, N, K, y, y_dtype, acc_out, pdl,
                     pdl, stream);
+}
+
+// Checks of one problem of a grouped call (the same rules as the forward).
+bitnet_status check_problem(const bitnet_linear_problem& q) {
+  bitnet_status st = check_shape(q.M, q.N, q.K);
+  if (st != BITNET_OK) return st;
+  if (q.M == 0) return BITNET_OK;
+  if (!q.x || !q.W_packed || !q.s_w || !q.y || !ok_dtype(q.x_dtype) || !ok_dtype(q.y_dtype) ||
+      !(q.eps >= 0.0f) || q.eps > 3.0e38f)
+    return BITNET_ERR_INVALID_ARG;
+  if (!aligned(q.x, 16) || (q.gamma && !aligned(q.gamma, 16)) || !aligned(q.W_packed, 16) ||
+      !aligned(q.s_w, 4) || !aligned(q.y, 16))
+    return BITNET_ERR_MISALIGNED;
+  return BITNET_OK;
+}
+
+size_t grouped_workspace(int count, const bitnet_linear_problem* problems) {
+  size_t total = 0;
+  for (int i = 0; i < count; ++i) {
+    const bitnet_linear_problem& q = problems[i];
+    if (q.M > 0) total += fwd_layout(q.M, q.N, q.K).total;
+  }
+  return total;
+}
+
+bitnet_status forward_grouped_impl(int count, const bitnet_linear_problem* problems,
+                                   void* workspace, size_t workspace_bytes, int phases,
+                                   cudaStream_t stream) {
+  if (count < 0 || count > BITNET_MAX_GROUP || (count > 0 && !problems))
+    return BITNET_ERR_INVALID_ARG;
+  if (phases < BITNET_PHASE_QUANTIZE || phases > BITNET_PHASE_ALL) return BITNET_ERR_INVALID_ARG;
+  const bool do_quant = (phases & BITNET_PHASE_QUANTIZE) != 0;
+  const bool do_matmul = (phases & BITNET_PHASE_MATMUL) != 0;
+  for (int i = 0; i < count; ++i) {
+    const bitnet_status st = check_problem(problems[i]);
+    if (st != BITNET_OK) return st;
+  }
+  const size_t need = grouped_workspace(count, problems);
+  if (need == 0) return BITNET_OK;
+  if (!workspace || workspace_bytes < need) return BITNET_ERR_WORKSPACE;
+  if (!aligned(workspace, 256)) return BITNET_ERR_MISALIGNED;
+  DeviceState* ds = device_state();
+  if (!ds) return BITNET_ERR_CUDA;
+  uint8_t* base = static_cast<uint8_t*>(workspace);
+
+  // Decode problems: one grouped quant launch, one grouped matmul launch.
+  QuantLaunch QL{};
+  GemvLaunch GL{};
+  int qblocks = 0, gblocks = 0, n = 0;
+  size_t smem = 0;
+  size_t off = 0;
+  for (int i = 0; i < count; ++i) {
+    const bitnet_linear_problem& q = problems[i];
+    if (q.M == 0) continue;
+    const FwdWorkspace L = fwd_layout(q.M, q.N, q.K);
+    uint8_t* ws = base + off;
+    off += L.total;
+    if (q.M > kGemvMaxM) continue;
+    const GemvPlan pl = plan_gemv(q.N, q.K, ds->num_sms);
+    size_t zbytes = 0;
+    void* zero = pl.ksplit > 1 ? splitk_region(ws, L, &zbytes) : nullptr;
+    QuantProblem& qp = QL.prob[n];
+    qp.x = q.x;
+    qp.gamma = q.gamma;
+    qp.xi = reinterpret_cast<int8_t*>(ws + L.xq);
+    qp.s_x = reinterpret_cast<float*>(ws + L.sx);
+    qp.rowsum = reinterpret_cast<int32_t*>(ws + L.rs);
+    qp.zero16 = static_cast<uint4*>(zero);
+    qp.n_zero16 = zero ? static_cast<int64_t>(zbytes / 16) : 0;
+    qp.eps = q.eps;
+    qp.M = static_cast<int>(q.M);
+    qp.K = static_cast<int>(q.K);
+    qp.x_bf16 = (q.x_dtype == BITNET_BF16) ? 1 : 0;
+    qp.block_begin = qblocks;
+    qp.zero_blocks = static_cast<int>(zero ? zero_blocks(zbytes) : 0);
+    qblocks += qp.M + qp.zero_blocks;
+    fill_gemv_problem(GL.prob[n], pl, q.W_packed, ws, L, qp.s_x, q.s_w, q.M, q.N, q.K, q.y,
+                      q.y_dtype, nullptr, gblocks);
+    gblocks += pl.blocks;
+    smem = std::max(smem, pl.smem);
+    ++n;
+  }
+  if (n > 0) {
+    QL.count = n;
+    QL.trigger_dependents = do_matmul ? 1 : 0;
+    GL.count = n;
+    if (do_quant) {
+      rmsnorm_quant_grouped_kernel<<<static_cast<unsigned>(qblocks), kActThreads, 0, stream>>>(
+          QL);
+      const bitnet_status st = launch_status();
+      if (st != BITNET_OK) return st;
+    }
+    if (do_matmul) {
+      // When the quant grid was just queued it started after every earlier
+      // write to the weights, so the copies may begin before waiting on it.
+      const bitnet_status st = launch_gemv_group(*ds, GL, gblocks, smem, true, do_quant, stream);
+      if (st != BITNET_OK) return st;
+    }
+  }
+  if (!do_matmul) return BITNET_OK;
+  // Prefill problems: the tensor-core GEMM, one after another.
+  off = 0;
+  for (int i = 0; i < count; ++i) {
+    const bitnet_linear_problem& q = problems[i];
+    if (q.M == 0) continue;
+    const FwdWorkspace L = fwd_layout(q.M, q.N, q.K);
+    uint8_t* ws = base + off;
+    off += L.total;
+    if (q.M <= kGemvMaxM) continue;
+    const bitnet_status st =
+        forward_impl(q.x, q.x_dtype, q.gamma, q.eps, q.W_packed, q.s_w, q.M, q.N, q.K, q.y,
+                     q.y_dtype, ws, L.total, nullptr, nullptr, nullptr, BITNET_PATH_GEMM, stream);
+    if (st != BITNET_OK) return st;
+  }
+  return BITNET_OK;
 }
 
 }  // namespace
@@ -488,6 +662,22 @@ BITNET_API bitnet_status bitnet_linear_matmul(const uint8_t* W_packed, const flo
                     as_stream(stream));
 }
 
+BITNET_API size_t bitnet_linear_forward_grouped_workspace_bytes(
+    int count, const bitnet_linear_problem* problems) {
+  if (count < 0 || count > BITNET_MAX_GROUP || (count > 0 && !problems)) return 0;
+  for (int i = 0; i < count; ++i)
+    if (problems[i].M < 0 || problems[i].N < 0 || problems[i].K < 0) return 0;
+  return grouped_workspace(count, problems);
+}
+
+BITNET_API bitnet_status bitnet_linear_forward_grouped(int count,
+                                                       const bitnet_linear_problem* problems,
+                                                       void* workspace, size_t workspace_bytes,
+                                                       int phases, bitnet_stream_t stream) {
+  return forward_grouped_impl(count, problems, workspace, workspace_bytes, phases,
+                              as_stream(stream));
+}
+
 BITNET_API bitnet_status bitnet_linear_forward_debug(
     const void* x, int x_dtype, const float* gamma, float eps, const uint8_t* W_packed,
     const float* s_w, int64_t M, int64_t N, int64_t K, void* y, int y_dtype, void* workspace,
@@ -518,7 +708,8 @@ BITNET_API bitnet_status bitnet_ternary_matmul_i32(const int8_t* x_q, const uint
   cudaStream_t s = as_stream(stream);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   size_t zbytes = 0;
-  void* zero = (path == BITNET_PATH_GEMV) ? splitk_region(ws, L, &zbytes) : nullptr;
+  void* zero = needs_zeroed_partials(*ds, path, M, N, K) ? splitk_region(ws, L, &zbytes)
+                                                          : nullptr;
   const int64_t zb = zero ? zero_blocks(zbytes) : 0;
   interleave_rowsum_kernel<<<static_cast<unsigned>(M + zb), kActThreads, 0, s>>>(
       x_q, M, K, reinterpret_cast<int8_t*>(ws + L.xq), reinterpret_cast<int32_t*>(ws + L.rs),

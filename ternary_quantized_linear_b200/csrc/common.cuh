@@ -19,6 +19,7 @@ enum DeviceDetail : int {
   DEV_TIMEOUT_EPILOGUE = 4,
   DEV_TIMEOUT_DRAIN = 5,
   DEV_TIMEOUT_SELFTEST = 6,
+  DEV_TIMEOUT_GEMV = 7,
 };
 
 // Default limit of one on-chip wait (nanoseconds of %globaltimer).  Real
@@ -109,6 +110,19 @@ __device__ __forceinline__ void tma_load_2d(void* smem_dst, const CUtensorMap* m
       "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
       " [%0], [%1, {%2, %3}], [%4];" ::"r"(smem_u32(smem_dst)),
       "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(smem_u32(bar))
+      : "memory");
+}
+
+// 1-D bulk copy (no tensor map, no multicast) of `bytes` contiguous bytes
+// from global memory into this CTA's shared memory, completing as
+// transaction bytes on `bar`.  Both addresses 16-byte aligned, bytes a
+// multiple of 16.
+__device__ __forceinline__ void bulk_load(void* smem_dst, const void* gmem_src, uint32_t bytes,
+                                          uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::
+          "r"(smem_u32(smem_dst)),
+      "l"(gmem_src), "r"(bytes), "r"(smem_u32(bar))
       : "memory");
 }
 
@@ -233,6 +247,17 @@ __device__ __forceinline__ uint4 ldg_stream_u4(const void* p) {
   asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
                : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
                : "l"(p));
+  return v;
+}
+
+// 16-byte load through L1 (data written by the preceding grid: not the
+// non-coherent path).
+__device__ __forceinline__ uint4 ldg_u4(const void* p) {
+  uint4 v;
+  asm volatile("ld.global.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p)
+               : "memory");
   return v;
 }
 

@@ -1,33 +1,41 @@
-// gemm_tc.cuh -- prefill-path ternary matmul on the 5th-generation tensor
-// cores: tcgen05.mma kind::i8 with int32 accumulators in tensor memory.
+// gemm_tc.cuh -- ternary matmul on the 5th-generation tensor cores for any
+// token count: tcgen05.mma kind::i8, A = unpacked weights held in TENSOR
+// MEMORY, B = activations in shared memory, int32 accumulators in TMEM.
 //
 // Method: "LLM を 1.58 ビットにファインチューニング：BitNet による極端な量子化",
 // sections 計算パラダイム (integer matmul), 推論最適化とカスタムカーネル
 // (weights unpacked on the fly inside the kernel), タイル化行列乗算 (tiles
-// staged in fast shared memory to avoid redundant global traffic),
+// staged in fast on-chip memory so global memory is read once),
 // 量子化の仕組み (rescale by both scales).
 //
-// One CTA computes a 128 (weight rows) x BN (tokens) tile of acc^T:
-//   warp 0      TMA producer: per 128-k step, the activation tile
-//               (BN x 128 int8, 128-byte swizzle, straight into the MMA's
-//               canonical K-major layout) and the packed weight tile
-//               (128 rows x 32 bytes) into a STAGES-deep ring;
-//   warp 1      allocates TMEM; one thread issues 4 MMAs (K = 32 each) per
-//               step with A = unpacked weights, B = activations, and
-//               commits each stage back to the producer;
-//   warps 4-7   unpack: thread i expands row i's 32 packed bytes to 128 int8
-//               codes (shift + mask, no table) written into the swizzled A
-//               tile, then fences the async proxy and arrives; after the last
-//               step the same warps read TMEM (one lane = one weight row) and
-//               write y = (acc - rowsum) / (s_x * s_w) coalesced along N.
-// The unpacked codes are t+1 in {0,1,2}, in the same k-interleaved order as
-// the activations (see act_quant.cuh), so the MMA pairs equal k and the row
-// sum correction restores sum x*t exactly.
+// A CTA computes a 128 (weight rows, TMEM lanes) x BN (tokens) tile of
+// acc^T over a range of K, in KSTEP-k steps (512 for BN <= 64, else 128):
+//   warp 0      TMA producer: per step the packed weight tile (128 rows x
+//               KSTEP/4 bytes) and the activation tile (BN rows of KSTEP int8
+//               as 128-byte swizzle atoms = the MMA's canonical K-major
+//               layout) into a STAGES-deep shared-memory ring;
+//   warp 1      allocates TMEM; one thread issues KSTEP/32 MMAs (K = 32 each)
+//               per step reading A from TMEM and B from shared memory;
+//   warps 4-11  unpack: each thread expands 16 packed bytes of its weight
+//               row (half a step) into 16 words of int8 codes t+1 (shift +
+//               mask, no table) and stores them with tcgen05.st into one of
+//               A_STAGES TMEM stages, so the unpack runs that many steps ahead
+//               of the MMAs; after the last step the same warps read the
+//               accumulators from TMEM (one lane = one weight row) and write
+//               y = (acc - rowsum) / (s_x * s_w) coalesced along N.
+// Keeping A in TMEM means the unpacked weights (4x the packed bytes) never
+// touch shared memory; only the packed tile and the activation tile do.
+// Code byte order: word r of packed word w holds k = 16w + 4i + r in byte i,
+// stored to TMEM column 4w + r, i.e. k-position 16w + 4r + i -- the same
+// k-interleaved order the activation kernel writes, so the MMA pairs equal k.
+//
+// Split-K (few row blocks): each CTA adds its int32 tile into a workspace
+// with atomics; the last CTA of a row/token block (arrival counter, no
+// waiting) reads back, re-zeroes and finishes the dequant.
 //
 // Every wait is bounded: on a timeout the thread records the failure in the
-// device status word, raises a CTA abort flag (so the other roles stop
-// waiting), and the kernel drains in-flight copies and MMAs before it frees
-// TMEM and exits without writing results.
+// device status word and raises a CTA abort flag; the kernel drains in-flight
+// copies and MMAs, frees TMEM and exits without writing results.
 #pragma once
 
 #include "common.cuh"
@@ -42,28 +50,50 @@ struct GemmParams {
   void* y;                // [M][N] or null
   int y_bf16;
   int32_t* acc_out;       // [M][N] debug or null
+  int ksplit;             // CTAs along K (gridDim.z)
+  int steps_per_split;    // KSTEP-k steps per CTA
+  int32_t* ws_acc;        // [M][N] split-K partials, zero on entry (ksplit > 1)
+  unsigned* ws_cnt;       // [row blocks * token blocks] counters, zero on entry
   int* status;            // device status word
   uint64_t wait_limit_ns;
 };
 
 template <int BN>
 struct GemmCfg {
-  static constexpr int BM = 128;                 // weight rows per CTA (MMA M)
-  static constexpr int BK = 128;                 // k per pipeline stage (one swizzle row)
-  static constexpr int STAGES = BN >= 256 ? 4 : (BN >= 128 ? 5 : 4);
-  static constexpr int X_BYTES = BN * BK;        // activation tile
-  static constexpr int A_BYTES = BM * BK;        // unpacked weight tile
-  static constexpr int WP_BYTES = BM * BK / 4;   // packed weight tile
+  static constexpr int BM = 128;                 // weight rows per CTA (MMA M, TMEM lanes)
+  // k per pipeline step: small token tiles stream 512 k per step so each TMA
+  // weight box has 128-byte rows (32-byte rows starve the copy engine);
+  // large tiles are tensor-bound and keep 128-k steps to fit the activations.
+  static constexpr int KSTEP = BN <= 64 ? 512 : 128;
+  static constexpr int ATOMS = KSTEP / 128;      // 128-byte swizzle atoms per activation tile
+  static constexpr int X_ATOM = BN * 128;        // bytes of one activation atom
+  static constexpr int X_BYTES = BN * KSTEP;     // activation tile
+  static constexpr int WP_ROW = KSTEP / 4;       // packed bytes per weight row per step
+  static constexpr int WP_BYTES = BM * WP_ROW;   // packed weight tile
+  static constexpr int STAGES = BN <= 16 ? 8 : (BN <= 32 ? 6 : (BN <= 64 ? 4 : (BN <= 128 ? 8 : 5)));
+  // TMEM: A_STAGES stages of KSTEP/4 columns of unpacked weights (four int8
+  // k per 32-bit column, one lane per weight row), then BN int32 accumulator
+  // columns.  One CTA owns all 512 columns.
+  static constexpr int A_COLS = KSTEP / 4;
+  static constexpr int A_STAGES = BN <= 64 ? 3 : 8;
+  static constexpr uint32_t A_COL = 0;
+  static constexpr uint32_t D_COL = A_COLS * A_STAGES;
+  static constexpr uint32_t TMEM_COLS = 512;
+  static constexpr int UNPACK_WARPS = 8;         // two per TMEM lane quarter
+  static constexpr int THREADS = 128 + 32 * UNPACK_WARPS;
+  static constexpr int PART = WP_ROW / 2;        // packed bytes per unpack thread per step
   static constexpr int OFF_X = 0;
-  static constexpr int OFF_A = OFF_X + STAGES * X_BYTES;
-  static constexpr int OFF_WP = OFF_A + STAGES * A_BYTES;
+  static constexpr int OFF_WP = OFF_X + STAGES * X_BYTES;
   static constexpr int OFF_BAR = OFF_WP + STAGES * WP_BYTES;
-  static constexpr int NBAR = 3 * STAGES + 1;
+  static constexpr int NBAR = 2 * STAGES + 2 * A_STAGES + 1;  // full/empty, aready/afree, accfull
   static constexpr int OFF_MISC = OFF_BAR + 8 * NBAR;
   static constexpr int BYTES = OFF_MISC + 16;
   static constexpr int SMEM_DYN = BYTES + 1024;  // slack for 1024-byte alignment
-  static constexpr uint32_t TMEM_COLS = BN;      // power of two >= 32
-  static_assert(BN == 64 || BN == 128 || BN == 256, "BN");
+  static_assert(BN == 16 || BN == 32 || BN == 64 || BN == 128 || BN == 256, "BN");
+  static_assert(D_COL + BN <= TMEM_COLS, "tensor memory");
+  static_assert(X_ATOM % 1024 == 0, "swizzle atoms must stay 1024-byte aligned");
+  static_assert(PART % 16 == 0, "unpack reads 16-byte words");
+  static_assert(WP_ROW == 128 || WP_ROW == 32, "weight tile swizzle");
   static_assert(SMEM_DYN <= 232448, "shared memory");
 };
 
@@ -72,8 +102,66 @@ __device__ __forceinline__ void gemm_fail(volatile int* abort_flag, int* status,
   record_failure(status, detail);
 }
 
+// All 32 lanes wait on `bar`; the verdict is made warp-uniform (tcgen05
+// loads/stores that follow are warp-collective).
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity,
+                                          const volatile int* abort_flag, uint64_t limit) {
+  const bool ok = mbar_wait_bounded(bar, parity, abort_flag, limit);
+  return __all_sync(0xFFFFFFFFu, ok);
+}
+
+__device__ __forceinline__ void tmem_st_32x32b_x32(uint32_t taddr, const uint32_t (&v)[32]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+      "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
+      "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]),
+      "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]),
+      "r"(v[15]), "r"(v[16]), "r"(v[17]), "r"(v[18]), "r"(v[19]), "r"(v[20]), "r"(v[21]),
+      "r"(v[22]), "r"(v[23]), "r"(v[24]), "r"(v[25]), "r"(v[26]), "r"(v[27]), "r"(v[28]),
+      "r"(v[29]), "r"(v[30]), "r"(v[31])
+      : "memory");
+}
+
+__device__ __forceinline__ void tmem_st_32x32b_x16(uint32_t taddr, const uint32_t (&v)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr),
+      "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]),
+      "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]),
+      "r"(v[15])
+      : "memory");
+}
+
+__device__ __forceinline__ void tmem_st_wait() {
+  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+
+// D[tmem] (+)= A[tmem] * B[smem desc]^T, int8 x int8 -> int32, one CTA.
+__device__ __forceinline__ void tc_mma_i8_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                             uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::i8 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+__device__ __forceinline__ void gemm_store(const GemmParams& p, float sw, int m, int n, int acc) {
+  const int64_t o = static_cast<int64_t>(m) * p.N + n;
+  if (p.acc_out) p.acc_out[o] = acc;
+  if (p.y) {
+    const float yv = __fdiv_rn(__int2float_rn(acc), __fmul_rn(p.s_x[m], sw));
+    if (p.y_bf16)
+      reinterpret_cast<__nv_bfloat16*>(p.y)[o] = __float2bfloat16_rn(yv);
+    else
+      reinterpret_cast<float*>(p.y)[o] = yv;
+  }
+}
+
 template <int BN>
-__global__ void __launch_bounds__(256, 1)
+__global__ void __launch_bounds__(GemmCfg<BN>::THREADS, 1)
 ternary_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x,
                        const __grid_constant__ CUtensorMap tmap_w, const GemmParams p) {
   using C = GemmCfg<BN>;
@@ -81,26 +169,33 @@ ternary_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x,
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   uint8_t* xs = smem + C::OFF_X;
-  uint8_t* as = smem + C::OFF_A;
   uint8_t* wps = smem + C::OFF_WP;
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
-  uint64_t* aready = full + C::STAGES;
-  uint64_t* empty = aready + C::STAGES;
-  uint64_t* accfull = empty + C::STAGES;
+  uint64_t* empty = full + C::STAGES;
+  uint64_t* aready = empty + C::STAGES;
+  uint64_t* afree = aready + C::A_STAGES;
+  uint64_t* accfull = afree + C::A_STAGES;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
+  int* is_last = reinterpret_cast<int*>(smem + C::OFF_MISC + 8);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int n0 = blockIdx.x * C::BM;
   const int m0 = blockIdx.y * BN;
-  const int nk = (p.K + C::BK - 1) / C::BK;
+  const int total_steps = (p.K + C::KSTEP - 1) / C::KSTEP;
+  const int kb0 = blockIdx.z * p.steps_per_split;
+  const int kb1 = min(kb0 + p.steps_per_split, total_steps);
+  const int nk = kb1 - kb0;
   const uint64_t limit = p.wait_limit_ns;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::STAGES; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&aready[s], 128);
-      mbar_init(&empty[s], 1);
+      mbar_init(&empty[s], 1 + C::UNPACK_WARPS);  // MMA commit + one per unpack warp
+    }
+    for (int a = 0; a < C::A_STAGES; ++a) {
+      mbar_init(&aready[a], C::UNPACK_WARPS);     // one arrival per unpack warp
+      mbar_init(&afree[a], 1);                    // MMA commit
     }
     mbar_init(accfull, 1);
     *abort_flag = 0;
@@ -117,30 +212,34 @@ ternary_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x,
   tc_fence_before_sync();
   __syncthreads();
   tc_fence_after_sync();
-  const uint32_t tmem_d = *tmem_slot;
+  const uint32_t tmem_base = *tmem_slot;
 
   if (warp == 0) {
     if (lane == 0) {
       // ------------------------------------------------------------ producer
       int issued = 0;
-      for (int kb = 0; kb < nk; ++kb) {
-        const int s = kb % C::STAGES;
-        const uint32_t use = static_cast<uint32_t>(kb / C::STAGES);
-        if (kb >= C::STAGES && !mbar_wait_bounded(&empty[s], (use - 1u) & 1u, abort_flag, limit)) {
+      for (int j = 0; j < nk; ++j) {
+        const int s = j % C::STAGES;
+        const uint32_t use = static_cast<uint32_t>(j / C::STAGES);
+        if (j >= C::STAGES && !mbar_wait_bounded(&empty[s], (use - 1u) & 1u, abort_flag, limit)) {
           gemm_fail(abort_flag, p.status, DEV_TIMEOUT_PRODUCER);
           break;
         }
+        const int kb = kb0 + j;
         mbar_arrive_expect_tx(&full[s], C::X_BYTES + C::WP_BYTES);
-        tma_load_2d(xs + s * C::X_BYTES, &tmap_x, kb * C::BK, m0, &full[s]);
-        tma_load_2d(wps + s * C::WP_BYTES, &tmap_w, kb * (C::BK / 4), n0, &full[s]);
-        issued = kb + 1;
+#pragma unroll
+        for (int at = 0; at < C::ATOMS; ++at)
+          tma_load_2d(xs + s * C::X_BYTES + at * C::X_ATOM, &tmap_x, kb * C::KSTEP + 128 * at, m0,
+                      &full[s]);
+        tma_load_2d(wps + s * C::WP_BYTES, &tmap_w, kb * C::WP_ROW, n0, &full[s]);
+        issued = j + 1;
       }
       if (*abort_flag) {
         // Let the copies already in flight land before the CTA exits.
         const int first = issued > C::STAGES ? issued - C::STAGES : 0;
-        for (int kb = first; kb < issued; ++kb) {
-          const int s = kb % C::STAGES;
-          if (!mbar_wait_bounded(&full[s], static_cast<uint32_t>(kb / C::STAGES) & 1u, nullptr,
+        for (int j = first; j < issued; ++j) {
+          const int s = j % C::STAGES;
+          if (!mbar_wait_bounded(&full[s], static_cast<uint32_t>(j / C::STAGES) & 1u, nullptr,
                                  limit))
             record_failure(p.status, DEV_TIMEOUT_DRAIN);
         }
@@ -150,24 +249,26 @@ ternary_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x,
     if (lane == 0) {
       // ------------------------------------------------------- MMA issuer
       const uint32_t idesc = umma_idesc_i8(C::BM, BN);
-      for (int kb = 0; kb < nk; ++kb) {
-        const int s = kb % C::STAGES;
-        const uint32_t par = static_cast<uint32_t>(kb / C::STAGES) & 1u;
-        if (!mbar_wait_bounded(&full[s], par, abort_flag, limit) ||
-            !mbar_wait_bounded(&aready[s], par, abort_flag, limit)) {
+      const uint32_t d_tmem = tmem_base + C::D_COL;
+      for (int j = 0; j < nk; ++j) {
+        const int s = j % C::STAGES, a = j % C::A_STAGES;
+        if (!mbar_wait_bounded(&aready[a], static_cast<uint32_t>(j / C::A_STAGES) & 1u,
+                               abort_flag, limit) ||
+            !mbar_wait_bounded(&full[s], static_cast<uint32_t>(j / C::STAGES) & 1u, abort_flag,
+                               limit)) {
           gemm_fail(abort_flag, p.status, DEV_TIMEOUT_MMA);
           break;
         }
         tc_fence_after_sync();
-        const uint32_t a_base = smem_u32(as + s * C::A_BYTES);
+        const uint32_t a_tmem = tmem_base + C::A_COL + static_cast<uint32_t>(C::A_COLS) * a;
         const uint32_t b_base = smem_u32(xs + s * C::X_BYTES);
 #pragma unroll
-        for (int kk = 0; kk < C::BK / 32; ++kk) {
-          tc_mma_i8(tmem_d, umma_desc_sw128_kmajor(a_base + 32 * kk),
-                    umma_desc_sw128_kmajor(b_base + 32 * kk), idesc,
-                    (kb > 0 || kk > 0) ? 1u : 0u);
-        }
+        for (int kk = 0; kk < C::KSTEP / 32; ++kk)
+          tc_mma_i8_ts(d_tmem, a_tmem + 8u * kk,
+                       umma_desc_sw128_kmajor(b_base + (kk >> 2) * C::X_ATOM + 32 * (kk & 3)),
+                       idesc, (j > 0 || kk > 0) ? 1u : 0u);
         tc_commit(&empty[s]);
+        tc_commit(&afree[a]);
       }
       // Signals the epilogue; on an abort it still marks that every MMA
       // issued so far has finished with TMEM and shared memory.
@@ -175,59 +276,78 @@ ternary_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x,
     }
   } else if (warp >= 4) {
     // ------------------------------------------------------------- unpack
-    const int i = threadIdx.x - 128;  // weight row inside the tile
-    const int sw = i & 7;
-    for (int kb = 0; kb < nk; ++kb) {
-      const int s = kb % C::STAGES;
-      const uint32_t par = static_cast<uint32_t>(kb / C::STAGES) & 1u;
-      if (!mbar_wait_bounded(&full[s], par, abort_flag, limit)) {
+    // Warp 4+u: TMEM lane quarter q = u % 4 (rows 32q..32q+31), half h = u / 4
+    // of each step's packed bytes (PART bytes -> PART TMEM columns).
+    const int u = warp - 4;
+    const int q = u & 3, h = u >> 2;
+    const int i = 32 * q + lane;        // weight row inside the tile
+    const uint32_t lane_addr = static_cast<uint32_t>(32 * q) << 16;
+    for (int j = 0; j < nk; ++j) {
+      const int s = j % C::STAGES, a = j % C::A_STAGES;
+      if (!warp_wait(&full[s], static_cast<uint32_t>(j / C::STAGES) & 1u, abort_flag, limit) ||
+          (j >= C::A_STAGES &&
+           !warp_wait(&afree[a], static_cast<uint32_t>(j / C::A_STAGES - 1) & 1u, abort_flag,
+                      limit))) {
         gemm_fail(abort_flag, p.status, DEV_TIMEOUT_UNPACK);
         break;
       }
-      const uint4* src = reinterpret_cast<const uint4*>(wps + s * C::WP_BYTES + i * 32);
-      const uint4 q0 = src[0], q1 = src[1];
-      uint8_t* dst = as + s * C::A_BYTES + i * 128;
-      const uint32_t words[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
+      tc_fence_after_sync();
+      constexpr int NV = C::PART / 16;  // 16-byte words of packed codes per thread
+      uint4 pk[NV];
 #pragma unroll
-      for (int w = 0; w < 8; ++w) {
-        const uint32_t P = words[w];
-        *reinterpret_cast<uint4*>(dst + ((w ^ sw) << 4)) =
-            make_uint4(P & 0x03030303u, (P >> 2) & 0x03030303u, (P >> 4) & 0x03030303u,
-                       (P >> 6) & 0x03030303u);
+      for (int t = 0; t < NV; ++t) {
+        // The copy engine wrote the tile swizzled (128-byte rows: chunk ^ row%8;
+        // 32-byte rows: chunk ^ (row/4)%2) so a warp's 32 rows hit distinct banks.
+        const int c = (C::PART / 16) * h + t;
+        const int pc = C::WP_ROW == 128 ? (c ^ (i & 7)) : (c ^ ((i >> 2) & 1));
+        pk[t] = *reinterpret_cast<const uint4*>(wps + s * C::WP_BYTES + i * C::WP_ROW + 16 * pc);
       }
-      fence_proxy_async_smem();
-      mbar_arrive(&aready[s]);
+      // The packed bytes are in registers: release the shared-memory stage.
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[s]);
+      const uint32_t col = tmem_base + lane_addr + C::A_COL + static_cast<uint32_t>(C::A_COLS) * a +
+                           static_cast<uint32_t>(C::PART) * h;
+#pragma unroll
+      for (int t = 0; t < NV; ++t) {
+        const uint32_t words[4] = {pk[t].x, pk[t].y, pk[t].z, pk[t].w};
+        uint32_t v[16];
+#pragma unroll
+        for (int w = 0; w < 4; ++w)
+#pragma unroll
+          for (int r = 0; r < 4; ++r) v[4 * w + r] = (words[w] >> (2 * r)) & 0x03030303u;
+        tmem_st_32x32b_x16(col + 16u * t, v);
+      }
+      tmem_st_wait();
+      tc_fence_before_sync();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&aready[a]);
     }
     // ----------------------------------------------------------- epilogue
-    const bool done = mbar_wait_bounded(accfull, 0u, nullptr, limit);
+    // Warps of half h take accumulator columns [h*BN/2, (h+1)*BN/2) (all of
+    // them when BN == 16, with half 1 idle).
+    const bool done = warp_wait(accfull, 0u, nullptr, limit);
     if (!done) gemm_fail(abort_flag, p.status, DEV_TIMEOUT_EPILOGUE);
     tc_fence_after_sync();
-    // tcgen05.ld is warp-collective: decide once per warp.
     const bool write = __all_sync(0xFFFFFFFFu, done && *abort_flag == 0);
-    if (write) {
-      const int wq = warp - 4;
-      const int n = n0 + wq * 32 + lane;
+    constexpr int kHalf = BN >= 32 ? BN / 2 : BN;
+    if (write && (BN >= 32 || h == 0)) {
+      const int n = n0 + i;
       const float swv = (p.y && p.s_w) ? *p.s_w : 0.0f;
-      for (int c0 = 0; c0 < BN; c0 += 16) {
+      const bool split = p.ksplit > 1;
+      for (int c0 = h * kHalf; c0 < (h + 1) * kHalf; c0 += 16) {
         if (m0 + c0 >= p.M) break;  // uniform across the warp
         uint32_t r[16];
-        tmem_ld_32x32b_x16(tmem_d + (static_cast<uint32_t>(wq * 32) << 16) + c0, r);
+        tmem_ld_32x32b_x16(tmem_base + lane_addr + C::D_COL + c0, r);
         tmem_ld_wait();
         if (n < p.N) {
 #pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            const int m = m0 + c0 + j;
+          for (int jj = 0; jj < 16; ++jj) {
+            const int m = m0 + c0 + jj;
             if (m < p.M) {
-              const int acc = static_cast<int>(r[j]) - p.rowsum[m];
-              const int64_t o = static_cast<int64_t>(m) * p.N + n;
-              if (p.acc_out) p.acc_out[o] = acc;
-              if (p.y) {
-                const float yv = __fdiv_rn(__int2float_rn(acc), __fmul_rn(p.s_x[m], swv));
-                if (p.y_bf16)
-                  reinterpret_cast<__nv_bfloat16*>(p.y)[o] = __float2bfloat16_rn(yv);
-                else
-                  reinterpret_cast<float*>(p.y)[o] = yv;
-              }
+              if (split)
+                atomicAdd(p.ws_acc + static_cast<int64_t>(m) * p.N + n, static_cast<int>(r[jj]));
+              else
+                gemm_store(p, swv, m, n, static_cast<int>(r[jj]) - p.rowsum[m]);
             }
           }
         }
@@ -239,7 +359,29 @@ ternary_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x,
   __syncthreads();
   if (warp == 1) {
     tc_fence_after_sync();
-    tmem_dealloc(tmem_d, C::TMEM_COLS);
+    tmem_dealloc(tmem_base, C::TMEM_COLS);
+  }
+
+  // Split-K: the last CTA of this output tile finishes (no waiting).
+  if (p.ksplit > 1) {
+    const int ok = __syncthreads_and(*abort_flag == 0 ? 1 : 0);
+    if (!ok) return;
+    const int tile = blockIdx.y * gridDim.x + blockIdx.x;
+    __threadfence();
+    __syncthreads();
+    if (threadIdx.x == 0)
+      *is_last = (atomicAdd(p.ws_cnt + tile, 1u) == static_cast<unsigned>(p.ksplit - 1)) ? 1 : 0;
+    __syncthreads();
+    if (!*is_last) return;
+    __threadfence();
+    const float swv = (p.y && p.s_w) ? *p.s_w : 0.0f;
+    const int rows = min(C::BM, p.N - n0), toks = min(BN, p.M - m0);
+    for (int idx = threadIdx.x; idx < rows * toks; idx += blockDim.x) {
+      const int r = idx % rows, mm = m0 + idx / rows, n = n0 + r;
+      const int v = atomicExch(p.ws_acc + static_cast<int64_t>(mm) * p.N + n, 0);
+      gemm_store(p, swv, mm, n, v - p.rowsum[mm]);
+    }
+    if (threadIdx.x == 0) p.ws_cnt[tile] = 0u;  // ready for the next call
   }
 }
 

@@ -119,3 +119,33 @@ def test_binding_refuses_cpu_tensors(lib):
     W = torch.zeros(64, 128)
     with pytest.raises(ValueError):
         tql.bitnet_quantize_pack_weights(W)
+
+
+def test_grouped_validation_and_workspace(lib):
+    import ctypes as C
+    P = tql.LinearProblem
+    arr = (P * 17)()
+    for i in range(17):
+        arr[i] = P(FAKE, 1, None, 1e-5, FAKE, FAKE, 4, 64, 256, FAKE, 1)
+    ptr = C.cast(arr, C.c_void_p)
+    assert lib.bitnet_linear_forward_grouped(17, ptr, C.c_void_p(FAKE), 1 << 30, 3, None) == \
+        tql.BITNET_ERR_INVALID_ARG
+    assert lib.bitnet_linear_forward_grouped(2, ptr, C.c_void_p(FAKE), 1 << 30, 0, None) == \
+        tql.BITNET_ERR_INVALID_ARG
+    arr[1].K = 100
+    assert lib.bitnet_linear_forward_grouped(2, ptr, C.c_void_p(FAKE), 1 << 30, 3, None) == \
+        tql.BITNET_ERR_UNSUPPORTED_SHAPE
+    arr[1].K = 256
+    arr[1].y = FAKE + 4
+    assert lib.bitnet_linear_forward_grouped(2, ptr, C.c_void_p(FAKE), 1 << 30, 3, None) == \
+        tql.BITNET_ERR_MISALIGNED
+    arr[1].y = FAKE
+    one = tql.bitnet_linear_forward_workspace_bytes(4, 64, 256)
+    assert tql.bitnet_linear_forward_grouped_workspace_bytes(arr, 2) == 2 * one
+    assert lib.bitnet_linear_forward_grouped(2, ptr, C.c_void_p(FAKE), 2 * one - 1, 3, None) == \
+        tql.BITNET_ERR_WORKSPACE
+    # empty groups and empty problems queue nothing
+    assert lib.bitnet_linear_forward_grouped(0, None, None, 0, 3, None) == tql.BITNET_OK
+    arr[0].M = 0
+    arr[1].M = 0
+    assert lib.bitnet_linear_forward_grouped(2, ptr, None, 0, 3, None) == tql.BITNET_OK

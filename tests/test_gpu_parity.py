@@ -278,3 +278,70 @@ def test_bounded_wait_reports_timeout():
 def test_no_device_failure_recorded():
     code, detail = tql.bitnet_device_status(reset=False)
     assert code == tql.BITNET_OK, detail
+
+
+# ------------------------------------------------------------- grouped
+
+def _grouped_items(case, extra=()):
+    items, meta = [], []
+    packed = {}
+    for si, K, N, M in workloads.all_problems(case):
+        if si not in packed:
+            packed[si] = (workloads.weights(case, si),) + _dev_weights(workloads.weights(case, si))
+        xh = workloads.activations(case, si, M)
+        y = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+        items.append((x_to_device(xh), None, workloads.DEFAULT_EPS, packed[si][1], packed[si][2], y))
+        meta.append((xh, packed[si][0], K, N, M))
+    for (M, N, K, ydt) in extra:
+        rng = np.random.default_rng(M * 13 + N)
+        W = (rng.standard_normal((N, K)) * 0.02).astype(np.float32)
+        xh = rng.standard_normal((M, K)).astype(np.float32)
+        W_p, s_w = _dev_weights(W)
+        y = torch.empty((M, N), dtype=ydt, device="cuda")
+        items.append((x_to_device(xh), None, workloads.DEFAULT_EPS, W_p, s_w, y))
+        meta.append((xh, W, K, N, M))
+    return items, meta
+
+
+@pytest.mark.parametrize("ci", [1, 2])
+@pytest.mark.parametrize("split", [False, True])
+def test_grouped_forward_matches_single_calls_and_oracle(ci, split):
+    case = workloads.CASES[ci]
+    # plus an fp32 decode problem, a prefill-sized one (tensor-core path) and an empty one
+    items, meta = _grouped_items(case, extra=[(5, 96, 320, torch.float32),
+                                              (40, 300, 512, torch.bfloat16),
+                                              (0, 64, 256, torch.bfloat16)])
+    if split:
+        ws = torch.empty(1 << 26, dtype=torch.uint8, device="cuda")
+        tql.bitnet_linear_forward_grouped(items, workspace=ws, phases=tql.BITNET_PHASE_QUANTIZE)
+        tql.bitnet_linear_forward_grouped(items, workspace=ws, phases=tql.BITNET_PHASE_MATMUL)
+    else:
+        tql.bitnet_linear_forward_grouped(items)
+    torch.cuda.synchronize()
+    for (x, g, eps, W_p, s_w, y), (xh, W, K, N, M) in zip(items, meta):
+        if M == 0:
+            continue
+        y1 = tql.bitnet_linear_forward(x, g, eps, W_p, s_w, y_dtype=y.dtype)
+        torch.cuda.synchronize()
+        if y.dtype == torch.bfloat16:
+            assert torch.equal(y.view(torch.int16), y1.view(torch.int16))
+        else:
+            assert torch.equal(y, y1)
+        ref_p, ref_s = oracle_weights(W)
+        cols = None if N <= 4096 else sample_columns(N, 256, seed=N)
+        ref = oracle.linear_forward(xh, None, eps, ref_p, ref_s, K, cols)
+        _check_y(y, ref["y"], ref["y_bf16"], cols)
+
+
+def test_grouped_rejects_bad_problem_and_queues_nothing():
+    case = workloads.CASES[1]
+    items, _ = _grouped_items(case)
+    for it in items:
+        it[5].fill_(0)
+    bad = list(items)
+    x, g, eps, W_p, s_w, y = bad[4]
+    bad[4] = (x, g, -1.0, W_p, s_w, y)  # eps < 0
+    with pytest.raises(tql.BitnetError):
+        tql.bitnet_linear_forward_grouped(bad)
+    torch.cuda.synchronize()
+    assert all(int(it[5].count_nonzero()) == 0 for it in items)
