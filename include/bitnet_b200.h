@@ -86,7 +86,7 @@ typedef enum { BITNET_F32 = 0, BITNET_BF16 = 1 } bitnet_dtype;
 
 /* Matmul path selection for the debug entry point (results never depend on it). */
 typedef enum {
-    BITNET_PATH_AUTO = 0,  /* decode GEMV for M <= 16, tensor-core GEMM above */
+    BITNET_PATH_AUTO = 0,  /* decode GEMV for M <= 16 and <= 32 MB of packed weights, else tcgen05 */
     BITNET_PATH_GEMV = 1,  /* tensor-core (mma.sync) streaming GEMV; needs M <= 16 */
     BITNET_PATH_GEMM = 2   /* tcgen05 + TMA GEMM with TMEM accumulators */
 } bitnet_path;
@@ -167,8 +167,9 @@ BITNET_API bitnet_status bitnet_rmsnorm_quant_act(const void *x, int x_dtype, co
 
 /* ------------------------------------------------------------------------
  * bitnet_linear_forward -- the whole BitLinear forward, y = dequant(
- *   quant(rmsnorm(x)) * ternary(W)^T ).  Picks the decode GEMV for M <= 16
- *   and the tcgen05 GEMM above; both give identical bits.
+ *   quant(rmsnorm(x)) * ternary(W)^T ).  Picks the warp-MMA decode GEMV for
+ *   M <= 16 with at most 32 MB of packed weights and the tcgen05 kernel
+ *   otherwise; both give identical bits.
  *
  *   x, x_dtype, gamma, eps   as bitnet_rmsnorm_quant_act.
  *   W_packed, s_w            as produced by bitnet_quantize_pack_weights
@@ -222,7 +223,7 @@ BITNET_API bitnet_status bitnet_linear_matmul(const uint8_t *W_packed, const flo
  * activation-quant launch and one matmul launch, so their weight streams
  * overlap instead of paying one launch latency each.  Typical use: the
  * projections of one decode step (q, k, v, o, gate, up, down).  Problems
- * with M > 16 run afterwards on the tensor-core GEMM, one at a time.
+ * with M > 16 run afterwards on the tcgen05 kernel, one at a time.
  *
  *   count      0 <= count <= BITNET_MAX_GROUP.
  *   problems   host array of `count` problem descriptions (each field as in

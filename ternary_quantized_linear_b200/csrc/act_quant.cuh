@@ -289,25 +289,20 @@ __device__ __forceinline__ void quant_row(const void* __restrict__ x,
   }
 }
 
-// Chunks per thread held in registers: 16 for bf16 rows (K <= 32768), 4 for
-// fp32 rows (K <= 8192); longer rows re-read.
-template <bool kBF16>
-__host__ __device__ constexpr int quant_cache_chunks() { return kBF16 ? 16 : 4; }
-
-template <bool kBF16, bool kInterleave>
-__device__ __forceinline__ void quant_row_any(const void* x, const float* gamma, float eps,
-                                              int64_t m, int64_t K, int8_t* x_q, float* s_x,
-                                              int32_t* rowsum, float* redf, int* redi) {
-  constexpr int C = quant_cache_chunks<kBF16>();
-  if ((K >> 3) <= static_cast<int64_t>(C) * kActThreads)
-    quant_row<kBF16, kInterleave, C>(x, gamma, eps, m, K, x_q, s_x, rowsum, redf, redi);
-  else
-    quant_row<kBF16, kInterleave, 0>(x, gamma, eps, m, K, x_q, s_x, rowsum, redf, redi);
+// Chunks per thread held in registers: the launch picks the smallest of
+// 1, 2, 4, 8, 16 that covers the row (bf16 rows up to 32 Ki elements; fp32
+// rows up to 4, i.e. K <= 8192), so the executed path stays short -- these
+// kernels run on few SMs with cold instruction caches.  Longer rows re-read.
+__host__ __device__ constexpr int quant_cache_for(int64_t K, bool bf16) {
+  const int64_t per = (K / 8 + kActThreads - 1) / kActThreads;
+  const int64_t cap = bf16 ? 16 : 4;
+  if (per > cap) return 0;
+  return per <= 1 ? 1 : (per <= 2 ? 2 : (per <= 4 ? 4 : (per <= 8 ? 8 : 16)));
 }
 
 // One CTA per row (blocks >= M zero `zero16` instead).  x: [M][K] (fp32 or
 // bf16 bits), gamma: [K] or null.
-template <bool kBF16, bool kInterleave>
+template <bool kBF16, bool kInterleave, int CACHE>
 __global__ void __launch_bounds__(kActThreads)
 rmsnorm_quant_kernel(const void* __restrict__ x, const float* __restrict__ gamma, float eps,
                      int64_t M, int64_t K, int8_t* __restrict__ x_q, float* __restrict__ s_x,
@@ -321,7 +316,7 @@ rmsnorm_quant_kernel(const void* __restrict__ x, const float* __restrict__ gamma
                      static_cast<int64_t>(gridDim.x) - M);
     return;
   }
-  quant_row_any<kBF16, kInterleave>(x, gamma, eps, blockIdx.x, K, x_q, s_x, rowsum, redf, redi);
+  quant_row<kBF16, kInterleave, CACHE>(x, gamma, eps, blockIdx.x, K, x_q, s_x, rowsum, redf, redi);
 }
 
 constexpr int kQuantMaxGroup = 16;
@@ -349,6 +344,7 @@ struct QuantLaunch {
 
 // Several independent problems in one launch: rows of every problem, then
 // each problem's zero-fill blocks, laid out by block_begin.
+template <int CACHE>
 __global__ void __launch_bounds__(kActThreads)
 rmsnorm_quant_grouped_kernel(const __grid_constant__ QuantLaunch L) {
   __shared__ float redf[kActThreads];
@@ -363,11 +359,13 @@ rmsnorm_quant_grouped_kernel(const __grid_constant__ QuantLaunch L) {
     zero_fill_blocks(q.zero16, q.n_zero16, local - q.M, q.zero_blocks);
     return;
   }
+  // CACHE covers every bf16 row of the launch; fp32 rows (rare: small
+  // problems) re-read.
   if (q.x_bf16)
-    quant_row_any<true, true>(q.x, q.gamma, q.eps, local, q.K, q.xi, q.s_x, q.rowsum, redf, redi);
+    quant_row<true, true, CACHE>(q.x, q.gamma, q.eps, local, q.K, q.xi, q.s_x, q.rowsum, redf,
+                                 redi);
   else
-    quant_row_any<false, true>(q.x, q.gamma, q.eps, local, q.K, q.xi, q.s_x, q.rowsum, redf,
-                               redi);
+    quant_row<false, true, 0>(q.x, q.gamma, q.eps, local, q.K, q.xi, q.s_x, q.rowsum, redf, redi);
 }
 
 // Natural-order x_q -> k-interleaved copy plus per-row sums (used when the

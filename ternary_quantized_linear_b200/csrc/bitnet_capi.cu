@@ -65,7 +65,7 @@ DeviceState* device_state() {
               cudaSuccess;
     ok = ok && cudaDeviceGetAttribute(&st.num_sms, cudaDevAttrMultiProcessorCount, dev) ==
                    cudaSuccess;
-    ok = ok && set_smem(ternary_gemv_kernel, kGemvRows * gemv_row_stride(kGemvMaxIps));
+    ok = ok && set_smem(ternary_gemv_kernel, gemv_smem_bytes(16));
     ok = ok && set_smem(ternary_gemm_tc_kernel<16>, GemmCfg<16>::SMEM_DYN);
     ok = ok && set_smem(ternary_gemm_tc_kernel<32>, GemmCfg<32>::SMEM_DYN);
     ok = ok && set_smem(ternary_gemm_tc_kernel<64>, GemmCfg<64>::SMEM_DYN);
@@ -153,32 +153,37 @@ bool ok_dtype(int d) { return d == BITNET_F32 || d == BITNET_BF16; }
 // ------------------------------------------------------------ launchers
 
 struct GemvPlan {
-  int rb, ksplit, ips, blocks;
-  size_t smem;
+  int rb, ksplit, steps, blocks;
 };
 
-// Row blocks of 16 weight rows; K is split across CTAs only when a slice
-// would not fit (more than kGemvMaxIps 256-k steps) or when there are too few
-// row blocks to give every SM a CTA.
-GemvPlan plan_gemv(int64_t N, int64_t K, int num_sms) {
+// Row blocks of 64 weight rows streaming K in 512-k steps.  K is split
+// across CTAs only when the whole launch has fewer row blocks than two per
+// SM (then the int32 partials go through the workspace).
+GemvPlan plan_gemv(int64_t N, int64_t K, int num_sms, int64_t launch_row_blocks = 0) {
   GemvPlan pl{};
   pl.rb = static_cast<int>((N + kGemvRows - 1) / kGemvRows);
-  const int iters = static_cast<int>((K + 255) / 256);
-  int ks = (iters + kGemvMaxIps - 1) / kGemvMaxIps;
-  if (pl.rb * ks < num_sms) ks = std::max(ks, std::min(iters, (num_sms + pl.rb - 1) / pl.rb));
-  pl.ips = (iters + ks - 1) / ks;
-  pl.ksplit = (iters + pl.ips - 1) / pl.ips;
+  const int total = static_cast<int>((K + kGemvKStep - 1) / kGemvKStep);
+  const int64_t lrb = launch_row_blocks > 0 ? launch_row_blocks : pl.rb;
+  int ks = 1;
+  if (lrb < 2 * num_sms)
+    ks = std::max(1, std::min(total, static_cast<int>((2 * num_sms + lrb - 1) / lrb)));
+  pl.steps = (total + ks - 1) / ks;
+  pl.ksplit = (total + pl.steps - 1) / pl.steps;
   pl.blocks = pl.rb * pl.ksplit;
-  pl.smem = static_cast<size_t>(kGemvRows) * gemv_row_stride(pl.ips);
   return pl;
 }
 
-void fill_gemv_problem(GemvProblem& q, const GemvPlan& pl, const uint8_t* Wp, uint8_t* ws,
+bool fill_gemv_problem(GemvProblem& q, const GemvPlan& pl, const uint8_t* Wp, uint8_t* ws,
                        const FwdWorkspace& L, const float* s_x, const float* s_w, int64_t M,
-                       int64_t N, int64_t K, void* y, int y_dtype, int32_t* acc_out,
+                       int64_t N, int64_t K, int mt, void* y, int y_dtype, int32_t* acc_out,
                        int block_begin) {
-  q.Wp = Wp;
-  q.xi = reinterpret_cast<const int8_t*>(ws + L.xq);
+  if (!make_tmap_u8(&q.tmap_w, Wp, static_cast<uint64_t>(K / 4), static_cast<uint64_t>(N),
+                    static_cast<uint64_t>(K / 4), 128, kGemvRows, CU_TENSOR_MAP_SWIZZLE_128B))
+    return false;
+  if (!make_tmap_u8(&q.tmap_x, ws + L.xq, static_cast<uint64_t>(K), static_cast<uint64_t>(M),
+                    static_cast<uint64_t>(K), 128, static_cast<uint32_t>(mt),
+                    CU_TENSOR_MAP_SWIZZLE_128B))
+    return false;
   q.rowsum = reinterpret_cast<const int32_t*>(ws + L.rs);
   q.s_x = s_x;
   q.s_w = s_w;
@@ -192,20 +197,21 @@ void fill_gemv_problem(GemvProblem& q, const GemvPlan& pl, const uint8_t* Wp, ui
   q.y_bf16 = (y_dtype == BITNET_BF16) ? 1 : 0;
   q.rb = pl.rb;
   q.ksplit = pl.ksplit;
-  q.ips = pl.ips;
+  q.steps = pl.steps;
   q.block_begin = block_begin;
+  return true;
 }
 
-bitnet_status launch_gemv_group(const DeviceState& ds, GemvLaunch& L, int blocks, size_t smem,
-                                bool pdl, bool early_weights, cudaStream_t stream) {
+bitnet_status launch_gemv_group(const DeviceState& ds, GemvLaunch& L, int blocks, bool pdl,
+                                bool early_weights, cudaStream_t stream) {
   L.use_pdl = pdl ? 1 : 0;
   L.early_weights = (pdl && early_weights) ? 1 : 0;
   L.status = ds.status;
   L.wait_limit_ns = kWaitLimitNs;
   cudaLaunchConfig_t cfg{};
   cfg.gridDim = dim3(static_cast<unsigned>(blocks), 1, 1);
-  cfg.blockDim = dim3(kGemvWarps * 32, 1, 1);
-  cfg.dynamicSmemBytes = smem;
+  cfg.blockDim = dim3(kGemvThreads, 1, 1);
+  cfg.dynamicSmemBytes = gemv_smem_bytes(L.mt);
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -221,10 +227,13 @@ bitnet_status launch_gemv(const DeviceState& ds, const uint8_t* Wp, const float*
                           const FwdWorkspace& Lw, void* y, int y_dtype, int32_t* acc_out,
                           bool pdl, bool early_weights, cudaStream_t stream) {
   const GemvPlan pl = plan_gemv(N, K, ds.num_sms);
-  GemvLaunch L{};
+  static thread_local GemvLaunch L;  // ~6 KB: keep it off the stack
   L.count = 1;
-  fill_gemv_problem(L.prob[0], pl, Wp, ws, Lw, s_x, s_w, M, N, K, y, y_dtype, acc_out, 0);
-  return launch_gemv_group(ds, L, pl.blocks, pl.smem, pdl, early_weights, stream);
+  L.mt = M <= 8 ? 8 : 16;
+  if (!fill_gemv_problem(L.prob[0], pl, Wp, ws, Lw, s_x, s_w, M, N, K, L.mt, y, y_dtype, acc_out,
+                         0))
+    return BITNET_ERR_CUDA;
+  return launch_gemv_group(ds, L, pl.blocks, pdl, early_weights, stream);
 }
 
 struct GemmPlan {
@@ -238,13 +247,16 @@ GemmPlan plan_gemm(int64_t M, int64_t N, int64_t K, int num_sms) {
   pl.BN = M <= 16 ? 16 : (M <= 32 ? 32 : (M <= 64 ? 64 : (M <= 128 ? 128 : 256)));
   pl.rb = static_cast<int>((N + 127) / 128);
   pl.tb = static_cast<int>((M + pl.BN - 1) / pl.BN);
-  const int kstep = pl.BN <= 64 ? 512 : 128;  // GemmCfg<BN>::KSTEP
+  const bool small = pl.BN <= 64;            // GemmCfg<BN>::SMALL
+  const int kstep = 256;                      // GemmCfg<BN>::KSTEP
   const int steps = static_cast<int>((K + kstep - 1) / kstep);
   int ks = 1;
   if (M <= kGemvMaxM) {
-    const int target = num_sms;  // one CTA per SM (each owns all of TMEM)
+    // Resident slots: two CTAs per SM for small token tiles.  Split K so the
+    // grid fills the slots without starting a partial second wave.
+    const int slots = (small ? 2 : 1) * num_sms;
     const int tiles = pl.rb * pl.tb;
-    ks = std::max(1, std::min(steps, (target + tiles - 1) / tiles));
+    if (tiles < slots) ks = std::max(1, std::min(steps, slots / tiles));
   }
   pl.steps_per_split = (steps + ks - 1) / ks;
   pl.ksplit = (steps + pl.steps_per_split - 1) / pl.steps_per_split;
@@ -254,29 +266,36 @@ GemmPlan plan_gemm(int64_t M, int64_t N, int64_t K, int num_sms) {
 template <int BN>
 bitnet_status launch_gemm_bn(const CUtensorMap& tx, const CUtensorMap& tw, const GemmParams& p,
                              const GemmPlan& pl, cudaStream_t stream) {
-  dim3 grid(static_cast<unsigned>(pl.rb), static_cast<unsigned>(pl.tb),
-            static_cast<unsigned>(pl.ksplit));
-  ternary_gemm_tc_kernel<BN><<<grid, GemmCfg<BN>::THREADS, GemmCfg<BN>::SMEM_DYN, stream>>>(
-      tx, tw, p);
-  return launch_status();
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(static_cast<unsigned>(pl.rb), static_cast<unsigned>(pl.tb),
+                     static_cast<unsigned>(pl.ksplit));
+  cfg.blockDim = dim3(GemmCfg<BN>::THREADS, 1, 1);
+  cfg.dynamicSmemBytes = GemmCfg<BN>::SMEM_DYN;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = p.use_pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, ternary_gemm_tc_kernel<BN>, tx, tw, p) == cudaSuccess
+             ? BITNET_OK
+             : BITNET_ERR_CUDA;
 }
 
 bitnet_status launch_gemm(const DeviceState& ds, const uint8_t* Wp, const int8_t* xi,
                           const int32_t* rowsum, const float* s_x, const float* s_w, int64_t M,
                           int64_t N, int64_t K, uint8_t* ws, const FwdWorkspace& Lw, void* y,
-                          int y_dtype, int32_t* acc_out, cudaStream_t stream) {
+                          int y_dtype, int32_t* acc_out, bool pdl, cudaStream_t stream) {
   const GemmPlan pl = plan_gemm(M, N, K, ds.num_sms);
   CUtensorMap tx, tw;
   if (!make_tmap_u8(&tx, xi, static_cast<uint64_t>(K), static_cast<uint64_t>(M),
                     static_cast<uint64_t>(K), 128, static_cast<uint32_t>(pl.BN),
                     CU_TENSOR_MAP_SWIZZLE_128B))
     return BITNET_ERR_CUDA;
-  // GemmCfg<BN>::WP_ROW bytes per row, swizzled so the unpack reads are
+  // GemmCfg<BN>::WP_ROW = 64 bytes per row, swizzled so the unpack reads are
   // bank-conflict free.
-  const uint32_t wp_row = pl.BN <= 64 ? 128 : 32;
   if (!make_tmap_u8(&tw, Wp, static_cast<uint64_t>(K / 4), static_cast<uint64_t>(N),
-                    static_cast<uint64_t>(K / 4), wp_row, 128,
-                    wp_row == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_32B))
+                    static_cast<uint64_t>(K / 4), 64, 128, CU_TENSOR_MAP_SWIZZLE_64B))
     return BITNET_ERR_CUDA;
   GemmParams p{};
   p.rowsum = rowsum;
@@ -294,6 +313,7 @@ bitnet_status launch_gemm(const DeviceState& ds, const uint8_t* Wp, const int8_t
   p.ws_cnt = reinterpret_cast<unsigned*>(ws + Lw.cnt);
   p.status = ds.status;
   p.wait_limit_ns = kWaitLimitNs;
+  p.use_pdl = pdl ? 1 : 0;
   switch (pl.BN) {
     case 16: return launch_gemm_bn<16>(tx, tw, p, pl, stream);
     case 32: return launch_gemm_bn<32>(tx, tw, p, pl, stream);
@@ -329,21 +349,25 @@ bitnet_status launch_act_quant(const void* x, int x_dtype, const float* gamma, f
   const int trig = trigger ? 1 : 0;
   uint4* z = static_cast<uint4*>(zero);
   const int64_t n16 = zero ? static_cast<int64_t>(zero_bytes / 16) : 0;
-  if (x_dtype == BITNET_BF16) {
-    if (interleave)
-      rmsnorm_quant_kernel<true, true><<<grid, block, 0, stream>>>(x, gamma, eps, M, K, x_q,
-                                                                   s_x, rowsum, z, n16, trig);
-    else
-      rmsnorm_quant_kernel<true, false><<<grid, block, 0, stream>>>(x, gamma, eps, M, K, x_q,
-                                                                    s_x, rowsum, z, n16, trig);
-  } else {
-    if (interleave)
-      rmsnorm_quant_kernel<false, true><<<grid, block, 0, stream>>>(x, gamma, eps, M, K, x_q,
-                                                                    s_x, rowsum, z, n16, trig);
-    else
-      rmsnorm_quant_kernel<false, false><<<grid, block, 0, stream>>>(x, gamma, eps, M, K, x_q,
-                                                                     s_x, rowsum, z, n16, trig);
+#define BITNET_QUANT(BF, IL, C)                                                        \
+  rmsnorm_quant_kernel<BF, IL, C><<<grid, block, 0, stream>>>(x, gamma, eps, M, K, x_q, s_x, \
+                                                              rowsum, z, n16, trig)
+#define BITNET_QUANT_C(BF, IL)                                    \
+  switch (quant_cache_for(K, BF)) {                               \
+    case 1: BITNET_QUANT(BF, IL, 1); break;                       \
+    case 2: BITNET_QUANT(BF, IL, 2); break;                       \
+    case 4: BITNET_QUANT(BF, IL, 4); break;                       \
+    case 8: BITNET_QUANT(BF, IL, 8); break;                       \
+    case 16: BITNET_QUANT(BF, IL, 16); break;                     \
+    default: BITNET_QUANT(BF, IL, 0); break;                      \
   }
+  if (x_dtype == BITNET_BF16) {
+    if (interleave) { BITNET_QUANT_C(true, true) } else { BITNET_QUANT_C(true, false) }
+  } else {
+    if (interleave) { BITNET_QUANT_C(false, true) } else { BITNET_QUANT_C(false, false) }
+  }
+#undef BITNET_QUANT_C
+#undef BITNET_QUANT
   return launch_status();
 }
 
@@ -364,12 +388,19 @@ bitnet_status run_matmul(const DeviceState& ds, int path, const uint8_t* Wp, uin
                        early_weights, stream);
   const int8_t* xi = reinterpret_cast<const int8_t*>(ws + L.xq);
   const int32_t* rs = reinterpret_cast<const int32_t*>(ws + L.rs);
-  return launch_gemm(ds, Wp, xi, rs, s_x, s_w, M, N, K, ws, L, y, y_dtype, acc_out, stream);
+  return launch_gemm(ds, Wp, xi, rs, s_x, s_w, M, N, K, ws, L, y, y_dtype, acc_out, pdl,
+                     stream);
 }
 
-int resolve_path(int path, int64_t M) {
-  if (path == BITNET_PATH_AUTO) return M <= kGemvMaxM ? BITNET_PATH_GEMV : BITNET_PATH_GEMM;
-  return path;
+// Decode GEMV (warp-level MMA) for M <= 16 unless the matrix is large: above
+// ~32 MB of packed weights the tcgen05 kernel streams faster (measured on
+// B200), and for M > 16 it is the only path.
+constexpr int64_t kGemvAutoMaxBytes = int64_t(32) << 20;
+
+int resolve_path(int path, int64_t M, int64_t N = 0, int64_t K = 0) {
+  if (path != BITNET_PATH_AUTO) return path;
+  if (M > kGemvMaxM) return BITNET_PATH_GEMM;
+  return (N * (K / 4) <= kGemvAutoMaxBytes) ? BITNET_PATH_GEMV : BITNET_PATH_GEMM;
 }
 
 bitnet_status forward_impl(const void* x, int x_dtype, const float* gamma, float eps,
@@ -384,7 +415,7 @@ bitnet_status forward_impl(const void* x, int x_dtype, const float* gamma, float
     return BITNET_ERR_INVALID_ARG;
   if (y && !ok_dtype(y_dtype)) return BITNET_ERR_INVALID_ARG;
   if (path < BITNET_PATH_AUTO || path > BITNET_PATH_GEMM) return BITNET_ERR_INVALID_ARG;
-  path = resolve_path(path, M);
+  path = resolve_path(path, M, N, K);
   if (path == BITNET_PATH_GEMV && M > kGemvMaxM) return BITNET_ERR_INVALID_ARG;
   if (!aligned(x, 16) || (gamma && !aligned(gamma, 16)) || !aligned(W_packed, 16) ||
       !aligned(s_w, 4) || (y && !aligned(y, 16)) || (x_q_out && !aligned(x_q_out, 16)) ||
@@ -404,7 +435,7 @@ bitnet_status forward_impl(const void* x, int x_dtype, const float* gamma, float
                           nullptr, 0, stream);
     if (st != BITNET_OK) return st;
   }
-  const bool pdl = (path == BITNET_PATH_GEMV);
+  const bool pdl = true;  // the matmul launch follows the quant launch directly
   float* sx = reinterpret_cast<float*>(ws + L.sx);
   size_t zbytes = 0;
   void* zero = needs_zeroed_partials(*ds, path, M, N, K) ? splitk_region(ws, L, &zbytes)
@@ -462,10 +493,19 @@ bitnet_status forward_grouped_impl(int count, const bitnet_linear_problem* probl
   uint8_t* base = static_cast<uint8_t*>(workspace);
 
   // Decode problems: one grouped quant launch, one grouped matmul launch.
-  QuantLaunch QL{};
-  GemvLaunch GL{};
+  static thread_local QuantLaunch QL;
+  static thread_local GemvLaunch GL;
+  QL = QuantLaunch{};
+  GL.count = 0;
   int qblocks = 0, gblocks = 0, n = 0;
-  size_t smem = 0;
+  int64_t launch_rb = 0;
+  int mt = 8;
+  for (int i = 0; i < count; ++i) {
+    const bitnet_linear_problem& q = problems[i];
+    if (q.M == 0 || q.M > kGemvMaxM) continue;
+    launch_rb += (q.N + kGemvRows - 1) / kGemvRows;
+    if (q.M > 8) mt = 16;
+  }
   size_t off = 0;
   for (int i = 0; i < count; ++i) {
     const bitnet_linear_problem& q = problems[i];
@@ -474,7 +514,7 @@ bitnet_status forward_grouped_impl(int count, const bitnet_linear_problem* probl
     uint8_t* ws = base + off;
     off += L.total;
     if (q.M > kGemvMaxM) continue;
-    const GemvPlan pl = plan_gemv(q.N, q.K, ds->num_sms);
+    const GemvPlan pl = plan_gemv(q.N, q.K, ds->num_sms, launch_rb);
     size_t zbytes = 0;
     void* zero = pl.ksplit > 1 ? splitk_region(ws, L, &zbytes) : nullptr;
     QuantProblem& qp = QL.prob[n];
@@ -492,31 +532,45 @@ bitnet_status forward_grouped_impl(int count, const bitnet_linear_problem* probl
     qp.block_begin = qblocks;
     qp.zero_blocks = static_cast<int>(zero ? zero_blocks(zbytes) : 0);
     qblocks += qp.M + qp.zero_blocks;
-    fill_gemv_problem(GL.prob[n], pl, q.W_packed, ws, L, qp.s_x, q.s_w, q.M, q.N, q.K, q.y,
-                      q.y_dtype, nullptr, gblocks);
+    if (!fill_gemv_problem(GL.prob[n], pl, q.W_packed, ws, L, qp.s_x, q.s_w, q.M, q.N, q.K, mt,
+                           q.y, q.y_dtype, nullptr, gblocks))
+      return BITNET_ERR_CUDA;
     gblocks += pl.blocks;
-    smem = std::max(smem, pl.smem);
     ++n;
   }
   if (n > 0) {
     QL.count = n;
     QL.trigger_dependents = do_matmul ? 1 : 0;
     GL.count = n;
+    GL.mt = mt;
     if (do_quant) {
-      rmsnorm_quant_grouped_kernel<<<static_cast<unsigned>(qblocks), kActThreads, 0, stream>>>(
-          QL);
+      int cache = 1;  // 0 = some bf16 row is too long to hold in registers
+      for (int i = 0; i < n; ++i) {
+        if (!QL.prob[i].x_bf16) continue;
+        const int c = quant_cache_for(QL.prob[i].K, true);
+        cache = (c == 0 || cache == 0) ? 0 : std::max(cache, c);
+      }
+      const dim3 qg(static_cast<unsigned>(qblocks));
+      switch (cache) {
+        case 1: rmsnorm_quant_grouped_kernel<1><<<qg, kActThreads, 0, stream>>>(QL); break;
+        case 2: rmsnorm_quant_grouped_kernel<2><<<qg, kActThreads, 0, stream>>>(QL); break;
+        case 4: rmsnorm_quant_grouped_kernel<4><<<qg, kActThreads, 0, stream>>>(QL); break;
+        case 8: rmsnorm_quant_grouped_kernel<8><<<qg, kActThreads, 0, stream>>>(QL); break;
+        case 16: rmsnorm_quant_grouped_kernel<16><<<qg, kActThreads, 0, stream>>>(QL); break;
+        default: rmsnorm_quant_grouped_kernel<0><<<qg, kActThreads, 0, stream>>>(QL); break;
+      }
       const bitnet_status st = launch_status();
       if (st != BITNET_OK) return st;
     }
     if (do_matmul) {
       // When the quant grid was just queued it started after every earlier
       // write to the weights, so the copies may begin before waiting on it.
-      const bitnet_status st = launch_gemv_group(*ds, GL, gblocks, smem, true, do_quant, stream);
+      const bitnet_status st = launch_gemv_group(*ds, GL, gblocks, true, do_quant, stream);
       if (st != BITNET_OK) return st;
     }
   }
   if (!do_matmul) return BITNET_OK;
-  // Prefill problems: the tensor-core GEMM, one after another.
+  // Larger problems: the tcgen05 kernel, one after another.
   off = 0;
   for (int i = 0; i < count; ++i) {
     const bitnet_linear_problem& q = problems[i];
@@ -656,7 +710,7 @@ BITNET_API bitnet_status bitnet_linear_matmul(const uint8_t* W_packed, const flo
   DeviceState* ds = device_state();
   if (!ds) return BITNET_ERR_CUDA;
   uint8_t* ws = static_cast<uint8_t*>(workspace);
-  const int path = resolve_path(BITNET_PATH_AUTO, M);
+  const int path = resolve_path(BITNET_PATH_AUTO, M, N, K);
   return run_matmul(*ds, path, W_packed, ws, L, reinterpret_cast<const float*>(ws + L.sx), s_w,
                     M, N, K, y, y_dtype, nullptr, path == BITNET_PATH_GEMV, false,
                     as_stream(stream));
@@ -696,7 +750,7 @@ BITNET_API bitnet_status bitnet_ternary_matmul_i32(const int8_t* x_q, const uint
   if (M == 0) return BITNET_OK;
   if (!x_q || !W_packed || !acc) return BITNET_ERR_INVALID_ARG;
   if (path < BITNET_PATH_AUTO || path > BITNET_PATH_GEMM) return BITNET_ERR_INVALID_ARG;
-  path = resolve_path(path, M);
+  path = resolve_path(path, M, N, K);
   if (path == BITNET_PATH_GEMV && M > kGemvMaxM) return BITNET_ERR_INVALID_ARG;
   if (!aligned(x_q, 16) || !aligned(W_packed, 16) || !aligned(acc, 16))
     return BITNET_ERR_MISALIGNED;

@@ -9,7 +9,7 @@
 // 量子化の仕組み (rescale by both scales).
 //
 // A CTA computes a 128 (weight rows, TMEM lanes) x BN (tokens) tile of
-// acc^T over a range of K, in KSTEP-k steps (512 for BN <= 64, else 128):
+// acc^T over a range of K, in 256-k steps:
 //   warp 0      TMA producer: per step the packed weight tile (128 rows x
 //               KSTEP/4 bytes) and the activation tile (BN rows of KSTEP int8
 //               as 128-byte swizzle atoms = the MMA's canonical K-major
@@ -56,45 +56,51 @@ struct GemmParams {
   unsigned* ws_cnt;       // [row blocks * token blocks] counters, zero on entry
   int* status;            // device status word
   uint64_t wait_limit_ns;
+  int use_pdl;            // wait for the preceding grid before touching its outputs
 };
 
 template <int BN>
 struct GemmCfg {
   static constexpr int BM = 128;                 // weight rows per CTA (MMA M, TMEM lanes)
-  // k per pipeline step: small token tiles stream 512 k per step so each TMA
-  // weight box has 128-byte rows (32-byte rows starve the copy engine);
-  // large tiles are tensor-bound and keep 128-k steps to fit the activations.
-  static constexpr int KSTEP = BN <= 64 ? 512 : 128;
+  static constexpr bool SMALL = BN <= 64;        // decode-sized token tile
+  // 256 k per pipeline step: each TMA weight box has 64-byte rows (narrower
+  // rows starve the copy engine) and each step issues 8 MMAs, amortising the
+  // per-step barrier traffic.  Small token tiles are bound by the MMA issue
+  // rate (a fixed cost per instruction), so two CTAs share each SM to
+  // interleave their MMA streams; large tiles are tensor-bound, one CTA/SM.
+  static constexpr int KSTEP = 256;
   static constexpr int ATOMS = KSTEP / 128;      // 128-byte swizzle atoms per activation tile
   static constexpr int X_ATOM = BN * 128;        // bytes of one activation atom
   static constexpr int X_BYTES = BN * KSTEP;     // activation tile
   static constexpr int WP_ROW = KSTEP / 4;       // packed bytes per weight row per step
   static constexpr int WP_BYTES = BM * WP_ROW;   // packed weight tile
-  static constexpr int STAGES = BN <= 16 ? 8 : (BN <= 32 ? 6 : (BN <= 64 ? 4 : (BN <= 128 ? 8 : 5)));
+  static constexpr int STAGES = BN <= 16 ? 8 : (BN <= 32 ? 6 : (BN <= 64 ? 4 : (BN <= 128 ? 5 : 3)));
   // TMEM: A_STAGES stages of KSTEP/4 columns of unpacked weights (four int8
   // k per 32-bit column, one lane per weight row), then BN int32 accumulator
-  // columns.  One CTA owns all 512 columns.
+  // columns.
   static constexpr int A_COLS = KSTEP / 4;
-  static constexpr int A_STAGES = BN <= 64 ? 3 : 8;
+  static constexpr int A_STAGES = SMALL ? 3 : STAGES;
   static constexpr uint32_t A_COL = 0;
   static constexpr uint32_t D_COL = A_COLS * A_STAGES;
-  static constexpr uint32_t TMEM_COLS = 512;
+  static constexpr uint32_t TMEM_COLS = SMALL ? 256 : 512;
+  static constexpr int MIN_BLOCKS = SMALL ? 2 : 1;
   static constexpr int UNPACK_WARPS = 8;         // two per TMEM lane quarter
   static constexpr int THREADS = 128 + 32 * UNPACK_WARPS;
   static constexpr int PART = WP_ROW / 2;        // packed bytes per unpack thread per step
   static constexpr int OFF_X = 0;
   static constexpr int OFF_WP = OFF_X + STAGES * X_BYTES;
   static constexpr int OFF_BAR = OFF_WP + STAGES * WP_BYTES;
-  static constexpr int NBAR = 2 * STAGES + 2 * A_STAGES + 1;  // full/empty, aready/afree, accfull
+  static constexpr int NBAR = 2 * STAGES + A_STAGES + 1;  // full/done, aready, accfull
   static constexpr int OFF_MISC = OFF_BAR + 8 * NBAR;
   static constexpr int BYTES = OFF_MISC + 16;
   static constexpr int SMEM_DYN = BYTES + 1024;  // slack for 1024-byte alignment
   static_assert(BN == 16 || BN == 32 || BN == 64 || BN == 128 || BN == 256, "BN");
+  static_assert(A_STAGES <= STAGES, "A stages are recycled through the stage barriers");
   static_assert(D_COL + BN <= TMEM_COLS, "tensor memory");
   static_assert(X_ATOM % 1024 == 0, "swizzle atoms must stay 1024-byte aligned");
   static_assert(PART % 16 == 0, "unpack reads 16-byte words");
-  static_assert(WP_ROW == 128 || WP_ROW == 32, "weight tile swizzle");
-  static_assert(SMEM_DYN <= 232448, "shared memory");
+  static_assert(WP_ROW == 64, "weight tile swizzle");
+  static_assert(SMEM_DYN * MIN_BLOCKS <= 232448, "shared memory");
 };
 
 __device__ __forceinline__ void gemm_fail(volatile int* abort_flag, int* status, int detail) {
@@ -161,7 +167,7 @@ __device__ __forceinline__ void gemm_store(const GemmParams& p, float sw, int m,
 }
 
 template <int BN>
-__global__ void __launch_bounds__(GemmCfg<BN>::THREADS, 1)
+__global__ void __launch_bounds__(GemmCfg<BN>::THREADS, GemmCfg<BN>::MIN_BLOCKS)
 ternary_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x,
                        const __grid_constant__ CUtensorMap tmap_w, const GemmParams p) {
   using C = GemmCfg<BN>;
@@ -170,11 +176,16 @@ ternary_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x,
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   uint8_t* xs = smem + C::OFF_X;
   uint8_t* wps = smem + C::OFF_WP;
+  // full[s]: both tiles of a step landed (TMA transaction bytes).
+  // done[s]: the step's MMAs completed (one tcgen05.commit) -- which also
+  //          means the unpack warps had finished reading its weight tile,
+  //          since the MMAs waited for them; it frees the shared-memory stage
+  //          for the producer and, A_STAGES steps later, the TMEM A stage.
+  // aready[a]: the unpack warps stored TMEM A stage a.
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
-  uint64_t* empty = full + C::STAGES;
-  uint64_t* aready = empty + C::STAGES;
-  uint64_t* afree = aready + C::A_STAGES;
-  uint64_t* accfull = afree + C::A_STAGES;
+  uint64_t* done = full + C::STAGES;
+  uint64_t* aready = done + C::STAGES;
+  uint64_t* accfull = aready + C::A_STAGES;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
   int* is_last = reinterpret_cast<int*>(smem + C::OFF_MISC + 8);
@@ -191,12 +202,9 @@ ternary_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x,
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::STAGES; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&empty[s], 1 + C::UNPACK_WARPS);  // MMA commit + one per unpack warp
+      mbar_init(&done[s], 1);                     // MMA commit
     }
-    for (int a = 0; a < C::A_STAGES; ++a) {
-      mbar_init(&aready[a], C::UNPACK_WARPS);     // one arrival per unpack warp
-      mbar_init(&afree[a], 1);                    // MMA commit
-    }
+    for (int a = 0; a < C::A_STAGES; ++a) mbar_init(&aready[a], C::UNPACK_WARPS);
     mbar_init(accfull, 1);
     *abort_flag = 0;
     fence_mbarrier_init();
@@ -213,6 +221,9 @@ ternary_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x,
   __syncthreads();
   tc_fence_after_sync();
   const uint32_t tmem_base = *tmem_slot;
+  // Set-up above overlaps the preceding grid; its outputs (activations, row
+  // sums, scales) are read only after this point.
+  if (p.use_pdl) pdl_wait_prior_grid();
 
   if (warp == 0) {
     if (lane == 0) {
@@ -221,7 +232,7 @@ ternary_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x,
       for (int j = 0; j < nk; ++j) {
         const int s = j % C::STAGES;
         const uint32_t use = static_cast<uint32_t>(j / C::STAGES);
-        if (j >= C::STAGES && !mbar_wait_bounded(&empty[s], (use - 1u) & 1u, abort_flag, limit)) {
+        if (j >= C::STAGES && !mbar_wait_bounded(&done[s], (use - 1u) & 1u, abort_flag, limit)) {
           gemm_fail(abort_flag, p.status, DEV_TIMEOUT_PRODUCER);
           break;
         }
@@ -252,6 +263,9 @@ ternary_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x,
       const uint32_t d_tmem = tmem_base + C::D_COL;
       for (int j = 0; j < nk; ++j) {
         const int s = j % C::STAGES, a = j % C::A_STAGES;
+        // aready implies full[s] already completed (the unpack warps waited
+        // on it); the MMA thread still observes full[s] itself so the copy
+        // engine's writes are ordered before its own tensor-core reads.
         if (!mbar_wait_bounded(&aready[a], static_cast<uint32_t>(j / C::A_STAGES) & 1u,
                                abort_flag, limit) ||
             !mbar_wait_bounded(&full[s], static_cast<uint32_t>(j / C::STAGES) & 1u, abort_flag,
@@ -267,8 +281,7 @@ ternary_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x,
           tc_mma_i8_ts(d_tmem, a_tmem + 8u * kk,
                        umma_desc_sw128_kmajor(b_base + (kk >> 2) * C::X_ATOM + 32 * (kk & 3)),
                        idesc, (j > 0 || kk > 0) ? 1u : 0u);
-        tc_commit(&empty[s]);
-        tc_commit(&afree[a]);
+        tc_commit(&done[s]);
       }
       // Signals the epilogue; on an abort it still marks that every MMA
       // issued so far has finished with TMEM and shared memory.
@@ -284,10 +297,12 @@ ternary_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x,
     const uint32_t lane_addr = static_cast<uint32_t>(32 * q) << 16;
     for (int j = 0; j < nk; ++j) {
       const int s = j % C::STAGES, a = j % C::A_STAGES;
+      // A stage a was last used by step j - A_STAGES; its MMAs completed when
+      // done[] of that step's shared-memory stage did.
+      const int jp = j - C::A_STAGES;
       if (!warp_wait(&full[s], static_cast<uint32_t>(j / C::STAGES) & 1u, abort_flag, limit) ||
-          (j >= C::A_STAGES &&
-           !warp_wait(&afree[a], static_cast<uint32_t>(j / C::A_STAGES - 1) & 1u, abort_flag,
-                      limit))) {
+          (jp >= 0 && !warp_wait(&done[jp % C::STAGES],
+                                 static_cast<uint32_t>(jp / C::STAGES) & 1u, abort_flag, limit))) {
         gemm_fail(abort_flag, p.status, DEV_TIMEOUT_UNPACK);
         break;
       }
@@ -296,15 +311,12 @@ ternary_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x,
       uint4 pk[NV];
 #pragma unroll
       for (int t = 0; t < NV; ++t) {
-        // The copy engine wrote the tile swizzled (128-byte rows: chunk ^ row%8;
-        // 32-byte rows: chunk ^ (row/4)%2) so a warp's 32 rows hit distinct banks.
+        // The copy engine wrote the tile swizzled (64-byte rows: chunk ^
+        // (row/2)%4) so a warp's 32 rows hit distinct banks.
         const int c = (C::PART / 16) * h + t;
-        const int pc = C::WP_ROW == 128 ? (c ^ (i & 7)) : (c ^ ((i >> 2) & 1));
+        const int pc = c ^ ((i >> 1) & 3);
         pk[t] = *reinterpret_cast<const uint4*>(wps + s * C::WP_BYTES + i * C::WP_ROW + 16 * pc);
       }
-      // The packed bytes are in registers: release the shared-memory stage.
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&empty[s]);
       const uint32_t col = tmem_base + lane_addr + C::A_COL + static_cast<uint32_t>(C::A_COLS) * a +
                            static_cast<uint32_t>(C::PART) * h;
 #pragma unroll
