@@ -12,6 +12,7 @@
 #include <algorithm>
 #include <cstdint>
 #include <mutex>
+#include <vector>
 
 #include "act_quant.cuh"
 #include "common.cuh"
@@ -45,6 +46,7 @@ struct DeviceState {
   bool ok = false;
   int* status = nullptr;  // device address of g_device_status
   int num_sms = 148;
+  int gemv_occ[2] = {1, 1};  // resident decode-GEMV CTAs per SM (1 / 2 token tiles)
 };
 DeviceState g_dev[kMaxDevices];
 
@@ -65,7 +67,13 @@ DeviceState* device_state() {
               cudaSuccess;
     ok = ok && cudaDeviceGetAttribute(&st.num_sms, cudaDevAttrMultiProcessorCount, dev) ==
                    cudaSuccess;
-    ok = ok && set_smem(ternary_gemv_kernel, gemv_smem_bytes(16));
+    for (int nt = 0; nt < 2 && ok; ++nt) {
+      int occ = 0;
+      ok = cudaOccupancyMaxActiveBlocksPerMultiprocessor(
+               &occ, nt ? ternary_gemv_kernel<2> : ternary_gemv_kernel<1>, kGemvThreads, 0) ==
+           cudaSuccess;
+      st.gemv_occ[nt] = std::max(1, occ);
+    }
     ok = ok && set_smem(ternary_gemm_tc_kernel<16>, GemmCfg<16>::SMEM_DYN);
     ok = ok && set_smem(ternary_gemm_tc_kernel<32>, GemmCfg<32>::SMEM_DYN);
     ok = ok && set_smem(ternary_gemm_tc_kernel<64>, GemmCfg<64>::SMEM_DYN);
@@ -152,38 +160,114 @@ bool ok_dtype(int d) { return d == BITNET_F32 || d == BITNET_BF16; }
 
 // ------------------------------------------------------------ launchers
 
-struct GemvPlan {
-  int rb, ksplit, steps, blocks;
-};
+// ------------------------------------------------------------ decode GEMV
 
-// Row blocks of 64 weight rows streaming K in 512-k steps.  K is split
-// across CTAs only when the whole launch has fewer row blocks than two per
-// SM (then the int32 partials go through the workspace).
-GemvPlan plan_gemv(int64_t N, int64_t K, int num_sms, int64_t launch_row_blocks = 0) {
-  GemvPlan pl{};
-  pl.rb = static_cast<int>((N + kGemvRows - 1) / kGemvRows);
-  const int total = static_cast<int>((K + kGemvKStep - 1) / kGemvKStep);
-  const int64_t lrb = launch_row_blocks > 0 ? launch_row_blocks : pl.rb;
-  int ks = 1;
-  if (lrb < 2 * num_sms)
-    ks = std::max(1, std::min(total, static_cast<int>((2 * num_sms + lrb - 1) / lrb)));
-  pl.steps = (total + ks - 1) / ks;
-  pl.ksplit = (total + pl.steps - 1) / pl.steps;
-  pl.blocks = pl.rb * pl.ksplit;
-  return pl;
+// Work a stream-K launch loses to its cross-CTA finish (partials through
+// the workspace, a fence, a counter, a read-back), in 4 KiB units per CTA.
+constexpr long long kGemvSplitPenaltyUnits = 24;
+
+// Deal whole row blocks, largest first, to the least-loaded CTA (at most
+// kGemvMaxSegs each).  Returns the largest CTA load in units, or -1 when
+// the launch does not fit the explicit list.
+long long plan_gemv_listed(GemvLaunch& L, long long G) {
+  int total = 0;
+  for (int i = 0; i < L.count; ++i) total += L.prob[i].rb;
+  if (total > kGemvMaxTasks || G > kGemvMaxCtas || G < 1) return -1;
+  // Problems by decreasing row-block size.
+  int order[kGemvMaxGroup];
+  for (int i = 0; i < L.count; ++i) order[i] = i;
+  std::sort(order, order + L.count,
+            [&L](int a, int b) { return L.prob[a].kc > L.prob[b].kc; });
+  // Min-heap of (load, cta).
+  std::vector<std::pair<long long, int>> heap;
+  heap.reserve(static_cast<size_t>(G));
+  for (int c = 0; c < G; ++c) heap.emplace_back(0LL, c);
+  std::vector<std::vector<uint16_t>> lists(static_cast<size_t>(G));
+  auto cmp = [](const std::pair<long long, int>& a, const std::pair<long long, int>& b) {
+    return a.first != b.first ? a.first > b.first : a.second > b.second;
+  };
+  std::make_heap(heap.begin(), heap.end(), cmp);
+  long long worst = 0;
+  for (int oi = 0; oi < L.count; ++oi) {
+    const GemvProblem& P = L.prob[order[oi]];
+    for (int r = 0; r < P.rb; ++r) {
+      if (heap.empty()) return -1;
+      std::pop_heap(heap.begin(), heap.end(), cmp);
+      auto top = heap.back();
+      heap.pop_back();
+      lists[static_cast<size_t>(top.second)].push_back(static_cast<uint16_t>(P.rb_begin + r));
+      top.first += P.kc;
+      worst = std::max(worst, top.first);
+      if (lists[static_cast<size_t>(top.second)].size() < static_cast<size_t>(kGemvMaxSegs)) {
+        heap.push_back(top);
+        std::push_heap(heap.begin(), heap.end(), cmp);
+      }
+    }
+  }
+  int pos = 0;
+  for (long long c = 0; c < G; ++c) {
+    L.cta_begin[c] = static_cast<uint16_t>(pos);
+    auto& v = lists[static_cast<size_t>(c)];
+    std::sort(v.begin(), v.end());
+    for (uint16_t r : v) L.task[pos++] = r;
+  }
+  L.cta_begin[G] = static_cast<uint16_t>(pos);
+  return worst;
 }
 
-bool fill_gemv_problem(GemvProblem& q, const GemvPlan& pl, const uint8_t* Wp, uint8_t* ws,
-                       const FwdWorkspace& L, const float* s_x, const float* s_w, int64_t M,
-                       int64_t N, int64_t K, int mt, void* y, int y_dtype, int32_t* acc_out,
-                       int block_begin) {
-  if (!make_tmap_u8(&q.tmap_w, Wp, static_cast<uint64_t>(K / 4), static_cast<uint64_t>(N),
-                    static_cast<uint64_t>(K / 4), 128, kGemvRows, CU_TENSOR_MAP_SWIZZLE_128B))
-    return false;
-  if (!make_tmap_u8(&q.tmap_x, ws + L.xq, static_cast<uint64_t>(K), static_cast<uint64_t>(M),
-                    static_cast<uint64_t>(K), 128, static_cast<uint32_t>(mt),
-                    CU_TENSOR_MAP_SWIZZLE_128B))
-    return false;
+// Shape fields of prob[0..count) must be set.  Lays the problems' units end
+// to end and returns the CTA count.  Whole row blocks per CTA when that
+// balances within the cost of splitting; otherwise stream-K: one CTA per 8
+// units (a unit per warp) up to the resident capacity, and enough CTAs that
+// no CTA's share touches more than kGemvMaxSegs row blocks.
+long long plan_gemv_launch(GemvLaunch& L, long long capacity) {
+  long long U = 0;
+  int rbs = 0, kc_min = 1 << 30;
+  for (int i = 0; i < L.count; ++i) {
+    GemvProblem& P = L.prob[i];
+    P.rb = (P.N + kGemvRows - 1) / kGemvRows;
+    P.kc = (P.K + kGemvUnitK - 1) / kGemvUnitK;
+    P.unit_begin = U;
+    P.rb_begin = rbs;
+    U += static_cast<long long>(P.rb) * P.kc;
+    rbs += P.rb;
+    kc_min = std::min(kc_min, P.kc);
+  }
+  L.units = U;
+  long long G = std::min((U + kGemvWarps - 1) / kGemvWarps, std::max(1LL, capacity));
+  // A share of n <= (kGemvMaxSegs - 1) * kc_min units touches at most
+  // kGemvMaxSegs row blocks.
+  const long long per = static_cast<long long>(kGemvMaxSegs - 1) * kc_min;
+  G = std::max(G, (U + per - 1) / per);
+  G = std::max(1LL, std::min(G, U));
+  const long long split_cost = (U + G - 1) / G + kGemvSplitPenaltyUnits;
+  const long long Gl = std::min<long long>(std::max(1LL, capacity), rbs);
+  const long long listed_cost = plan_gemv_listed(L, Gl);
+  if (listed_cost >= 0 && listed_cost <= split_cost) {
+    L.listed = 1;
+    return Gl;
+  }
+  L.listed = 0;
+  return G;
+}
+
+// Whether a CTA boundary of a G-CTA launch falls inside a row block of
+// problem i (its partials then go through the workspace, which must start
+// at zero).
+bool gemv_problem_shared(const GemvLaunch& L, int i, long long G) {
+  if (L.listed) return false;
+  const GemvProblem& P = L.prob[i];
+  const long long U = L.units, lo = P.unit_begin, hi = lo + static_cast<long long>(P.rb) * P.kc;
+  for (long long b = gemv_cta_of(lo, U, G) + 1; b <= gemv_cta_of(hi - 1, U, G); ++b)
+    if ((b * U / G - lo) % P.kc != 0) return true;
+  return false;
+}
+
+void fill_gemv_problem(GemvProblem& q, const uint8_t* Wp, uint8_t* ws, const FwdWorkspace& L,
+                       const float* s_x, const float* s_w, int64_t M, int64_t N, int64_t K,
+                       void* y, int y_dtype, int32_t* acc_out) {
+  q.W = Wp;
+  q.xq = reinterpret_cast<const int8_t*>(ws + L.xq);
   q.rowsum = reinterpret_cast<const int32_t*>(ws + L.rs);
   q.s_x = s_x;
   q.s_w = s_w;
@@ -195,45 +279,61 @@ bool fill_gemv_problem(GemvProblem& q, const GemvPlan& pl, const uint8_t* Wp, ui
   q.N = static_cast<int>(N);
   q.K = static_cast<int>(K);
   q.y_bf16 = (y_dtype == BITNET_BF16) ? 1 : 0;
-  q.rb = pl.rb;
-  q.ksplit = pl.ksplit;
-  q.steps = pl.steps;
-  q.block_begin = block_begin;
-  return true;
 }
 
-bitnet_status launch_gemv_group(const DeviceState& ds, GemvLaunch& L, int blocks, bool pdl,
+// Token tiles of a launch: two n8 tiles when any problem has more than 8.
+int gemv_tiles(const GemvLaunch& L) {
+  for (int i = 0; i < L.count; ++i)
+    if (L.prob[i].M > 8) return 2;
+  return 1;
+}
+
+// Bytes of whole row blocks each CTA asks the copy engine to stream into L2
+// at entry (the launch total stays well inside the 126 MB L2).
+constexpr unsigned kGemvPrefetchBytes = 256u << 10;
+
+bitnet_status launch_gemv_group(const DeviceState& ds, GemvLaunch& L, long long G, bool pdl,
                                 bool early_weights, cudaStream_t stream) {
   L.use_pdl = pdl ? 1 : 0;
   L.early_weights = (pdl && early_weights) ? 1 : 0;
-  L.status = ds.status;
-  L.wait_limit_ns = kWaitLimitNs;
+  L.prefetch_bytes = kGemvPrefetchBytes;
   cudaLaunchConfig_t cfg{};
-  cfg.gridDim = dim3(static_cast<unsigned>(blocks), 1, 1);
+  cfg.gridDim = dim3(static_cast<unsigned>(G), 1, 1);
   cfg.blockDim = dim3(kGemvThreads, 1, 1);
-  cfg.dynamicSmemBytes = gemv_smem_bytes(L.mt);
+  cfg.dynamicSmemBytes = 0;
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = pdl ? 1 : 0;
-  return cudaLaunchKernelEx(&cfg, ternary_gemv_kernel, L) == cudaSuccess ? BITNET_OK
-                                                                         : BITNET_ERR_CUDA;
+  const cudaError_t e = gemv_tiles(L) == 2 ? cudaLaunchKernelEx(&cfg, ternary_gemv_kernel<2>, L)
+                                           : cudaLaunchKernelEx(&cfg, ternary_gemv_kernel<1>, L);
+  return e == cudaSuccess ? BITNET_OK : BITNET_ERR_CUDA;
+}
+
+long long gemv_capacity(const DeviceState& ds, int M) {
+  return static_cast<long long>(ds.num_sms) * (M > 8 ? ds.gemv_occ[1] : ds.gemv_occ[0]);
+}
+
+// One problem: its plan (count = 1) in *L.
+long long plan_gemv_single(const DeviceState& ds, GemvLaunch& L, int64_t M, int64_t N,
+                           int64_t K) {
+  L.count = 1;
+  L.prob[0].M = static_cast<int>(M);
+  L.prob[0].N = static_cast<int>(N);
+  L.prob[0].K = static_cast<int>(K);
+  return plan_gemv_launch(L, gemv_capacity(ds, static_cast<int>(M)));
 }
 
 bitnet_status launch_gemv(const DeviceState& ds, const uint8_t* Wp, const float* s_x,
                           const float* s_w, int64_t M, int64_t N, int64_t K, uint8_t* ws,
                           const FwdWorkspace& Lw, void* y, int y_dtype, int32_t* acc_out,
                           bool pdl, bool early_weights, cudaStream_t stream) {
-  const GemvPlan pl = plan_gemv(N, K, ds.num_sms);
-  static thread_local GemvLaunch L;  // ~6 KB: keep it off the stack
-  L.count = 1;
-  L.mt = M <= 8 ? 8 : 16;
-  if (!fill_gemv_problem(L.prob[0], pl, Wp, ws, Lw, s_x, s_w, M, N, K, L.mt, y, y_dtype, acc_out,
-                         0))
-    return BITNET_ERR_CUDA;
-  return launch_gemv_group(ds, L, pl.blocks, pdl, early_weights, stream);
+  static thread_local GemvLaunch L;  // ~2 KB: keep it off the stack
+  fill_gemv_problem(L.prob[0], Wp, ws, Lw, s_x, s_w, M, N, K, y, y_dtype, acc_out);
+  const long long G = plan_gemv_single(ds, L, M, N, K);
+  return launch_gemv_group(ds, L, G, pdl, early_weights, stream);
 }
 
 struct GemmPlan {
@@ -327,7 +427,11 @@ bitnet_status launch_gemm(const DeviceState& ds, const uint8_t* Wp, const int8_t
 // in the workspace (which must then start at zero).
 bool needs_zeroed_partials(const DeviceState& ds, int path, int64_t M, int64_t N, int64_t K) {
   if (M > kGemvMaxM) return false;
-  if (path == BITNET_PATH_GEMV) return plan_gemv(N, K, ds.num_sms).ksplit > 1;
+  if (path == BITNET_PATH_GEMV) {
+    static thread_local GemvLaunch L;
+    const long long G = plan_gemv_single(ds, L, M, N, K);
+    return gemv_problem_shared(L, 0, G);
+  }
   return plan_gemm(M, N, K, ds.num_sms).ksplit > 1;
 }
 
@@ -497,16 +601,23 @@ bitnet_status forward_grouped_impl(int count, const bitnet_linear_problem* probl
   static thread_local GemvLaunch GL;
   QL = QuantLaunch{};
   GL.count = 0;
-  int qblocks = 0, gblocks = 0, n = 0;
-  int64_t launch_rb = 0;
-  int mt = 8;
+  // First pass: the matmul plan (it decides which partial regions need
+  // zeroing by the quant launch).
+  int n = 0, mmax = 0;
   for (int i = 0; i < count; ++i) {
     const bitnet_linear_problem& q = problems[i];
     if (q.M == 0 || q.M > kGemvMaxM) continue;
-    launch_rb += (q.N + kGemvRows - 1) / kGemvRows;
-    if (q.M > 8) mt = 16;
+    GL.prob[n].M = static_cast<int>(q.M);
+    GL.prob[n].N = static_cast<int>(q.N);
+    GL.prob[n].K = static_cast<int>(q.K);
+    mmax = std::max(mmax, static_cast<int>(q.M));
+    ++n;
   }
+  GL.count = n;
+  const long long G = n > 0 ? plan_gemv_launch(GL, gemv_capacity(*ds, mmax)) : 0;
+  int qblocks = 0;
   size_t off = 0;
+  n = 0;
   for (int i = 0; i < count; ++i) {
     const bitnet_linear_problem& q = problems[i];
     if (q.M == 0) continue;
@@ -514,9 +625,8 @@ bitnet_status forward_grouped_impl(int count, const bitnet_linear_problem* probl
     uint8_t* ws = base + off;
     off += L.total;
     if (q.M > kGemvMaxM) continue;
-    const GemvPlan pl = plan_gemv(q.N, q.K, ds->num_sms, launch_rb);
     size_t zbytes = 0;
-    void* zero = pl.ksplit > 1 ? splitk_region(ws, L, &zbytes) : nullptr;
+    void* zero = gemv_problem_shared(GL, n, G) ? splitk_region(ws, L, &zbytes) : nullptr;
     QuantProblem& qp = QL.prob[n];
     qp.x = q.x;
     qp.gamma = q.gamma;
@@ -532,17 +642,13 @@ bitnet_status forward_grouped_impl(int count, const bitnet_linear_problem* probl
     qp.block_begin = qblocks;
     qp.zero_blocks = static_cast<int>(zero ? zero_blocks(zbytes) : 0);
     qblocks += qp.M + qp.zero_blocks;
-    if (!fill_gemv_problem(GL.prob[n], pl, q.W_packed, ws, L, qp.s_x, q.s_w, q.M, q.N, q.K, mt,
-                           q.y, q.y_dtype, nullptr, gblocks))
-      return BITNET_ERR_CUDA;
-    gblocks += pl.blocks;
+    fill_gemv_problem(GL.prob[n], q.W_packed, ws, L, qp.s_x, q.s_w, q.M, q.N, q.K, q.y,
+                      q.y_dtype, nullptr);
     ++n;
   }
   if (n > 0) {
     QL.count = n;
     QL.trigger_dependents = do_matmul ? 1 : 0;
-    GL.count = n;
-    GL.mt = mt;
     if (do_quant) {
       int cache = 1;  // 0 = some bf16 row is too long to hold in registers
       for (int i = 0; i < n; ++i) {
@@ -564,8 +670,8 @@ bitnet_status forward_grouped_impl(int count, const bitnet_linear_problem* probl
     }
     if (do_matmul) {
       // When the quant grid was just queued it started after every earlier
-      // write to the weights, so the copies may begin before waiting on it.
-      const bitnet_status st = launch_gemv_group(*ds, GL, gblocks, true, do_quant, stream);
+      // write to the weights, so the loads may begin before waiting on it.
+      const bitnet_status st = launch_gemv_group(*ds, GL, G, true, do_quant, stream);
       if (st != BITNET_OK) return st;
     }
   }

@@ -207,6 +207,8 @@ RAGGED = [
     (1, 1, 64), (2, 33, 64), (3, 100, 192), (5, 31, 320), (7, 129, 1088), (9, 257, 8640),
     (16, 1000, 3200), (17, 130, 256), (63, 127, 576), (65, 255, 1216), (129, 300, 704),
     (200, 1, 128), (300, 520, 8640),
+    # few rows, long K: the decode matmul splits row blocks across CTAs
+    (1, 64, 16384), (4, 100, 20480), (13, 130, 32768),
 ]
 
 
