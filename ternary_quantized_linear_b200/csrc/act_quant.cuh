@@ -289,34 +289,144 @@ __device__ __forceinline__ void quant_row(const void* __restrict__ x,
   }
 }
 
-// Chunks per thread held in registers: the launch picks the smallest of
-// 1, 2, 4, 8, 16 that covers the row (bf16 rows up to 32 Ki elements; fp32
-// rows up to 4, i.e. K <= 8192), so the executed path stays short -- these
-// kernels run on few SMs with cold instruction caches.  Longer rows re-read.
-__host__ __device__ constexpr int quant_cache_for(int64_t K, bool bf16) {
-  const int64_t per = (K / 8 + kActThreads - 1) / kActThreads;
-  const int64_t cap = bf16 ? 16 : 4;
-  if (per > cap) return 0;
-  return per <= 1 ? 1 : (per <= 2 ? 2 : (per <= 4 ? 4 : (per <= 8 ? 8 : 16)));
+// Shared-memory bytes to stage a row (and gamma) of K elements; rows above
+// kQuantStageMax take the re-reading path instead.
+constexpr uint32_t kQuantStageMax = 160u << 10;
+__host__ __device__ constexpr uint32_t quant_stage_bytes(int64_t K, bool bf16, bool gamma) {
+  return static_cast<uint32_t>(K * ((bf16 ? 2 : 4) + (gamma ? 4 : 0)));
+}
+
+// RMSNorm + absmax quantization of row m, staged: one thread brings the row
+// (and gamma) into shared memory with bulk asynchronous copies, then three
+// short loops read it there.  The executed code stays small, which matters:
+// each row's CTA usually runs alone on an SM with a cold instruction cache.
+// Same arithmetic and reduction order as quant_row.  Returns false (nothing
+// written) when the copy did not land within the wait limit.
+template <bool kBF16, bool kInterleave>
+__device__ bool quant_row_staged(const void* __restrict__ x, const float* __restrict__ gamma,
+                                 float eps, int64_t m, int64_t K, int8_t* __restrict__ x_q,
+                                 float* __restrict__ s_x, int32_t* __restrict__ rowsum,
+                                 float* redf, int* redi, uint8_t* stage, uint64_t* bar,
+                                 uint64_t wait_limit_ns) {
+  constexpr int ES = kBF16 ? 2 : 4;
+  const int tid = threadIdx.x;
+  const uint32_t xbytes = static_cast<uint32_t>(K * ES);
+  const float* sg = reinterpret_cast<const float*>(stage + xbytes);
+  if (tid == 0) {
+    mbar_init(bar, 1);
+    fence_mbarrier_init();
+  }
+  __syncthreads();
+  if (tid == 0) {
+    mbar_arrive_expect_tx(bar, xbytes + (gamma ? static_cast<uint32_t>(K * 4) : 0u));
+    bulk_load(stage, static_cast<const uint8_t*>(x) + m * K * ES, xbytes, bar);
+    if (gamma) bulk_load(stage + xbytes, gamma, static_cast<uint32_t>(K * 4), bar);
+  }
+  const bool landed = mbar_wait_bounded(bar, 0u, nullptr, wait_limit_ns);
+  if (!__syncthreads_and(landed ? 1 : 0)) return false;
+
+  const int64_t nchunk = K >> 3;
+  const int iters = static_cast<int>((nchunk + kActThreads - 1) / kActThreads);
+  auto chunk = [&](int64_t c, float (&v)[8]) {
+    RawChunk<kBF16> r;
+    const uint4* src = reinterpret_cast<const uint4*>(stage + c * 8 * ES);
+    r.w[0] = src[0];
+    if (!kBF16) r.w[kBF16 ? 0 : 1] = src[1];
+    widen8<kBF16>(r, v);
+  };
+  auto gam = [&](int64_t c, float (&g)[8]) {
+#pragma unroll
+    for (int j = 0; j < 8; ++j) g[j] = gamma ? sg[8 * c + j] : 1.0f;
+  };
+
+  // Pass 1: sum of squares, partial = this thread's chunks in increasing k.
+  float p = 0.0f;
+#pragma unroll 1
+  for (int64_t c = tid; c < nchunk; c += kActThreads) {
+    float v[8];
+    chunk(c, v);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) p = __fmaf_rn(v[j], v[j], p);
+  }
+  const float ss = block_tree_sum_f32(p, redf);
+  const float ms = __fdiv_rn(ss, static_cast<float>(K));
+  const float d = __fadd_rn(ms, eps);
+  const bool zero_row = (d == 0.0f);
+  const float r = zero_row ? 0.0f : __fdiv_rn(1.0f, __fsqrt_rn(d));
+
+  // Pass 2: max |x_n|.
+  float amax = 0.0f;
+  if (!zero_row) {
+#pragma unroll 1
+    for (int64_t c = tid; c < nchunk; c += kActThreads) {
+      float v[8], g[8];
+      chunk(c, v);
+      gam(c, g);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) amax = fmaxf(amax, fabsf(__fmul_rn(__fmul_rn(v[j], r), g[j])));
+    }
+  }
+  amax = block_max_f32(amax, redf);
+  amax = fmaxf(amax, 1e-5f);
+  const float sx = __fdiv_rn(127.0f, amax);
+
+  // Pass 3: quantize, store, row sum (every lane runs every iteration: the
+  // interleaved store exchanges bytes between lane pairs).
+  int sum = 0;
+  int8_t* xq_row = x_q + m * K;
+#pragma unroll 1
+  for (int it = 0; it < iters; ++it) {
+    const int64_t c = tid + static_cast<int64_t>(kActThreads) * it;
+    const bool valid = c < nchunk;
+    int8_t q[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+    if (valid && !zero_row) {
+      float v[8], g[8];
+      chunk(c, v);
+      gam(c, g);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        q[j] = quant_one(__fmul_rn(__fmul_rn(v[j], r), g[j]), sx);
+        sum += q[j];
+      }
+    }
+    Chunk8 ch{pack4(q[0], q[1], q[2], q[3]), pack4(q[4], q[5], q[6], q[7])};
+    store_chunk8<kInterleave>(xq_row, 8 * c, ch, valid);
+  }
+  sum = block_sum_i32(sum, redi);
+  if (tid == 0) {
+    if (s_x) s_x[m] = sx;
+    if (rowsum) rowsum[m] = sum;
+  }
+  return true;
 }
 
 // One CTA per row (blocks >= M zero `zero16` instead).  x: [M][K] (fp32 or
-// bf16 bits), gamma: [K] or null.
-template <bool kBF16, bool kInterleave, int CACHE>
+// bf16 bits), gamma: [K] or null.  STAGED: the row goes through shared
+// memory (dynamic, quant_stage_bytes); otherwise each pass re-reads it.
+template <bool kBF16, bool kInterleave, bool STAGED>
 __global__ void __launch_bounds__(kActThreads)
 rmsnorm_quant_kernel(const void* __restrict__ x, const float* __restrict__ gamma, float eps,
                      int64_t M, int64_t K, int8_t* __restrict__ x_q, float* __restrict__ s_x,
                      int32_t* __restrict__ rowsum, uint4* __restrict__ zero16, int64_t n_zero16,
-                     int trigger_dependents) {
+                     int trigger_dependents, int* status, uint64_t wait_limit_ns) {
   __shared__ float redf[kActThreads];
   __shared__ int redi[kActThreads / 32];
+  __shared__ __align__(8) uint64_t bar;
+  extern __shared__ __align__(16) uint8_t stage[];
   if (trigger_dependents) pdl_launch_dependents();
   if (static_cast<int64_t>(blockIdx.x) >= M) {
     zero_fill_blocks(zero16, n_zero16, static_cast<int64_t>(blockIdx.x) - M,
                      static_cast<int64_t>(gridDim.x) - M);
     return;
   }
-  quant_row<kBF16, kInterleave, CACHE>(x, gamma, eps, blockIdx.x, K, x_q, s_x, rowsum, redf, redi);
+  if (STAGED) {
+    if (!quant_row_staged<kBF16, kInterleave>(x, gamma, eps, blockIdx.x, K, x_q, s_x, rowsum,
+                                              redf, redi, stage, &bar, wait_limit_ns) &&
+        threadIdx.x == 0)
+      record_failure(status, DEV_TIMEOUT_QUANT);
+  } else {
+    quant_row<kBF16, kInterleave, 0>(x, gamma, eps, blockIdx.x, K, x_q, s_x, rowsum, redf, redi);
+  }
 }
 
 constexpr int kQuantMaxGroup = 16;
@@ -339,16 +449,21 @@ struct QuantProblem {
 struct QuantLaunch {
   int count;
   int trigger_dependents;
+  int* status;              // device status word (bounded waits)
+  uint64_t wait_limit_ns;
   QuantProblem prob[kQuantMaxGroup];
 };
 
 // Several independent problems in one launch: rows of every problem, then
-// each problem's zero-fill blocks, laid out by block_begin.
-template <int CACHE>
+// each problem's zero-fill blocks, laid out by block_begin.  STAGED: every
+// row of the launch fits the dynamic shared-memory stage.
+template <bool STAGED>
 __global__ void __launch_bounds__(kActThreads)
 rmsnorm_quant_grouped_kernel(const __grid_constant__ QuantLaunch L) {
   __shared__ float redf[kActThreads];
   __shared__ int redi[kActThreads / 32];
+  __shared__ __align__(8) uint64_t bar;
+  extern __shared__ __align__(16) uint8_t stage[];
   if (L.trigger_dependents) pdl_launch_dependents();
   int pi = 0;
   for (int i = 1; i < L.count; ++i)
@@ -359,13 +474,19 @@ rmsnorm_quant_grouped_kernel(const __grid_constant__ QuantLaunch L) {
     zero_fill_blocks(q.zero16, q.n_zero16, local - q.M, q.zero_blocks);
     return;
   }
-  // CACHE covers every bf16 row of the launch; fp32 rows (rare: small
-  // problems) re-read.
-  if (q.x_bf16)
-    quant_row<true, true, CACHE>(q.x, q.gamma, q.eps, local, q.K, q.xi, q.s_x, q.rowsum, redf,
-                                 redi);
-  else
+  if (STAGED) {
+    const bool ok =
+        q.x_bf16 ? quant_row_staged<true, true>(q.x, q.gamma, q.eps, local, q.K, q.xi, q.s_x,
+                                                q.rowsum, redf, redi, stage, &bar, L.wait_limit_ns)
+                 : quant_row_staged<false, true>(q.x, q.gamma, q.eps, local, q.K, q.xi, q.s_x,
+                                                 q.rowsum, redf, redi, stage, &bar,
+                                                 L.wait_limit_ns);
+    if (!ok && threadIdx.x == 0) record_failure(L.status, DEV_TIMEOUT_QUANT);
+  } else if (q.x_bf16) {
+    quant_row<true, true, 0>(q.x, q.gamma, q.eps, local, q.K, q.xi, q.s_x, q.rowsum, redf, redi);
+  } else {
     quant_row<false, true, 0>(q.x, q.gamma, q.eps, local, q.K, q.xi, q.s_x, q.rowsum, redf, redi);
+  }
 }
 
 // Natural-order x_q -> k-interleaved copy plus per-row sums (used when the

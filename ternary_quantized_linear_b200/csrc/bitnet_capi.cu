@@ -74,6 +74,11 @@ DeviceState* device_state() {
            cudaSuccess;
       st.gemv_occ[nt] = std::max(1, occ);
     }
+    ok = ok && set_smem(rmsnorm_quant_kernel<true, true, true>, kQuantStageMax);
+    ok = ok && set_smem(rmsnorm_quant_kernel<true, false, true>, kQuantStageMax);
+    ok = ok && set_smem(rmsnorm_quant_kernel<false, true, true>, kQuantStageMax);
+    ok = ok && set_smem(rmsnorm_quant_kernel<false, false, true>, kQuantStageMax);
+    ok = ok && set_smem(rmsnorm_quant_grouped_kernel<true>, kQuantStageMax);
     ok = ok && set_smem(ternary_gemm_tc_kernel<16>, GemmCfg<16>::SMEM_DYN);
     ok = ok && set_smem(ternary_gemm_tc_kernel<32>, GemmCfg<32>::SMEM_DYN);
     ok = ok && set_smem(ternary_gemm_tc_kernel<64>, GemmCfg<64>::SMEM_DYN);
@@ -453,24 +458,27 @@ bitnet_status launch_act_quant(const void* x, int x_dtype, const float* gamma, f
   const int trig = trigger ? 1 : 0;
   uint4* z = static_cast<uint4*>(zero);
   const int64_t n16 = zero ? static_cast<int64_t>(zero_bytes / 16) : 0;
-#define BITNET_QUANT(BF, IL, C)                                                        \
-  rmsnorm_quant_kernel<BF, IL, C><<<grid, block, 0, stream>>>(x, gamma, eps, M, K, x_q, s_x, \
-                                                              rowsum, z, n16, trig)
-#define BITNET_QUANT_C(BF, IL)                                    \
-  switch (quant_cache_for(K, BF)) {                               \
-    case 1: BITNET_QUANT(BF, IL, 1); break;                       \
-    case 2: BITNET_QUANT(BF, IL, 2); break;                       \
-    case 4: BITNET_QUANT(BF, IL, 4); break;                       \
-    case 8: BITNET_QUANT(BF, IL, 8); break;                       \
-    case 16: BITNET_QUANT(BF, IL, 16); break;                     \
-    default: BITNET_QUANT(BF, IL, 0); break;                      \
-  }
-  if (x_dtype == BITNET_BF16) {
-    if (interleave) { BITNET_QUANT_C(true, true) } else { BITNET_QUANT_C(true, false) }
+  const bool bf16 = x_dtype == BITNET_BF16;
+  const uint32_t stage = quant_stage_bytes(K, bf16, gamma != nullptr);
+  const bool staged = stage <= kQuantStageMax;
+  int* status = device_state() ? device_state()->status : nullptr;
+  const size_t dyn = staged ? stage : 0;
+#define BITNET_QUANT(BF, IL, ST)                                                             \
+  rmsnorm_quant_kernel<BF, IL, ST><<<grid, block, dyn, stream>>>(                           \
+      x, gamma, eps, M, K, x_q, s_x, rowsum, z, n16, trig, status, kWaitLimitNs)
+  if (bf16) {
+    if (interleave) {
+      if (staged) BITNET_QUANT(true, true, true); else BITNET_QUANT(true, true, false);
+    } else {
+      if (staged) BITNET_QUANT(true, false, true); else BITNET_QUANT(true, false, false);
+    }
   } else {
-    if (interleave) { BITNET_QUANT_C(false, true) } else { BITNET_QUANT_C(false, false) }
+    if (interleave) {
+      if (staged) BITNET_QUANT(false, true, true); else BITNET_QUANT(false, true, false);
+    } else {
+      if (staged) BITNET_QUANT(false, false, true); else BITNET_QUANT(false, false, false);
+    }
   }
-#undef BITNET_QUANT_C
 #undef BITNET_QUANT
   return launch_status();
 }
@@ -650,21 +658,17 @@ bitnet_status forward_grouped_impl(int count, const bitnet_linear_problem* probl
     QL.count = n;
     QL.trigger_dependents = do_matmul ? 1 : 0;
     if (do_quant) {
-      int cache = 1;  // 0 = some bf16 row is too long to hold in registers
-      for (int i = 0; i < n; ++i) {
-        if (!QL.prob[i].x_bf16) continue;
-        const int c = quant_cache_for(QL.prob[i].K, true);
-        cache = (c == 0 || cache == 0) ? 0 : std::max(cache, c);
-      }
+      uint32_t stage = 0;
+      for (int i = 0; i < n; ++i)
+        stage = std::max(stage, quant_stage_bytes(QL.prob[i].K, QL.prob[i].x_bf16 != 0,
+                                                  QL.prob[i].gamma != nullptr));
+      QL.status = ds->status;
+      QL.wait_limit_ns = kWaitLimitNs;
       const dim3 qg(static_cast<unsigned>(qblocks));
-      switch (cache) {
-        case 1: rmsnorm_quant_grouped_kernel<1><<<qg, kActThreads, 0, stream>>>(QL); break;
-        case 2: rmsnorm_quant_grouped_kernel<2><<<qg, kActThreads, 0, stream>>>(QL); break;
-        case 4: rmsnorm_quant_grouped_kernel<4><<<qg, kActThreads, 0, stream>>>(QL); break;
-        case 8: rmsnorm_quant_grouped_kernel<8><<<qg, kActThreads, 0, stream>>>(QL); break;
-        case 16: rmsnorm_quant_grouped_kernel<16><<<qg, kActThreads, 0, stream>>>(QL); break;
-        default: rmsnorm_quant_grouped_kernel<0><<<qg, kActThreads, 0, stream>>>(QL); break;
-      }
+      if (stage <= kQuantStageMax)
+        rmsnorm_quant_grouped_kernel<true><<<qg, kActThreads, stage, stream>>>(QL);
+      else
+        rmsnorm_quant_grouped_kernel<false><<<qg, kActThreads, 0, stream>>>(QL);
       const bitnet_status st = launch_status();
       if (st != BITNET_OK) return st;
     }

@@ -20,6 +20,7 @@ enum DeviceDetail : int {
   DEV_TIMEOUT_DRAIN = 5,
   DEV_TIMEOUT_SELFTEST = 6,
   DEV_TIMEOUT_GEMV = 7,
+  DEV_TIMEOUT_QUANT = 8,  // activation-quant row copy
 };
 
 // Default limit of one on-chip wait (nanoseconds of %globaltimer).  Real
@@ -254,6 +255,16 @@ __device__ __forceinline__ uint4 ldg_stream_u4(const void* p) {
 // use; the copy engine does it asynchronously and nothing waits on it.
 __device__ __forceinline__ void prefetch_l2_bulk(const void* p, uint32_t bytes) {
   asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
+}
+
+// 16-byte load through L1 without a compiler memory barrier: for data that
+// nothing in this kernel writes (after the wait on the preceding grid).
+__device__ __forceinline__ uint4 ldg_u4_ro(const void* p) {
+  uint4 v;
+  asm volatile("ld.global.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p));
+  return v;
 }
 
 // 16-byte load through L1 (data written by the preceding grid: not the

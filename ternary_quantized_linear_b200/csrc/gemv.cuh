@@ -14,8 +14,8 @@
 //     one) in one of two ways: whole row blocks dealt out greedily, largest
 //     first, to the least-loaded CTA (no cross-CTA reduction at all), or,
 //     when that balances badly, every CTA an equal contiguous share of the
-//     units laid end to end ("stream-K").  Warp w of a CTA takes units w,
-//     w+8, ... of its segment list.
+//     units laid end to end ("stream-K").  The units of a CTA's segment list
+//     are split into eight equal contiguous ranges, one per warp.
 //   * No shared-memory staging.  Lane (4g + t) loads 16 bytes (64 k) of rows
 //     g and g+8 of each of the unit's four 16-row groups straight into
 //     registers (eight 16-byte loads, every 32-byte sector used) and the
@@ -58,6 +58,12 @@ constexpr int kGemvThreads = 32 * kGemvWarps;
 constexpr int kGemvMaxSegs = 8;      // row blocks one CTA's share may touch
 constexpr int kGemvMaxGroup = 16;    // problems per grouped launch
 constexpr uint32_t kCodeMask = 0x03030303u;
+// Two register buffers per warp (next unit's loads in flight during the
+// MMAs, one CTA per SM), or one buffer and two CTAs per SM.
+#ifndef BITNET_GEMV_DOUBLE_BUFFER
+#define BITNET_GEMV_DOUBLE_BUFFER 1
+#endif
+constexpr bool kGemvDoubleBuffer = BITNET_GEMV_DOUBLE_BUFFER != 0;
 
 struct GemvProblem {
   const uint8_t* W;       // W_packed [N][K/4]
@@ -122,19 +128,22 @@ __device__ __forceinline__ GemvUnit gemv_unit(const GemvProblem* prob, int count
   return r;
 }
 
+// Weight load of any unit.  No lane branches around its loads: rows past N
+// read row N-1 (their outputs are never written) and a segment past K reads
+// k = 0 (its activations are zeroed in gemv_load_x, so it adds nothing).
 template <int NT>
 __device__ __forceinline__ void gemv_load_w(GemvBuf<NT>& b, const GemvProblem& P, int rbl, int c,
                                             int g, int t) {
   const int kseg = c * kGemvUnitK + 64 * t;
-  const bool kval = kseg < P.K;  // K % 64 == 0: a segment is all in or all out
+  const int kk = kseg < P.K ? kseg : 0;  // K % 64 == 0: a segment is all in or all out
   const size_t rowb = static_cast<size_t>(P.K) / 4;
   const int r = rbl * kGemvRows + g;
-  const uint8_t* base = P.W + static_cast<size_t>(r) * rowb + kseg / 4;
-  const uint4 z = make_uint4(0u, 0u, 0u, 0u);
+  const uint8_t* base = P.W + kk / 4;
 #pragma unroll
   for (int rg = 0; rg < 4; ++rg) {
-    b.wa[rg] = (kval && r + 16 * rg < P.N) ? ldg_stream_u4(base + (16 * rg) * rowb) : z;
-    b.wb[rg] = (kval && r + 16 * rg + 8 < P.N) ? ldg_stream_u4(base + (16 * rg + 8) * rowb) : z;
+    const int ra = min(r + 16 * rg, P.N - 1), rb = min(r + 16 * rg + 8, P.N - 1);
+    b.wa[rg] = ldg_stream_u4(base + static_cast<size_t>(ra) * rowb);
+    b.wb[rg] = ldg_stream_u4(base + static_cast<size_t>(rb) * rowb);
   }
 }
 
@@ -151,18 +160,24 @@ __device__ __forceinline__ void gemv_load_w_full(GemvBuf<NT>& b, const uint8_t* 
   }
 }
 
+// Activation load: token 8 nt + g, this lane's 64 k.  Tokens past M read
+// token M-1 (their output columns are never written); a segment past K
+// reads zeros.  No lane branches around the loads.
 template <int NT>
 __device__ __forceinline__ void gemv_load_x(GemvBuf<NT>& b, const GemvProblem& P, int c, int g,
                                             int t) {
   const int kseg = c * kGemvUnitK + 64 * t;
   const bool kval = kseg < P.K;
-  const uint4 z = make_uint4(0u, 0u, 0u, 0u);
+  const int kk = kval ? kseg : 0;
 #pragma unroll
   for (int nt = 0; nt < NT; ++nt) {
-    const int m = 8 * nt + g;
-    const int8_t* px = P.xq + static_cast<size_t>(m) * P.K + kseg;
+    const int m = min(8 * nt + g, P.M - 1);
+    const int8_t* px = P.xq + static_cast<size_t>(m) * P.K + kk;
 #pragma unroll
-    for (int q = 0; q < 4; ++q) b.x[nt][q] = (kval && m < P.M) ? ldg_u4(px + 16 * q) : z;
+    for (int q = 0; q < 4; ++q) {
+      const uint4 v = ldg_u4_ro(px + 16 * q);
+      b.x[nt][q] = kval ? v : make_uint4(0u, 0u, 0u, 0u);
+    }
   }
 }
 
@@ -221,13 +236,13 @@ __device__ __forceinline__ void gemv_mma_unit(int (&acc)[4][NT][4], int (&acc16)
 }
 
 // Add a warp's accumulators into the row block's shared sums and clear them.
-template <int NT>
+template <int NT, int TILES>
 __device__ __forceinline__ void gemv_flush(int (&acc)[4][NT][4], int (&acc16)[4][NT][4], int* red,
                                            int M, int g, int t) {
 #pragma unroll
   for (int rg = 0; rg < 4; ++rg) {
 #pragma unroll
-    for (int nt = 0; nt < NT; ++nt) {
+    for (int nt = 0; nt < TILES; ++nt) {
       const int r0 = 16 * rg + g, c0 = 8 * nt + 2 * t;
       int v[4];
 #pragma unroll
@@ -266,7 +281,7 @@ __host__ __device__ __forceinline__ long long gemv_cta_of(long long u, long long
 }
 
 template <int NT>
-__global__ void __launch_bounds__(kGemvThreads, 1)
+__global__ void __launch_bounds__(kGemvThreads, kGemvDoubleBuffer ? 1 : 2)
 ternary_gemv_kernel(const __grid_constant__ GemvLaunch L) {
   __shared__ int red[kGemvMaxSegs * kGemvRows * 16];  // [segment][row][token]
   // The problem table and this CTA's segments live in shared memory: the
@@ -360,18 +375,29 @@ ternary_gemv_kernel(const __grid_constant__ GemvLaunch L) {
     gemv_load_x(buf, prob[seg_p[x.s]], seg_lo[x.s] + x.off, g, t);
   };
 
+  // Warp w takes the w-th of eight equal contiguous ranges of the CTA's units
+  // (in segment order): it touches one or two segments, and its loads walk
+  // along the rows.
+  int n_units = 0;
+  for (int i = 0; i < nseg; ++i) n_units += seg_n[i];
+  const int u_begin = warp * n_units / kGemvWarps;
+  const int u_count = (warp + 1) * n_units / kGemvWarps - u_begin;
+
   // Before the activations exist: the weights of this warp's first two
   // units go to registers, and one thread asks the copy engine to stream the
   // CTA's whole row blocks (up to L.prefetch_bytes) into L2.
   GemvBuf<NT> bufA, bufB;
   Cursor xA{0, 0};
-  advance(xA, warp);
+  advance(xA, u_begin);
+  if (u_count == 0) xA.s = nseg;
+  int left = u_count;  // units of this warp not yet loaded (xA counts as loaded)
   Cursor xB = xA;
-  advance(xB, kGemvWarps);
+  if (left > 1) advance(xB, 1);
+  else xB.s = nseg;
   const bool early = L.early_weights != 0;
   if (early) {
-    if (xA.s < nseg) load_w(bufA, xA);
-    if (xB.s < nseg) load_w(bufB, xB);
+    if (u_count > 0) load_w(bufA, xA);
+    if (kGemvDoubleBuffer && u_count > 1) load_w(bufB, xB);
   }
   if (tid == 0 && L.prefetch_bytes > 0) {
     uint32_t left = L.prefetch_bytes;
@@ -382,11 +408,11 @@ ternary_gemv_kernel(const __grid_constant__ GemvLaunch L) {
   if (L.use_pdl) pdl_wait_prior_grid();
   __syncthreads();
 
-  if (xA.s < nseg) {
+  if (u_count > 0) {
     if (!early) load_w(bufA, xA);
     load_x(bufA, xA);
   }
-  bool preB = early && xB.s < nseg;  // bufB already holds the next unit's weights
+  bool preB = early && u_count > 1;  // bufB already holds the next unit's weights
   int acc[4][NT][4], acc16[4][NT][4];
 #pragma unroll
   for (int rg = 0; rg < 4; ++rg)
@@ -395,9 +421,17 @@ ternary_gemv_kernel(const __grid_constant__ GemvLaunch L) {
 #pragma unroll
       for (int j = 0; j < 4; ++j) acc[rg][nt][j] = acc16[rg][nt][j] = 0;
   int cur_seg = -1, cur_m = 0;
+  auto flush = [&]() {
+    if (cur_seg < 0) return;
+    int* dst = red + cur_seg * kGemvRows * 16;
+    if (NT == 2 && cur_m > 8)
+      gemv_flush<NT, NT>(acc, acc16, dst, cur_m, g, t);
+    else
+      gemv_flush<NT, 1>(acc, acc16, dst, cur_m, g, t);
+  };
   auto enter = [&](int seg) {
     if (seg != cur_seg) {
-      if (cur_seg >= 0) gemv_flush<NT>(acc, acc16, red + cur_seg * kGemvRows * 16, cur_m, g, t);
+      flush();
       cur_seg = seg;
       cur_m = prob[seg_p[seg]].M;
     }
@@ -410,30 +444,49 @@ ternary_gemv_kernel(const __grid_constant__ GemvLaunch L) {
       gemv_mma_unit<NT, 1>(acc, acc16, buf);
   };
 
-  while (xA.s < nseg) {
-    if (!preB) {
-      xB = xA;
-      advance(xB, kGemvWarps);
+  // left = units of this warp from xA on.
+  if (!kGemvDoubleBuffer) {
+    // One register buffer: load a unit, compute it; the other warps of the
+    // SM (two CTAs) cover the load latency.
+    bool loaded = u_count > 0;  // bufA holds xA (weights and activations)
+    while (left > 0) {
+      if (!loaded) {
+        load_w(bufA, xA);
+        load_x(bufA, xA);
+      }
+      loaded = false;
+      enter(xA.s);
+      mma(bufA);
+      if (--left > 0) advance(xA, 1);
     }
-    const bool hasB = xB.s < nseg;
+    left = 0;
+  }
+  while (left > 0) {
+    const bool hasB = left > 1;
     if (hasB) {
-      if (!preB) load_w(bufB, xB);
+      if (!preB) {
+        xB = xA;
+        advance(xB, 1);
+        load_w(bufB, xB);
+      }
       load_x(bufB, xB);
     }
     preB = false;
     enter(xA.s);
     mma(bufA);
     if (!hasB) break;
-    xA = xB;
-    advance(xA, kGemvWarps);
-    if (xA.s < nseg) {
+    const bool hasA = left > 2;
+    if (hasA) {
+      xA = xB;
+      advance(xA, 1);
       load_w(bufA, xA);
       load_x(bufA, xA);
     }
     enter(xB.s);
     mma(bufB);
+    left -= 2;
   }
-  if (cur_seg >= 0) gemv_flush<NT>(acc, acc16, red + cur_seg * kGemvRows * 16, cur_m, g, t);
+  flush();
   __syncthreads();
 
   // Finish this CTA's segments: whole row blocks straight from the shared
