@@ -21,7 +21,9 @@
 // (mask-and-shift of a 32-bit word of 16 codes yields four words holding the
 // codes with k = 4i + r for a fixed r), so integer dot products pair the same
 // k on both sides.  rowsum[m] = sum_k x_q[m,k] lets the matmul use the raw
-// codes t+1 in {0,1,2} and subtract rowsum afterwards.
+// codes t+1 in {0,1,2} and subtract rowsum afterwards.  The decode matmul
+// additionally wants its 16-byte blocks permuted inside every 256-byte span
+// (see x_block_pos) so that its shared-memory reads hit distinct banks.
 #pragma once
 
 #include "common.cuh"
@@ -51,12 +53,18 @@ struct Chunk8 {
 // (lanes l and l^1) holding the halves of a 16-element group swap four bytes
 // each so that every lane writes 8 contiguous output bytes.  All 32 lanes of
 // the warp must call this (valid or not).
+// perm: -1 keeps the block order; 0 / 1 applies x_block_pos with that
+// token parity.
 template <bool kInterleave>
-__device__ __forceinline__ void store_chunk8(int8_t* xq_row, int64_t k, Chunk8 c, bool valid) {
+__device__ __forceinline__ void store_chunk8(int8_t* xq_row, int64_t k, Chunk8 c, bool valid,
+                                             int perm = -1) {
   if (!kInterleave) {
     if (valid) *reinterpret_cast<uint2*>(xq_row + k) = make_uint2(c.lo, c.hi);
     return;
   }
+  if (perm >= 0)
+    k = (k & ~static_cast<int64_t>(255)) +
+        16 * x_block_pos(static_cast<int>((k & 255) >> 4), perm) + (k & 15);
   const int h = static_cast<int>((k >> 3) & 1);   // which half of the 16-group
   // A = bytes (q0, q4, q1, q5), B = (q2, q6, q3, q7) of this half.
   const uint32_t A = __byte_perm(c.lo, c.hi, 0x5140);
@@ -193,7 +201,7 @@ __device__ __forceinline__ void quant_row(const void* __restrict__ x,
                                           const float* __restrict__ gamma, float eps, int64_t m,
                                           int64_t K, int8_t* __restrict__ x_q,
                                           float* __restrict__ s_x, int32_t* __restrict__ rowsum,
-                                          float* redf, int* redi) {
+                                          float* redf, int* redi, bool perm = false) {
   const int tid = threadIdx.x;
   const int64_t nchunk = K >> 3;
   const int iters = static_cast<int>((nchunk + kActThreads - 1) / kActThreads);
@@ -279,7 +287,7 @@ __device__ __forceinline__ void quant_row(const void* __restrict__ x,
         }
       }
       Chunk8 ch{pack4(q[0], q[1], q[2], q[3]), pack4(q[4], q[5], q[6], q[7])};
-      store_chunk8<kInterleave>(xq_row, 8 * c, ch, valid);
+      store_chunk8<kInterleave>(xq_row, 8 * c, ch, valid, perm ? static_cast<int>(m & 1) : -1);
     }
   }
   sum = block_sum_i32(sum, redi);
@@ -307,7 +315,7 @@ __device__ bool quant_row_staged(const void* __restrict__ x, const float* __rest
                                  float eps, int64_t m, int64_t K, int8_t* __restrict__ x_q,
                                  float* __restrict__ s_x, int32_t* __restrict__ rowsum,
                                  float* redf, int* redi, uint8_t* stage, uint64_t* bar,
-                                 uint64_t wait_limit_ns) {
+                                 uint64_t wait_limit_ns, bool perm) {
   constexpr int ES = kBF16 ? 2 : 4;
   const int tid = threadIdx.x;
   const uint32_t xbytes = static_cast<uint32_t>(K * ES);
@@ -390,7 +398,7 @@ __device__ bool quant_row_staged(const void* __restrict__ x, const float* __rest
       }
     }
     Chunk8 ch{pack4(q[0], q[1], q[2], q[3]), pack4(q[4], q[5], q[6], q[7])};
-    store_chunk8<kInterleave>(xq_row, 8 * c, ch, valid);
+    store_chunk8<kInterleave>(xq_row, 8 * c, ch, valid, perm ? static_cast<int>(m & 1) : -1);
   }
   sum = block_sum_i32(sum, redi);
   if (tid == 0) {
@@ -408,7 +416,7 @@ __global__ void __launch_bounds__(kActThreads)
 rmsnorm_quant_kernel(const void* __restrict__ x, const float* __restrict__ gamma, float eps,
                      int64_t M, int64_t K, int8_t* __restrict__ x_q, float* __restrict__ s_x,
                      int32_t* __restrict__ rowsum, uint4* __restrict__ zero16, int64_t n_zero16,
-                     int trigger_dependents, int* status, uint64_t wait_limit_ns) {
+                     int trigger_dependents, int* status, uint64_t wait_limit_ns, int perm) {
   __shared__ float redf[kActThreads];
   __shared__ int redi[kActThreads / 32];
   __shared__ __align__(8) uint64_t bar;
@@ -421,11 +429,13 @@ rmsnorm_quant_kernel(const void* __restrict__ x, const float* __restrict__ gamma
   }
   if (STAGED) {
     if (!quant_row_staged<kBF16, kInterleave>(x, gamma, eps, blockIdx.x, K, x_q, s_x, rowsum,
-                                              redf, redi, stage, &bar, wait_limit_ns) &&
+                                              redf, redi, stage, &bar, wait_limit_ns,
+                                              perm != 0) &&
         threadIdx.x == 0)
       record_failure(status, DEV_TIMEOUT_QUANT);
   } else {
-    quant_row<kBF16, kInterleave, 0>(x, gamma, eps, blockIdx.x, K, x_q, s_x, rowsum, redf, redi);
+    quant_row<kBF16, kInterleave, 0>(x, gamma, eps, blockIdx.x, K, x_q, s_x, rowsum, redf, redi,
+                                     perm != 0);
   }
 }
 
@@ -442,6 +452,7 @@ struct QuantProblem {
   float eps;
   int M, K;
   int x_bf16;
+  int perm;               // decode-matmul block order (x_block_pos)
   int block_begin;        // first block of this problem
   int zero_blocks;        // blocks after the M row blocks that clear zero16
 };
@@ -477,15 +488,18 @@ rmsnorm_quant_grouped_kernel(const __grid_constant__ QuantLaunch L) {
   if (STAGED) {
     const bool ok =
         q.x_bf16 ? quant_row_staged<true, true>(q.x, q.gamma, q.eps, local, q.K, q.xi, q.s_x,
-                                                q.rowsum, redf, redi, stage, &bar, L.wait_limit_ns)
+                                                q.rowsum, redf, redi, stage, &bar, L.wait_limit_ns,
+                                                q.perm != 0)
                  : quant_row_staged<false, true>(q.x, q.gamma, q.eps, local, q.K, q.xi, q.s_x,
                                                  q.rowsum, redf, redi, stage, &bar,
-                                                 L.wait_limit_ns);
+                                                 L.wait_limit_ns, q.perm != 0);
     if (!ok && threadIdx.x == 0) record_failure(L.status, DEV_TIMEOUT_QUANT);
   } else if (q.x_bf16) {
-    quant_row<true, true, 0>(q.x, q.gamma, q.eps, local, q.K, q.xi, q.s_x, q.rowsum, redf, redi);
+    quant_row<true, true, 0>(q.x, q.gamma, q.eps, local, q.K, q.xi, q.s_x, q.rowsum, redf, redi,
+                             q.perm != 0);
   } else {
-    quant_row<false, true, 0>(q.x, q.gamma, q.eps, local, q.K, q.xi, q.s_x, q.rowsum, redf, redi);
+    quant_row<false, true, 0>(q.x, q.gamma, q.eps, local, q.K, q.xi, q.s_x, q.rowsum, redf, redi,
+                              q.perm != 0);
   }
 }
 
@@ -494,7 +508,7 @@ rmsnorm_quant_grouped_kernel(const __grid_constant__ QuantLaunch L) {
 __global__ void __launch_bounds__(kActThreads)
 interleave_rowsum_kernel(const int8_t* __restrict__ x_q, int64_t M, int64_t K,
                          int8_t* __restrict__ xi, int32_t* __restrict__ rowsum,
-                         uint4* __restrict__ zero16, int64_t n_zero16) {
+                         uint4* __restrict__ zero16, int64_t n_zero16, int perm) {
   __shared__ int redi[kActThreads / 32];
   if (static_cast<int64_t>(blockIdx.x) >= M) {
     zero_fill_blocks(zero16, n_zero16, static_cast<int64_t>(blockIdx.x) - M,
@@ -520,7 +534,7 @@ interleave_rowsum_kernel(const int8_t* __restrict__ x_q, int64_t M, int64_t K,
         sum += static_cast<int8_t>((u.y >> (8 * j)) & 0xFF);
       }
     }
-    store_chunk8<true>(xi + m * K, 8 * c, ch, valid);
+    store_chunk8<true>(xi + m * K, 8 * c, ch, valid, perm ? static_cast<int>(m & 1) : -1);
   }
   sum = block_sum_i32(sum, redi);
   if (tid == 0) rowsum[m] = sum;

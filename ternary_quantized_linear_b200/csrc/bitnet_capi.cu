@@ -50,10 +50,16 @@ struct DeviceState {
 };
 DeviceState g_dev[kMaxDevices];
 
+// Dynamic shared-memory opt-in, and the largest shared-memory carve-out for
+// every kernel: kernels that follow one another on an SM then share one L1 /
+// shared split, so an SM need not drain to switch between them (the decode
+// matmul starts early, next to the activation-quant kernel it depends on).
 template <typename K>
 bool set_smem(K kernel, int bytes) {
   return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) ==
-         cudaSuccess;
+             cudaSuccess &&
+         cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                              cudaSharedmemCarveoutMaxShared) == cudaSuccess;
 }
 
 // Set up the current device once: status-word address, SM count, and the
@@ -67,10 +73,13 @@ DeviceState* device_state() {
               cudaSuccess;
     ok = ok && cudaDeviceGetAttribute(&st.num_sms, cudaDevAttrMultiProcessorCount, dev) ==
                    cudaSuccess;
+    ok = ok && set_smem(ternary_gemv_kernel<1>, gemv_smem_bytes(1));
+    ok = ok && set_smem(ternary_gemv_kernel<2>, gemv_smem_bytes(2));
     for (int nt = 0; nt < 2 && ok; ++nt) {
       int occ = 0;
       ok = cudaOccupancyMaxActiveBlocksPerMultiprocessor(
-               &occ, nt ? ternary_gemv_kernel<2> : ternary_gemv_kernel<1>, kGemvThreads, 0) ==
+               &occ, nt ? ternary_gemv_kernel<2> : ternary_gemv_kernel<1>, kGemvThreads,
+               gemv_smem_bytes(nt + 1)) ==
            cudaSuccess;
       st.gemv_occ[nt] = std::max(1, occ);
     }
@@ -79,6 +88,12 @@ DeviceState* device_state() {
     ok = ok && set_smem(rmsnorm_quant_kernel<false, true, true>, kQuantStageMax);
     ok = ok && set_smem(rmsnorm_quant_kernel<false, false, true>, kQuantStageMax);
     ok = ok && set_smem(rmsnorm_quant_grouped_kernel<true>, kQuantStageMax);
+    ok = ok && set_smem(rmsnorm_quant_grouped_kernel<false>, 0);
+    ok = ok && set_smem(rmsnorm_quant_kernel<true, true, false>, 0);
+    ok = ok && set_smem(rmsnorm_quant_kernel<true, false, false>, 0);
+    ok = ok && set_smem(rmsnorm_quant_kernel<false, true, false>, 0);
+    ok = ok && set_smem(rmsnorm_quant_kernel<false, false, false>, 0);
+    ok = ok && set_smem(interleave_rowsum_kernel, 0);
     ok = ok && set_smem(ternary_gemm_tc_kernel<16>, GemmCfg<16>::SMEM_DYN);
     ok = ok && set_smem(ternary_gemm_tc_kernel<32>, GemmCfg<32>::SMEM_DYN);
     ok = ok && set_smem(ternary_gemm_tc_kernel<64>, GemmCfg<64>::SMEM_DYN);
@@ -171,6 +186,10 @@ bool ok_dtype(int d) { return d == BITNET_F32 || d == BITNET_BF16; }
 // the workspace, a fence, a counter, a read-back), in 4 KiB units per CTA.
 constexpr long long kGemvSplitPenaltyUnits = 24;
 
+// Relative time of one unit: two token tiles take about half again as long
+// as one (measured on the decode shapes).
+long long gemv_unit_cost(const GemvProblem& P) { return P.M > 8 ? 3 : 2; }
+
 // Deal whole row blocks, largest first, to the least-loaded CTA (at most
 // kGemvMaxSegs each).  Returns the largest CTA load in units, or -1 when
 // the launch does not fit the explicit list.
@@ -181,8 +200,9 @@ long long plan_gemv_listed(GemvLaunch& L, long long G) {
   // Problems by decreasing row-block size.
   int order[kGemvMaxGroup];
   for (int i = 0; i < L.count; ++i) order[i] = i;
-  std::sort(order, order + L.count,
-            [&L](int a, int b) { return L.prob[a].kc > L.prob[b].kc; });
+  std::sort(order, order + L.count, [&L](int a, int b) {
+    return gemv_unit_cost(L.prob[a]) * L.prob[a].kc > gemv_unit_cost(L.prob[b]) * L.prob[b].kc;
+  });
   // Min-heap of (load, cta).
   std::vector<std::pair<long long, int>> heap;
   heap.reserve(static_cast<size_t>(G));
@@ -201,7 +221,7 @@ long long plan_gemv_listed(GemvLaunch& L, long long G) {
       auto top = heap.back();
       heap.pop_back();
       lists[static_cast<size_t>(top.second)].push_back(static_cast<uint16_t>(P.rb_begin + r));
-      top.first += P.kc;
+      top.first += gemv_unit_cost(P) * P.kc;
       worst = std::max(worst, top.first);
       if (lists[static_cast<size_t>(top.second)].size() < static_cast<size_t>(kGemvMaxSegs)) {
         heap.push_back(top);
@@ -239,14 +259,20 @@ long long plan_gemv_launch(GemvLaunch& L, long long capacity) {
     kc_min = std::min(kc_min, P.kc);
   }
   L.units = U;
-  long long G = std::min((U + kGemvWarps - 1) / kGemvWarps, std::max(1LL, capacity));
+  capacity = std::max(1LL, capacity);
+  long long G = std::min((U + kGemvWarps - 1) / kGemvWarps, capacity);
   // A share of n <= (kGemvMaxSegs - 1) * kc_min units touches at most
   // kGemvMaxSegs row blocks.
   const long long per = static_cast<long long>(kGemvMaxSegs - 1) * kc_min;
   G = std::max(G, (U + per - 1) / per);
   G = std::max(1LL, std::min(G, U));
-  const long long split_cost = (U + G - 1) / G + kGemvSplitPenaltyUnits;
-  const long long Gl = std::min<long long>(std::max(1LL, capacity), rbs);
+  long long W = 0;  // total weighted cost
+  for (int i = 0; i < L.count; ++i)
+    W += gemv_unit_cost(L.prob[i]) * static_cast<long long>(L.prob[i].rb) * L.prob[i].kc;
+  // CTAs beyond the resident capacity run as a later wave: cost per wave.
+  const long long waves = (G + capacity - 1) / capacity;
+  const long long split_cost = waves * ((W + G - 1) / G + 2 * kGemvSplitPenaltyUnits);
+  const long long Gl = std::min<long long>(capacity, rbs);
   const long long listed_cost = plan_gemv_listed(L, Gl);
   if (listed_cost >= 0 && listed_cost <= split_cost) {
     L.listed = 1;
@@ -268,9 +294,20 @@ bool gemv_problem_shared(const GemvLaunch& L, int i, long long G) {
   return false;
 }
 
-void fill_gemv_problem(GemvProblem& q, const uint8_t* Wp, uint8_t* ws, const FwdWorkspace& L,
+// nt: token tiles of the launch (the activation box has 8 nt rows).
+bool fill_gemv_problem(GemvProblem& q, const uint8_t* Wp, uint8_t* ws, const FwdWorkspace& L,
                        const float* s_x, const float* s_w, int64_t M, int64_t N, int64_t K,
-                       void* y, int y_dtype, int32_t* acc_out) {
+                       void* y, int y_dtype, int32_t* acc_out, int nt) {
+  // One unit = a 64-row x 64-byte weight box and a 256-byte x 8 nt-row
+  // activation box; rows past N or M and bytes past K read as zero.
+  if (!make_tmap_u8(&q.tmap_w, Wp, static_cast<uint64_t>(K / 4), static_cast<uint64_t>(N),
+                    static_cast<uint64_t>(K / 4), kGemvUnitK / 4, kGemvRows,
+                    CU_TENSOR_MAP_SWIZZLE_NONE))
+    return false;
+  if (!make_tmap_u8(&q.tmap_x, ws + L.xq, static_cast<uint64_t>(K), static_cast<uint64_t>(M),
+                    static_cast<uint64_t>(K), kGemvUnitK, static_cast<uint32_t>(8 * nt),
+                    CU_TENSOR_MAP_SWIZZLE_NONE))
+    return false;
   q.W = Wp;
   q.xq = reinterpret_cast<const int8_t*>(ws + L.xq);
   q.rowsum = reinterpret_cast<const int32_t*>(ws + L.rs);
@@ -284,6 +321,7 @@ void fill_gemv_problem(GemvProblem& q, const uint8_t* Wp, uint8_t* ws, const Fwd
   q.N = static_cast<int>(N);
   q.K = static_cast<int>(K);
   q.y_bf16 = (y_dtype == BITNET_BF16) ? 1 : 0;
+  return true;
 }
 
 // Token tiles of a launch: two n8 tiles when any problem has more than 8.
@@ -293,27 +331,25 @@ int gemv_tiles(const GemvLaunch& L) {
   return 1;
 }
 
-// Bytes of whole row blocks each CTA asks the copy engine to stream into L2
-// at entry (the launch total stays well inside the 126 MB L2).
-constexpr unsigned kGemvPrefetchBytes = 256u << 10;
-
 bitnet_status launch_gemv_group(const DeviceState& ds, GemvLaunch& L, long long G, bool pdl,
                                 bool early_weights, cudaStream_t stream) {
   L.use_pdl = pdl ? 1 : 0;
   L.early_weights = (pdl && early_weights) ? 1 : 0;
-  L.prefetch_bytes = kGemvPrefetchBytes;
+  L.status = ds.status;
+  L.wait_limit_ns = kWaitLimitNs;
   cudaLaunchConfig_t cfg{};
   cfg.gridDim = dim3(static_cast<unsigned>(G), 1, 1);
   cfg.blockDim = dim3(kGemvThreads, 1, 1);
-  cfg.dynamicSmemBytes = 0;
+  const int nt = gemv_tiles(L);
+  cfg.dynamicSmemBytes = gemv_smem_bytes(nt);
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = pdl ? 1 : 0;
-  const cudaError_t e = gemv_tiles(L) == 2 ? cudaLaunchKernelEx(&cfg, ternary_gemv_kernel<2>, L)
-                                           : cudaLaunchKernelEx(&cfg, ternary_gemv_kernel<1>, L);
+  const cudaError_t e = nt == 2 ? cudaLaunchKernelEx(&cfg, ternary_gemv_kernel<2>, L)
+                                : cudaLaunchKernelEx(&cfg, ternary_gemv_kernel<1>, L);
   return e == cudaSuccess ? BITNET_OK : BITNET_ERR_CUDA;
 }
 
@@ -335,8 +371,10 @@ bitnet_status launch_gemv(const DeviceState& ds, const uint8_t* Wp, const float*
                           const float* s_w, int64_t M, int64_t N, int64_t K, uint8_t* ws,
                           const FwdWorkspace& Lw, void* y, int y_dtype, int32_t* acc_out,
                           bool pdl, bool early_weights, cudaStream_t stream) {
-  static thread_local GemvLaunch L;  // ~2 KB: keep it off the stack
-  fill_gemv_problem(L.prob[0], Wp, ws, Lw, s_x, s_w, M, N, K, y, y_dtype, acc_out);
+  static thread_local GemvLaunch L;  // ~9 KB: keep it off the stack
+  if (!fill_gemv_problem(L.prob[0], Wp, ws, Lw, s_x, s_w, M, N, K, y, y_dtype, acc_out,
+                         M > 8 ? 2 : 1))
+    return BITNET_ERR_CUDA;
   const long long G = plan_gemv_single(ds, L, M, N, K);
   return launch_gemv_group(ds, L, G, pdl, early_weights, stream);
 }
@@ -447,12 +485,17 @@ int64_t zero_blocks(size_t bytes) {
   return std::min<int64_t>(256, (static_cast<int64_t>(bytes) + per_block - 1) / per_block);
 }
 
+// Layouts of the quantized activations a launch writes.
+enum XLayout { kXNatural = 0, kXInterleaved = 1, kXDecode = 2 };  // decode: + x_block_pos
+
 // zero/zero_bytes: a 16-byte aligned range (multiple of 16 bytes) cleared by
 // extra blocks of the same launch, or null/0.
 bitnet_status launch_act_quant(const void* x, int x_dtype, const float* gamma, float eps,
                                int64_t M, int64_t K, int8_t* x_q, float* s_x, int32_t* rowsum,
-                               bool interleave, bool trigger, void* zero, size_t zero_bytes,
+                               int layout, bool trigger, void* zero, size_t zero_bytes,
                                cudaStream_t stream) {
+  const bool interleave = layout != kXNatural;
+  const int perm = layout == kXDecode ? 1 : 0;
   const int64_t zb = zero ? zero_blocks(zero_bytes) : 0;
   dim3 grid(static_cast<unsigned>(M + zb)), block(kActThreads);
   const int trig = trigger ? 1 : 0;
@@ -465,7 +508,7 @@ bitnet_status launch_act_quant(const void* x, int x_dtype, const float* gamma, f
   const size_t dyn = staged ? stage : 0;
 #define BITNET_QUANT(BF, IL, ST)                                                             \
   rmsnorm_quant_kernel<BF, IL, ST><<<grid, block, dyn, stream>>>(                           \
-      x, gamma, eps, M, K, x_q, s_x, rowsum, z, n16, trig, status, kWaitLimitNs)
+      x, gamma, eps, M, K, x_q, s_x, rowsum, z, n16, trig, status, kWaitLimitNs, perm)
   if (bf16) {
     if (interleave) {
       if (staged) BITNET_QUANT(true, true, true); else BITNET_QUANT(true, true, false);
@@ -543,8 +586,8 @@ bitnet_status forward_impl(const void* x, int x_dtype, const float* gamma, float
   if (x_q_out || s_x_out) {
     // Debug export in natural k order (same arithmetic as the fused pass).
     int8_t* xq_nat = x_q_out ? x_q_out : reinterpret_cast<int8_t*>(ws + L.xq);
-    st = launch_act_quant(x, x_dtype, gamma, eps, M, K, xq_nat, s_x_out, nullptr, false, false,
-                          nullptr, 0, stream);
+    st = launch_act_quant(x, x_dtype, gamma, eps, M, K, xq_nat, s_x_out, nullptr, kXNatural,
+                          false, nullptr, 0, stream);
     if (st != BITNET_OK) return st;
   }
   const bool pdl = true;  // the matmul launch follows the quant launch directly
@@ -553,7 +596,9 @@ bitnet_status forward_impl(const void* x, int x_dtype, const float* gamma, float
   void* zero = needs_zeroed_partials(*ds, path, M, N, K) ? splitk_region(ws, L, &zbytes)
                                                           : nullptr;
   st = launch_act_quant(x, x_dtype, gamma, eps, M, K, reinterpret_cast<int8_t*>(ws + L.xq), sx,
-                        reinterpret_cast<int32_t*>(ws + L.rs), true, pdl, zero, zbytes, stream);
+                        reinterpret_cast<int32_t*>(ws + L.rs),
+                        path == BITNET_PATH_GEMV ? kXDecode : kXInterleaved, pdl, zero, zbytes,
+                        stream);
   if (st != BITNET_OK) return st;
   // The activation-quant kernel just queued started after every earlier
   // write to W_packed, so the GEMV may fetch weights before waiting on it.
@@ -647,11 +692,13 @@ bitnet_status forward_grouped_impl(int count, const bitnet_linear_problem* probl
     qp.M = static_cast<int>(q.M);
     qp.K = static_cast<int>(q.K);
     qp.x_bf16 = (q.x_dtype == BITNET_BF16) ? 1 : 0;
+    qp.perm = 1;  // decode matmul
     qp.block_begin = qblocks;
     qp.zero_blocks = static_cast<int>(zero ? zero_blocks(zbytes) : 0);
     qblocks += qp.M + qp.zero_blocks;
-    fill_gemv_problem(GL.prob[n], q.W_packed, ws, L, qp.s_x, q.s_w, q.M, q.N, q.K, q.y,
-                      q.y_dtype, nullptr);
+    if (!fill_gemv_problem(GL.prob[n], q.W_packed, ws, L, qp.s_x, q.s_w, q.M, q.N, q.K, q.y,
+                           q.y_dtype, nullptr, mmax > 8 ? 2 : 1))
+      return BITNET_ERR_CUDA;
     ++n;
   }
   if (n > 0) {
@@ -762,7 +809,7 @@ BITNET_API bitnet_status bitnet_rmsnorm_quant_act(const void* x, int x_dtype, co
   if (!aligned(x, 16) || (gamma && !aligned(gamma, 16)) || !aligned(x_q, 16) || !aligned(s_x, 4))
     return BITNET_ERR_MISALIGNED;
   if (!device_state()) return BITNET_ERR_CUDA;
-  return launch_act_quant(x, x_dtype, gamma, eps, M, K, x_q, s_x, nullptr, false, false,
+  return launch_act_quant(x, x_dtype, gamma, eps, M, K, x_q, s_x, nullptr, kXNatural, false,
                           nullptr, 0, as_stream(stream));
 }
 
@@ -799,10 +846,12 @@ BITNET_API bitnet_status bitnet_linear_quantize_input(const void* x, int x_dtype
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   size_t zbytes = 0;
   void* zero = (M <= kGemvMaxM) ? splitk_region(ws, L, &zbytes) : nullptr;
+  const int path = resolve_path(BITNET_PATH_AUTO, M, N, K);  // the same as the matmul phase
   return launch_act_quant(x, x_dtype, gamma, eps, M, K, reinterpret_cast<int8_t*>(ws + L.xq),
                           reinterpret_cast<float*>(ws + L.sx),
-                          reinterpret_cast<int32_t*>(ws + L.rs), true, M <= kGemvMaxM, zero,
-                          zbytes, as_stream(stream));
+                          reinterpret_cast<int32_t*>(ws + L.rs),
+                          path == BITNET_PATH_GEMV ? kXDecode : kXInterleaved, M <= kGemvMaxM,
+                          zero, zbytes, as_stream(stream));
 }
 
 BITNET_API bitnet_status bitnet_linear_matmul(const uint8_t* W_packed, const float* s_w,
@@ -877,7 +926,8 @@ BITNET_API bitnet_status bitnet_ternary_matmul_i32(const int8_t* x_q, const uint
   const int64_t zb = zero ? zero_blocks(zbytes) : 0;
   interleave_rowsum_kernel<<<static_cast<unsigned>(M + zb), kActThreads, 0, s>>>(
       x_q, M, K, reinterpret_cast<int8_t*>(ws + L.xq), reinterpret_cast<int32_t*>(ws + L.rs),
-      static_cast<uint4*>(zero), zero ? static_cast<int64_t>(zbytes / 16) : 0);
+      static_cast<uint4*>(zero), zero ? static_cast<int64_t>(zbytes / 16) : 0,
+      path == BITNET_PATH_GEMV ? 1 : 0);
   st = launch_status();
   if (st != BITNET_OK) return st;
   return run_matmul(*ds, path, W_packed, ws, L, nullptr, nullptr, M, N, K, nullptr, BITNET_F32,

@@ -278,6 +278,17 @@ __device__ __forceinline__ uint4 ldg_u4(const void* p) {
   return v;
 }
 
+// ------------------------------------------------- decode activation order
+
+// Decode-matmul block order: inside every 256-byte span of a token row of
+// k-interleaved x_q, 16-byte block b is stored at block x_block_pos(b, m & 1).
+// A lane (g, t) of the decode matmul reads blocks 4t + q of token g; with
+// this order the eight lanes of a quarter warp (two tokens of opposite
+// parity, t = 0..3) hit eight different 16-byte bank groups for every q.
+__host__ __device__ __forceinline__ int x_block_pos(int b, int parity) {
+  return b ^ (((b >> 3) & 1) << 1) ^ parity;
+}
+
 // ---------------------------------------------------------- float helpers
 
 __device__ __forceinline__ float bf16_bits_to_f32(uint32_t h) {

@@ -15,15 +15,18 @@
 //     first, to the least-loaded CTA (no cross-CTA reduction at all), or,
 //     when that balances badly, every CTA an equal contiguous share of the
 //     units laid end to end ("stream-K").  The units of a CTA's segment list
-//     are split into eight equal contiguous ranges, one per warp.
-//   * No shared-memory staging.  Lane (4g + t) loads 16 bytes (64 k) of rows
-//     g and g+8 of each of the unit's four 16-row groups straight into
-//     registers (eight 16-byte loads, every 32-byte sector used) and the
-//     matching 64 bytes of x_q for token g (from L2: every row block reads
-//     the same activations).  The next unit's loads are issued before the
-//     current unit's MMAs (two register buffers).  At entry one thread asks
-//     the copy engine to stream the share's whole row blocks (contiguous
-//     64 x K/4 bytes each, one bulk operation per row block) into L2.
+//     are split into eight equal contiguous ranges, one per compute warp.
+//   * Operands move by TMA: each warp has its own ring of kGemvStages stages
+//     and its lane 0 issues, per unit, one 2-D box of weights (64 rows x 64
+//     bytes) and one of activations (the unit's 256 bytes of 8 or 16 token
+//     rows), refilling a stage as soon as the warp has read it.  Eight
+//     issuing lanes per SM keep enough copies in flight (one issuing thread
+//     cannot: each copy costs it a few hundred nanoseconds), and rows past N,
+//     tokens past M or k past K arrive as zeros.
+//   * Lane (4g + t) reads 16 bytes (64 k) of rows g and g+8 of each 16-row
+//     group (64-byte rows: conflict-free) and the 64 bytes of token g for the
+//     same k, which the activation-quant kernel stored in the decode block
+//     order (x_block_pos) so that these reads are conflict-free too.
 //   * Unpack in registers with masks: byte i of a packed word holds the codes
 //     t+1 of k = 4i..4i+3 of a 16-k group at bits 2r; P & 0x03030303 and
 //     (P >> 2) & 0x03030303 are words of four int8 codes (r = 0, 1), and
@@ -32,19 +35,18 @@
 //     k-interleaved (byte 4r+i of each 16-group holds k = 4i+r), so the
 //     matching activation word is a plain 4-byte slice.
 //   * Warp-level int8 MMA m16n8k32 in swap-AB form: 16 weight rows are the
-//     MMA's M, up to 16 tokens its N (one or two n8 tiles).  The four row
-//     groups are four independent accumulator chains.  sum x*(t+1) minus the
-//     token's row sum sum x gives sum x*t exactly.
-//   * Before waiting on the activation-quant grid (programmatic dependent
-//     launch) each warp already loads its first two units' weights and the
-//     L2 stream starts, so the weight traffic overlaps that grid.
-//   * A warp adds its accumulators to its CTA's per-row-block sums in shared
-//     memory when it moves to another row block.  At the end, a row block
-//     that lies inside the CTA's share is finished directly
-//     (y = acc / (s_x * s_w)); one shared with neighbouring CTAs adds its
-//     partials into an int32 workspace and the last CTA to arrive (arrival
-//     counter, no waiting) reads them back, re-zeroes them and finishes.
-//   * Nothing in this kernel waits on a flag or barrier another CTA sets.
+//     MMA's M, up to 16 tokens its N (one or two n8 tiles).  Eight
+//     independent accumulator chains.  sum x*(t+1) minus the token's row sum
+//     sum x gives sum x*t exactly.
+//   * The weight copies start before waiting on the activation-quant grid
+//     (programmatic dependent launch): only the activation copies wait.
+//   * A warp adds its accumulators to its CTA's per-segment sums in shared
+//     memory when it moves to another segment.  At the end, whole row blocks
+//     are finished directly (y = acc / (s_x * s_w)); a part of a row block
+//     (stream-K ends) adds its partials into an int32 workspace and the last
+//     CTA to arrive (arrival counter, no waiting) reads them back, re-zeroes
+//     them and finishes.
+//   * Every wait on a copy is bounded; nothing waits on another CTA.
 #pragma once
 
 #include "common.cuh"
@@ -55,17 +57,21 @@ constexpr int kGemvRows = 64;        // weight rows per unit
 constexpr int kGemvUnitK = 256;      // k per unit
 constexpr int kGemvWarps = 8;
 constexpr int kGemvThreads = 32 * kGemvWarps;
-constexpr int kGemvMaxSegs = 8;      // row blocks one CTA's share may touch
+constexpr int kGemvMaxSegs = 6;      // row blocks one CTA's share may touch
 constexpr int kGemvMaxGroup = 16;    // problems per grouped launch
 constexpr uint32_t kCodeMask = 0x03030303u;
-// Two register buffers per warp (next unit's loads in flight during the
-// MMAs, one CTA per SM), or one buffer and two CTAs per SM.
-#ifndef BITNET_GEMV_DOUBLE_BUFFER
-#define BITNET_GEMV_DOUBLE_BUFFER 1
-#endif
-constexpr bool kGemvDoubleBuffer = BITNET_GEMV_DOUBLE_BUFFER != 0;
+constexpr int kGemvStages = 3;      // ring stages per warp
+constexpr int kGemvUnitBytes = kGemvRows * (kGemvUnitK / 4);  // 4 KiB of weights
+// A stage: the unit's weights, then its activations (8 or 16 token rows of
+// 256 bytes).
+__host__ __device__ constexpr int gemv_stage_bytes(int nt) { return kGemvUnitBytes + nt * 2048; }
+__host__ __device__ constexpr int gemv_smem_bytes(int nt) {
+  return kGemvWarps * kGemvStages * gemv_stage_bytes(nt) + 1024;  // + alignment slack
+}
 
 struct GemvProblem {
+  CUtensorMap tmap_w;     // W_packed [N][K/4] bytes, box 64 x 64 rows, no swizzle
+  CUtensorMap tmap_x;     // x_q [M][K] bytes (decode block order), box 256 x 8*NT rows
   const uint8_t* W;       // W_packed [N][K/4]
   const int8_t* xq;       // x_q k-interleaved [M][K]
   const int32_t* rowsum;  // [M]
@@ -91,8 +97,9 @@ struct GemvLaunch {
   long long units;        // total units of the launch
   int count;              // problems in this launch
   int use_pdl;            // wait for the preceding grid before reading activations
-  int early_weights;      // start the weight loads before that wait
-  unsigned prefetch_bytes;  // per CTA: whole row blocks streamed into L2 at entry
+  int early_weights;      // start the weight copies before that wait
+  int* status;            // device status word (bounded waits)
+  uint64_t wait_limit_ns;
   int listed;             // 1: CTA b owns row blocks task[cta_begin[b] .. cta_begin[b+1])
                           // 0: CTA b owns units [b U / G, (b+1) U / G)
   uint16_t cta_begin[kGemvMaxCtas + 1];
@@ -104,6 +111,8 @@ struct GemvBuf {
   uint4 wa[4], wb[4];  // rows g and g+8 of the four row groups
   uint4 x[NT][4];      // token 8 nt + g, 64 k
 };
+
+
 
 __device__ __forceinline__ uint32_t word_of(const uint4& v, int w) {
   return w == 0 ? v.x : (w == 1 ? v.y : (w == 2 ? v.z : v.w));
@@ -128,70 +137,31 @@ __device__ __forceinline__ GemvUnit gemv_unit(const GemvProblem* prob, int count
   return r;
 }
 
-// Weight load of any unit.  No lane branches around its loads: rows past N
-// read row N-1 (their outputs are never written) and a segment past K reads
-// k = 0 (its activations are zeroed in gemv_load_x, so it adds nothing).
+// Activations of one unit from its stage: token 8 nt + g, this lane's 64 k
+// (blocks 4t + q of the 256-byte span, stored at x_block_pos; tokens past M
+// and k past K arrived as zeros).
+template <int NT, int TILES>
+__device__ __forceinline__ void gemv_read_stage_x(GemvBuf<NT>& b, const uint8_t* xs, int g,
+                                                  int t) {
+#pragma unroll
+  for (int nt = 0; nt < TILES; ++nt)
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+      b.x[nt][q] = *reinterpret_cast<const uint4*>(
+          xs + (8 * nt + g) * 256 + 16 * x_block_pos(4 * t + q, g & 1));
+}
+
+// Weights of one unit from its stage: rows g and g+8 of each 16-row group,
+// this lane's 16 bytes.  64-byte rows: the eight lanes of a quarter warp
+// (g = 2j, 2j+1; t = 0..3) hit 32 distinct banks.
 template <int NT>
-__device__ __forceinline__ void gemv_load_w(GemvBuf<NT>& b, const GemvProblem& P, int rbl, int c,
-                                            int g, int t) {
-  const int kseg = c * kGemvUnitK + 64 * t;
-  const int kk = kseg < P.K ? kseg : 0;  // K % 64 == 0: a segment is all in or all out
-  const size_t rowb = static_cast<size_t>(P.K) / 4;
-  const int r = rbl * kGemvRows + g;
-  const uint8_t* base = P.W + kk / 4;
+__device__ __forceinline__ void gemv_read_stage(GemvBuf<NT>& b, const uint8_t* stage, int g,
+                                                int t) {
 #pragma unroll
   for (int rg = 0; rg < 4; ++rg) {
-    const int ra = min(r + 16 * rg, P.N - 1), rb = min(r + 16 * rg + 8, P.N - 1);
-    b.wa[rg] = ldg_stream_u4(base + static_cast<size_t>(ra) * rowb);
-    b.wb[rg] = ldg_stream_u4(base + static_cast<size_t>(rb) * rowb);
+    b.wa[rg] = *reinterpret_cast<const uint4*>(stage + (16 * rg + g) * 64 + 16 * t);
+    b.wb[rg] = *reinterpret_cast<const uint4*>(stage + (16 * rg + g + 8) * 64 + 16 * t);
   }
-}
-
-// Weight load of a unit inside a full row block with K % 256 == 0: no
-// bounds tests.  base = row g of the row block, at this lane's 16 bytes.
-template <int NT>
-__device__ __forceinline__ void gemv_load_w_full(GemvBuf<NT>& b, const uint8_t* base,
-                                                 size_t rowb) {
-  const size_t r8 = 8 * rowb;
-#pragma unroll
-  for (int rg = 0; rg < 4; ++rg) {
-    b.wa[rg] = ldg_stream_u4(base + 2 * rg * r8);
-    b.wb[rg] = ldg_stream_u4(base + (2 * rg + 1) * r8);
-  }
-}
-
-// Activation load: token 8 nt + g, this lane's 64 k.  Tokens past M read
-// token M-1 (their output columns are never written); a segment past K
-// reads zeros.  No lane branches around the loads.
-template <int NT>
-__device__ __forceinline__ void gemv_load_x(GemvBuf<NT>& b, const GemvProblem& P, int c, int g,
-                                            int t) {
-  const int kseg = c * kGemvUnitK + 64 * t;
-  const bool kval = kseg < P.K;
-  const int kk = kval ? kseg : 0;
-#pragma unroll
-  for (int nt = 0; nt < NT; ++nt) {
-    const int m = min(8 * nt + g, P.M - 1);
-    const int8_t* px = P.xq + static_cast<size_t>(m) * P.K + kk;
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const uint4 v = ldg_u4_ro(px + 16 * q);
-      b.x[nt][q] = kval ? v : make_uint4(0u, 0u, 0u, 0u);
-    }
-  }
-}
-
-// Ask the copy engine to bring row block rbl of P (64 rows x K/4 bytes,
-// contiguous) into L2, clipped to `limit` bytes; one bulk operation.
-__device__ __forceinline__ uint32_t gemv_prefetch_rows(const GemvProblem& P, int rbl,
-                                                       uint32_t limit) {
-  const size_t rowb = static_cast<size_t>(P.K) / 4;
-  const int rows = min(kGemvRows, P.N - rbl * kGemvRows);
-  size_t bytes = static_cast<size_t>(rows) * rowb;  // multiple of 16 (K % 64 == 0)
-  if (bytes > limit) bytes = limit & ~15u;
-  if (bytes) prefetch_l2_bulk(P.W + static_cast<size_t>(rbl) * kGemvRows * rowb,
-                              static_cast<uint32_t>(bytes));
-  return static_cast<uint32_t>(bytes);
 }
 
 // The MMAs of one unit for TILES token tiles.  Unpack: Q = P >> 2 once per
@@ -261,13 +231,15 @@ __device__ __forceinline__ void gemv_flush(int (&acc)[4][NT][4], int (&acc16)[4]
   }
 }
 
-__device__ __forceinline__ void gemv_finish(const GemvProblem& p, float sw, int m, int n,
-                                            int acc_codes) {
-  const int acc = acc_codes - p.rowsum[m];
+// rs, sx: token m's row sum and scale (read once per segment into shared
+// memory); sw the weight scale.
+__device__ __forceinline__ void gemv_finish(const GemvProblem& p, float sw, float sx, int rs,
+                                            int m, int n, int acc_codes) {
+  const int acc = acc_codes - rs;
   const int64_t o = static_cast<int64_t>(m) * p.N + n;
   if (p.acc_out) p.acc_out[o] = acc;
   if (p.y) {
-    const float yv = __fdiv_rn(__int2float_rn(acc), __fmul_rn(p.s_x[m], sw));
+    const float yv = __fdiv_rn(__int2float_rn(acc), __fmul_rn(sx, sw));
     if (p.y_bf16)
       reinterpret_cast<__nv_bfloat16*>(p.y)[o] = __float2bfloat16_rn(yv);
     else
@@ -281,24 +253,38 @@ __host__ __device__ __forceinline__ long long gemv_cta_of(long long u, long long
 }
 
 template <int NT>
-__global__ void __launch_bounds__(kGemvThreads, kGemvDoubleBuffer ? 1 : 2)
+__global__ void __launch_bounds__(kGemvThreads, 1)
 ternary_gemv_kernel(const __grid_constant__ GemvLaunch L) {
+  extern __shared__ uint8_t gemv_smem_raw[];
+  uint8_t* ring = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(gemv_smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   __shared__ int red[kGemvMaxSegs * kGemvRows * 16];  // [segment][row][token]
+  __shared__ __align__(8) uint64_t full[kGemvWarps][kGemvStages];
   // The problem table and this CTA's segments live in shared memory: the
   // walk indexes them by run-time numbers, which kernel-parameter space
-  // serves slowly.
+  // serves slowly (the copy engine still reads the tensor maps from the
+  // parameters).
   __shared__ GemvProblem sprob[kGemvMaxGroup];
   __shared__ int seg_p[kGemvMaxSegs], seg_rbl[kGemvMaxSegs];
   __shared__ int seg_lo[kGemvMaxSegs], seg_n[kGemvMaxSegs], seg_owned[kGemvMaxSegs];
-  __shared__ int seg_full[kGemvMaxSegs];  // 64 rows inside N and K % 256 == 0
   __shared__ int seg_count, seg_last[kGemvMaxSegs];
+  __shared__ int seg_rs[kGemvMaxSegs][16];    // row sums of the segment's tokens
+  __shared__ float seg_sx[kGemvMaxSegs][16];  // their scales
+  __shared__ float seg_sw[kGemvMaxSegs];      // the weight scale
+  __shared__ volatile int abort_flag;
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int g = lane >> 2, t = lane & 3;
   const long long U = L.units, G = gridDim.x, b = blockIdx.x;
   const long long ub = b * U / G, ue = (b + 1) * U / G;  // stream-K share
   const int count = L.count;
+  const uint64_t limit = L.wait_limit_ns;
   if (tid < count) sprob[tid] = L.prob[tid];
+  if (tid < kGemvWarps * kGemvStages) mbar_init(&full[0][0] + tid, 1);
+  if (tid == 0) {
+    abort_flag = 0;
+    fence_mbarrier_init();
+  }
   __syncthreads();
   const GemvProblem* prob = sprob;
   if (tid == 0) {
@@ -338,11 +324,8 @@ ternary_gemv_kernel(const __grid_constant__ GemvLaunch L) {
       }
     }
     seg_count = n;
-    for (int i = 0; i < n; ++i) {
-      const GemvProblem& P = prob[seg_p[i]];
-      seg_full[i] = ((seg_rbl[i] + 1) * kGemvRows <= P.N && P.K % kGemvUnitK == 0) ? 1 : 0;
-    }
   }
+  for (int i = tid; i < kGemvMaxSegs * kGemvRows * 16; i += kGemvThreads) red[i] = 0;
   __syncthreads();
   const int nseg = seg_count;  // <= kGemvMaxSegs (host)
   if (nseg == 0) return;       // uniform over the CTA
@@ -358,61 +341,68 @@ ternary_gemv_kernel(const __grid_constant__ GemvLaunch L) {
       ++x.s;
     }
   };
-  auto load_w = [&](GemvBuf<NT>& buf, const Cursor& x) {
-    const GemvProblem& P = prob[seg_p[x.s]];
-    const int c = seg_lo[x.s] + x.off;
-    if (seg_full[x.s]) {
-      const size_t rowb = static_cast<size_t>(P.K) / 4;
-      gemv_load_w_full(buf,
-                       P.W + static_cast<size_t>(seg_rbl[x.s] * kGemvRows + g) * rowb +
-                           c * (kGemvUnitK / 4) + 16 * t,
-                       rowb);
-    } else {
-      gemv_load_w(buf, P, seg_rbl[x.s], c, g, t);
-    }
-  };
-  auto load_x = [&](GemvBuf<NT>& buf, const Cursor& x) {
-    gemv_load_x(buf, prob[seg_p[x.s]], seg_lo[x.s] + x.off, g, t);
-  };
-
-  // Warp w takes the w-th of eight equal contiguous ranges of the CTA's units
-  // (in segment order): it touches one or two segments, and its loads walk
-  // along the rows.
+  // Warp w takes the w-th of eight equal contiguous ranges of the CTA's
+  // units.
   int n_units = 0;
   for (int i = 0; i < nseg; ++i) n_units += seg_n[i];
-  const int u_begin = warp * n_units / kGemvWarps;
-  const int u_count = (warp + 1) * n_units / kGemvWarps - u_begin;
+  auto range_of = [&](int w, Cursor& x0) {
+    const int u0 = w * n_units / kGemvWarps;
+    x0 = Cursor{0, 0};
+    advance(x0, u0);
+    return (w + 1) * n_units / kGemvWarps - u0;
+  };
 
-  // Before the activations exist: the weights of this warp's first two
-  // units go to registers, and one thread asks the copy engine to stream the
-  // CTA's whole row blocks (up to L.prefetch_bytes) into L2.
-  GemvBuf<NT> bufA, bufB;
-  Cursor xA{0, 0};
-  advance(xA, u_begin);
-  if (u_count == 0) xA.s = nseg;
-  int left = u_count;  // units of this warp not yet loaded (xA counts as loaded)
-  Cursor xB = xA;
-  if (left > 1) advance(xB, 1);
-  else xB.s = nseg;
-  const bool early = L.early_weights != 0;
-  if (early) {
-    if (u_count > 0) load_w(bufA, xA);
-    if (kGemvDoubleBuffer && u_count > 1) load_w(bufB, xB);
+  // Warp w streams its range through its own ring: lane 0 issues the copies
+  // (weights as soon as the CTA starts, activations once the preceding grid
+  // is done), all lanes consume.
+  constexpr int kStage = gemv_stage_bytes(NT);
+  uint8_t* myring = ring + warp * kGemvStages * kStage;
+  Cursor xA;
+  const int n = range_of(warp, xA);
+  Cursor xI = xA;  // next unit to issue
+  int issued = 0;
+  auto issue_w = [&](int j) {  // lane 0: unit j (cursor xI) weights into stage j % S
+    const int st = j % kGemvStages;
+    const int p = seg_p[xI.s];
+    mbar_arrive_expect_tx(&full[warp][st], kStage);
+    tma_load_2d(myring + st * kStage, &L.prob[p].tmap_w, (seg_lo[xI.s] + xI.off) * (kGemvUnitK / 4),
+                seg_rbl[xI.s] * kGemvRows, &full[warp][st]);
+  };
+  auto issue_x = [&](int j, const Cursor& x) {
+    const int st = j % kGemvStages;
+    tma_load_2d(myring + st * kStage + kGemvUnitBytes, &L.prob[seg_p[x.s]].tmap_x,
+                (seg_lo[x.s] + x.off) * kGemvUnitK, 0, &full[warp][st]);
+  };
+  const int pre = min(n, kGemvStages);
+  const bool early = L.early_weights != 0 || !L.use_pdl;
+  if (lane == 0 && early) {
+    Cursor c0 = xI;
+    for (int j = 0; j < pre; ++j) {
+      issue_w(j);
+      if (j + 1 < pre) advance(xI, 1);
+    }
+    xI = c0;
   }
-  if (tid == 0 && L.prefetch_bytes > 0) {
-    uint32_t left = L.prefetch_bytes;
-    for (int s = 0; s < nseg && left > 0; ++s)
-      if (seg_owned[s]) left -= gemv_prefetch_rows(prob[seg_p[s]], seg_rbl[s], left);
-  }
-  for (int i = tid; i < nseg * kGemvRows * 16; i += kGemvThreads) red[i] = 0;
   if (L.use_pdl) pdl_wait_prior_grid();
-  __syncthreads();
-
-  if (u_count > 0) {
-    if (!early) load_w(bufA, xA);
-    load_x(bufA, xA);
+  if (warp < nseg) {
+    // This warp reads segment `warp`'s row sums and scales for the finish.
+    const GemvProblem& P = prob[seg_p[warp]];
+    if (lane < P.M) {
+      seg_rs[warp][lane] = P.rowsum[lane];
+      seg_sx[warp][lane] = P.s_x ? P.s_x[lane] : 0.0f;
+    }
+    if (lane == 0) seg_sw[warp] = (P.y && P.s_w) ? P.s_w[0] : 0.0f;
   }
-  bool preB = early && u_count > 1;  // bufB already holds the next unit's weights
+  if (lane == 0) {
+    for (int j = 0; j < pre; ++j) {
+      if (!early) issue_w(j);
+      issue_x(j, xI);
+      if (j + 1 < n) advance(xI, 1);
+    }
+  }
+  issued = pre;
+
+  GemvBuf<NT> buf;
   int acc[4][NT][4], acc16[4][NT][4];
 #pragma unroll
   for (int rg = 0; rg < 4; ++rg)
@@ -429,65 +419,56 @@ ternary_gemv_kernel(const __grid_constant__ GemvLaunch L) {
     else
       gemv_flush<NT, 1>(acc, acc16, dst, cur_m, g, t);
   };
-  auto enter = [&](int seg) {
+  int k = 0;
+  for (; k < n; ++k) {
+    const int st = k % kGemvStages;
+    // The MMAs below are warp-collective: the wait verdict is made uniform
+    // across the warp.
+    const bool got = mbar_wait_bounded(&full[warp][st], static_cast<uint32_t>(k / kGemvStages) & 1u,
+                                       &abort_flag, limit);
+    if (!__all_sync(0xFFFFFFFFu, got)) {
+      abort_flag = 1;
+      if (lane == 0) record_failure(L.status, DEV_TIMEOUT_GEMV);
+      break;
+    }
+    const uint8_t* sp = myring + st * kStage;
+    const int seg = xA.s;
     if (seg != cur_seg) {
       flush();
       cur_seg = seg;
       cur_m = prob[seg_p[seg]].M;
     }
-  };
-  // One token tile unless this problem has more than 8 tokens (uniform).
-  auto mma = [&](const GemvBuf<NT>& buf) {
-    if (NT == 2 && cur_m > 8)
+    const bool two = NT == 2 && cur_m > 8;
+    gemv_read_stage(buf, sp, g, t);
+    if (two)
+      gemv_read_stage_x<NT, NT>(buf, sp + kGemvUnitBytes, g, t);
+    else
+      gemv_read_stage_x<NT, 1>(buf, sp + kGemvUnitBytes, g, t);
+    // Refill this stage with unit k + S once every lane's reads are done.
+    __syncwarp();
+    if (lane == 0 && issued < n) {
+      fence_proxy_async_smem();
+      issue_w(issued);
+      issue_x(issued, xI);
+      if (issued + 1 < n) advance(xI, 1);
+    }
+    if (issued < n) ++issued;
+    if (k + 1 < n) advance(xA, 1);
+    if (two)
       gemv_mma_unit<NT, NT>(acc, acc16, buf);
     else
       gemv_mma_unit<NT, 1>(acc, acc16, buf);
-  };
-
-  // left = units of this warp from xA on.
-  if (!kGemvDoubleBuffer) {
-    // One register buffer: load a unit, compute it; the other warps of the
-    // SM (two CTAs) cover the load latency.
-    bool loaded = u_count > 0;  // bufA holds xA (weights and activations)
-    while (left > 0) {
-      if (!loaded) {
-        load_w(bufA, xA);
-        load_x(bufA, xA);
-      }
-      loaded = false;
-      enter(xA.s);
-      mma(bufA);
-      if (--left > 0) advance(xA, 1);
-    }
-    left = 0;
-  }
-  while (left > 0) {
-    const bool hasB = left > 1;
-    if (hasB) {
-      if (!preB) {
-        xB = xA;
-        advance(xB, 1);
-        load_w(bufB, xB);
-      }
-      load_x(bufB, xB);
-    }
-    preB = false;
-    enter(xA.s);
-    mma(bufA);
-    if (!hasB) break;
-    const bool hasA = left > 2;
-    if (hasA) {
-      xA = xB;
-      advance(xA, 1);
-      load_w(bufA, xA);
-      load_x(bufA, xA);
-    }
-    enter(xB.s);
-    mma(bufB);
-    left -= 2;
   }
   flush();
-  __syncthreads();
+  if (abort_flag && lane == 0) {
+    // Let the copies already in flight land before the CTA exits.
+    for (int j = k; j < issued; ++j)
+      if (!mbar_wait_bounded(&full[warp][j % kGemvStages],
+                             static_cast<uint32_t>(j / kGemvStages) & 1u, nullptr, limit))
+        record_failure(L.status, DEV_TIMEOUT_DRAIN);
+  }
+  const int all_ok = __syncthreads_and(abort_flag == 0 ? 1 : 0);
+  if (!all_ok) return;  // a timed-out copy: results would be garbage
 
   // Finish this CTA's segments: whole row blocks straight from the shared
   // sums; a part of a row block (stream-K ends) adds its partials to the
@@ -500,10 +481,9 @@ ternary_gemv_kernel(const __grid_constant__ GemvLaunch L) {
     const int nout = kGemvRows * P.M;
     const int n0 = seg_rbl[s] * kGemvRows;
     if (seg_owned[s]) {
-      const float sw = (P.y && P.s_w) ? __ldg(P.s_w) : 0.0f;
       for (int idx = tid; idx < nout; idx += kGemvThreads) {
         const int r = idx % kGemvRows, m = idx / kGemvRows, n = n0 + r;
-        if (n < P.N) gemv_finish(P, sw, m, n, rs[r * 16 + m]);
+        if (n < P.N) gemv_finish(P, seg_sw[s], seg_sx[s][m], seg_rs[s][m], m, n, rs[r * 16 + m]);
       }
       continue;
     }
@@ -534,14 +514,13 @@ ternary_gemv_kernel(const __grid_constant__ GemvLaunch L) {
   for (int s = 0; s < nseg; ++s) {
     if (!seg_last[s]) continue;
     const GemvProblem& P = prob[seg_p[s]];
-    const float sw = (P.y && P.s_w) ? __ldg(P.s_w) : 0.0f;
     const int nout = kGemvRows * P.M;
     const int n0 = seg_rbl[s] * kGemvRows;
     for (int idx = tid; idx < nout; idx += kGemvThreads) {
       const int r = idx % kGemvRows, m = idx / kGemvRows, n = n0 + r;
       if (n < P.N) {
         const int v = atomicExch(P.ws_acc + static_cast<int64_t>(m) * P.N + n, 0);
-        gemv_finish(P, sw, m, n, v);
+        gemv_finish(P, seg_sw[s], seg_sx[s][m], seg_rs[s][m], m, n, v);
       }
     }
     if (tid == 0) P.ws_cnt[seg_rbl[s]] = 0u;  // ready for the next call
