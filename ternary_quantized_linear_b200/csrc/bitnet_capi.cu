@@ -196,7 +196,7 @@ long long gemv_unit_cost(const GemvProblem& P) { return P.M > 8 ? 3 : 2; }
 long long plan_gemv_listed(GemvLaunch& L, long long G) {
   int total = 0;
   for (int i = 0; i < L.count; ++i) total += L.prob[i].rb;
-  if (total > kGemvMaxTasks || G > kGemvMaxCtas || G < 1) return -1;
+  if (total > G * kGemvMaxSegs || G > kGemvMaxCtas || G < 1 || total >= 65536) return -1;
   // Problems by decreasing row-block size.
   int order[kGemvMaxGroup];
   for (int i = 0; i < L.count; ++i) order[i] = i;
@@ -229,14 +229,12 @@ long long plan_gemv_listed(GemvLaunch& L, long long G) {
       }
     }
   }
-  int pos = 0;
   for (long long c = 0; c < G; ++c) {
-    L.cta_begin[c] = static_cast<uint16_t>(pos);
     auto& v = lists[static_cast<size_t>(c)];
     std::sort(v.begin(), v.end());
-    for (uint16_t r : v) L.task[pos++] = r;
+    L.ntask[c] = static_cast<uint8_t>(v.size());
+    for (size_t i = 0; i < v.size(); ++i) L.task[c][i] = v[i];
   }
-  L.cta_begin[G] = static_cast<uint16_t>(pos);
   return worst;
 }
 
@@ -294,18 +292,18 @@ bool gemv_problem_shared(const GemvLaunch& L, int i, long long G) {
   return false;
 }
 
-// nt: token tiles of the launch (the activation box has 8 nt rows).
-bool fill_gemv_problem(GemvProblem& q, const uint8_t* Wp, uint8_t* ws, const FwdWorkspace& L,
-                       const float* s_x, const float* s_w, int64_t M, int64_t N, int64_t K,
-                       void* y, int y_dtype, int32_t* acc_out, int nt) {
+// The activation box has the problem's own token tiles (8 or 16 rows).
+bool fill_gemv_problem(GemvMaps& maps, GemvProblem& q, const uint8_t* Wp, uint8_t* ws,
+                       const FwdWorkspace& L, const float* s_x, const float* s_w, int64_t M,
+                       int64_t N, int64_t K, void* y, int y_dtype, int32_t* acc_out) {
   // One unit = a 64-row x 64-byte weight box and a 256-byte x 8 nt-row
   // activation box; rows past N or M and bytes past K read as zero.
-  if (!make_tmap_u8(&q.tmap_w, Wp, static_cast<uint64_t>(K / 4), static_cast<uint64_t>(N),
+  if (!make_tmap_u8(&maps.tmap_w, Wp, static_cast<uint64_t>(K / 4), static_cast<uint64_t>(N),
                     static_cast<uint64_t>(K / 4), kGemvUnitK / 4, kGemvRows,
                     CU_TENSOR_MAP_SWIZZLE_NONE))
     return false;
-  if (!make_tmap_u8(&q.tmap_x, ws + L.xq, static_cast<uint64_t>(K), static_cast<uint64_t>(M),
-                    static_cast<uint64_t>(K), kGemvUnitK, static_cast<uint32_t>(8 * nt),
+  if (!make_tmap_u8(&maps.tmap_x, ws + L.xq, static_cast<uint64_t>(K), static_cast<uint64_t>(M),
+                    static_cast<uint64_t>(K), kGemvUnitK, M > 8 ? 16u : 8u,
                     CU_TENSOR_MAP_SWIZZLE_NONE))
     return false;
   q.W = Wp;
@@ -372,8 +370,8 @@ bitnet_status launch_gemv(const DeviceState& ds, const uint8_t* Wp, const float*
                           const FwdWorkspace& Lw, void* y, int y_dtype, int32_t* acc_out,
                           bool pdl, bool early_weights, cudaStream_t stream) {
   static thread_local GemvLaunch L;  // ~9 KB: keep it off the stack
-  if (!fill_gemv_problem(L.prob[0], Wp, ws, Lw, s_x, s_w, M, N, K, y, y_dtype, acc_out,
-                         M > 8 ? 2 : 1))
+  if (!fill_gemv_problem(L.maps[0], L.prob[0], Wp, ws, Lw, s_x, s_w, M, N, K, y, y_dtype,
+                         acc_out))
     return BITNET_ERR_CUDA;
   const long long G = plan_gemv_single(ds, L, M, N, K);
   return launch_gemv_group(ds, L, G, pdl, early_weights, stream);
@@ -696,8 +694,8 @@ bitnet_status forward_grouped_impl(int count, const bitnet_linear_problem* probl
     qp.block_begin = qblocks;
     qp.zero_blocks = static_cast<int>(zero ? zero_blocks(zbytes) : 0);
     qblocks += qp.M + qp.zero_blocks;
-    if (!fill_gemv_problem(GL.prob[n], q.W_packed, ws, L, qp.s_x, q.s_w, q.M, q.N, q.K, q.y,
-                           q.y_dtype, nullptr, mmax > 8 ? 2 : 1))
+    if (!fill_gemv_problem(GL.maps[n], GL.prob[n], q.W_packed, ws, L, qp.s_x, q.s_w, q.M, q.N,
+                           q.K, q.y, q.y_dtype, nullptr))
       return BITNET_ERR_CUDA;
     ++n;
   }

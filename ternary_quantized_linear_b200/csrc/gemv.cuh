@@ -16,7 +16,7 @@
 //     when that balances badly, every CTA an equal contiguous share of the
 //     units laid end to end ("stream-K").  The units of a CTA's segment list
 //     are split into eight equal contiguous ranges, one per compute warp.
-//   * Operands move by TMA: each warp has its own ring of kGemvStages stages
+//   * Operands move by TMA: each warp has its own ring of stages (gemv_stages)
 //     and its lane 0 issues, per unit, one 2-D box of weights (64 rows x 64
 //     bytes) and one of activations (the unit's 256 bytes of 8 or 16 token
 //     rows), refilling a stage as soon as the warp has read it.  Eight
@@ -60,18 +60,26 @@ constexpr int kGemvThreads = 32 * kGemvWarps;
 constexpr int kGemvMaxSegs = 6;      // row blocks one CTA's share may touch
 constexpr int kGemvMaxGroup = 16;    // problems per grouped launch
 constexpr uint32_t kCodeMask = 0x03030303u;
-constexpr int kGemvStages = 3;      // ring stages per warp
+constexpr int kGemvStagesMax = 3;
 constexpr int kGemvUnitBytes = kGemvRows * (kGemvUnitK / 4);  // 4 KiB of weights
+// Ring stages per warp: three with one token tile, two with two, so that a
+// decode CTA still fits on an SM beside an activation-quant CTA (the two
+// overlap under programmatic dependent launch).
+__host__ __device__ constexpr int gemv_stages(int nt) { return nt == 1 ? 3 : 2; }
 // A stage: the unit's weights, then its activations (8 or 16 token rows of
 // 256 bytes).
 __host__ __device__ constexpr int gemv_stage_bytes(int nt) { return kGemvUnitBytes + nt * 2048; }
 __host__ __device__ constexpr int gemv_smem_bytes(int nt) {
-  return kGemvWarps * kGemvStages * gemv_stage_bytes(nt) + 1024;  // + alignment slack
+  return kGemvWarps * gemv_stages(nt) * gemv_stage_bytes(nt) + 1024;  // + alignment slack
 }
 
-struct GemvProblem {
+// The copy engine reads these from the kernel parameters.
+struct GemvMaps {
   CUtensorMap tmap_w;     // W_packed [N][K/4] bytes, box 64 x 64 rows, no swizzle
-  CUtensorMap tmap_x;     // x_q [M][K] bytes (decode block order), box 256 x 8*NT rows
+  CUtensorMap tmap_x;     // x_q [M][K] bytes (decode block order), box 256 x 8 or 16 rows
+};
+
+struct GemvProblem {
   const uint8_t* W;       // W_packed [N][K/4]
   const int8_t* xq;       // x_q k-interleaved [M][K]
   const int32_t* rowsum;  // [M]
@@ -89,10 +97,10 @@ struct GemvProblem {
   int rb_begin;           // first row block of this problem in the launch
 };
 
-constexpr int kGemvMaxCtas = 1024;   // CTAs of a launch with an explicit row-block list
-constexpr int kGemvMaxTasks = 2048;  // row blocks of such a launch
+constexpr int kGemvMaxCtas = 296;    // CTAs of a launch with an explicit row-block list
 
 struct GemvLaunch {
+  GemvMaps maps[kGemvMaxGroup];
   GemvProblem prob[kGemvMaxGroup];
   long long units;        // total units of the launch
   int count;              // problems in this launch
@@ -100,10 +108,10 @@ struct GemvLaunch {
   int early_weights;      // start the weight copies before that wait
   int* status;            // device status word (bounded waits)
   uint64_t wait_limit_ns;
-  int listed;             // 1: CTA b owns row blocks task[cta_begin[b] .. cta_begin[b+1])
+  int listed;             // 1: CTA b owns row blocks task[b][0 .. ntask[b])
                           // 0: CTA b owns units [b U / G, (b+1) U / G)
-  uint16_t cta_begin[kGemvMaxCtas + 1];
-  uint16_t task[kGemvMaxTasks];  // global row block ids
+  uint8_t ntask[kGemvMaxCtas];
+  uint16_t task[kGemvMaxCtas][kGemvMaxSegs];  // global row block ids
 };
 
 template <int NT>
@@ -259,7 +267,7 @@ ternary_gemv_kernel(const __grid_constant__ GemvLaunch L) {
   uint8_t* ring = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(gemv_smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   __shared__ int red[kGemvMaxSegs * kGemvRows * 16];  // [segment][row][token]
-  __shared__ __align__(8) uint64_t full[kGemvWarps][kGemvStages];
+  __shared__ __align__(8) uint64_t full[kGemvWarps][kGemvStagesMax];
   // The problem table and this CTA's segments live in shared memory: the
   // walk indexes them by run-time numbers, which kernel-parameter space
   // serves slowly (the copy engine still reads the tensor maps from the
@@ -280,28 +288,32 @@ ternary_gemv_kernel(const __grid_constant__ GemvLaunch L) {
   const int count = L.count;
   const uint64_t limit = L.wait_limit_ns;
   if (tid < count) sprob[tid] = L.prob[tid];
-  if (tid < kGemvWarps * kGemvStages) mbar_init(&full[0][0] + tid, 1);
+  if (tid < kGemvWarps * kGemvStagesMax) mbar_init(&full[0][0] + tid, 1);
   if (tid == 0) {
     abort_flag = 0;
     fence_mbarrier_init();
   }
   __syncthreads();
   const GemvProblem* prob = sprob;
-  if (tid == 0) {
-    int n = 0;
-    if (L.listed) {
-      const int t0 = L.cta_begin[b], t1 = L.cta_begin[b + 1];
-      for (int i = t0; i < t1 && n < kGemvMaxSegs; ++i, ++n) {
-        const int R = L.task[i];
+  if (L.listed) {
+    // One thread per listed row block: the parameter reads go out together.
+    if (tid < kGemvMaxSegs) {
+      const int n = L.ntask[b];
+      if (tid == 0) seg_count = n;
+      if (tid < n) {
+        const int R = L.task[b][tid];
         int p = 0;
         while (p + 1 < count && R >= prob[p + 1].rb_begin) ++p;
-        seg_p[n] = p;
-        seg_rbl[n] = R - prob[p].rb_begin;
-        seg_lo[n] = 0;
-        seg_n[n] = prob[p].kc;
-        seg_owned[n] = 1;
+        seg_p[tid] = p;
+        seg_rbl[tid] = R - prob[p].rb_begin;
+        seg_lo[tid] = 0;
+        seg_n[tid] = prob[p].kc;
+        seg_owned[tid] = 1;
       }
-    } else if (ub < ue) {
+    }
+  } else if (tid == 0) {
+    int n = 0;
+    if (ub < ue) {
       int p = 0;
       const GemvUnit first = gemv_unit(prob, count, ub, p);
       const GemvUnit last = gemv_unit(prob, count, ue - 1, p);
@@ -341,21 +353,36 @@ ternary_gemv_kernel(const __grid_constant__ GemvLaunch L) {
       ++x.s;
     }
   };
-  // Warp w takes the w-th of eight equal contiguous ranges of the CTA's
-  // units.
-  int n_units = 0;
-  for (int i = 0; i < nseg; ++i) n_units += seg_n[i];
+  // Warp w takes the w-th of eight contiguous ranges of the CTA's units, of
+  // equal cost: a unit of a problem with two token tiles counts 3, one with
+  // one tile 2 (the MMA work is half again as large).
+  auto unit_cost = [&](int sg) { return prob[seg_p[sg]].M > 8 ? 3 : 2; };
+  int total_cost = 0;
+  for (int i = 0; i < nseg; ++i) total_cost += seg_n[i] * unit_cost(i);
+  // First unit (as a count of units before it) whose cost prefix reaches c.
+  auto unit_at = [&](int c) {
+    int u = 0;
+    for (int i = 0; i < nseg; ++i) {
+      const int w = unit_cost(i), segc = seg_n[i] * w;
+      if (c <= segc) return u + (c + w - 1) / w;
+      c -= segc;
+      u += seg_n[i];
+    }
+    return u;
+  };
   auto range_of = [&](int w, Cursor& x0) {
-    const int u0 = w * n_units / kGemvWarps;
+    const int u0 = unit_at(w * total_cost / kGemvWarps);
+    const int u1 = unit_at((w + 1) * total_cost / kGemvWarps);
     x0 = Cursor{0, 0};
     advance(x0, u0);
-    return (w + 1) * n_units / kGemvWarps - u0;
+    return u1 - u0;
   };
 
   // Warp w streams its range through its own ring: lane 0 issues the copies
   // (weights as soon as the CTA starts, activations once the preceding grid
   // is done), all lanes consume.
   constexpr int kStage = gemv_stage_bytes(NT);
+  constexpr int kGemvStages = gemv_stages(NT);
   uint8_t* myring = ring + warp * kGemvStages * kStage;
   Cursor xA;
   const int n = range_of(warp, xA);
@@ -364,13 +391,14 @@ ternary_gemv_kernel(const __grid_constant__ GemvLaunch L) {
   auto issue_w = [&](int j) {  // lane 0: unit j (cursor xI) weights into stage j % S
     const int st = j % kGemvStages;
     const int p = seg_p[xI.s];
-    mbar_arrive_expect_tx(&full[warp][st], kStage);
-    tma_load_2d(myring + st * kStage, &L.prob[p].tmap_w, (seg_lo[xI.s] + xI.off) * (kGemvUnitK / 4),
+    // The activation box has 8 or 16 rows: the problem's own token tiles.
+    mbar_arrive_expect_tx(&full[warp][st], kGemvUnitBytes + (prob[p].M > 8 ? 4096 : 2048));
+    tma_load_2d(myring + st * kStage, &L.maps[p].tmap_w, (seg_lo[xI.s] + xI.off) * (kGemvUnitK / 4),
                 seg_rbl[xI.s] * kGemvRows, &full[warp][st]);
   };
   auto issue_x = [&](int j, const Cursor& x) {
     const int st = j % kGemvStages;
-    tma_load_2d(myring + st * kStage + kGemvUnitBytes, &L.prob[seg_p[x.s]].tmap_x,
+    tma_load_2d(myring + st * kStage + kGemvUnitBytes, &L.maps[seg_p[x.s]].tmap_x,
                 (seg_lo[x.s] + x.off) * kGemvUnitK, 0, &full[warp][st]);
   };
   const int pre = min(n, kGemvStages);
