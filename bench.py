@@ -29,10 +29,11 @@ METRIC = "BitLinear fwd: decode HBM GB/s & tok/s, prefill int8 TOPS (% of B200 p
 WORKLOAD = "decode_bitnet3b"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
-# DRAM traffic per GEMV launch from an ncu capture of this workload (bytes,
-# averaged over the nine problems), valid only for the kernel source it was
-# measured on (sha256 of csrc/gemv.cuh); None until measured.
-GEMV_TRAFFIC = {"src_sha256": None, "bytes_per_launch": None}
+# DRAM bytes (read + write) of one grouped GEMV launch of this workload from
+# an ncu capture (summary under profiles/), valid only for the kernel source
+# it was measured on (sha256 of csrc/gemv.cuh); reported as null otherwise.
+GEMV_TRAFFIC = {"src_sha256": "b9e8b916d1ea9e52ddd205c6a91647a872128d6a5ee73d25747b8c4b7a85a262",
+                "bytes_per_launch": 49548032}
 
 
 # ------------------------------------------------------------------ helpers
@@ -334,25 +335,35 @@ def run_ours(args):
     launches = 2 * args.steps
 
     # ---- kernel durations with CUDA events: the grouped matmul (dominant
-    # kernel) and the grouped activation quant, launched as separate phases
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(R)]
-    q_ms, m_ms = [], []
-    with torch.cuda.stream(stream):
-        sp = P(stream.cuda_stream)
-        for i in range(args.steps + args.warmup):
-            r = i % R
-            torch.cuda._sleep(1_000_000)  # queue the step while the GPU is busy
-            evs[r][0].record(stream)
-            grouped(r, sp, tql.BITNET_PHASE_QUANTIZE)
-            evs[r][1].record(stream)
-            grouped(r, sp, tql.BITNET_PHASE_MATMUL)
-            evs[r][2].record(stream)
+    # kernel) and the grouped activation quant, each captured alone as CUDA
+    # graphs over the rotation sets (the matmul phase reads the activations
+    # the full steps above left in each set's workspace) and replayed
+    # back to back: the average launch duration in a steady stream.
+    def phase_ms(phases):
+        gs = []
+        with torch.cuda.stream(stream):
+            for r in range(R):
+                g = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(g, stream=stream):
+                    grouped(r, P(torch.cuda.current_stream().cuda_stream), phases)
+                gs.append(g)
+            for i in range(args.warmup):
+                gs[i % R].replay()
             stream.synchronize()
-            if i >= args.warmup:
-                q_ms.append(evs[r][0].elapsed_time(evs[r][1]))
-                m_ms.append(evs[r][1].elapsed_time(evs[r][2]))
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            for i in range(args.steps):
+                gs[i % R].replay()
+            b.record(stream)
+            stream.synchronize()
+        ms = a.elapsed_time(b) / args.steps
+        del gs
+        return ms
+
+    m_avg = phase_ms(tql.BITNET_PHASE_MATMUL)
+    q_avg = phase_ms(tql.BITNET_PHASE_QUANTIZE)
     gemv_b = sum(gemv_bytes(M, N, K) for _, K, N, M in probs)
-    m_avg = statistics.mean(m_ms)
     peaks, peak_src = load_peaks()
     hbm_peak = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
     achieved = gemv_b / (m_avg * 1e-3) / 1e9
@@ -394,7 +405,9 @@ def run_ours(args):
                 "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)",
                 "algorithmic_bytes_per_launch": gemv_b,
                 "avg_launch_us": round(1e3 * m_avg, 2),
-                "quant_kernel_us": round(1e3 * statistics.mean(q_ms), 2),
+                "quant_kernel_us": round(1e3 * q_avg, 2),
+                "how": "CUDA events around back-to-back CUDA-graph replays of the matmul "
+                       "phase alone (6 rotating weight sets), average per launch",
                 "single_problem_launches": single}
 
     # ---- end to end through the public call with host buffers
