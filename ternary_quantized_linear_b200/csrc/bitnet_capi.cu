@@ -381,14 +381,19 @@ struct GemmPlan {
   int BN, rb, tb, ksplit, steps_per_split;
 };
 
-// Token tile BN from M; K is split across CTAs only for small M (then the
-// int32 partials go through the workspace), to give every SM work.
+// Token tile BN from M (and K: above 128 tokens, 128-token tiles two per
+// SM while K <= 8192 or M <= 1024, where per-tile pipeline fill and
+// epilogue dominate; 256-token tiles otherwise -- measured on the prefill
+// shapes).  K is
+// split across CTAs only for small M (then the int32 partials go through the
+// workspace), to give every SM work.
 GemmPlan plan_gemm(int64_t M, int64_t N, int64_t K, int num_sms) {
   GemmPlan pl{};
-  pl.BN = M <= 16 ? 16 : (M <= 32 ? 32 : (M <= 64 ? 64 : (M <= 128 ? 128 : 256)));
+  pl.BN = M <= 16 ? 16
+        : (M <= 32 ? 32 : (M <= 64 ? 64 : (M <= 1024 || K <= 8192 ? 128 : 256)));
   pl.rb = static_cast<int>((N + 127) / 128);
   pl.tb = static_cast<int>((M + pl.BN - 1) / pl.BN);
-  const bool small = pl.BN <= 64;            // GemmCfg<BN>::SMALL
+  const bool small = pl.BN <= 128;           // GemmCfg<BN>::TWO_PER_SM
   const int kstep = 256;                      // GemmCfg<BN>::KSTEP
   const int steps = static_cast<int>((K + kstep - 1) / kstep);
   int ks = 1;

@@ -65,25 +65,29 @@ struct GemmCfg {
   static constexpr bool SMALL = BN <= 64;        // decode-sized token tile
   // 256 k per pipeline step: each TMA weight box has 64-byte rows (narrower
   // rows starve the copy engine) and each step issues 8 MMAs, amortising the
-  // per-step barrier traffic.  Small token tiles are bound by the MMA issue
-  // rate (a fixed cost per instruction), so two CTAs share each SM to
-  // interleave their MMA streams; large tiles are tensor-bound, one CTA/SM.
+  // per-step barrier traffic.  Token tiles up to 128 run two CTAs per SM:
+  // small tiles are bound by the MMA issue rate (a fixed cost per
+  // instruction) and interleave two MMA streams; 128-token tiles overlap one
+  // CTA's pipeline fill and epilogue with the other's main loop (the host
+  // picks them for short K, where those per-tile costs dominate); 256-token
+  // tiles are tensor-bound, one CTA/SM.
   static constexpr int KSTEP = 256;
   static constexpr int ATOMS = KSTEP / 128;      // 128-byte swizzle atoms per activation tile
   static constexpr int X_ATOM = BN * 128;        // bytes of one activation atom
   static constexpr int X_BYTES = BN * KSTEP;     // activation tile
   static constexpr int WP_ROW = KSTEP / 4;       // packed bytes per weight row per step
   static constexpr int WP_BYTES = BM * WP_ROW;   // packed weight tile
-  static constexpr int STAGES = BN <= 16 ? 8 : (BN <= 32 ? 6 : (BN <= 64 ? 4 : (BN <= 128 ? 5 : 3)));
+  static constexpr bool TWO_PER_SM = BN <= 128;
+  static constexpr int STAGES = BN <= 16 ? 8 : (BN <= 32 ? 6 : (BN <= 64 ? 4 : (BN <= 128 ? 2 : 3)));
   // TMEM: A_STAGES stages of KSTEP/4 columns of unpacked weights (four int8
   // k per 32-bit column, one lane per weight row), then BN int32 accumulator
   // columns.
   static constexpr int A_COLS = KSTEP / 4;
-  static constexpr int A_STAGES = SMALL ? 3 : STAGES;
+  static constexpr int A_STAGES = SMALL ? 3 : (TWO_PER_SM ? 2 : STAGES);
   static constexpr uint32_t A_COL = 0;
   static constexpr uint32_t D_COL = A_COLS * A_STAGES;
-  static constexpr uint32_t TMEM_COLS = SMALL ? 256 : 512;
-  static constexpr int MIN_BLOCKS = SMALL ? 2 : 1;
+  static constexpr uint32_t TMEM_COLS = TWO_PER_SM ? 256 : 512;
+  static constexpr int MIN_BLOCKS = TWO_PER_SM ? 2 : 1;
   static constexpr int UNPACK_WARPS = 8;         // two per TMEM lane quarter
   static constexpr int THREADS = 128 + 32 * UNPACK_WARPS;
   static constexpr int PART = WP_ROW / 2;        // packed bytes per unpack thread per step
