@@ -222,8 +222,13 @@ BITNET_API bitnet_status bitnet_linear_matmul(const uint8_t *W_packed, const flo
  * each problem in order, but the decode problems (M <= 16) share one
  * activation-quant launch and one matmul launch, so their weight streams
  * overlap instead of paying one launch latency each.  Typical use: the
- * projections of one decode step (q, k, v, o, gate, up, down).  Problems
- * with M > 16 run afterwards on the tcgen05 kernel, one at a time.
+ * projections of one decode step (q, k, v, o, gate, up, down).  Decode
+ * problems with the same x, x_dtype, gamma, eps, M and K (q/k/v, gate/up)
+ * share one activation quantization.  The host-side plan of a call is
+ * cached per thread (a few entries, keyed by every field of every problem
+ * and the workspace), so a decode loop that repeats the same call plans it
+ * once.  Problems with M > 16 run afterwards on the tcgen05 kernel, one at a
+ * time.
  *
  *   count      0 <= count <= BITNET_MAX_GROUP.
  *   problems   host array of `count` problem descriptions (each field as in

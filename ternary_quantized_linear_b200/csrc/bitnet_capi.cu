@@ -11,6 +11,7 @@
 
 #include <algorithm>
 #include <cstdint>
+#include <cstring>
 #include <mutex>
 #include <vector>
 
@@ -293,22 +294,26 @@ bool gemv_problem_shared(const GemvLaunch& L, int i, long long G) {
 }
 
 // The activation box has the problem's own token tiles (8 or 16 rows).
-bool fill_gemv_problem(GemvMaps& maps, GemvProblem& q, const uint8_t* Wp, uint8_t* ws,
-                       const FwdWorkspace& L, const float* s_x, const float* s_w, int64_t M,
-                       int64_t N, int64_t K, void* y, int y_dtype, int32_t* acc_out) {
+// xws / xL: the workspace holding this problem's quantized activations (its
+// own, or that of an earlier problem of the launch with the same input);
+// ws / L: its own workspace (split-K partials).
+bool fill_gemv_problem(GemvMaps& maps, GemvProblem& q, const uint8_t* Wp, uint8_t* xws,
+                       const FwdWorkspace& xL, uint8_t* ws, const FwdWorkspace& L,
+                       const float* s_x, const float* s_w, int64_t M, int64_t N, int64_t K,
+                       void* y, int y_dtype, int32_t* acc_out) {
   // One unit = a 64-row x 64-byte weight box and a 256-byte x 8 nt-row
   // activation box; rows past N or M and bytes past K read as zero.
   if (!make_tmap_u8(&maps.tmap_w, Wp, static_cast<uint64_t>(K / 4), static_cast<uint64_t>(N),
                     static_cast<uint64_t>(K / 4), kGemvUnitK / 4, kGemvRows,
                     CU_TENSOR_MAP_SWIZZLE_NONE))
     return false;
-  if (!make_tmap_u8(&maps.tmap_x, ws + L.xq, static_cast<uint64_t>(K), static_cast<uint64_t>(M),
+  if (!make_tmap_u8(&maps.tmap_x, xws + xL.xq, static_cast<uint64_t>(K), static_cast<uint64_t>(M),
                     static_cast<uint64_t>(K), kGemvUnitK, M > 8 ? 16u : 8u,
                     CU_TENSOR_MAP_SWIZZLE_NONE))
     return false;
   q.W = Wp;
-  q.xq = reinterpret_cast<const int8_t*>(ws + L.xq);
-  q.rowsum = reinterpret_cast<const int32_t*>(ws + L.rs);
+  q.xq = reinterpret_cast<const int8_t*>(xws + xL.xq);
+  q.rowsum = reinterpret_cast<const int32_t*>(xws + xL.rs);
   q.s_x = s_x;
   q.s_w = s_w;
   q.y = y;
@@ -370,7 +375,7 @@ bitnet_status launch_gemv(const DeviceState& ds, const uint8_t* Wp, const float*
                           const FwdWorkspace& Lw, void* y, int y_dtype, int32_t* acc_out,
                           bool pdl, bool early_weights, cudaStream_t stream) {
   static thread_local GemvLaunch L;  // ~9 KB: keep it off the stack
-  if (!fill_gemv_problem(L.maps[0], L.prob[0], Wp, ws, Lw, s_x, s_w, M, N, K, y, y_dtype,
+  if (!fill_gemv_problem(L.maps[0], L.prob[0], Wp, ws, Lw, ws, Lw, s_x, s_w, M, N, K, y, y_dtype,
                          acc_out))
     return BITNET_ERR_CUDA;
   const long long G = plan_gemv_single(ds, L, M, N, K);
@@ -632,6 +637,151 @@ size_t grouped_workspace(int count, const bitnet_linear_problem* problems) {
   return total;
 }
 
+// The launches of the decode problems of one grouped call.
+struct DecodePlan {
+  bool valid = false;
+  int dev = -1;
+  int count = 0;
+  uint8_t* ws = nullptr;
+  size_t ws_bytes = 0;
+  bitnet_linear_problem probs[BITNET_MAX_GROUP];
+  QuantLaunch QL;
+  GemvLaunch GL;
+  long long G = 0;
+  int n = 0;        // decode problems
+  int qblocks = 0;  // blocks of the quant launch
+  uint32_t stage = 0;
+};
+
+constexpr int kPlanCacheSize = 8;
+thread_local DecodePlan g_plans[kPlanCacheSize];
+thread_local int g_plan_next = 0;
+
+bool same_problem(const bitnet_linear_problem& a, const bitnet_linear_problem& b) {
+  return a.x == b.x && a.x_dtype == b.x_dtype && a.gamma == b.gamma &&
+         std::memcmp(&a.eps, &b.eps, sizeof(float)) == 0 && a.W_packed == b.W_packed &&
+         a.s_w == b.s_w && a.M == b.M && a.N == b.N && a.K == b.K && a.y == b.y &&
+         a.y_dtype == b.y_dtype;
+}
+
+// Whether problems a and b quantize the same activations identically.
+bool same_input(const bitnet_linear_problem& a, const bitnet_linear_problem& b) {
+  return a.x == b.x && a.x_dtype == b.x_dtype && a.gamma == b.gamma &&
+         std::memcmp(&a.eps, &b.eps, sizeof(float)) == 0 && a.M == b.M && a.K == b.K;
+}
+
+DecodePlan* cached_decode_plan(int count, const bitnet_linear_problem* problems, uint8_t* ws,
+                               size_t ws_bytes) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) return nullptr;
+  for (DecodePlan& p : g_plans) {
+    if (!p.valid || p.dev != dev || p.count != count || p.ws != ws || p.ws_bytes != ws_bytes)
+      continue;
+    bool same = true;
+    for (int i = 0; i < count && same; ++i) same = same_problem(p.probs[i], problems[i]);
+    if (same) return &p;
+  }
+  return nullptr;
+}
+
+DecodePlan* new_decode_plan_slot(int count, const bitnet_linear_problem* problems, uint8_t* ws,
+                                 size_t ws_bytes) {
+  DecodePlan& p = g_plans[g_plan_next];
+  g_plan_next = (g_plan_next + 1) % kPlanCacheSize;
+  p.valid = false;
+  if (cudaGetDevice(&p.dev) != cudaSuccess) p.dev = -1;
+  p.count = count;
+  p.ws = ws;
+  p.ws_bytes = ws_bytes;
+  for (int i = 0; i < count; ++i) p.probs[i] = problems[i];
+  return &p;
+}
+
+// Plans the decode problems (M <= 16) of a grouped call: the matmul's work
+// split, which partial regions the quant launch must clear, and one quant
+// entry per distinct input (problems with the same x, dtype, gamma, eps, M
+// and K share one quantization -- e.g. q/k/v or gate/up of one token batch).
+bool build_decode_plan(const DeviceState& ds, int count, const bitnet_linear_problem* problems,
+                       uint8_t* base, DecodePlan& plan) {
+  QuantLaunch& QL = plan.QL;
+  GemvLaunch& GL = plan.GL;
+  QL = QuantLaunch{};
+  GL.count = 0;
+  // First pass: the matmul plan (it decides which partial regions need
+  // zeroing by the quant launch).
+  int n = 0, mmax = 0;
+  for (int i = 0; i < count; ++i) {
+    const bitnet_linear_problem& q = problems[i];
+    if (q.M == 0 || q.M > kGemvMaxM) continue;
+    GL.prob[n].M = static_cast<int>(q.M);
+    GL.prob[n].N = static_cast<int>(q.N);
+    GL.prob[n].K = static_cast<int>(q.K);
+    mmax = std::max(mmax, static_cast<int>(q.M));
+    ++n;
+  }
+  GL.count = n;
+  plan.n = n;
+  plan.G = n > 0 ? plan_gemv_launch(GL, gemv_capacity(ds, mmax)) : 0;
+  int qblocks = 0, qn = 0;
+  uint32_t stage = 0;
+  size_t off = 0;
+  int src[BITNET_MAX_GROUP];            // problem index of each decode problem
+  uint8_t* qws[BITNET_MAX_GROUP];       // its quantized-activation workspace
+  FwdWorkspace qL[BITNET_MAX_GROUP];
+  n = 0;
+  for (int i = 0; i < count; ++i) {
+    const bitnet_linear_problem& q = problems[i];
+    if (q.M == 0) continue;
+    const FwdWorkspace L = fwd_layout(q.M, q.N, q.K);
+    uint8_t* ws = base + off;
+    off += L.total;
+    if (q.M > kGemvMaxM) continue;
+    const bool shared_rows = gemv_problem_shared(GL, n, plan.G);
+    int owner = -1;
+    if (!shared_rows)
+      for (int j = 0; j < n && owner < 0; ++j)
+        if (same_input(problems[src[j]], q)) owner = j;
+    src[n] = i;
+    if (owner >= 0) {
+      // Reuse that problem's quantization.
+      qws[n] = qws[owner];
+      qL[n] = qL[owner];
+    } else {
+      qws[n] = ws;
+      qL[n] = L;
+      size_t zbytes = 0;
+      void* zero = shared_rows ? splitk_region(ws, L, &zbytes) : nullptr;
+      QuantProblem& qp = QL.prob[qn++];
+      qp.x = q.x;
+      qp.gamma = q.gamma;
+      qp.xi = reinterpret_cast<int8_t*>(ws + L.xq);
+      qp.s_x = reinterpret_cast<float*>(ws + L.sx);
+      qp.rowsum = reinterpret_cast<int32_t*>(ws + L.rs);
+      qp.zero16 = static_cast<uint4*>(zero);
+      qp.n_zero16 = zero ? static_cast<int64_t>(zbytes / 16) : 0;
+      qp.eps = q.eps;
+      qp.M = static_cast<int>(q.M);
+      qp.K = static_cast<int>(q.K);
+      qp.x_bf16 = (q.x_dtype == BITNET_BF16) ? 1 : 0;
+      qp.perm = 1;  // decode matmul
+      qp.block_begin = qblocks;
+      qp.zero_blocks = static_cast<int>(zero ? zero_blocks(zbytes) : 0);
+      qblocks += qp.M + qp.zero_blocks;
+      stage = std::max(stage, quant_stage_bytes(q.K, qp.x_bf16 != 0, q.gamma != nullptr));
+    }
+    const float* sx = reinterpret_cast<const float*>(qws[n] + qL[n].sx);
+    if (!fill_gemv_problem(GL.maps[n], GL.prob[n], q.W_packed, qws[n], qL[n], ws, L, sx, q.s_w,
+                           q.M, q.N, q.K, q.y, q.y_dtype, nullptr))
+      return false;
+    ++n;
+  }
+  QL.count = qn;
+  plan.qblocks = qblocks;
+  plan.stage = stage;
+  plan.valid = true;
+  return true;
+}
+
 bitnet_status forward_grouped_impl(int count, const bitnet_linear_problem* problems,
                                    void* workspace, size_t workspace_bytes, int phases,
                                    cudaStream_t stream) {
@@ -652,71 +802,26 @@ bitnet_status forward_grouped_impl(int count, const bitnet_linear_problem* probl
   if (!ds) return BITNET_ERR_CUDA;
   uint8_t* base = static_cast<uint8_t*>(workspace);
 
-  // Decode problems: one grouped quant launch, one grouped matmul launch.
-  static thread_local QuantLaunch QL;
-  static thread_local GemvLaunch GL;
-  QL = QuantLaunch{};
-  GL.count = 0;
-  // First pass: the matmul plan (it decides which partial regions need
-  // zeroing by the quant launch).
-  int n = 0, mmax = 0;
-  for (int i = 0; i < count; ++i) {
-    const bitnet_linear_problem& q = problems[i];
-    if (q.M == 0 || q.M > kGemvMaxM) continue;
-    GL.prob[n].M = static_cast<int>(q.M);
-    GL.prob[n].N = static_cast<int>(q.N);
-    GL.prob[n].K = static_cast<int>(q.K);
-    mmax = std::max(mmax, static_cast<int>(q.M));
-    ++n;
-  }
-  GL.count = n;
-  const long long G = n > 0 ? plan_gemv_launch(GL, gemv_capacity(*ds, mmax)) : 0;
-  int qblocks = 0;
-  size_t off = 0;
-  n = 0;
-  for (int i = 0; i < count; ++i) {
-    const bitnet_linear_problem& q = problems[i];
-    if (q.M == 0) continue;
-    const FwdWorkspace L = fwd_layout(q.M, q.N, q.K);
-    uint8_t* ws = base + off;
-    off += L.total;
-    if (q.M > kGemvMaxM) continue;
-    size_t zbytes = 0;
-    void* zero = gemv_problem_shared(GL, n, G) ? splitk_region(ws, L, &zbytes) : nullptr;
-    QuantProblem& qp = QL.prob[n];
-    qp.x = q.x;
-    qp.gamma = q.gamma;
-    qp.xi = reinterpret_cast<int8_t*>(ws + L.xq);
-    qp.s_x = reinterpret_cast<float*>(ws + L.sx);
-    qp.rowsum = reinterpret_cast<int32_t*>(ws + L.rs);
-    qp.zero16 = static_cast<uint4*>(zero);
-    qp.n_zero16 = zero ? static_cast<int64_t>(zbytes / 16) : 0;
-    qp.eps = q.eps;
-    qp.M = static_cast<int>(q.M);
-    qp.K = static_cast<int>(q.K);
-    qp.x_bf16 = (q.x_dtype == BITNET_BF16) ? 1 : 0;
-    qp.perm = 1;  // decode matmul
-    qp.block_begin = qblocks;
-    qp.zero_blocks = static_cast<int>(zero ? zero_blocks(zbytes) : 0);
-    qblocks += qp.M + qp.zero_blocks;
-    if (!fill_gemv_problem(GL.maps[n], GL.prob[n], q.W_packed, ws, L, qp.s_x, q.s_w, q.M, q.N,
-                           q.K, q.y, q.y_dtype, nullptr))
+  // Decode problems: one grouped quant launch, one grouped matmul launch,
+  // planned once per distinct problem set (the plan is cached per thread).
+  DecodePlan* plan = cached_decode_plan(count, problems, base, workspace_bytes);
+  if (!plan) {
+    plan = new_decode_plan_slot(count, problems, base, workspace_bytes);
+    if (!build_decode_plan(*ds, count, problems, base, *plan)) {
+      plan->valid = false;
       return BITNET_ERR_CUDA;
-    ++n;
+    }
   }
-  if (n > 0) {
-    QL.count = n;
+  if (plan->n > 0) {
+    QuantLaunch& QL = plan->QL;
+    GemvLaunch& GL = plan->GL;
     QL.trigger_dependents = do_matmul ? 1 : 0;
-    if (do_quant) {
-      uint32_t stage = 0;
-      for (int i = 0; i < n; ++i)
-        stage = std::max(stage, quant_stage_bytes(QL.prob[i].K, QL.prob[i].x_bf16 != 0,
-                                                  QL.prob[i].gamma != nullptr));
+    if (do_quant && QL.count > 0) {
       QL.status = ds->status;
       QL.wait_limit_ns = kWaitLimitNs;
-      const dim3 qg(static_cast<unsigned>(qblocks));
-      if (stage <= kQuantStageMax)
-        rmsnorm_quant_grouped_kernel<true><<<qg, kActThreads, stage, stream>>>(QL);
+      const dim3 qg(static_cast<unsigned>(plan->qblocks));
+      if (plan->stage <= kQuantStageMax)
+        rmsnorm_quant_grouped_kernel<true><<<qg, kActThreads, plan->stage, stream>>>(QL);
       else
         rmsnorm_quant_grouped_kernel<false><<<qg, kActThreads, 0, stream>>>(QL);
       const bitnet_status st = launch_status();
@@ -725,13 +830,13 @@ bitnet_status forward_grouped_impl(int count, const bitnet_linear_problem* probl
     if (do_matmul) {
       // When the quant grid was just queued it started after every earlier
       // write to the weights, so the loads may begin before waiting on it.
-      const bitnet_status st = launch_gemv_group(*ds, GL, G, true, do_quant, stream);
+      const bitnet_status st = launch_gemv_group(*ds, GL, plan->G, true, do_quant, stream);
       if (st != BITNET_OK) return st;
     }
   }
   if (!do_matmul) return BITNET_OK;
   // Larger problems: the tcgen05 kernel, one after another.
-  off = 0;
+  size_t off = 0;
   for (int i = 0; i < count; ++i) {
     const bitnet_linear_problem& q = problems[i];
     if (q.M == 0) continue;

@@ -347,3 +347,47 @@ def test_grouped_rejects_bad_problem_and_queues_nothing():
         tql.bitnet_linear_forward_grouped(bad)
     torch.cuda.synchronize()
     assert all(int(it[5].count_nonzero()) == 0 for it in items)
+
+
+@pytest.mark.parametrize("M", [1, 13])
+def test_grouped_shared_input_and_repeated_calls(M):
+    # q/k/v- and gate/up-style problems read the same x (one quantization is
+    # shared); the call is repeated with the same problems (cached plan) and
+    # then with new output buffers (a different plan): every result must be
+    # the single-call result.
+    rng = np.random.default_rng(77 + M)
+    K = 1024
+    x = x_to_device(workloads._to_bf16_bits(rng.standard_normal((M, K)).astype(np.float32)))
+    x2 = x_to_device(workloads._to_bf16_bits(rng.standard_normal((M, K)).astype(np.float32)))
+    gamma = torch.from_numpy(workloads.random_gamma(K)).cuda()
+    mats = []
+    for N in (1024, 256, 256, 2816, 2816):
+        W = (rng.standard_normal((N, K)) * 0.02).astype(np.float32)
+        mats.append(_dev_weights(W))
+
+    def items_for(outs):
+        its = []
+        for j, ((W_p, s_w), y) in enumerate(zip(mats, outs)):
+            xin, g = (x, gamma) if j < 3 else (x2, None)
+            its.append((xin, g, 1e-5, W_p, s_w, y))
+        return its
+
+    def fresh():
+        return [torch.empty((M, W_p.shape[0]), dtype=torch.bfloat16, device="cuda")
+                for W_p, _ in mats]
+
+    ys = fresh()
+    ws = torch.empty(1 << 24, dtype=torch.uint8, device="cuda")
+    for _ in range(2):
+        for y in ys:
+            y.fill_(0)
+        tql.bitnet_linear_forward_grouped(items_for(ys), workspace=ws)
+    ys2 = fresh()
+    tql.bitnet_linear_forward_grouped(items_for(ys2), workspace=ws)
+    torch.cuda.synchronize()
+    for j, (W_p, s_w) in enumerate(mats):
+        xin, g = (x, gamma) if j < 3 else (x2, None)
+        y1 = tql.bitnet_linear_forward(xin, g, 1e-5, W_p, s_w, y_dtype=torch.bfloat16)
+        torch.cuda.synchronize()
+        assert torch.equal(ys[j].view(torch.int16), y1.view(torch.int16))
+        assert torch.equal(ys2[j].view(torch.int16), y1.view(torch.int16))
