@@ -164,13 +164,13 @@ class ClockSampler:
 
 # --------------------------------------------------------------- CPU oracle
 
-def time_oracle(probs, budget_s, max_steps=None, per_problem=False):
+def time_oracle(probs, budget_s, max_steps=None, per_problem=False, threads=1):
     """Run the CPU oracle over the workload: whole steps (or single problems,
-    cycling, when per_problem) until budget_s is spent.  Returns
-    (bytes, seconds, units, threads)."""
+    cycling, when per_problem) until budget_s is spent, its integer matmul on
+    `threads` threads.  Returns (bytes, seconds, units, threads in effect)."""
     import oracle
     from ternary_quantized_linear_b200 import workloads
-    threads = oracle.set_threads(1)
+    threads = oracle.set_threads(threads)
     case = workloads.CASE_BY_NAME[WORKLOAD]
     prepared = []
     wcache = {}
@@ -490,6 +490,12 @@ def run_ours(args):
         cpu = {"value": b / s / 1e9, "unit": "GB/s", "cores": threads, "kind": "oracle",
                "sample": f"{units} full decode step(s) (all nine problems) of the plain C "
                          f"oracle, {threads} thread(s), {s:.1f} s"}
+        # the same oracle with its integer matmul spread over every host core
+        ncores = os.cpu_count() or 1
+        b, s, units, threads = time_oracle(probs, args.cpu_budget / 2, threads=ncores)
+        cpu["all_cores"] = {"value": b / s / 1e9, "unit": "GB/s", "cores": threads,
+                            "sample": f"{units} full decode step(s), integer matmul on "
+                                      f"{threads} thread(s), {s:.1f} s"}
 
     if world > 1:
         import torch.distributed as dist
