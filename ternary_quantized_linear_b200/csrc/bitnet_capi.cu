@@ -187,9 +187,9 @@ bool ok_dtype(int d) { return d == BITNET_F32 || d == BITNET_BF16; }
 // the workspace, a fence, a counter, a read-back), in 4 KiB units per CTA.
 constexpr long long kGemvSplitPenaltyUnits = 24;
 
-// Relative time of one unit: two token tiles take about half again as long
-// as one (measured on the decode shapes).
-long long gemv_unit_cost(const GemvProblem& P) { return P.M > 8 ? 3 : 2; }
+// Relative time of one unit: two token tiles take about 1.2 times as long as
+// one (fitted to in-kernel timestamps of the decode shapes).
+long long gemv_unit_cost(const GemvProblem& P) { return P.M > 8 ? 6 : 5; }
 
 // Deal whole row blocks, largest first, to the least-loaded CTA (at most
 // kGemvMaxSegs each).  Returns the largest CTA load in units, or -1 when

@@ -354,9 +354,9 @@ ternary_gemv_kernel(const __grid_constant__ GemvLaunch L) {
     }
   };
   // Warp w takes the w-th of eight contiguous ranges of the CTA's units, of
-  // equal cost: a unit of a problem with two token tiles counts 3, one with
-  // one tile 2 (the MMA work is half again as large).
-  auto unit_cost = [&](int sg) { return prob[seg_p[sg]].M > 8 ? 3 : 2; };
+  // equal cost: a unit of a problem with two token tiles counts 6, one with
+  // one tile 5 (the host's dealing uses the same weights).
+  auto unit_cost = [&](int sg) { return prob[seg_p[sg]].M > 8 ? 6 : 5; };
   int total_cost = 0;
   for (int i = 0; i < nseg; ++i) total_cost += seg_n[i] * unit_cost(i);
   // First unit (as a count of units before it) whose cost prefix reaches c.
