@@ -316,6 +316,22 @@ BITNET_API bitnet_status bitnet_device_status(bitnet_stream_t stream, int reset,
  * ---------------------------------------------------------------------- */
 BITNET_API bitnet_status bitnet_selftest_bounded_wait(uint64_t limit_ns, bitnet_stream_t stream);
 
+/* ------------------------------------------------------------------------
+ * bitnet_selftest_divide -- q[i] = a[i] / b[i] through the division the
+ * decode epilogue uses for y = acc / (s_x * s_w): the correctly rounded
+ * reciprocal of b and two fused residual corrections (Markstein's method),
+ * which rounds to nearest even exactly like an IEEE binary32 division for
+ * finite a and normal b > 0 whose quotient is zero or normal.  Lets a test
+ * check that claim against a host IEEE division.
+ *
+ *   a, b, q   device fp32 arrays of n elements (16-byte aligned), caller-owned.
+ *   n         >= 0.
+ * Queues one kernel on `stream`; BITNET_ERR_INVALID_ARG / _MISALIGNED on bad
+ * arguments (nothing queued).
+ * ---------------------------------------------------------------------- */
+BITNET_API bitnet_status bitnet_selftest_divide(const float *a, const float *b, float *q,
+                                                int64_t n, bitnet_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -41,7 +41,7 @@ EXPORTED = (
     "bitnet_rmsnorm_quant_act", "bitnet_linear_forward_workspace_bytes",
     "bitnet_linear_forward", "bitnet_linear_quantize_input", "bitnet_linear_matmul",
     "bitnet_linear_forward_debug", "bitnet_ternary_matmul_i32",
-    "bitnet_device_status", "bitnet_selftest_bounded_wait",
+    "bitnet_device_status", "bitnet_selftest_bounded_wait", "bitnet_selftest_divide",
     "bitnet_quantize_pack_weights_static",
     "bitnet_linear_forward_grouped_workspace_bytes", "bitnet_linear_forward_grouped",
 )
@@ -99,6 +99,7 @@ def load_library(path: str = LIB_PATH):
             "bitnet_ternary_matmul_i32": ([P, P, I64, I64, I64, P, P, SZ, I, P], I),
             "bitnet_device_status": ([P, I, ctypes.POINTER(I)], I),
             "bitnet_selftest_bounded_wait": ([ctypes.c_uint64, P], I),
+            "bitnet_selftest_divide": ([P, P, P, I64, P], I),
             "bitnet_quantize_pack_weights_static": ([P, I64, I64, P, P, P], I),
             "bitnet_linear_forward_grouped_workspace_bytes": ([I, P], SZ),
             "bitnet_linear_forward_grouped": ([I, P, P, SZ, I, P], I),
@@ -363,6 +364,18 @@ def bitnet_device_status(reset=True, stream=None):
 def bitnet_selftest_bounded_wait(limit_ns: int, stream=None):
     _check("bitnet_selftest_bounded_wait",
            load_library().bitnet_selftest_bounded_wait(int(limit_ns), _stream(stream)))
+
+
+def bitnet_selftest_divide(a, b, stream=None):
+    """a / b (fp32 CUDA tensors) through the decode epilogue's division."""
+    _need_cuda(a, b)
+    a = a.contiguous()
+    b = b.contiguous()
+    q = torch.empty_like(a)
+    _check("bitnet_selftest_divide",
+           load_library().bitnet_selftest_divide(_ptr(a), _ptr(b), _ptr(q), a.numel(),
+                                                 _stream(stream)))
+    return q
 
 
 class BitLinear:

@@ -133,6 +133,38 @@ __device__ __forceinline__ float block_max_f32(float v, float* red) {
   return r;
 }
 
+// block_tree_sum_f32 of p (same order, same result) and the block max of m
+// through the same barriers.
+__device__ __forceinline__ float2 block_sum_max_f32(float p, float m, float* red, int* redm) {
+  const int tid = threadIdx.x;
+#pragma unroll
+  for (int s = 16; s >= 1; s >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, s));
+  red[tid] = p;
+  if ((tid & 31) == 0) redm[tid >> 5] = __float_as_int(m);
+  __syncthreads();
+#pragma unroll
+  for (int s = 128; s >= 32; s >>= 1) {
+    if (tid < s) red[tid] = __fadd_rn(red[tid], red[tid + s]);
+    __syncthreads();
+  }
+  if (tid < 32) {
+    float v = red[tid];
+#pragma unroll
+    for (int s = 16; s >= 1; s >>= 1) v = __fadd_rn(v, __shfl_down_sync(0xFFFFFFFFu, v, s));
+    float w = (tid < kActThreads / 32) ? __int_as_float(redm[tid]) : 0.0f;
+#pragma unroll
+    for (int s = 16; s >= 1; s >>= 1) w = fmaxf(w, __shfl_xor_sync(0xFFFFFFFFu, w, s));
+    if (tid == 0) {
+      red[0] = v;
+      redm[0] = __float_as_int(w);
+    }
+  }
+  __syncthreads();
+  const float2 r = make_float2(red[0], __int_as_float(redm[0]));
+  __syncthreads();
+  return r;
+}
+
 __device__ __forceinline__ int block_sum_i32(int v, int* red) {
   const int tid = threadIdx.x;
 #pragma unroll
@@ -347,34 +379,51 @@ __device__ bool quant_row_staged(const void* __restrict__ x, const float* __rest
     for (int j = 0; j < 8; ++j) g[j] = gamma ? sg[8 * c + j] : 1.0f;
   };
 
-  // Pass 1: sum of squares, partial = this thread's chunks in increasing k.
-  float p = 0.0f;
+  // Pass 1: sum of squares, partial = this thread's chunks in increasing k;
+  // without gamma also max |x| (then max |x_n| = max |x| * r exactly: a
+  // correctly rounded product is monotonic in |x|).
+  float p = 0.0f, xmax = 0.0f;
 #pragma unroll 1
   for (int64_t c = tid; c < nchunk; c += kActThreads) {
     float v[8];
     chunk(c, v);
 #pragma unroll
-    for (int j = 0; j < 8; ++j) p = __fmaf_rn(v[j], v[j], p);
+    for (int j = 0; j < 8; ++j) {
+      p = __fmaf_rn(v[j], v[j], p);
+      xmax = fmaxf(xmax, fabsf(v[j]));
+    }
   }
-  const float ss = block_tree_sum_f32(p, redf);
+  float ss;
+  if (gamma) {
+    ss = block_tree_sum_f32(p, redf);
+  } else {
+    const float2 sm = block_sum_max_f32(p, xmax, redf, redi);
+    ss = sm.x;
+    xmax = sm.y;
+  }
   const float ms = __fdiv_rn(ss, static_cast<float>(K));
   const float d = __fadd_rn(ms, eps);
   const bool zero_row = (d == 0.0f);
   const float r = zero_row ? 0.0f : __fdiv_rn(1.0f, __fsqrt_rn(d));
 
-  // Pass 2: max |x_n|.
+  // Pass 2 (with gamma): max |x_n|.
   float amax = 0.0f;
-  if (!zero_row) {
+  if (!gamma) {
+    amax = zero_row ? 0.0f : __fmul_rn(xmax, r);
+  } else {
+    if (!zero_row) {
 #pragma unroll 1
-    for (int64_t c = tid; c < nchunk; c += kActThreads) {
-      float v[8], g[8];
-      chunk(c, v);
-      gam(c, g);
+      for (int64_t c = tid; c < nchunk; c += kActThreads) {
+        float v[8], g[8];
+        chunk(c, v);
+        gam(c, g);
 #pragma unroll
-      for (int j = 0; j < 8; ++j) amax = fmaxf(amax, fabsf(__fmul_rn(__fmul_rn(v[j], r), g[j])));
+        for (int j = 0; j < 8; ++j)
+          amax = fmaxf(amax, fabsf(__fmul_rn(__fmul_rn(v[j], r), g[j])));
+      }
     }
+    amax = block_max_f32(amax, redf);
   }
-  amax = block_max_f32(amax, redf);
   amax = fmaxf(amax, 1e-5f);
   const float sx = __fdiv_rn(127.0f, amax);
 

@@ -1075,6 +1075,31 @@ __global__ void bounded_wait_selftest_kernel(int* status, uint64_t limit_ns) {
 }  // namespace
 }  // namespace bitnet
 
+namespace bitnet {
+namespace {
+__global__ void divide_selftest_kernel(const float* __restrict__ a, const float* __restrict__ b,
+                                       float* __restrict__ q, int64_t n) {
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x)
+    q[i] = div_rn_by_recip(a[i], b[i], __frcp_rn(b[i]));
+}
+}  // namespace
+}  // namespace bitnet
+
+extern "C" BITNET_API bitnet_status bitnet_selftest_divide(const float* a, const float* b,
+                                                           float* q, int64_t n,
+                                                           bitnet_stream_t stream) {
+  if (n < 0 || (n > 0 && (!a || !b || !q))) return BITNET_ERR_INVALID_ARG;
+  if (n == 0) return BITNET_OK;
+  if (!aligned(a, 16) || !aligned(b, 16) || !aligned(q, 16)) return BITNET_ERR_MISALIGNED;
+  DeviceState* ds = device_state();
+  if (!ds) return BITNET_ERR_CUDA;
+  const int64_t blocks = std::min<int64_t>((n + 255) / 256, 4 * ds->num_sms);
+  divide_selftest_kernel<<<static_cast<unsigned>(blocks), 256, 0, as_stream(stream)>>>(a, b, q,
+                                                                                        n);
+  return launch_status();
+}
+
 extern "C" BITNET_API bitnet_status bitnet_selftest_bounded_wait(uint64_t limit_ns,
                                                                  bitnet_stream_t stream) {
   if (limit_ns < 1000ull || limit_ns > 1000000000ull) return BITNET_ERR_INVALID_ARG;

@@ -278,6 +278,23 @@ __device__ __forceinline__ uint4 ldg_u4(const void* p) {
   return v;
 }
 
+// ------------------------------------------------------------ division
+
+// a / b rounded to nearest even (binary32), for finite a and normal b > 0
+// whose quotient is zero or normal, given y = RN(1 / b): Markstein's method
+// (P. Markstein, "Computation of elementary functions on the IBM RISC
+// System/6000 processor", IBM J. Res. Dev. 34(1), 1990): with y within half
+// an ulp of 1/b and q within one ulp of a/b, the residual a - b q is exact
+// under a fused multiply-add and RN(q + (a - b q) y) = RN(a / b).  One
+// correction brings RN(a y) within one ulp; the second rounds correctly.
+__device__ __forceinline__ float div_rn_by_recip(float a, float b, float y) {
+  float q = __fmul_rn(a, y);
+  float r = __fmaf_rn(-q, b, a);
+  q = __fmaf_rn(r, y, q);
+  r = __fmaf_rn(-q, b, a);
+  return __fmaf_rn(r, y, q);
+}
+
 // ------------------------------------------------- decode activation order
 
 // Decode-matmul block order: inside every 256-byte span of a token row of

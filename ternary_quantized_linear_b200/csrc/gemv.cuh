@@ -239,15 +239,15 @@ __device__ __forceinline__ void gemv_flush(int (&acc)[4][NT][4], int (&acc16)[4]
   }
 }
 
-// rs, sx: token m's row sum and scale (read once per segment into shared
-// memory); sw the weight scale.
-__device__ __forceinline__ void gemv_finish(const GemvProblem& p, float sw, float sx, int rs,
+// rs: token m's row sum; d = RN(s_x[m] * s_w) and rd = RN(1 / d), read and
+// computed once per segment into shared memory.
+__device__ __forceinline__ void gemv_finish(const GemvProblem& p, float d, float rd, int rs,
                                             int m, int n, int acc_codes) {
   const int acc = acc_codes - rs;
   const int64_t o = static_cast<int64_t>(m) * p.N + n;
   if (p.acc_out) p.acc_out[o] = acc;
   if (p.y) {
-    const float yv = __fdiv_rn(__int2float_rn(acc), __fmul_rn(sx, sw));
+    const float yv = div_rn_by_recip(__int2float_rn(acc), d, rd);
     if (p.y_bf16)
       reinterpret_cast<__nv_bfloat16*>(p.y)[o] = __float2bfloat16_rn(yv);
     else
@@ -277,8 +277,8 @@ ternary_gemv_kernel(const __grid_constant__ GemvLaunch L) {
   __shared__ int seg_lo[kGemvMaxSegs], seg_n[kGemvMaxSegs], seg_owned[kGemvMaxSegs];
   __shared__ int seg_count, seg_last[kGemvMaxSegs];
   __shared__ int seg_rs[kGemvMaxSegs][16];    // row sums of the segment's tokens
-  __shared__ float seg_sx[kGemvMaxSegs][16];  // their scales
-  __shared__ float seg_sw[kGemvMaxSegs];      // the weight scale
+  __shared__ float seg_d[kGemvMaxSegs][16];   // their dequant divisors s_x * s_w
+  __shared__ float seg_rd[kGemvMaxSegs][16];  // and RN(1 / divisor)
   __shared__ volatile int abort_flag;
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -417,9 +417,10 @@ ternary_gemv_kernel(const __grid_constant__ GemvLaunch L) {
     const GemvProblem& P = prob[seg_p[warp]];
     if (lane < P.M) {
       seg_rs[warp][lane] = P.rowsum[lane];
-      seg_sx[warp][lane] = P.s_x ? P.s_x[lane] : 0.0f;
+      const float d = (P.y && P.s_x && P.s_w) ? __fmul_rn(P.s_x[lane], P.s_w[0]) : 1.0f;
+      seg_d[warp][lane] = d;
+      seg_rd[warp][lane] = __frcp_rn(d);
     }
-    if (lane == 0) seg_sw[warp] = (P.y && P.s_w) ? P.s_w[0] : 0.0f;
   }
   if (lane == 0) {
     for (int j = 0; j < pre; ++j) {
@@ -511,7 +512,7 @@ ternary_gemv_kernel(const __grid_constant__ GemvLaunch L) {
     if (seg_owned[s]) {
       for (int idx = tid; idx < nout; idx += kGemvThreads) {
         const int r = idx % kGemvRows, m = idx / kGemvRows, n = n0 + r;
-        if (n < P.N) gemv_finish(P, seg_sw[s], seg_sx[s][m], seg_rs[s][m], m, n, rs[r * 16 + m]);
+        if (n < P.N) gemv_finish(P, seg_d[s][m], seg_rd[s][m], seg_rs[s][m], m, n, rs[r * 16 + m]);
       }
       continue;
     }
@@ -548,7 +549,7 @@ ternary_gemv_kernel(const __grid_constant__ GemvLaunch L) {
       const int r = idx % kGemvRows, m = idx / kGemvRows, n = n0 + r;
       if (n < P.N) {
         const int v = atomicExch(P.ws_acc + static_cast<int64_t>(m) * P.N + n, 0);
-        gemv_finish(P, seg_sw[s], seg_sx[s][m], seg_rs[s][m], m, n, v);
+        gemv_finish(P, seg_d[s][m], seg_rd[s][m], seg_rs[s][m], m, n, v);
       }
     }
     if (tid == 0) P.ws_cnt[seg_rbl[s]] = 0u;  // ready for the next call

@@ -112,6 +112,12 @@ def test_other_entry_points_reject_bad_arguments(lib):
     assert lib.bitnet_ternary_matmul_i32(P(FAKE), P(FAKE), 4, 64, 128, P(FAKE), P(FAKE), 1 << 30,
                                          9, None) == tql.BITNET_ERR_INVALID_ARG
     assert lib.bitnet_selftest_bounded_wait(10, None) == tql.BITNET_ERR_INVALID_ARG
+    assert lib.bitnet_selftest_divide(P(FAKE), P(FAKE), P(FAKE), -1, None) == \
+        tql.BITNET_ERR_INVALID_ARG
+    assert lib.bitnet_selftest_divide(None, P(FAKE), P(FAKE), 4, None) == tql.BITNET_ERR_INVALID_ARG
+    assert lib.bitnet_selftest_divide(P(FAKE + 4), P(FAKE), P(FAKE), 4, None) == \
+        tql.BITNET_ERR_MISALIGNED
+    assert lib.bitnet_selftest_divide(None, None, None, 0, None) == tql.BITNET_OK
 
 
 def test_binding_refuses_cpu_tensors(lib):

@@ -391,3 +391,34 @@ def test_grouped_shared_input_and_repeated_calls(M):
         torch.cuda.synchronize()
         assert torch.equal(ys[j].view(torch.int16), y1.view(torch.int16))
         assert torch.equal(ys2[j].view(torch.int16), y1.view(torch.int16))
+
+
+def test_epilogue_division_matches_ieee_division():
+    # The decode epilogue divides through a correctly rounded reciprocal and
+    # two residual corrections; it must equal an IEEE binary32 division
+    # (numpy on the host) for every value the dequant can see: integer
+    # numerators up to 2^27 and divisors from products of scales, plus
+    # significands at the edges (all ones, powers of two, near-midpoint
+    # quotients) and random finite floats.
+    rng = np.random.default_rng(2024)
+    n = 1 << 22
+    a_int = rng.integers(-(1 << 27), 1 << 27, n).astype(np.float32)
+    sx = (127.0 / rng.uniform(1e-3, 300.0, n)).astype(np.float32)
+    sw = rng.uniform(1.0, 400.0, n).astype(np.float32)
+    b_prod = (sx * sw).astype(np.float32)
+    ones = np.float32(2.0 ** 24 - 1) * np.power(np.float32(2.0), rng.integers(-30, 8, n).astype(np.float32))
+    pow2 = np.power(np.float32(2.0), rng.integers(-20, 20, n).astype(np.float32))
+    rnd_a = (rng.standard_normal(n) * np.exp(rng.uniform(-20, 20, n))).astype(np.float32)
+    rnd_b = np.exp(rng.uniform(-20, 20, n)).astype(np.float32)
+    a_mid = ((rng.integers(1, 1 << 24, n) * 2 + 1) * np.float32(0.5)).astype(np.float32)
+    cases = [(a_int, b_prod), (a_int, ones.astype(np.float32)), (a_int, pow2.astype(np.float32)),
+             (rnd_a, rnd_b), (a_mid, np.float32(3.0) * pow2.astype(np.float32)),
+             (np.zeros(n, np.float32), b_prod)]
+    for a, b in cases:
+        ref = (a / b).astype(np.float32)
+        assert np.all(np.isfinite(ref))
+        q = tql.bitnet_selftest_divide(torch.from_numpy(a).cuda(), torch.from_numpy(b).cuda())
+        torch.cuda.synchronize()
+        got = q.cpu().numpy()
+        bad = np.nonzero(got.view(np.uint32) != ref.view(np.uint32))[0]
+        assert bad.size == 0, (a[bad[:5]], b[bad[:5]], got[bad[:5]], ref[bad[:5]])
