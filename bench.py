@@ -32,8 +32,8 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # DRAM bytes (read + write) of one grouped GEMV launch of this workload from
 # an ncu capture (summary under profiles/), valid only for the kernel source
 # it was measured on (sha256 of csrc/gemv.cuh); reported as null otherwise.
-GEMV_TRAFFIC = {"src_sha256": "b9e8b916d1ea9e52ddd205c6a91647a872128d6a5ee73d25747b8c4b7a85a262",
-                "bytes_per_launch": 49548032}
+GEMV_TRAFFIC = {"src_sha256": "98667b7979eccb6645044ce749447ee19b1ef880903737271b3b5bfe55394e29",
+                "bytes_per_launch": 49537280}
 
 
 # ------------------------------------------------------------------ helpers
