@@ -32,7 +32,7 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # DRAM bytes (read + write) of one grouped GEMV launch of this workload from
 # an ncu capture (summary under profiles/), valid only for the kernel source
 # it was measured on (sha256 of csrc/gemv.cuh); reported as null otherwise.
-GEMV_TRAFFIC = {"src_sha256": "98667b7979eccb6645044ce749447ee19b1ef880903737271b3b5bfe55394e29",
+GEMV_TRAFFIC = {"src_sha256": "d5f0e05da58c50699640b00f12d8cc0c624cb952e6282a088a857f01a4bb1d51",
                 "bytes_per_launch": 49537280}
 
 

@@ -241,43 +241,6 @@ __device__ __forceinline__ void mma_m16n8k32_s8(int (&d)[4], uint32_t a0, uint32
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
-// 16-byte streaming load of packed weights (read once per call; keep it out
-// of L1).
-__device__ __forceinline__ uint4 ldg_stream_u4(const void* p) {
-  uint4 v;
-  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
-               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-               : "l"(p));
-  return v;
-}
-
-// Hint: bring `bytes` (a multiple of 16, 16-byte aligned) into L2 ahead of
-// use; the copy engine does it asynchronously and nothing waits on it.
-__device__ __forceinline__ void prefetch_l2_bulk(const void* p, uint32_t bytes) {
-  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
-}
-
-// 16-byte load through L1 without a compiler memory barrier: for data that
-// nothing in this kernel writes (after the wait on the preceding grid).
-__device__ __forceinline__ uint4 ldg_u4_ro(const void* p) {
-  uint4 v;
-  asm volatile("ld.global.v4.u32 {%0,%1,%2,%3}, [%4];"
-               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-               : "l"(p));
-  return v;
-}
-
-// 16-byte load through L1 (data written by the preceding grid: not the
-// non-coherent path).
-__device__ __forceinline__ uint4 ldg_u4(const void* p) {
-  uint4 v;
-  asm volatile("ld.global.v4.u32 {%0,%1,%2,%3}, [%4];"
-               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-               : "l"(p)
-               : "memory");
-  return v;
-}
-
 // ------------------------------------------------------------ division
 
 // a / b rounded to nearest even (binary32), for finite a and normal b > 0

@@ -127,8 +127,7 @@ __device__ __forceinline__ uint32_t word_of(const uint4& v, int w) {
 }
 
 // Unit u of the launch: its problem (p advances monotonically from a hint),
-// row block and k chunk.  Used once per warp; the walk then advances a
-// cursor (no division per unit).
+// row block and k chunk.  Used for the two ends of a stream-K share.
 struct GemvUnit {
   int p, rbl, c;
 };
