@@ -241,6 +241,12 @@ __device__ __forceinline__ void mma_m16n8k32_s8(int (&d)[4], uint32_t a0, uint32
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
+// Barrier `id` (1..15) over `count` threads (a multiple of 32): lets a
+// subset of a CTA's warps synchronise without the others.
+__device__ __forceinline__ void named_barrier_sync(int id, int count) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+
 // ------------------------------------------------------------ division
 
 // a / b rounded to nearest even (binary32), for finite a and normal b > 0

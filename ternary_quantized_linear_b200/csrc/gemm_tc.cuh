@@ -22,7 +22,9 @@
 //               A_STAGES TMEM stages, so the unpack runs that many steps ahead
 //               of the MMAs; after the last step the same warps read the
 //               accumulators from TMEM (one lane = one weight row) and write
-//               y = (acc - rowsum) / (s_x * s_w) coalesced along N.
+//               y = (acc - rowsum) / (s_x * s_w) coalesced along N, the
+//               row sums, divisors and their reciprocals taken from a
+//               per-tile shared-memory table built before the main loop.
 // Keeping A in TMEM means the unpacked weights (4x the packed bytes) never
 // touch shared memory; only the packed tile and the activation tile do.
 // Code byte order: word r of packed word w holds k = 16w + 4i + r in byte i,
@@ -96,11 +98,13 @@ struct GemmCfg {
   static constexpr int OFF_BAR = OFF_WP + STAGES * WP_BYTES;
   static constexpr int NBAR = 2 * STAGES + A_STAGES + 1;  // full/done, aready, accfull
   static constexpr int OFF_MISC = OFF_BAR + 8 * NBAR;
-  static constexpr int BYTES = OFF_MISC + 16;
+  static constexpr int OFF_TAB = (OFF_MISC + 16 + 15) & ~15;  // epilogue table: one int4 per token
+  static constexpr int BYTES = OFF_TAB + 16 * BN;
   static constexpr int SMEM_DYN = BYTES + 1024;  // slack for 1024-byte alignment
   static_assert(BN == 16 || BN == 32 || BN == 64 || BN == 128 || BN == 256, "BN");
   static_assert(A_STAGES <= STAGES, "A stages are recycled through the stage barriers");
   static_assert(D_COL + BN <= TMEM_COLS, "tensor memory");
+  static_assert(OFF_TAB % 16 == 0, "the epilogue table is read as int4");
   static_assert(X_ATOM % 1024 == 0, "swizzle atoms must stay 1024-byte aligned");
   static_assert(PART % 16 == 0, "unpack reads 16-byte words");
   static_assert(WP_ROW == 64, "weight tile swizzle");
@@ -158,11 +162,15 @@ __device__ __forceinline__ void tc_mma_i8_ts(uint32_t d_tmem, uint32_t a_tmem, u
       : "memory");
 }
 
-__device__ __forceinline__ void gemm_store(const GemmParams& p, float sw, int m, int n, int acc) {
+// One output: e = the tile's epilogue entry of token m, {row sum, divisor
+// s_x * s_w, RN(1 / divisor)} (the last two as float bits).
+__device__ __forceinline__ void gemm_store(const GemmParams& p, int4 e, int m, int n, int acc_codes) {
+  const int acc = acc_codes - e.x;
   const int64_t o = static_cast<int64_t>(m) * p.N + n;
   if (p.acc_out) p.acc_out[o] = acc;
   if (p.y) {
-    const float yv = __fdiv_rn(__int2float_rn(acc), __fmul_rn(p.s_x[m], sw));
+    const float yv =
+        div_rn_by_recip(__int2float_rn(acc), __int_as_float(e.y), __int_as_float(e.z));
     if (p.y_bf16)
       reinterpret_cast<__nv_bfloat16*>(p.y)[o] = __float2bfloat16_rn(yv);
     else
@@ -193,6 +201,7 @@ ternary_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x,
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
   int* is_last = reinterpret_cast<int*>(smem + C::OFF_MISC + 8);
+  int4* tab = reinterpret_cast<int4*>(smem + C::OFF_TAB);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int n0 = blockIdx.x * C::BM;
@@ -299,6 +308,24 @@ ternary_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x,
     const int q = u & 3, h = u >> 2;
     const int i = 32 * q + lane;        // weight row inside the tile
     const uint32_t lane_addr = static_cast<uint32_t>(32 * q) << 16;
+    // Epilogue table of this tile's tokens, built while the first copies are
+    // in flight: row sum, divisor s_x * s_w and its correctly rounded
+    // reciprocal, so each output costs a multiply and four FMAs instead of
+    // a division.  Only the unpack warps read it before the final barrier.
+    {
+      const float swv = (p.y && p.s_w) ? *p.s_w : 0.0f;
+      for (int c = threadIdx.x - 128; c < BN; c += 32 * C::UNPACK_WARPS) {
+        const int m = m0 + c;
+        int rs = 0;
+        float d = 1.0f;
+        if (m < p.M) {
+          rs = p.rowsum[m];
+          if (p.y) d = __fmul_rn(p.s_x[m], swv);
+        }
+        tab[c] = make_int4(rs, __float_as_int(d), __float_as_int(__frcp_rn(d)), 0);
+      }
+      named_barrier_sync(1, 32 * C::UNPACK_WARPS);
+    }
     for (int j = 0; j < nk; ++j) {
       const int s = j % C::STAGES, a = j % C::A_STAGES;
       // A stage a was last used by step j - A_STAGES; its MMAs completed when
@@ -348,7 +375,6 @@ ternary_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x,
     constexpr int kHalf = BN >= 32 ? BN / 2 : BN;
     if (write && (BN >= 32 || h == 0)) {
       const int n = n0 + i;
-      const float swv = (p.y && p.s_w) ? *p.s_w : 0.0f;
       const bool split = p.ksplit > 1;
       for (int c0 = h * kHalf; c0 < (h + 1) * kHalf; c0 += 16) {
         if (m0 + c0 >= p.M) break;  // uniform across the warp
@@ -363,7 +389,7 @@ ternary_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x,
               if (split)
                 atomicAdd(p.ws_acc + static_cast<int64_t>(m) * p.N + n, static_cast<int>(r[jj]));
               else
-                gemm_store(p, swv, m, n, static_cast<int>(r[jj]) - p.rowsum[m]);
+                gemm_store(p, tab[c0 + jj], m, n, static_cast<int>(r[jj]));
             }
           }
         }
@@ -390,12 +416,11 @@ ternary_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x,
     __syncthreads();
     if (!*is_last) return;
     __threadfence();
-    const float swv = (p.y && p.s_w) ? *p.s_w : 0.0f;
     const int rows = min(C::BM, p.N - n0), toks = min(BN, p.M - m0);
     for (int idx = threadIdx.x; idx < rows * toks; idx += blockDim.x) {
-      const int r = idx % rows, mm = m0 + idx / rows, n = n0 + r;
-      const int v = atomicExch(p.ws_acc + static_cast<int64_t>(mm) * p.N + n, 0);
-      gemm_store(p, swv, mm, n, v - p.rowsum[mm]);
+      const int r = idx % rows, c = idx / rows, n = n0 + r;
+      const int v = atomicExch(p.ws_acc + static_cast<int64_t>(m0 + c) * p.N + n, 0);
+      gemm_store(p, tab[c], m0 + c, n, v);
     }
     if (threadIdx.x == 0) p.ws_cnt[tile] = 0u;  // ready for the next call
   }
