@@ -114,8 +114,8 @@ class ClockSampler:
                0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
                0x100: "display_clock_setting"}
 
-    def __init__(self, index, period_s=0.002):
-        self.index, self.period = index, period_s
+    def __init__(self, index, period_s=0.001, window=""):
+        self.index, self.period, self.window = index, period_s, window
         self.samples, self.reasons = [], 0
         self.max_mhz = None
         self._stop = threading.Event()
@@ -141,16 +141,23 @@ class ClockSampler:
                 pass
             time.sleep(self.period)
 
-    def __enter__(self):
-        if self.ok:
+    def start(self):
+        if self.ok and self._t is None:
             self._t = threading.Thread(target=self._run, daemon=True)
             self._t.start()
         return self
 
-    def __exit__(self, *exc):
+    def stop(self):
         if self._t is not None:
             self._stop.set()
             self._t.join()
+            self._t = None
+
+    def __enter__(self):
+        return self.start()
+
+    def __exit__(self, *exc):
+        self.stop()
 
     def summary(self):
         if not self.ok:
@@ -159,7 +166,7 @@ class ClockSampler:
         names = [n for bit, n in self.REASONS.items() if self.reasons & bit and n != "gpu_idle"]
         return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
                 "sm_max_mhz": self.max_mhz, "reasons": names, "samples": len(self.samples),
-                "source": "nvml"}
+                "source": "nvml", "window": self.window}
 
 
 # --------------------------------------------------------------- CPU oracle
@@ -322,7 +329,12 @@ def run_ours(args):
             import torch.distributed as dist
             dist.barrier(device_ids=[local_rank])
 
-    # ---- warm-up, then exactly K timed steps (graph replays)
+    # ---- warm-up, then exactly K timed steps (graph replays).  The clock
+    # sampler runs from the warm-up through the kernel-timing replays below:
+    # the timed steps alone last a few milliseconds, about one NVML sample.
+    clocks = ClockSampler(local_rank, window="warm-up, the timed steps and the kernel-timing "
+                                              "graph replays (all back-to-back GPU work)")
+    clocks.start()
     with torch.cuda.stream(stream):
         run_steps(args.warmup)
     stream.synchronize()
@@ -330,12 +342,11 @@ def run_ours(args):
     torch.cuda.synchronize()
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
-    with ClockSampler(local_rank) as clocks:
-        with torch.cuda.stream(stream):
-            e0.record(stream)
-            run_steps(args.steps)
-            e1.record(stream)
-        stream.synchronize()
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        run_steps(args.steps)
+        e1.record(stream)
+    stream.synchronize()
     torch.cuda.synchronize()
     barrier()
     local_ms = e0.elapsed_time(e1)
@@ -374,6 +385,7 @@ def run_ours(args):
 
     m_avg = phase_ms(tql.BITNET_PHASE_MATMUL)
     q_avg = phase_ms(tql.BITNET_PHASE_QUANTIZE)
+    clocks.stop()
     gemv_b = sum(gemv_bytes(M, N, K) for _, K, N, M in probs)
     peaks, peak_src = load_peaks()
     hbm_peak = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
