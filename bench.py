@@ -506,50 +506,93 @@ def run_ours(args):
             # events order upload -> call -> download and gate the reuse of
             # its buffers: an upload waits for the set's previous call (its
             # input buffer is free), a call for the set's previous download
-            # (its output buffer is free).
+            # (its output buffer is free).  The copies and event operations go
+            # straight to the CUDA driver (handles and pointers resolved before
+            # the loop) so the host keeps ahead of the device.
+            cu = ctypes.CDLL("libcuda.so.1")
+            VP, U64, SZ = ctypes.c_void_p, ctypes.c_uint64, ctypes.c_size_t
+            h2d_copy, d2h_copy = cu.cuMemcpyHtoDAsync_v2, cu.cuMemcpyDtoHAsync_v2
+            h2d_copy.argtypes = [U64, VP, SZ, VP]
+            d2h_copy.argtypes = [VP, U64, SZ, VP]
+            ev_create, ev_record, ev_destroy = cu.cuEventCreate, cu.cuEventRecord, cu.cuEventDestroy_v2
+            ev_create.argtypes = [ctypes.POINTER(VP), ctypes.c_uint]
+            ev_record.argtypes = [VP, VP]
+            ev_destroy.argtypes = [VP]
+            wait_ev = cu.cuStreamWaitEvent
+            wait_ev.argtypes = [VP, VP, ctypes.c_uint]
+
+            def ok(rc, what):
+                if rc != 0:
+                    raise RuntimeError(f"{what} returned CUDA driver error {rc}")
+
             s_up, s_dn = torch.cuda.Stream(device), torch.cuda.Stream(device)
-            up = [torch.cuda.Event() for _ in range(R)]
-            called = [torch.cuda.Event() for _ in range(R)]
-            down = [torch.cuda.Event() for _ in range(R)]
+            h_up, h_c, h_dn = VP(s_up.cuda_stream), VP(stream.cuda_stream), VP(s_dn.cuda_stream)
+            events = []
+
+            def new_event():
+                e = VP()
+                ok(ev_create(ctypes.byref(e), 2), "cuEventCreate")  # CU_EVENT_DISABLE_TIMING
+                events.append(e)
+                return e
+
+            up = [new_event() for _ in range(R)]
+            called = [new_event() for _ in range(R)]
+            down = [new_event() for _ in range(R)]
             used = [False] * R
+            plan = []
+            for r in range(R):
+                dx, dy, hx, hy, arr, count, ws, _ = e2e_sets[r]
+                nx, ny = dx.numel() * dx.element_size(), dy.numel() * dy.element_size()
+                assert nx == hx.numel() * hx.element_size() and hx.is_pinned()
+                assert ny == hy.numel() * hy.element_size() and hy.is_pinned()
+                plan.append((U64(dx.data_ptr()), VP(hx.data_ptr()), SZ(nx),
+                             VP(hy.data_ptr()), U64(dy.data_ptr()), SZ(ny),
+                             count, ctypes.cast(arr, P), P(ws.data_ptr()), ws.numel()))
+            call = lib.bitnet_linear_forward_grouped
+            phase = tql.BITNET_PHASE_ALL
 
             def step(r):
-                dx, dy, hx, hy = e2e_sets[r][:4]
+                dxp, hxp, nx, hyp, dyp, ny, count, arr_p, ws_p, nb = plan[r]
                 if used[r]:
-                    s_up.wait_event(called[r])
-                with torch.cuda.stream(s_up):
-                    dx.copy_(hx, non_blocking=True)
-                up[r].record(s_up)
-                stream.wait_event(up[r])
+                    ok(wait_ev(h_up, called[r], 0), "cuStreamWaitEvent")
+                ok(h2d_copy(dxp, hxp, nx, h_up), "cuMemcpyHtoDAsync")
+                ok(ev_record(up[r], h_up), "cuEventRecord")
+                ok(wait_ev(h_c, up[r], 0), "cuStreamWaitEvent")
                 if used[r]:
-                    stream.wait_event(down[r])
-                grouped_call(r, stream)
-                called[r].record(stream)
-                s_dn.wait_event(called[r])
-                with torch.cuda.stream(s_dn):
-                    hy.copy_(dy, non_blocking=True)
-                down[r].record(s_dn)
+                    ok(wait_ev(h_c, down[r], 0), "cuStreamWaitEvent")
+                rc = call(count, arr_p, ws_p, nb, phase, h_c)
+                if rc != 0:
+                    raise RuntimeError(tql.bitnet_status_string(rc))
+                ok(ev_record(called[r], h_c), "cuEventRecord")
+                ok(wait_ev(h_dn, called[r], 0), "cuStreamWaitEvent")
+                ok(d2h_copy(hyp, dyp, ny, h_dn), "cuMemcpyDtoHAsync")
+                ok(ev_record(down[r], h_dn), "cuEventRecord")
                 used[r] = True
 
             def join():
                 stream.wait_stream(s_up)
                 stream.wait_stream(s_dn)
 
-            for i in range(args.warmup):
-                step(i % R)
-            join()
-            torch.cuda.synchronize()
-            barrier()
-            a0 = torch.cuda.Event(enable_timing=True)
-            a1 = torch.cuda.Event(enable_timing=True)
-            a0.record(stream)
-            s_up.wait_stream(stream)
-            s_dn.wait_stream(stream)
-            for i in range(args.steps):
-                step(i % R)
-            join()
-            a1.record(stream)
-            torch.cuda.synchronize()
+            try:
+                for i in range(args.warmup):
+                    step(i % R)
+                join()
+                torch.cuda.synchronize()
+                barrier()
+                a0 = torch.cuda.Event(enable_timing=True)
+                a1 = torch.cuda.Event(enable_timing=True)
+                a0.record(stream)
+                s_up.wait_stream(stream)
+                s_dn.wait_stream(stream)
+                for i in range(args.steps):
+                    step(i % R)
+                join()
+                a1.record(stream)
+                torch.cuda.synchronize()
+            finally:
+                torch.cuda.synchronize()
+                for e in events:
+                    ev_destroy(e)
             # the downloads hold what the device path computed for each set
             for r in range(R):
                 if not used[r]:
@@ -567,14 +610,15 @@ def run_ours(args):
         how_pipe = ("per step: one pinned-host -> device copy of the nine inputs, one "
                     "bitnet_linear_forward_grouped call (C ABI, eager), one device -> "
                     "pinned-host copy of the nine outputs; uploads, calls and downloads on "
-                    "three streams ordered per rotation set by events, so step i's upload "
-                    "overlaps step i-1's call and download; every step's copies inside the "
-                    "timed region; outputs checked against the device path; device-timed")
+                    "three streams ordered per rotation set by events (copies and events "
+                    "issued through the CUDA driver API), so step i's upload overlaps step "
+                    "i-1's call and download; every step's copies inside the timed region; "
+                    "outputs checked against the device path; device-timed")
         note = None
         try:
             local = e2e_pipelined()
             how = how_pipe
-        except RuntimeError as exc:
+        except Exception as exc:  # noqa: BLE001 -- any failure: measure on one stream
             torch.cuda.synchronize()
             note = f"pipelined measurement failed ({exc}); serial measurement instead"
             local = e2e_serial()
