@@ -635,6 +635,14 @@ def run_ours(args):
     if not args.no_prefill:
         prefill = measure_prefill(args, device, stream, peaks, peak_src)
 
+    # ---- offline weight quant + pack, timed on its own (not in the metric)
+    weight_pack = None
+    if not args.no_weight_pack:
+        try:
+            weight_pack = measure_weight_pack(args, device, stream, hbm_peak)
+        except Exception as exc:  # noqa: BLE001 -- report, keep the line
+            weight_pack = {"error": str(exc)}
+
     # ---- CPU baseline (rank 0, one GPU only)
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -682,9 +690,60 @@ def run_ours(args):
             "gpu_launches": launches,
             "clocks": clocks.summary(),
             "prefill": prefill,
+            "weight_pack": weight_pack,
         }
         print(json.dumps(line), flush=True)
     return 0
+
+
+def measure_weight_pack(args, device, stream, hbm_peak):
+    """bitnet_quantize_pack_weights on the decode workload's three fp32
+    matrices (261 MB together, more than L2), cycled, outputs preallocated:
+    the absmean pass reads W, the quantize pass reads it again and writes the
+    packed codes (the scale must be known before any code is decided)."""
+    import torch
+
+    import ternary_quantized_linear_b200 as tql
+    from ternary_quantized_linear_b200 import workloads
+
+    case = workloads.CASE_BY_NAME[WORKLOAD]
+    mats = []
+    for si, (K, N) in enumerate(case.shapes):
+        W = torch.from_numpy(workloads.weights(case, si)).to(device)
+        W_p = torch.empty((N, K // 4), dtype=torch.uint8, device=device)
+        s_w = torch.empty((1,), dtype=torch.float32, device=device)
+        nb = max(tql.bitnet_quantize_pack_weights_workspace_bytes(N, K), 256)
+        ws = torch.empty(nb, dtype=torch.uint8, device=device)
+        mats.append((W, W_p, s_w, ws, N, K))
+    n = len(mats)
+    reps = max(3, min(args.steps, 30))
+    with torch.cuda.stream(stream):
+        for i in range(max(args.warmup, 3) * n):
+            W, W_p, s_w, ws, _, _ = mats[i % n]
+            tql.bitnet_quantize_pack_weights(W, W_p, s_w, ws, stream=stream)
+        stream.synchronize()
+        ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(reps * n)]
+        for i in range(reps * n):
+            W, W_p, s_w, ws, _, _ = mats[i % n]
+            ev[i][0].record(stream)
+            tql.bitnet_quantize_pack_weights(W, W_p, s_w, ws, stream=stream)
+            ev[i][1].record(stream)
+        stream.synchronize()
+    per = []
+    tot_b, tot_ms = 0, 0.0
+    for j, (W, W_p, _, _, N, K) in enumerate(mats):
+        ms = sum(ev[i][0].elapsed_time(ev[i][1]) for i in range(j, reps * n, n)) / reps
+        b = 2 * 4 * N * K + N * K // 4
+        tot_b += b
+        tot_ms += ms
+        per.append({"N": N, "K": K, "us": round(1e3 * ms, 2),
+                    "gbs": round(b / (ms * 1e-3) / 1e9, 1)})
+    gbs = tot_b / (tot_ms * 1e-3) / 1e9
+    return {"workload": f"{WORKLOAD} weights, fp32, cycled", "matrices": per,
+            "gbs": round(gbs, 1), "frac_of_hbm": round(gbs / hbm_peak, 4),
+            "bytes": "two reads of W (absmean, then quantize) + the packed write",
+            "how": "CUDA events around each call on the launching stream, "
+                   f"{reps} calls per matrix after warm-up"}
 
 
 def measure_prefill(args, device, stream, peaks, peak_src):
@@ -751,6 +810,7 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-prefill", action="store_true")
+    ap.add_argument("--no-weight-pack", action="store_true")
     args = ap.parse_args(argv)
     if args.warmup < 3 and args.impl == "ours":
         args.warmup = 3
