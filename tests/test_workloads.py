@@ -13,6 +13,7 @@ import torch
 
 from ternary_quantized_linear_b200 import workloads
 
+
 @pytest.mark.parametrize("K,expected", [(3200, 3), (4096, 4), (8192, 8), (8640, 9),
                                         (14336, 14), (28672, 29), (256, 1)])
 def test_outlier_channel_count(K, expected):
