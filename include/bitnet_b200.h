@@ -43,8 +43,9 @@
  *     status calls that say so).  Work is queued on `stream` (a
  *     cudaStream_t; NULL = the legacy default stream) and runs
  *     asynchronously.
- *   - Shapes: M >= 0 (M == 0 queues nothing and returns BITNET_OK), N >= 1,
- *     64 <= K <= BITNET_MAX_K and K % 64 == 0.
+ *   - Shapes: 0 <= M <= BITNET_MAX_M (M == 0 queues nothing and returns
+ *     BITNET_OK), 1 <= N <= BITNET_MAX_N, 64 <= K <= BITNET_MAX_K and
+ *     K % 64 == 0; outside these, BITNET_ERR_UNSUPPORTED_SHAPE.
  *   - Every tensor pointer must be 16-byte aligned (workspace: 256-byte).
  *   - Invalid arguments return a status and queue nothing.
  *   - Errors of the CUDA launch itself return BITNET_ERR_CUDA.
@@ -74,7 +75,7 @@ typedef struct CUstream_st *bitnet_stream_t;
 typedef enum {
     BITNET_OK = 0,
     BITNET_ERR_INVALID_ARG = 1,       /* null pointer, negative size, bad dtype, eps < 0 */
-    BITNET_ERR_UNSUPPORTED_SHAPE = 2, /* K % 64 != 0, K out of range, N < 1 */
+    BITNET_ERR_UNSUPPORTED_SHAPE = 2, /* K % 64 != 0, K, M or N out of range */
     BITNET_ERR_MISALIGNED = 3,        /* a pointer is not 16-byte (workspace 256-byte) aligned */
     BITNET_ERR_CUDA = 4,              /* a CUDA launch or query failed */
     BITNET_ERR_TIMEOUT = 5,           /* a bounded on-device wait gave up */
@@ -92,6 +93,10 @@ typedef enum {
 } bitnet_path;
 
 #define BITNET_MAX_K (1 << 20)
+/* Token rows of one call: 65535 tiles of 128 tokens (the tensor-core grid's
+ * token dimension); weight rows: 2^24. */
+#define BITNET_MAX_M (65535 * 128)
+#define BITNET_MAX_N (1 << 24)
 
 /* Human-readable name of a status code (static string, never NULL). */
 BITNET_API const char *bitnet_status_string(int status);

@@ -172,7 +172,7 @@ FwdWorkspace fwd_layout(int64_t M, int64_t N, int64_t K) {
 
 bitnet_status check_shape(int64_t M, int64_t N, int64_t K) {
   if (M < 0 || N < 0 || K < 0) return BITNET_ERR_INVALID_ARG;
-  if (N < 1 || N > (1 << 24) || M > (1 << 24)) return BITNET_ERR_UNSUPPORTED_SHAPE;
+  if (N < 1 || N > BITNET_MAX_N || M > BITNET_MAX_M) return BITNET_ERR_UNSUPPORTED_SHAPE;
   if (K < 64 || K > BITNET_MAX_K || (K % 64) != 0) return BITNET_ERR_UNSUPPORTED_SHAPE;
   return BITNET_OK;
 }

@@ -79,6 +79,10 @@ def test_forward_rejects_bad_arguments(lib):
     assert _fwd(lib, K=0) == tql.BITNET_ERR_UNSUPPORTED_SHAPE
     assert _fwd(lib, K=32) == tql.BITNET_ERR_UNSUPPORTED_SHAPE
     assert _fwd(lib, N=0) == tql.BITNET_ERR_UNSUPPORTED_SHAPE
+    # the tensor-core grid holds at most 65535 token tiles of 128
+    assert _fwd(lib, M=65535 * 128 + 1) == tql.BITNET_ERR_UNSUPPORTED_SHAPE
+    assert _fwd(lib, N=(1 << 24) + 1) == tql.BITNET_ERR_UNSUPPORTED_SHAPE
+    assert _fwd(lib, K=(1 << 20) + 64) == tql.BITNET_ERR_UNSUPPORTED_SHAPE
     assert _fwd(lib, M=-1) == tql.BITNET_ERR_INVALID_ARG
     assert _fwd(lib, x=0) == tql.BITNET_ERR_INVALID_ARG
     assert _fwd(lib, y=0) == tql.BITNET_ERR_INVALID_ARG
