@@ -26,6 +26,9 @@ BITNET_ERR_TIMEOUT = 5
 BITNET_ERR_WORKSPACE = 6
 BITNET_ERR_SCRATCH_LIMIT = 7
 BITNET_STATIC_SCRATCH_MAX_N = 65536
+BITNET_MAX_K = 1 << 20
+BITNET_MAX_M = 65535 * 128
+BITNET_MAX_N = 1 << 24
 
 BITNET_F32 = 0
 BITNET_BF16 = 1

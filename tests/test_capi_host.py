@@ -35,6 +35,13 @@ def test_header_declares_the_three_core_calls():
         assert n in names
 
 
+def test_binding_limits_mirror_the_header():
+    text = open(HEADER).read()
+    for name in ("BITNET_MAX_K", "BITNET_MAX_M", "BITNET_MAX_N"):
+        expr = re.search(rf"#define {name} (\(.*\))", text).group(1)
+        assert eval(expr) == getattr(tql, name), name  # arithmetic on integer literals
+
+
 def test_every_declared_symbol_is_exported(lib):
     out = subprocess.run(["nm", "-D", "--defined-only", tql.LIB_PATH], capture_output=True,
                          text=True, check=True).stdout
@@ -80,9 +87,9 @@ def test_forward_rejects_bad_arguments(lib):
     assert _fwd(lib, K=32) == tql.BITNET_ERR_UNSUPPORTED_SHAPE
     assert _fwd(lib, N=0) == tql.BITNET_ERR_UNSUPPORTED_SHAPE
     # the tensor-core grid holds at most 65535 token tiles of 128
-    assert _fwd(lib, M=65535 * 128 + 1) == tql.BITNET_ERR_UNSUPPORTED_SHAPE
-    assert _fwd(lib, N=(1 << 24) + 1) == tql.BITNET_ERR_UNSUPPORTED_SHAPE
-    assert _fwd(lib, K=(1 << 20) + 64) == tql.BITNET_ERR_UNSUPPORTED_SHAPE
+    assert _fwd(lib, M=tql.BITNET_MAX_M + 1) == tql.BITNET_ERR_UNSUPPORTED_SHAPE
+    assert _fwd(lib, N=tql.BITNET_MAX_N + 1) == tql.BITNET_ERR_UNSUPPORTED_SHAPE
+    assert _fwd(lib, K=tql.BITNET_MAX_K + 64) == tql.BITNET_ERR_UNSUPPORTED_SHAPE
     assert _fwd(lib, M=-1) == tql.BITNET_ERR_INVALID_ARG
     assert _fwd(lib, x=0) == tql.BITNET_ERR_INVALID_ARG
     assert _fwd(lib, y=0) == tql.BITNET_ERR_INVALID_ARG
