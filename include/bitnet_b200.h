@@ -175,6 +175,11 @@ BITNET_API bitnet_status bitnet_rmsnorm_quant_act(const void *x, int x_dtype, co
  *   quant(rmsnorm(x)) * ternary(W)^T ).  Picks the warp-MMA decode GEMV for
  *   M <= 16 with at most 32 MB of packed weights and the tcgen05 kernel
  *   otherwise; both give identical bits.
+ *   (The steps: first page, 量子化の仕組み -- normalise, absmax-quantize the
+ *    activations, ternary weights, rescale by both scales; 計算パラダイム --
+ *    integer additions in place of floating-point multiply-adds; 推論最適化と
+ *    カスタムカーネル -- weights unpacked on the fly inside the matmul; The Era
+ *    of 1-bit LLMs review, 提案手法 -- RMSNorm and absmean.)
  *
  *   x, x_dtype, gamma, eps   as bitnet_rmsnorm_quant_act.
  *   W_packed, s_w            as produced by bitnet_quantize_pack_weights
@@ -187,6 +192,9 @@ BITNET_API bitnet_status bitnet_rmsnorm_quant_act(const void *x, int x_dtype, co
  *                            overlap in time (use one per stream).
  * ---------------------------------------------------------------------- */
 BITNET_API size_t bitnet_linear_forward_workspace_bytes(int64_t M, int64_t N, int64_t K);
+/* The same size under the short name the forward's plan gives it (identical
+ * result for every M, N, K). */
+BITNET_API size_t bitnet_workspace_bytes(int64_t M, int64_t N, int64_t K);
 BITNET_API bitnet_status bitnet_linear_forward(const void *x, int x_dtype, const float *gamma,
                                                float eps, const uint8_t *W_packed,
                                                const float *s_w, int64_t M, int64_t N, int64_t K,
@@ -223,8 +231,10 @@ BITNET_API bitnet_status bitnet_linear_matmul(const uint8_t *W_packed, const flo
 
 /* ------------------------------------------------------------------------
  * bitnet_linear_forward_grouped -- several independent BitLinear forwards in
- * one call: the result is exactly that of calling bitnet_linear_forward on
- * each problem in order, but the decode problems (M <= 16) share one
+ * one call (each one the forward of the first page's 量子化の仕組み, as
+ * bitnet_linear_forward; the projections of one LLaMA-like block, The Era of
+ * 1-bit LLMs review, 提案手法, are the typical group): the result is exactly
+ * that of calling bitnet_linear_forward on each problem in order, but the decode problems (M <= 16) share one
  * activation-quant launch and one matmul launch, so their weight streams
  * overlap instead of paying one launch latency each.  Typical use: the
  * projections of one decode step (q, k, v, o, gate, up, down).  Decode
@@ -274,7 +284,9 @@ BITNET_API bitnet_status bitnet_linear_forward_grouped(int count,
 
 /* ------------------------------------------------------------------------
  * bitnet_linear_forward_debug -- bitnet_linear_forward that also exports the
- * intermediate results, and can force a matmul path.
+ * intermediate results, and can force a matmul path.  (The exported values
+ * are the quantized activations of the first page's 量子化の仕組み
+ * activations bullet and the integer accumulators of its 計算パラダイム.)
  *
  *   x_q_out  [M][K] int8 (natural k order) or NULL.
  *   s_x_out  [M] fp32 or NULL.
@@ -290,7 +302,10 @@ BITNET_API bitnet_status bitnet_linear_forward_debug(
 
 /* ------------------------------------------------------------------------
  * bitnet_ternary_matmul_i32 -- debug: acc = x_q * t^T on the integer path
- * alone (first page, 計算パラダイム).
+ * alone (first page, 計算パラダイム).  Unlike a plain (x_q, W_packed, acc)
+ * signature it takes a workspace (the library allocates nothing; the
+ * kernels need the activations in their interleaved order and, for few
+ * rows, split-K partials) and a path selector (to check both kernels).
  *
  *   x_q       [M][K] int8 (natural k order, any values in [-128, 127]).
  *   W_packed  [N][K/4].
@@ -311,6 +326,9 @@ BITNET_API bitnet_status bitnet_ternary_matmul_i32(const int8_t *x_q, const uint
  * and clears the word when reset != 0.  It is per device and per process.
  * ---------------------------------------------------------------------- */
 BITNET_API bitnet_status bitnet_device_status(bitnet_stream_t stream, int reset, int *detail);
+/* bitnet_device_status(stream, 0, NULL): synchronises `stream` and returns
+ * the recorded status without clearing it. */
+BITNET_API bitnet_status bitnet_last_device_status(bitnet_stream_t stream);
 
 /* ------------------------------------------------------------------------
  * bitnet_selftest_bounded_wait -- runs one tiny kernel that waits on an
@@ -326,8 +344,10 @@ BITNET_API bitnet_status bitnet_selftest_bounded_wait(uint64_t limit_ns, bitnet_
  * decode epilogue uses for y = acc / (s_x * s_w): the correctly rounded
  * reciprocal of b and two fused residual corrections (Markstein's method),
  * which rounds to nearest even exactly like an IEEE binary32 division for
- * finite a and normal b > 0 whose quotient is zero or normal.  Lets a test
- * check that claim against a host IEEE division.
+ * finite a and normal b > 0 whose quotient is zero or normal; outside that
+ * range (subnormal or huge divisors, quotients near overflow) the kernel
+ * falls back to the IEEE division itself.  Lets a test check that the
+ * result always equals a host IEEE division.
  *
  *   a, b, q   device fp32 arrays of n elements (16-byte aligned), caller-owned.
  *   n         >= 0.

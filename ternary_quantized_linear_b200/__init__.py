@@ -47,6 +47,7 @@ EXPORTED = (
     "bitnet_device_status", "bitnet_selftest_bounded_wait", "bitnet_selftest_divide",
     "bitnet_quantize_pack_weights_static",
     "bitnet_linear_forward_grouped_workspace_bytes", "bitnet_linear_forward_grouped",
+    "bitnet_workspace_bytes", "bitnet_last_device_status",
 )
 
 BITNET_MAX_GROUP = 16
@@ -106,6 +107,8 @@ def load_library(path: str = LIB_PATH):
             "bitnet_quantize_pack_weights_static": ([P, I64, I64, P, P, P], I),
             "bitnet_linear_forward_grouped_workspace_bytes": ([I, P], SZ),
             "bitnet_linear_forward_grouped": ([I, P, P, SZ, I, P], I),
+            "bitnet_workspace_bytes": ([I64, I64, I64], SZ),
+            "bitnet_last_device_status": ([P], I),
         }
         for name, (argtypes, restype) in sig.items():
             fn = getattr(lib, name)
@@ -144,6 +147,43 @@ def _need_cuda(*ts):
             raise ValueError("tensors must be contiguous CUDA tensors")
 
 
+def _expect(t, name, dtypes, numel=None, shape=None):
+    """Check a caller-supplied buffer before its pointer reaches the library,
+    which cannot see sizes or element types: a wrong dtype or a buffer too
+    small for what the call writes raises here instead of becoming an
+    out-of-range device access."""
+    if t is None:
+        raise ValueError(f"{name} is required")
+    if not isinstance(dtypes, tuple):
+        dtypes = (dtypes,)
+    if t.dtype not in dtypes:
+        raise TypeError(f"{name} must have dtype {' or '.join(str(d) for d in dtypes)}, "
+                        f"got {t.dtype}")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+    if numel is not None and t.numel() < numel:
+        raise ValueError(f"{name} holds {t.numel()} elements; the call needs {numel}")
+
+
+def _expect_gamma(gamma, K):
+    if gamma is not None:
+        _expect(gamma, "gamma", torch.float32, shape=(K,))
+
+
+def _expect_x(x):
+    if x.dim() != 2:
+        raise ValueError("x must be 2-D [M, K]")
+    _expect(x, "x", (torch.float32, torch.bfloat16))
+    return x.shape
+
+
+def _expect_packed(W_packed, K=None):
+    _expect(W_packed, "W_packed", torch.uint8)
+    if W_packed.dim() != 2 or (K is not None and W_packed.shape[1] * 4 != K):
+        raise ValueError("W_packed must be uint8 [N, K/4]")
+    return W_packed.shape[0]
+
+
 class Workspace:
     """Device scratch reused across stream-ordered calls (one buffer per
     device and stream, grown on demand; the library clears what it needs)."""
@@ -152,8 +192,12 @@ class Workspace:
         self._buf = {}
 
     def get(self, nbytes, device, stream=None):
-        key = (device.index if isinstance(device, torch.device) else int(device),
-               0 if stream is None else stream.cuda_stream)
+        # Key on the stream the call will actually run on (the current one
+        # when none is given): two streams must never share a buffer.
+        dev = torch.device("cuda", device.index if isinstance(device, torch.device)
+                           else int(device))
+        s = torch.cuda.current_stream(dev) if stream is None else stream
+        key = (dev.index, s.cuda_stream)
         buf = self._buf.get(key)
         if buf is None or buf.numel() < nbytes:
             buf = torch.empty(max(int(nbytes), 256), dtype=torch.uint8, device=device)
@@ -180,20 +224,30 @@ def bitnet_linear_forward_workspace_bytes(M: int, N: int, K: int) -> int:
     return int(load_library().bitnet_linear_forward_workspace_bytes(M, N, K))
 
 
+def _expect_weights(W):
+    if W.dim() != 2:
+        raise ValueError("W must be 2-D [N, K]")
+    _expect(W, "W", torch.float32)
+    return W.shape
+
+
 def bitnet_quantize_pack_weights(W, W_packed=None, s_w=None, workspace=None, stream=None):
     """W fp32 [N,K] -> (W_packed uint8 [N,K/4], s_w fp32 [1]) on W's device."""
-    if W.dtype != torch.float32 or W.dim() != 2:
-        raise TypeError("W must be a 2-D float32 tensor")
-    _need_cuda(W)
-    N, K = W.shape
+    N, K = _expect_weights(W)
+    if W_packed is not None:
+        _expect(W_packed, "W_packed", torch.uint8, numel=N * (K // 4))
+    if s_w is not None:
+        _expect(s_w, "s_w", torch.float32, numel=1)
+    nb = bitnet_quantize_pack_weights_workspace_bytes(N, K)
+    if workspace is not None:
+        _expect(workspace, "workspace", torch.uint8, numel=nb)
+    _need_cuda(W, W_packed, s_w, workspace)
     if W_packed is None:
         W_packed = torch.empty((N, K // 4), dtype=torch.uint8, device=W.device)
     if s_w is None:
         s_w = torch.empty((1,), dtype=torch.float32, device=W.device)
-    nb = bitnet_quantize_pack_weights_workspace_bytes(N, K)
     if workspace is None:
         workspace = torch.empty(max(nb, 256), dtype=torch.uint8, device=W.device)
-    _need_cuda(W_packed, s_w, workspace)
     _check("bitnet_quantize_pack_weights", load_library().bitnet_quantize_pack_weights(
         _ptr(W), N, K, _ptr(W_packed), _ptr(s_w), _ptr(workspace), workspace.numel(),
         _stream(stream)))
@@ -207,10 +261,10 @@ def bitnet_quantize_pack_weights_static(W, W_packed, s_w, stream=None):
     library's own static scratch (N <= 65536 rows) replaces the workspace.
     Calls on one device share that scratch, so calls that overlap on the GPU
     race."""
-    if W.dtype != torch.float32 or W.dim() != 2:
-        raise TypeError("W must be a 2-D float32 tensor")
+    N, K = _expect_weights(W)
+    _expect(W_packed, "W_packed", torch.uint8, numel=N * (K // 4))
+    _expect(s_w, "s_w", torch.float32, numel=1)
     _need_cuda(W, W_packed, s_w)
-    N, K = W.shape
     _check("bitnet_quantize_pack_weights_static",
            load_library().bitnet_quantize_pack_weights_static(
                _ptr(W), N, K, _ptr(W_packed), _ptr(s_w), _stream(stream)))
@@ -219,15 +273,17 @@ def bitnet_quantize_pack_weights_static(W, W_packed, s_w, stream=None):
 
 def bitnet_rmsnorm_quant_act(x, gamma=None, eps=1e-5, x_q=None, s_x=None, stream=None):
     """x [M,K] fp32/bf16 -> (x_q int8 [M,K], s_x fp32 [M])."""
-    if x.dim() != 2:
-        raise ValueError("x must be 2-D")
-    _need_cuda(x, gamma)
-    M, K = x.shape
+    M, K = _expect_x(x)
+    _expect_gamma(gamma, K)
+    if x_q is not None:
+        _expect(x_q, "x_q", torch.int8, numel=M * K)
+    if s_x is not None:
+        _expect(s_x, "s_x", torch.float32, numel=M)
+    _need_cuda(x, gamma, x_q, s_x)
     if x_q is None:
         x_q = torch.empty((M, K), dtype=torch.int8, device=x.device)
     if s_x is None:
         s_x = torch.empty((M,), dtype=torch.float32, device=x.device)
-    _need_cuda(x_q, s_x)
     _check("bitnet_rmsnorm_quant_act", load_library().bitnet_rmsnorm_quant_act(
         _ptr(x), _dtype_code(x.dtype), _ptr(gamma), float(eps), M, K, _ptr(x_q), _ptr(s_x),
         _stream(stream)))
@@ -238,21 +294,36 @@ def _ws_for(M, N, K, device, workspace, stream):
     nb = bitnet_linear_forward_workspace_bytes(M, N, K)
     if workspace is None:
         workspace = _default_ws.get(nb, device, stream)
+    _expect(workspace, "workspace", torch.uint8, numel=nb)
     _need_cuda(workspace)
     return workspace
+
+
+def _expect_y(y, M, N, dtypes=(torch.float32, torch.bfloat16)):
+    _expect(y, "y", dtypes, numel=M * N)
+    if y.dim() != 2 or tuple(y.shape) != (M, N):
+        raise ValueError(f"y must have shape ({M}, {N}), got {tuple(y.shape)}")
+
+
+def _expect_scale(s_w):
+    _expect(s_w, "s_w", torch.float32, numel=1)
 
 
 def bitnet_linear_forward(x, gamma, eps, W_packed, s_w, y_dtype=torch.bfloat16, y=None,
                           workspace=None, stream=None):
     """y = BitLinear(x) with packed ternary weights; y [M,N] in y_dtype."""
-    _need_cuda(x, gamma, W_packed, s_w)
-    M, K = x.shape
-    N = W_packed.shape[0]
-    if W_packed.shape[1] * 4 != K:
-        raise ValueError("W_packed must be [N, K/4]")
+    M, K = _expect_x(x)
+    _expect_gamma(gamma, K)
+    N = _expect_packed(W_packed, K)
+    _expect_scale(s_w)
+    if y is not None:
+        _expect_y(y, M, N)
+    if workspace is not None:
+        _expect(workspace, "workspace", torch.uint8,
+                numel=bitnet_linear_forward_workspace_bytes(M, N, K))
+    _need_cuda(x, gamma, W_packed, s_w, y, workspace)
     if y is None:
         y = torch.empty((M, N), dtype=y_dtype, device=x.device)
-    _need_cuda(y)
     ws = _ws_for(M, N, K, x.device, workspace, stream)
     _check("bitnet_linear_forward", load_library().bitnet_linear_forward(
         _ptr(x), _dtype_code(x.dtype), _ptr(gamma), float(eps), _ptr(W_packed), _ptr(s_w),
@@ -262,8 +333,11 @@ def bitnet_linear_forward(x, gamma, eps, W_packed, s_w, y_dtype=torch.bfloat16, 
 
 def bitnet_linear_quantize_input(x, gamma, eps, N, workspace, stream=None):
     """Phase 1 of the forward: quantize x [M,K] into `workspace` (sized for (M,N,K))."""
+    M, K = _expect_x(x)
+    _expect_gamma(gamma, K)
+    _expect(workspace, "workspace", torch.uint8,
+            numel=bitnet_linear_forward_workspace_bytes(M, int(N), K))
     _need_cuda(x, gamma, workspace)
-    M, K = x.shape
     _check("bitnet_linear_quantize_input", load_library().bitnet_linear_quantize_input(
         _ptr(x), _dtype_code(x.dtype), _ptr(gamma), float(eps), M, int(N), K, _ptr(workspace),
         workspace.numel(), _stream(stream)))
@@ -273,13 +347,18 @@ def bitnet_linear_quantize_input(x, gamma, eps, N, workspace, stream=None):
 def bitnet_linear_matmul(W_packed, s_w, M, K, workspace, y_dtype=torch.bfloat16, y=None,
                          stream=None):
     """Phase 2: y [M,N] = dequant(quantized input in `workspace` x ternary(W)^T)."""
-    _need_cuda(W_packed, s_w, workspace)
-    N = W_packed.shape[0]
+    M, K = int(M), int(K)
+    N = _expect_packed(W_packed, K)
+    _expect_scale(s_w)
+    _expect(workspace, "workspace", torch.uint8,
+            numel=bitnet_linear_forward_workspace_bytes(M, N, K))
+    if y is not None:
+        _expect_y(y, M, N)
+    _need_cuda(W_packed, s_w, workspace, y)
     if y is None:
         y = torch.empty((M, N), dtype=y_dtype, device=W_packed.device)
-    _need_cuda(y)
     _check("bitnet_linear_matmul", load_library().bitnet_linear_matmul(
-        _ptr(W_packed), _ptr(s_w), int(M), N, int(K), _ptr(y), _dtype_code(y.dtype),
+        _ptr(W_packed), _ptr(s_w), M, N, K, _ptr(y), _dtype_code(y.dtype),
         _ptr(workspace), workspace.numel(), _stream(stream)))
     return y
 
@@ -290,11 +369,15 @@ def grouped_problems(items):
     items = list(items)
     arr = (LinearProblem * max(1, len(items)))()
     for i, (x, gamma, eps, W_packed, s_w, y) in enumerate(items):
+        M, K = _expect_x(x)
+        _expect_gamma(gamma, K)
+        N = _expect_packed(W_packed, K)
+        _expect_scale(s_w)
+        _expect_y(y, M, N)
         _need_cuda(x, gamma, W_packed, s_w, y)
-        M, K = x.shape
         arr[i] = LinearProblem(x.data_ptr(), _dtype_code(x.dtype),
                                None if gamma is None else gamma.data_ptr(), float(eps),
-                               W_packed.data_ptr(), s_w.data_ptr(), M, W_packed.shape[0], K,
+                               W_packed.data_ptr(), s_w.data_ptr(), M, N, K,
                                y.data_ptr(), _dtype_code(y.dtype))
     return arr, len(items)
 
@@ -312,6 +395,7 @@ def bitnet_linear_forward_grouped(items, workspace=None, phases=BITNET_PHASE_ALL
     nb = bitnet_linear_forward_grouped_workspace_bytes(arr, count)
     if workspace is None:
         workspace = _default_ws.get(nb, items[0][0].device if items else 0, stream)
+    _expect(workspace, "workspace", torch.uint8, numel=nb)
     _need_cuda(workspace)
     _check("bitnet_linear_forward_grouped", load_library().bitnet_linear_forward_grouped(
         count, ctypes.cast(arr, ctypes.c_void_p), _ptr(workspace), workspace.numel(),
@@ -323,9 +407,15 @@ def bitnet_linear_forward_debug(x, gamma, eps, W_packed, s_w, y_dtype=torch.floa
                                 path=BITNET_PATH_AUTO, want_y=True, workspace=None,
                                 stream=None):
     """Forward that also returns x_q (natural order), s_x and the int32 accumulators."""
-    _need_cuda(x, gamma, W_packed, s_w)
-    M, K = x.shape
-    N = W_packed.shape[0]
+    M, K = _expect_x(x)
+    _expect_gamma(gamma, K)
+    N = _expect_packed(W_packed, K)
+    _expect_scale(s_w)
+    _dtype_code(y_dtype)
+    if workspace is not None:
+        _expect(workspace, "workspace", torch.uint8,
+                numel=bitnet_linear_forward_workspace_bytes(M, N, K))
+    _need_cuda(x, gamma, W_packed, s_w, workspace)
     dev = x.device
     y = torch.empty((M, N), dtype=y_dtype, device=dev) if want_y else None
     x_q = torch.empty((M, K), dtype=torch.int8, device=dev)
@@ -342,11 +432,17 @@ def bitnet_linear_forward_debug(x, gamma, eps, W_packed, s_w, y_dtype=torch.floa
 def bitnet_ternary_matmul_i32(x_q, W_packed, path=BITNET_PATH_AUTO, acc=None, workspace=None,
                               stream=None):
     """acc int32 [M,N] = x_q (int8 [M,K]) times the ternary weights transposed."""
-    _need_cuda(x_q, W_packed)
-    if x_q.dtype != torch.int8:
-        raise TypeError("x_q must be int8")
+    if x_q.dim() != 2:
+        raise ValueError("x_q must be 2-D [M, K]")
+    _expect(x_q, "x_q", torch.int8)
     M, K = x_q.shape
-    N = W_packed.shape[0]
+    N = _expect_packed(W_packed, K)
+    if acc is not None:
+        _expect(acc, "acc", torch.int32, numel=M * N)
+    if workspace is not None:
+        _expect(workspace, "workspace", torch.uint8,
+                numel=bitnet_linear_forward_workspace_bytes(M, N, K))
+    _need_cuda(x_q, W_packed, acc, workspace)
     if acc is None:
         acc = torch.empty((M, N), dtype=torch.int32, device=x_q.device)
     ws = _ws_for(M, N, K, x_q.device, workspace, stream)
@@ -371,6 +467,8 @@ def bitnet_selftest_bounded_wait(limit_ns: int, stream=None):
 
 def bitnet_selftest_divide(a, b, stream=None):
     """a / b (fp32 CUDA tensors) through the decode epilogue's division."""
+    _expect(a, "a", torch.float32)
+    _expect(b, "b", torch.float32, numel=a.numel())
     _need_cuda(a, b)
     a = a.contiguous()
     b = b.contiguous()

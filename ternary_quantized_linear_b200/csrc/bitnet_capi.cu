@@ -863,7 +863,9 @@ BITNET_API const char* bitnet_status_string(int status) {
   switch (status) {
     case BITNET_OK: return "ok";
     case BITNET_ERR_INVALID_ARG: return "invalid argument";
-    case BITNET_ERR_UNSUPPORTED_SHAPE: return "unsupported shape (need N >= 1, 64 <= K <= 2^20, K % 64 == 0)";
+    case BITNET_ERR_UNSUPPORTED_SHAPE:
+      return "unsupported shape (need M <= 65535*128, 1 <= N <= 2^24, 64 <= K <= 2^20, "
+             "K % 64 == 0)";
     case BITNET_ERR_MISALIGNED: return "misaligned pointer (tensors 16-byte, workspace 256-byte)";
     case BITNET_ERR_CUDA: return "CUDA error";
     case BITNET_ERR_TIMEOUT: return "bounded on-device wait timed out";
@@ -1040,6 +1042,14 @@ BITNET_API bitnet_status bitnet_ternary_matmul_i32(const int8_t* x_q, const uint
   if (st != BITNET_OK) return st;
   return run_matmul(*ds, path, W_packed, ws, L, nullptr, nullptr, M, N, K, nullptr, BITNET_F32,
                     acc, false, false, s);
+}
+
+BITNET_API size_t bitnet_workspace_bytes(int64_t M, int64_t N, int64_t K) {
+  return bitnet_linear_forward_workspace_bytes(M, N, K);
+}
+
+BITNET_API bitnet_status bitnet_last_device_status(bitnet_stream_t stream) {
+  return bitnet_device_status(stream, 0, nullptr);
 }
 
 BITNET_API bitnet_status bitnet_device_status(bitnet_stream_t stream, int reset, int* detail) {

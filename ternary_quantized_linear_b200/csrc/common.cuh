@@ -256,8 +256,17 @@ __device__ __forceinline__ void named_barrier_sync(int id, int count) {
 // an ulp of 1/b and q within one ulp of a/b, the residual a - b q is exact
 // under a fused multiply-add and RN(q + (a - b q) y) = RN(a / b).  One
 // correction brings RN(a y) within one ulp; the second rounds correctly.
+//
+// Outside that range (a divisor that is subnormal, zero or above 2^126, a
+// quotient or numerator near overflow or underflow -- reachable only with
+// extreme gains or weight magnitudes) the function returns the IEEE
+// division itself, so the result is always RN(a / b).
 __device__ __forceinline__ float div_rn_by_recip(float a, float b, float y) {
   float q = __fmul_rn(a, y);
+  const float ab = fabsf(b), aq = fabsf(q), aa = fabsf(a);
+  if (!(ab >= 0x1p-126f && ab <= 0x1p126f) ||
+      (a != 0.0f && !(aq >= 0x1p-100f && aq <= 0x1p126f && aa >= 0x1p-100f && aa <= 0x1p126f)))
+    return __fdiv_rn(a, b);
   float r = __fmaf_rn(-q, b, a);
   q = __fmaf_rn(r, y, q);
   r = __fmaf_rn(-q, b, a);

@@ -166,3 +166,66 @@ def test_grouped_validation_and_workspace(lib):
     arr[0].M = 0
     arr[1].M = 0
     assert lib.bitnet_linear_forward_grouped(2, ptr, None, 0, 3, None) == tql.BITNET_OK
+
+
+def test_unsupported_shape_message_names_every_limit(lib):
+    msg = tql.bitnet_status_string(tql.BITNET_ERR_UNSUPPORTED_SHAPE)
+    for part in ("65535*128", "2^24", "2^20", "K % 64"):
+        assert part in msg
+
+
+def test_spec_named_utilities_agree(lib):
+    for M, N, K in ((1, 64, 64), (16, 3200, 8640), (2048, 14336, 4096)):
+        assert lib.bitnet_workspace_bytes(M, N, K) == \
+            tql.bitnet_linear_forward_workspace_bytes(M, N, K)
+
+
+def _cpu(shape, dtype):
+    import torch
+    return torch.zeros(shape, dtype=dtype)
+
+
+def test_binding_rejects_wrong_buffers_before_the_library(lib):
+    # CPU tensors: every check below must fire before the CUDA-tensor check,
+    # i.e. before any pointer could reach the library.
+    import torch
+    M, N, K = 4, 64, 256
+    x = _cpu((M, K), torch.bfloat16)
+    W_p = _cpu((N, K // 4), torch.uint8)
+    s_w = _cpu((1,), torch.float32)
+    y = _cpu((M, N), torch.bfloat16)
+    cases = [
+        (TypeError, lambda: tql.bitnet_linear_forward(x, None, 1e-5, W_p.view(torch.int8), s_w, y=y)),
+        (ValueError, lambda: tql.bitnet_linear_forward(x, None, 1e-5, _cpu((N, K // 8), torch.uint8),
+                                                       s_w, y=y)),
+        (TypeError, lambda: tql.bitnet_linear_forward(x, None, 1e-5, W_p, s_w.double(), y=y)),
+        (ValueError, lambda: tql.bitnet_linear_forward(x, None, 1e-5, W_p, _cpu((0,), torch.float32),
+                                                       y=y)),
+        (ValueError, lambda: tql.bitnet_linear_forward(x, None, 1e-5, W_p, s_w,
+                                                       y=_cpu((M, N - 1), torch.bfloat16))),
+        (TypeError, lambda: tql.bitnet_linear_forward(x, None, 1e-5, W_p, s_w,
+                                                      y=_cpu((M, N), torch.float16))),
+        (ValueError, lambda: tql.bitnet_linear_forward(x, _cpu((K - 1,), torch.float32), 1e-5, W_p,
+                                                       s_w, y=y)),
+        (ValueError, lambda: tql.bitnet_linear_forward(x, None, 1e-5, W_p, s_w, y=y,
+                                                       workspace=_cpu((16,), torch.uint8))),
+        (TypeError, lambda: tql.bitnet_linear_forward(x.half(), None, 1e-5, W_p, s_w, y=y)),
+        (ValueError, lambda: tql.bitnet_quantize_pack_weights_static(
+            _cpu((N, K), torch.float32), _cpu((N, K // 4 - 1), torch.uint8), s_w)),
+        (TypeError, lambda: tql.bitnet_quantize_pack_weights_static(
+            _cpu((N, K), torch.float32), W_p, _cpu((1,), torch.float16))),
+        (ValueError, lambda: tql.bitnet_quantize_pack_weights(
+            _cpu((N, K), torch.float32), W_packed=_cpu((N, K // 4 - 1), torch.uint8))),
+        (ValueError, lambda: tql.bitnet_rmsnorm_quant_act(x, None, 1e-5,
+                                                          x_q=_cpu((M, K - 1), torch.int8))),
+        (ValueError, lambda: tql.bitnet_rmsnorm_quant_act(x, None, 1e-5,
+                                                          s_x=_cpu((M - 1,), torch.float32))),
+        (TypeError, lambda: tql.bitnet_ternary_matmul_i32(_cpu((M, K), torch.int8), W_p,
+                                                          acc=_cpu((M, N), torch.int64))),
+        (ValueError, lambda: tql.bitnet_linear_matmul(W_p, s_w, M, K, _cpu((16,), torch.uint8))),
+        (ValueError, lambda: tql.grouped_problems([(x, None, 1e-5, W_p, s_w,
+                                                    _cpu((M + 1, N), torch.bfloat16))])),
+    ]
+    for exc, call in cases:
+        with pytest.raises(exc):
+            call()

@@ -422,3 +422,82 @@ def test_epilogue_division_matches_ieee_division():
         got = q.cpu().numpy()
         bad = np.nonzero(got.view(np.uint32) != ref.view(np.uint32))[0]
         assert bad.size == 0, (a[bad[:5]], b[bad[:5]], got[bad[:5]], ref[bad[:5]])
+
+
+@pytest.mark.parametrize("M", [1, 16])
+def test_grouped_shared_quantization_matches_oracle(M):
+    # q/k/v read one x and gate/up another (Llama-3-8B decode shapes): the
+    # grouped call quantizes each distinct input once and the matmuls share
+    # it.  Every output is compared with the oracle element by element, in
+    # fp32 (<= 1e-6 relative) and bf16 (<= 1 ulp).
+    case = workloads.CASES[2]
+    xq = workloads.activations(case, 0, M)   # 4096 wide: the q/k/v input
+    xg = workloads.activations(case, 2, M)   # 4096 wide: the gate/up input
+    shapes = [(0, xq), (1, xq), (1, xq), (2, xg), (2, xg)]   # q, k, v, gate, up
+    rng = np.random.default_rng(31 + M)
+    items, refs = [], []
+    xd = {id(xq): x_to_device(xq), id(xg): x_to_device(xg)}
+    for j, (si, xh) in enumerate(shapes):
+        K, N = case.shapes[si]
+        W = (rng.standard_normal((N, K)) * 0.02).astype(np.float32)
+        W_p, s_w = _dev_weights(W)
+        ref_p, ref_s = oracle_weights(W)
+        ydt = torch.float32 if j % 2 == 0 else torch.bfloat16
+        y = torch.empty((M, N), dtype=ydt, device="cuda")
+        items.append((xd[id(xh)], None, workloads.DEFAULT_EPS, W_p, s_w, y))
+        refs.append(oracle.linear_forward(xh, None, workloads.DEFAULT_EPS, ref_p, ref_s, K))
+    arr, count = tql.grouped_problems(items)
+    nb = tql.bitnet_linear_forward_grouped_workspace_bytes(arr, count)
+    ws = torch.empty(nb, dtype=torch.uint8, device="cuda")
+    for _ in range(2):   # the second call replays the cached plan
+        for it in items:
+            it[5].fill_(0)
+        tql.bitnet_linear_forward_grouped(items, workspace=ws)
+        torch.cuda.synchronize()
+        for it, ref in zip(items, refs):
+            exact = _check_y(it[5], ref["y"], ref["y_bf16"])
+            assert exact == 1.0
+
+
+def test_default_workspace_is_per_stream():
+    # Two side streams with no ordering between them, both using the
+    # binding's default workspace: each must get its own buffer, and both
+    # results must match the oracle.
+    case = workloads.CASES[2]
+    outs, refs = [], []
+    streams = [torch.cuda.Stream(), torch.cuda.Stream()]
+    jobs = []
+    for j, si in enumerate((3, 0)):
+        K, N = case.shapes[si]
+        xh = workloads.activations(case, si, 16)
+        W = workloads.weights(case, si)
+        W_p, s_w = _dev_weights(W)
+        ref_p, ref_s = oracle_weights(W)
+        refs.append(oracle.linear_forward(xh, None, workloads.DEFAULT_EPS, ref_p, ref_s, K))
+        jobs.append((x_to_device(xh), W_p, s_w))
+    torch.cuda.synchronize()
+    for _ in range(3):
+        outs = []
+        for (x, W_p, s_w), st in zip(jobs, streams):
+            with torch.cuda.stream(st):
+                outs.append(tql.bitnet_linear_forward(x, None, workloads.DEFAULT_EPS, W_p, s_w,
+                                                      y_dtype=torch.float32))
+        torch.cuda.synchronize()
+        for y, ref in zip(outs, refs):
+            _check_y(y, ref["y"], ref["y_bf16"])
+
+
+def test_division_outside_the_fast_range_is_ieee():
+    # Subnormal and zero divisors, quotients that overflow, numerators near
+    # the range ends: the epilogue division falls back to IEEE division there.
+    a = np.array([1.0, -3.0, 1e30, 7.0, 1e-30, 3.0e38, 2.0, 0.0, 5.0, -1e20],
+                 np.float32)
+    b = np.array([1e-40, 1e-39, 1e-10, 0.0, 3.0, 0.5, 3.0e38, 1e-40, np.float32(2.0 ** -126),
+                  1e-20], np.float32)
+    with np.errstate(divide="ignore", over="ignore", invalid="ignore"):
+        ref = (a / b).astype(np.float32)
+    q = tql.bitnet_selftest_divide(torch.from_numpy(a).cuda(), torch.from_numpy(b).cuda())
+    torch.cuda.synchronize()
+    got = q.cpu().numpy()
+    same = (got.view(np.uint32) == ref.view(np.uint32)) | (np.isnan(got) & np.isnan(ref))
+    assert same.all(), (a[~same], b[~same], got[~same], ref[~same])
