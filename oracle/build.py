@@ -2,8 +2,9 @@
 
 Flags: -ffp-contract=off and no fast-math, so every product and sum in the C
 source is one IEEE-754 round-to-nearest-even operation.  OpenMP only spreads
-the integer matmul's output rows over threads (results are independent of
-the thread count because integer sums are exact).
+loops whose iterations each compute whole outputs sequentially (the integer
+matmul's rows, the BitDelta and group-scale outputs), so results do not
+depend on the thread count.
 """
 import os
 import subprocess
