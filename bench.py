@@ -1,12 +1,22 @@
 #!/usr/bin/env python
 """Benchmark of the B200 BitNet b1.58 BitLinear forward.
 
-Workload (one "step"): the decode forward (RMSNorm + absmax int8 quant,
-ternary matmul, dequant) of the BitNet-3B-shaped problems
-K=3200->N=3200, 3200->8640 and 8640->3200 at M = 1, 4 and 16 tokens each
-(nine problems), bf16 activations with 0.1% x20 outlier channels, bf16
-output, inputs resident in HBM.  Weights rotate over several distinct copies
-so that a step never reads weights that are still in L2.
+Headline workload (one "step"): the decode forward (RMSNorm + absmax int8
+quant, ternary matmul, dequant) of the 70B-shaped layers K=8192->N=28672 and
+K=28672->N=8192 at M = 1, 16 and 64 tokens each -- six forwards, bf16
+activations with 0.1% x20 outlier channels, bf16 output, packed weights in
+the tiled layout (converted once, offline), inputs resident in HBM, issued
+as one bitnet_linear_forward_grouped call per step.  Every forward of a step
+reads its own copy of the weights and the steps rotate over several such
+sets (more than 1 GB of packed weights), so no step reads weights still in
+L2.  The timed region (K steps) is repeated `--trials` times; the line
+reports the median and the spread.
+
+Besides the headline the line carries the roofline of the step's dominant
+kernel, the end-to-end number through the C ABI with host buffers, a
+per-configuration table for every workload of the suite (decode GB/s,
+prefill int8 TOPS against the measured tensor-core rate), the measured int8
+peak, the clocks seen during the timed regions, and the CPU oracle's rate.
 
 Prints one JSON line (rank 0).  `--impl reference` times the CPU oracle on
 the same metric instead.  Under torchrun each rank runs an independent
@@ -26,14 +36,15 @@ if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
 METRIC = "BitLinear fwd: decode HBM GB/s & tok/s, prefill int8 TOPS (% of B200 peak)"
-WORKLOAD = "decode_bitnet3b"
+HEADLINE = "sweep_70b"
+HEADLINE_MS = (1, 16, 64)
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
-# DRAM bytes (read + write) of one grouped GEMV launch of this workload from
-# an ncu capture (summary under profiles/), valid only for the kernel source
-# it was measured on (sha256 of csrc/gemv.cuh); reported as null otherwise.
-GEMV_TRAFFIC = {"src_sha256": "d5f0e05da58c50699640b00f12d8cc0c624cb952e6282a088a857f01a4bb1d51",
-                "bytes_per_launch": 49537280}
+# DRAM bytes (read + write) of one launch of the headline's dominant kernel
+# (the tiled decode matmul over the step's four M <= 16 forwards) from an
+# ncu capture (summary under profiles/), valid only for the kernel source it
+# was measured on (sha256 of csrc/gemv_tiled.cuh); reported as null otherwise.
+GT_TRAFFIC = {"src_sha256": None, "bytes_per_launch": None}
 
 
 # ------------------------------------------------------------------ helpers
@@ -65,22 +76,10 @@ def gemv_bytes(M, N, K, y_bytes=2):
     return N * K // 4 + M * K + 8 * M + 4 + M * N * y_bytes
 
 
-def quant_bytes(M, K, x_bytes=2):
-    return M * K * x_bytes + M * K + 8 * M
-
-
-def problems():
-    from ternary_quantized_linear_b200 import workloads
-    case = workloads.CASE_BY_NAME[WORKLOAD]
-    return case, list(workloads.all_problems(case))
-
-
-def step_bytes(probs):
-    return sum(forward_bytes(M, N, K) for _, K, N, M in probs)
-
-
-def step_tokens(probs):
-    return sum(M for _, _, _, M in probs)
+def file_sha256(path):
+    import hashlib
+    with open(path, "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()
 
 
 def max_over_ranks(value, world, device=None):
@@ -98,12 +97,6 @@ def max_over_ranks(value, world, device=None):
 def job_throughput(bytes_per_step_per_rank, steps, world, max_ms):
     """Whole-job GB/s: the bytes all ranks processed over the slowest rank's time."""
     return bytes_per_step_per_rank * steps * world / (max_ms * 1e-3) / 1e9
-
-
-def file_sha256(path):
-    import hashlib
-    with open(path, "rb") as f:
-        return hashlib.sha256(f.read()).hexdigest()
 
 
 class ClockSampler:
@@ -153,12 +146,6 @@ class ClockSampler:
             self._t.join()
             self._t = None
 
-    def __enter__(self):
-        return self.start()
-
-    def __exit__(self, *exc):
-        self.stop()
-
     def summary(self):
         if not self.ok:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0,
@@ -169,35 +156,41 @@ class ClockSampler:
                 "source": "nvml", "window": self.window}
 
 
+def case_problems(name, ms=None):
+    from ternary_quantized_linear_b200 import workloads
+    case = workloads.CASE_BY_NAME[name]
+    probs = [p for p in workloads.all_problems(case) if ms is None or p[3] in ms]
+    return case, probs
+
+
 # --------------------------------------------------------------- CPU oracle
 
-def time_oracle(probs, budget_s, max_steps=None, per_problem=False, threads=1):
-    """Run the CPU oracle over the workload: whole steps (or single problems,
-    cycling, when per_problem) until budget_s is spent, its integer matmul on
-    `threads` threads.  Returns (bytes, seconds, units, threads in effect)."""
+def time_oracle(case_name, probs, budget_s, max_steps=None, threads=1):
+    """Run the CPU oracle on the problems (cycling, one forward at a time)
+    until budget_s is spent or max_steps forwards ran, its integer matmul on
+    `threads` threads.  Returns (bytes, seconds, forwards, threads in effect)."""
     import oracle
     from ternary_quantized_linear_b200 import workloads
     threads = oracle.set_threads(threads)
-    case = workloads.CASE_BY_NAME[WORKLOAD]
-    prepared = []
-    wcache = {}
+    case = workloads.CASE_BY_NAME[case_name]
+    wcache, prepared = {}, []
     for si, K, N, M in probs:
         if si not in wcache:
             W = workloads.weights(case, si)
             s_w, _ = oracle.weight_scale(W)
             W_p, _ = oracle.quantize_pack(W, s_w)
             wcache[si] = (W_p, s_w)
+            del W
         prepared.append((workloads.activations(case, si, M), wcache[si], K, N, M))
     total_b, total_s, units = 0, 0.0, 0
     t_start = time.perf_counter()
     i = 0
     while True:
-        batch = [prepared[i % len(prepared)]] if per_problem else prepared
+        x, (W_p, s_w), K, N, M = prepared[i % len(prepared)]
         t0 = time.perf_counter()
-        for x, (W_p, s_w), K, N, M in batch:
-            oracle.linear_forward(x, None, workloads.DEFAULT_EPS, W_p, s_w, K)
-            total_b += forward_bytes(M, N, K)
+        oracle.linear_forward(x, None, workloads.DEFAULT_EPS, W_p, s_w, K)
         total_s += time.perf_counter() - t0
+        total_b += forward_bytes(M, N, K)
         units += 1
         i += 1
         if max_steps is not None and units >= max_steps:
@@ -211,22 +204,22 @@ def run_reference(args):
     rank, world, _ = env_rank()
     if rank != 0:
         return 0
-    case, probs = problems()
-    # warm-up steps (untimed), then exactly `steps` timed steps; one step here is
-    # one problem of the workload (cycling through the nine), so the run stays short
-    time_oracle(probs, 0, max_steps=max(args.warmup, 0) or 1, per_problem=True)
-    b, s, units, threads = time_oracle(probs, 0, max_steps=args.steps, per_problem=True)
+    case, probs = case_problems(HEADLINE, (1,))
+    # one step here is one M = 1 forward of the headline's layers (the
+    # oracle's full step would take minutes); warm-up untimed
+    time_oracle(HEADLINE, probs, 0, max_steps=max(args.warmup, 1))
+    b, s, units, threads = time_oracle(HEADLINE, probs, 0, max_steps=args.steps)
     gbs = b / s / 1e9
     line = {
         "metric": METRIC, "value": gbs, "unit": "GB/s", "n_gpus": args.gpus, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": 1e3 * s / units, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "i8", "data": "synthetic",
         "impl": "reference",
-        "config": {"workload": WORKLOAD + ": " + case.description, "x_dtype": "bf16",
+        "config": {"workload": HEADLINE + ": " + case.description, "x_dtype": "bf16",
                    "y_dtype": "bf16"},
         "cpu_baseline": {"value": gbs, "unit": "GB/s", "cores": threads, "kind": "oracle",
-                         "sample": f"{units} single-problem steps cycling through the nine "
-                                   "decode problems, plain C oracle, 1 thread"},
+                         "sample": f"{units} single forwards (M = 1) of the 70B-shaped layers, "
+                                   "cycling, plain C oracle, 1 thread"},
         "e2e": {"value": gbs, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -234,6 +227,102 @@ def run_reference(args):
 
 
 # -------------------------------------------------------------- GPU path
+
+class DecodeWorkload:
+    """Decode forwards of one case on tiled weights: `rot` rotation sets,
+    each forward of each set with its own weight copy, one grouped call per
+    set (= one step)."""
+
+    def __init__(self, tql, workloads, case_name, ms, rot, device, tiled_cache):
+        import numpy as np
+        import torch
+        self.case, self.probs = case_problems(case_name, ms)
+        self.rot = rot
+        self.sets = []
+        base = {}
+        for si, (K, N) in enumerate(self.case.shapes):
+            if not any(p[0] == si for p in self.probs):
+                continue
+            key = (case_name, si)
+            if key not in tiled_cache:
+                W = torch.from_numpy(workloads.weights(self.case, si)).to(device)
+                W_p, s_w = tql.bitnet_quantize_pack_weights(W)
+                del W
+                tiled_cache[key] = (tql.bitnet_tile_weights(W_p), s_w)
+                del W_p
+            base[si] = tiled_cache[key]
+        for r in range(rot):
+            items = []
+            for si, K, N, M in self.probs:
+                Wt, s_w = base[si]
+                Wc = tql.TiledWeights(Wt.data.clone(), Wt.N, Wt.K)
+                xh = workloads.activations(self.case, si, M)
+                x = torch.from_numpy(xh.view(np.int16).copy()).view(torch.bfloat16).to(device)
+                y = torch.empty((M, N), dtype=torch.bfloat16, device=device)
+                items.append((x, None, workloads.DEFAULT_EPS, Wc, s_w, y))
+            arr, count = tql.grouped_problems(items)
+            nb = tql.bitnet_linear_forward_grouped_workspace_bytes(arr, count)
+            ws = torch.empty(nb, dtype=torch.uint8, device=device)
+            self.sets.append({"items": items, "arr": arr, "count": count, "ws": ws})
+        self.weight_bytes = sum(it[3].data.numel() for s in self.sets for it in s["items"])
+
+    def step_bytes(self):
+        return sum(forward_bytes(M, N, K) for _, K, N, M in self.probs)
+
+    def tokens(self):
+        return sum(M for _, _, _, M in self.probs)
+
+
+def grouped_call(lib, tql, st, phases, stream_handle):
+    rc = lib.bitnet_linear_forward_grouped(st["count"], ctypes.cast(st["arr"], ctypes.c_void_p),
+                                           ctypes.c_void_p(st["ws"].data_ptr()),
+                                           st["ws"].numel(), phases, stream_handle)
+    if rc != 0:
+        raise RuntimeError(f"bitnet_linear_forward_grouped: {tql.bitnet_status_string(rc)}")
+
+
+def timed_graph_steps(torch, stream, calls, steps, warmup, trials):
+    """calls: R callables (one step each, taking a stream handle).  Captures
+    the R steps back to back in one CUDA graph (and single-step graphs for a
+    remainder), runs `warmup` untimed steps, then times exactly `steps` steps
+    `trials` times with CUDA events on `stream`.  Returns ms per trial."""
+    R = len(calls)
+    P = ctypes.c_void_p
+    with torch.cuda.stream(stream):
+        for c in calls:
+            c(P(stream.cuda_stream))
+        stream.synchronize()
+        rotation = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(rotation, stream=stream):
+            for c in calls:
+                c(P(torch.cuda.current_stream().cuda_stream))
+        singles = []
+        for c in calls[:steps % R]:
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream):
+                c(P(torch.cuda.current_stream().cuda_stream))
+            singles.append(g)
+
+        def run(k):
+            for _ in range(k // R):
+                rotation.replay()
+            for g in singles[:k % R]:
+                g.replay()
+
+        run(max(warmup, 1))
+        stream.synchronize()
+        out = []
+        for _ in range(trials):
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            run(steps)
+            e1.record(stream)
+            stream.synchronize()
+            out.append(e0.elapsed_time(e1))
+    del rotation, singles
+    return out
+
 
 def run_ours(args):
     import numpy as np
@@ -254,415 +343,111 @@ def run_ours(args):
 
     tql_build.build()
     lib = tql.load_library()
-    case, probs = problems()
-    R = args.rotations
-    eps = workloads.DEFAULT_EPS
-
-    # ---- inputs resident in HBM: R rotation sets x 9 problems
-    packed = {}
-    for si in range(len(case.shapes)):
-        W = torch.from_numpy(workloads.weights(case, si)).to(device)
-        packed[si] = tql.bitnet_quantize_pack_weights(W)
-        del W
-    sets = []
-    for r in range(R):
-        entries = []
-        for si, K, N, M in probs:
-            W_p, s_w = packed[si]
-            xh = workloads.activations(case, si, M)
-            x = torch.from_numpy(xh.view(np.int16).copy()).view(torch.bfloat16).to(device)
-            y = torch.empty((M, N), dtype=torch.bfloat16, device=device)
-            ws = torch.zeros(tql.bitnet_linear_forward_workspace_bytes(M, N, K),
-                             dtype=torch.uint8, device=device)
-            entries.append({"x": x, "W_p": W_p.clone(), "s_w": s_w, "y": y, "ws": ws,
-                            "M": M, "N": N, "K": K})
-        sets.append(entries)
-    torch.cuda.synchronize()
-    weight_mb_per_set = sum(e["W_p"].numel() for e in sets[0]) / 1e6
-
     stream = torch.cuda.Stream(device=device)
-    P = ctypes.c_void_p
-
-    # one grouped-forward description (and workspace) per rotation set
-    groups = []
-    for r in range(R):
-        items = [(e["x"], None, eps, e["W_p"], e["s_w"], e["y"]) for e in sets[r]]
-        arr, count = tql.grouped_problems(items)
-        nb = tql.bitnet_linear_forward_grouped_workspace_bytes(arr, count)
-        ws = torch.empty(nb, dtype=torch.uint8, device=device)
-        groups.append((arr, count, ws))
-
-    def grouped(r, sp, phases=tql.BITNET_PHASE_ALL):
-        arr, count, ws = groups[r]
-        rc = lib.bitnet_linear_forward_grouped(count, ctypes.cast(arr, P), P(ws.data_ptr()),
-                                               ws.numel(), phases, sp)
-        if rc != 0:
-            raise RuntimeError(f"bitnet_linear_forward_grouped: {tql.bitnet_status_string(rc)}")
-
-    # ---- CUDA graphs: one per rotation set (one step = one grouped call = 2
-    # launches) and one holding the R steps of a whole rotation back to back,
-    # so the timed loop pays one graph launch per R steps
-    graphs = []
-    with torch.cuda.stream(stream):
-        grouped(0, P(stream.cuda_stream))  # first call sets up the device state
-        stream.synchronize()
-        for r in range(R):
-            g = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(g, stream=stream):
-                grouped(r, P(torch.cuda.current_stream().cuda_stream))
-            graphs.append(g)
-        rotation = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(rotation, stream=stream):
-            for r in range(R):
-                grouped(r, P(torch.cuda.current_stream().cuda_stream))
-    torch.cuda.synchronize()
-
-    def run_steps(k):
-        # exactly k steps, cycling through the rotation sets
-        for _ in range(k // R):
-            rotation.replay()
-        for r in range(k % R):
-            graphs[r].replay()
+    peaks, peak_src = load_peaks()
+    hbm_peak = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+    tiled_cache = {}
 
     def barrier():
         if world > 1:
             import torch.distributed as dist
             dist.barrier(device_ids=[local_rank])
 
-    # ---- warm-up, then exactly K timed steps (graph replays).  The clock
-    # sampler runs from the warm-up through the kernel-timing replays below:
-    # the timed steps alone last a few milliseconds, about one NVML sample.
-    clocks = ClockSampler(local_rank, window="warm-up, the timed steps and the kernel-timing "
-                                              "graph replays (all back-to-back GPU work)")
+    # ---- headline: the 70B decode step, R rotation sets of six forwards
+    head = DecodeWorkload(tql, workloads, HEADLINE, HEADLINE_MS, args.rotations, device,
+                          tiled_cache)
+    torch.cuda.synchronize()
+    calls = [lambda h, st=st: grouped_call(lib, tql, st, tql.BITNET_PHASE_ALL, h)
+             for st in head.sets]
+    clocks = ClockSampler(local_rank, window="the headline's warm-up and timed trials, the "
+                                             "kernel timing and the per-config timings")
     clocks.start()
-    with torch.cuda.stream(stream):
-        run_steps(args.warmup)
-    stream.synchronize()
     barrier()
-    torch.cuda.synchronize()
-    e0 = torch.cuda.Event(enable_timing=True)
-    e1 = torch.cuda.Event(enable_timing=True)
-    with torch.cuda.stream(stream):
-        e0.record(stream)
-        run_steps(args.steps)
-        e1.record(stream)
-    stream.synchronize()
-    torch.cuda.synchronize()
+    trial_ms = timed_graph_steps(torch, stream, calls, args.steps, args.warmup, args.trials)
     barrier()
-    local_ms = e0.elapsed_time(e1)
-    max_ms = max_over_ranks(local_ms, world, device)
-    sb = step_bytes(probs)
+    med_ms = statistics.median(trial_ms)
+    max_ms = max_over_ranks(med_ms, world, device)
+    sb = head.step_bytes()
     value = job_throughput(sb, args.steps, world, max_ms)
+    trial_gbs = sorted(sb * args.steps / (t * 1e-3) / 1e9 for t in trial_ms)
     ms_per_step = max_ms / args.steps
-    launches = 2 * args.steps
+    # kernel launches per step: the grouped decode quant + the tiled decode
+    # matmul for the four M <= 16 forwards; quant + tcgen05 for each M = 64
+    n_big = sum(1 for p in head.probs if p[3] > 16)
+    launches_per_step = 2 + 2 * n_big
 
-    # ---- kernel durations with CUDA events: the grouped matmul (dominant
-    # kernel) and the grouped activation quant, each captured alone as CUDA
-    # graphs over the rotation sets (the matmul phase reads the activations
-    # the full steps above left in each set's workspace) and replayed
-    # back to back: the average launch duration in a steady stream.
-    def phase_ms(phases):
-        gs = []
-        with torch.cuda.stream(stream):
-            for r in range(R):
-                g = torch.cuda.CUDAGraph()
-                with torch.cuda.graph(g, stream=stream):
-                    grouped(r, P(torch.cuda.current_stream().cuda_stream), phases)
-                gs.append(g)
-            for i in range(args.warmup):
-                gs[i % R].replay()
-            stream.synchronize()
-            a = torch.cuda.Event(enable_timing=True)
-            b = torch.cuda.Event(enable_timing=True)
-            a.record(stream)
-            for i in range(args.steps):
-                gs[i % R].replay()
-            b.record(stream)
-            stream.synchronize()
-        ms = a.elapsed_time(b) / args.steps
-        del gs
-        return ms
-
-    m_avg = phase_ms(tql.BITNET_PHASE_MATMUL)
-    q_avg = phase_ms(tql.BITNET_PHASE_QUANTIZE)
-    clocks.stop()
-    gemv_b = sum(gemv_bytes(M, N, K) for _, K, N, M in probs)
-    peaks, peak_src = load_peaks()
-    hbm_peak = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
-    achieved = gemv_b / (m_avg * 1e-3) / 1e9
-    sha = file_sha256(os.path.join(ROOT, "ternary_quantized_linear_b200", "csrc", "gemv.cuh"))
-    traffic = GEMV_TRAFFIC["bytes_per_launch"] if GEMV_TRAFFIC["src_sha256"] == sha else None
-
-    # ---- the same nine problems one launch pair at a time (two-phase single API)
-    single = []
-    one = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in probs]
-    acc_q = {j: [] for j in range(len(probs))}
-    acc_m = {j: [] for j in range(len(probs))}
-    with torch.cuda.stream(stream):
-        for i in range(min(args.steps, 20) + 2):
-            r = i % R
-            torch.cuda._sleep(2_000_000)
-            for j, e in enumerate(sets[r]):
-                one[j][0].record(stream)
-                tql.bitnet_linear_quantize_input(e["x"], None, eps, e["N"], e["ws"],
-                                                 stream=stream)
-                one[j][1].record(stream)
-                tql.bitnet_linear_matmul(e["W_p"], e["s_w"], e["M"], e["K"], e["ws"], y=e["y"],
-                                         stream=stream)
-                one[j][2].record(stream)
-            stream.synchronize()
-            if i >= 2:
-                for j in range(len(probs)):
-                    acc_q[j].append(one[j][0].elapsed_time(one[j][1]))
-                    acc_m[j].append(one[j][1].elapsed_time(one[j][2]))
-    for j, (si, K, N, M) in enumerate(probs):
-        t = statistics.mean(acc_m[j])
-        single.append({"K": K, "N": N, "M": M, "matmul_us": round(1e3 * t, 2),
-                       "matmul_gbs": round(gemv_bytes(M, N, K) / (t * 1e-3) / 1e9, 1),
-                       "quant_us": round(1e3 * statistics.mean(acc_q[j]), 2)})
-
+    # ---- roofline: the tiled decode matmul of the four M <= 16 forwards
+    # (the dominant kernel: 4 x 58.7 MB of the step's 6 x 58.7 MB), timed
+    # alone as the matmul phase of a group holding just those forwards.
+    small_sets = []
+    for st in head.sets:
+        items = [it for it in st["items"] if it[0].shape[0] <= 16]
+        arr, count = tql.grouped_problems(items)
+        small_sets.append({"items": items, "arr": arr, "count": count, "ws": st["ws"]})
+    with torch.cuda.stream(stream):   # quantize once into each set's workspace
+        for st in small_sets:
+            grouped_call(lib, tql, st, tql.BITNET_PHASE_QUANTIZE, ctypes.c_void_p(stream.cuda_stream))
+        stream.synchronize()
+    mm_calls = [lambda h, st=st: grouped_call(lib, tql, st, tql.BITNET_PHASE_MATMUL, h)
+                for st in small_sets]
+    k_ms = timed_graph_steps(torch, stream, mm_calls, args.steps, args.warmup, args.trials)
+    gt_ms = statistics.median(k_ms) / args.steps
+    gt_b = sum(gemv_bytes(M, N, K) for _, K, N, M in head.probs if M <= 16)
+    achieved = gt_b / (gt_ms * 1e-3) / 1e9
+    sha = file_sha256(os.path.join(ROOT, "ternary_quantized_linear_b200", "csrc",
+                                   "gemv_tiled.cuh"))
+    traffic = GT_TRAFFIC["bytes_per_launch"] if GT_TRAFFIC["src_sha256"] == sha else None
     roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm_peak,
                 "unit": "GB/s", "frac": round(achieved / hbm_peak, 4), "traffic": traffic,
-                "kernel": "ternary_gemv_kernel, one grouped launch over the nine problems "
-                          "(matmul + fused dequant)",
-                "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)",
-                "algorithmic_bytes_per_launch": gemv_b,
-                "avg_launch_us": round(1e3 * m_avg, 2),
-                "quant_kernel_us": round(1e3 * q_avg, 2),
+                "kernel": "ternary_gemv_tiled_kernel, one launch over the step's four M <= 16 "
+                          "forwards (matmul + fused dequant)",
+                "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs, burst copy)",
+                "algorithmic_bytes_per_launch": gt_b,
+                "avg_launch_us": round(1e3 * gt_ms, 2),
                 "how": "CUDA events around back-to-back CUDA-graph replays of the matmul "
-                       "phase alone (6 rotating weight sets), average per launch",
-                "single_problem_launches": single}
+                       f"phase alone over {args.rotations} rotating weight sets, median of "
+                       f"{args.trials} trials of {args.steps} launches"}
 
-    # ---- end to end through the public call with host buffers: each set's
-    # nine inputs live in one pinned host buffer and one device buffer (and
-    # likewise the outputs), so a step is one upload, one grouped call and
-    # one download.
+    # ---- int8 tensor-core rate (the prefill roofline's denominator)
+    i8 = measure_int8_peak(tql, torch, stream)
+
+    # ---- per-configuration table
+    per_config = []
+    if not args.no_configs:
+        per_config = measure_configs(args, tql, lib, workloads, torch, stream, device, hbm_peak,
+                                     i8, tiled_cache, head, value, gt_ms, gt_b)
+    clocks.stop()
+
+    # ---- end to end through the C ABI with host buffers
     e2e = None
     if not args.no_e2e:
-        def packed(shapes, dtype):
-            # 128-byte aligned offsets of each tensor in one flat buffer
-            offs, n = [], 0
-            for shp in shapes:
-                offs.append(n)
-                n += -(-shp[0] * shp[1] // 64) * 64
-            return offs, n
+        e2e = measure_e2e(args, tql, lib, torch, stream, device, head, world, barrier)
 
-        e2e_sets, e2e_yoffs = [], []
-        for r in range(R):
-            xs = [tuple(e["x"].shape) for e in sets[r]]
-            ys = [tuple(e["y"].shape) for e in sets[r]]
-            xo, xn = packed(xs, torch.bfloat16)
-            yo, yn = packed(ys, torch.bfloat16)
-            dx = torch.empty(xn, dtype=torch.bfloat16, device=device)
-            dy = torch.empty(yn, dtype=torch.bfloat16, device=device)
-            hx = torch.empty(xn, dtype=torch.bfloat16).pin_memory()
-            hy = torch.empty(yn, dtype=torch.bfloat16).pin_memory()
-            items = []
-            for j, e in enumerate(sets[r]):
-                xv = dx[xo[j]:xo[j] + xs[j][0] * xs[j][1]].view(xs[j])
-                hx[xo[j]:xo[j] + xs[j][0] * xs[j][1]].view(xs[j]).copy_(e["x"].cpu())
-                yv = dy[yo[j]:yo[j] + ys[j][0] * ys[j][1]].view(ys[j])
-                items.append((xv, None, eps, e["W_p"], e["s_w"], yv))
-            arr, count = tql.grouped_problems(items)
-            nb = tql.bitnet_linear_forward_grouped_workspace_bytes(arr, count)
-            ws = torch.empty(nb, dtype=torch.uint8, device=device)
-            e2e_sets.append((dx, dy, hx, hy, arr, count, ws, items))
-            e2e_yoffs.append(yo)
-        h2d = sum(e["x"].numel() * 2 for e in sets[0])
-        d2h = sum(e["y"].numel() * 2 for e in sets[0])
-        def grouped_call(r, st):
-            _, _, _, _, arr, count, ws, _ = e2e_sets[r]
-            rc = lib.bitnet_linear_forward_grouped(count, ctypes.cast(arr, P), P(ws.data_ptr()),
-                                                   ws.numel(), tql.BITNET_PHASE_ALL,
-                                                   P(st.cuda_stream))
-            if rc != 0:
-                raise RuntimeError(tql.bitnet_status_string(rc))
-
-        def e2e_serial():
-            # one stream: upload, call, download, step after step
-            def step(r):
-                dx, dy, hx, hy = e2e_sets[r][:4]
-                dx.copy_(hx, non_blocking=True)
-                grouped_call(r, stream)
-                hy.copy_(dy, non_blocking=True)
-
-            with torch.cuda.stream(stream):
-                for i in range(args.warmup):
-                    step(i % R)
-                stream.synchronize()
-                barrier()
-                a0 = torch.cuda.Event(enable_timing=True)
-                a1 = torch.cuda.Event(enable_timing=True)
-                a0.record(stream)
-                for i in range(args.steps):
-                    step(i % R)
-                a1.record(stream)
-                stream.synchronize()
-            return a0.elapsed_time(a1)
-
-        def e2e_pipelined():
-            # Three streams -- uploads, grouped calls, downloads -- so step i's
-            # upload overlaps step i-1's call and download.  Per rotation set,
-            # events order upload -> call -> download and gate the reuse of
-            # its buffers: an upload waits for the set's previous call (its
-            # input buffer is free), a call for the set's previous download
-            # (its output buffer is free).  The copies and event operations go
-            # straight to the CUDA driver (handles and pointers resolved before
-            # the loop) so the host keeps ahead of the device.
-            cu = ctypes.CDLL("libcuda.so.1")
-            VP, U64, SZ = ctypes.c_void_p, ctypes.c_uint64, ctypes.c_size_t
-            h2d_copy, d2h_copy = cu.cuMemcpyHtoDAsync_v2, cu.cuMemcpyDtoHAsync_v2
-            h2d_copy.argtypes = [U64, VP, SZ, VP]
-            d2h_copy.argtypes = [VP, U64, SZ, VP]
-            ev_create, ev_record, ev_destroy = cu.cuEventCreate, cu.cuEventRecord, cu.cuEventDestroy_v2
-            ev_create.argtypes = [ctypes.POINTER(VP), ctypes.c_uint]
-            ev_record.argtypes = [VP, VP]
-            ev_destroy.argtypes = [VP]
-            wait_ev = cu.cuStreamWaitEvent
-            wait_ev.argtypes = [VP, VP, ctypes.c_uint]
-
-            def ok(rc, what):
-                if rc != 0:
-                    raise RuntimeError(f"{what} returned CUDA driver error {rc}")
-
-            s_up, s_dn = torch.cuda.Stream(device), torch.cuda.Stream(device)
-            h_up, h_c, h_dn = VP(s_up.cuda_stream), VP(stream.cuda_stream), VP(s_dn.cuda_stream)
-            events = []
-
-            def new_event():
-                e = VP()
-                ok(ev_create(ctypes.byref(e), 2), "cuEventCreate")  # CU_EVENT_DISABLE_TIMING
-                events.append(e)
-                return e
-
-            up = [new_event() for _ in range(R)]
-            called = [new_event() for _ in range(R)]
-            down = [new_event() for _ in range(R)]
-            used = [False] * R
-            plan = []
-            for r in range(R):
-                dx, dy, hx, hy, arr, count, ws, _ = e2e_sets[r]
-                nx, ny = dx.numel() * dx.element_size(), dy.numel() * dy.element_size()
-                assert nx == hx.numel() * hx.element_size() and hx.is_pinned()
-                assert ny == hy.numel() * hy.element_size() and hy.is_pinned()
-                plan.append((U64(dx.data_ptr()), VP(hx.data_ptr()), SZ(nx),
-                             VP(hy.data_ptr()), U64(dy.data_ptr()), SZ(ny),
-                             count, ctypes.cast(arr, P), P(ws.data_ptr()), ws.numel()))
-            call = lib.bitnet_linear_forward_grouped
-            phase = tql.BITNET_PHASE_ALL
-
-            def step(r):
-                dxp, hxp, nx, hyp, dyp, ny, count, arr_p, ws_p, nb = plan[r]
-                if used[r]:
-                    ok(wait_ev(h_up, called[r], 0), "cuStreamWaitEvent")
-                ok(h2d_copy(dxp, hxp, nx, h_up), "cuMemcpyHtoDAsync")
-                ok(ev_record(up[r], h_up), "cuEventRecord")
-                ok(wait_ev(h_c, up[r], 0), "cuStreamWaitEvent")
-                if used[r]:
-                    ok(wait_ev(h_c, down[r], 0), "cuStreamWaitEvent")
-                rc = call(count, arr_p, ws_p, nb, phase, h_c)
-                if rc != 0:
-                    raise RuntimeError(tql.bitnet_status_string(rc))
-                ok(ev_record(called[r], h_c), "cuEventRecord")
-                ok(wait_ev(h_dn, called[r], 0), "cuStreamWaitEvent")
-                ok(d2h_copy(hyp, dyp, ny, h_dn), "cuMemcpyDtoHAsync")
-                ok(ev_record(down[r], h_dn), "cuEventRecord")
-                used[r] = True
-
-            def join():
-                stream.wait_stream(s_up)
-                stream.wait_stream(s_dn)
-
-            try:
-                for i in range(args.warmup):
-                    step(i % R)
-                join()
-                torch.cuda.synchronize()
-                barrier()
-                a0 = torch.cuda.Event(enable_timing=True)
-                a1 = torch.cuda.Event(enable_timing=True)
-                a0.record(stream)
-                s_up.wait_stream(stream)
-                s_dn.wait_stream(stream)
-                for i in range(args.steps):
-                    step(i % R)
-                join()
-                a1.record(stream)
-                torch.cuda.synchronize()
-            finally:
-                torch.cuda.synchronize()
-                for e in events:
-                    ev_destroy(e)
-            # the downloads hold what the device path computed for each set
-            for r in range(R):
-                if not used[r]:
-                    continue
-                hy, items = e2e_sets[r][3], e2e_sets[r][7]
-                got = torch.cat([hy[o:o + it[5].numel()] for o, it in zip(e2e_yoffs[r], items)])
-                want = torch.cat([e["y"].reshape(-1).cpu() for e in sets[r]])
-                if not torch.equal(got.view(torch.int16), want.view(torch.int16)):
-                    raise RuntimeError(f"pipelined end-to-end outputs of set {r} differ")
-            return a0.elapsed_time(a1)
-
-        how_serial = ("per step: one pinned-host -> device copy of the nine inputs, one "
-                      "bitnet_linear_forward_grouped call (C ABI, eager), one device -> "
-                      "pinned-host copy of the nine outputs, all on one stream; device-timed")
-        how_pipe = ("per step: one pinned-host -> device copy of the nine inputs, one "
-                    "bitnet_linear_forward_grouped call (C ABI, eager), one device -> "
-                    "pinned-host copy of the nine outputs; uploads, calls and downloads on "
-                    "three streams ordered per rotation set by events (copies and events "
-                    "issued through the CUDA driver API), so step i's upload overlaps step "
-                    "i-1's call and download; every step's copies inside the timed region; "
-                    "outputs checked against the device path; device-timed")
-        note = None
-        try:
-            local = e2e_pipelined()
-            how = how_pipe
-        except Exception as exc:  # noqa: BLE001 -- any failure: measure on one stream
-            torch.cuda.synchronize()
-            note = f"pipelined measurement failed ({exc}); serial measurement instead"
-            local = e2e_serial()
-            how = how_serial
-        e2e_ms = max_over_ranks(local, world, device)
-        e2e = {"value": job_throughput(sb, args.steps, world, e2e_ms), "unit": "GB/s",
-               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-               "ms_per_step": e2e_ms / args.steps, "how": how}
-        if note:
-            e2e["note"] = note
-
-    # ---- prefill extra: tcgen05 GEMM TOPS on the Llama-3-8B FFN shapes
-    prefill = None
-    if not args.no_prefill:
-        prefill = measure_prefill(args, device, stream, peaks, peak_src)
-
-    # ---- offline weight quant + pack, timed on its own (not in the metric)
     weight_pack = None
     if not args.no_weight_pack:
         try:
-            weight_pack = measure_weight_pack(args, device, stream, hbm_peak)
+            weight_pack = measure_weight_pack(args, tql, workloads, torch, stream, device,
+                                              hbm_peak)
         except Exception as exc:  # noqa: BLE001 -- report, keep the line
             weight_pack = {"error": str(exc)}
 
-    # ---- CPU baseline (rank 0, one GPU only)
+    # ---- CPU baseline (rank 0, one GPU only): the oracle on a bounded
+    # sample of the headline workload
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        b, s, units, threads = time_oracle(probs, args.cpu_budget)
+        _, probs1 = case_problems(HEADLINE, (1,))
+        b, s, units, threads = time_oracle(HEADLINE, probs1, args.cpu_budget)
         cpu = {"value": b / s / 1e9, "unit": "GB/s", "cores": threads, "kind": "oracle",
-               "sample": f"{units} full decode step(s) (all nine problems) of the plain C "
-                         f"oracle, {threads} thread(s), {s:.1f} s"}
-        # the same oracle with its integer matmul spread over every host core
+               "sample": f"{units} single forwards (M = 1) of the two 70B-shaped layers, "
+                         f"cycling, plain C oracle, {threads} thread(s), {s:.1f} s"}
         ncores = os.cpu_count() or 1
-        b, s, units, threads = time_oracle(probs, args.cpu_budget / 2, threads=ncores)
+        b, s, units, threads = time_oracle(HEADLINE, probs1, args.cpu_budget / 2, threads=ncores)
         cpu["all_cores"] = {"value": b / s / 1e9, "unit": "GB/s", "cores": threads,
-                            "sample": f"{units} full decode step(s), integer matmul on "
-                                      f"{threads} thread(s), {s:.1f} s"}
+                            "sample": f"{units} forwards, integer matmul on {threads} "
+                                      f"thread(s), {s:.1f} s"}
 
     if world > 1:
         import torch.distributed as dist
-        for g in graphs:
-            del g
-        graphs.clear()
-        del rotation
         dist.barrier(device_ids=[local_rank])
         dist.destroy_process_group()
 
@@ -672,41 +457,314 @@ def run_ours(args):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "i8",
             "data": "synthetic",
-            "config": {"workload": WORKLOAD + ": " + case.description,
-                       "problems": [[K, N, M] for _, K, N, M in probs],
-                       "x_dtype": "bf16", "y_dtype": "bf16",
-                       "l2": f"inputs larger than L2: {R} rotating weight/activation sets, "
-                             f"{R * weight_mb_per_set:.0f} MB of packed weights",
-                       "launch": "one bitnet_linear_forward_grouped call per step (a grouped "
-                                 "activation-quant launch + a grouped matmul launch with "
-                                 "programmatic dependent launch); the R rotation steps "
-                                 "captured back to back in one CUDA graph, replayed "
-                                 "steps/R times (single-step graphs for a remainder)",
+            "config": {"workload": HEADLINE + ": " + head.case.description,
+                       "problems": [[K, N, M] for _, K, N, M in head.probs],
+                       "x_dtype": "bf16", "y_dtype": "bf16", "weights": "tiled layout",
+                       "l2": f"inputs larger than L2: {args.rotations} rotating sets, every "
+                             f"forward with its own weight copy, "
+                             f"{head.weight_bytes / 1e6:.0f} MB of packed weights",
+                       "launch": "one bitnet_linear_forward_grouped call per step; the R "
+                                 "rotation steps captured back to back in one CUDA graph",
                        "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
-            "tok_s": round(world * step_tokens(probs) * args.steps / (max_ms * 1e-3), 1),
+            "trials": {"count": args.trials, "median_gbs": round(statistics.median(trial_gbs), 1),
+                       "min_gbs": round(trial_gbs[0], 1), "max_gbs": round(trial_gbs[-1], 1)},
+            "tok_s": round(world * head.tokens() * args.steps / (max_ms * 1e-3), 1),
             "roofline": roofline,
+            "int8_peak": i8,
+            "per_config": per_config,
             "cpu_baseline": cpu,
             "e2e": e2e,
-            "gpu_launches": launches,
+            "gpu_launches": launches_per_step * args.steps,
             "clocks": clocks.summary(),
-            "prefill": prefill,
             "weight_pack": weight_pack,
         }
         print(json.dumps(line), flush=True)
     return 0
 
 
-def measure_weight_pack(args, device, stream, hbm_peak):
-    """bitnet_quantize_pack_weights on the decode workload's three fp32
-    matrices (261 MB together, more than L2), cycled, outputs preallocated:
-    the absmean pass reads W, the quantize pass reads it again and writes the
+def measure_int8_peak(tql, torch, stream):
+    """Dense int8 tensor-core rate: one CTA per SM issuing 128x256x32
+    tcgen05 MMAs back to back (A in shared memory, and in tensor memory as
+    the forward's kernels use it), timed with CUDA events."""
+    sms = torch.cuda.get_device_properties(stream.device).multi_processor_count
+    res = {}
+    for name, tmem in (("a_smem", False), ("a_tmem", True)):
+        iters = 20000
+        with torch.cuda.stream(stream):
+            tql.bitnet_selftest_mma_i8(1000, sms, tmem, stream=stream)
+            stream.synchronize()
+            best = None
+            for _ in range(3):
+                e0 = torch.cuda.Event(enable_timing=True)
+                e1 = torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
+                ops = tql.bitnet_selftest_mma_i8(iters, sms, tmem, stream=stream)
+                e1.record(stream)
+                stream.synchronize()
+                ms = e0.elapsed_time(e1)
+                best = ms if best is None else min(best, ms)
+        res[name] = round(ops / (best * 1e-3) / 1e12, 1)
+    code, _ = tql.bitnet_device_status(reset=False, stream=stream)
+    return {"tops": max(res.values()), "a_smem_tops": res["a_smem"],
+            "a_tmem_tops": res["a_tmem"], "source": "measured",
+            "how": f"bitnet_selftest_mma_i8: {sms} CTAs x 20000 tcgen05.mma kind::i8 "
+                   "128x256x32, best of 3, CUDA events", "status_ok": code == tql.BITNET_OK,
+            "spec_tops": 4500.0}
+
+
+def measure_configs(args, tql, lib, workloads, torch, stream, device, hbm_peak, i8, tiled_cache,
+                    head, head_value, head_gt_ms, head_gt_b):
+    """One entry per workload of the suite: decode GB/s (and the roofline of
+    its decode matmul launch), prefill int8 TOPS against the measured rate."""
+    import numpy as np
+    out = []
+    P = ctypes.c_void_p
+    steps, trials = max(6, args.steps // 2), max(3, args.trials // 2)
+
+    # tiny: one fp32 forward through the plain C-ABI call
+    x, W = workloads.tiny_inputs()
+    W_p, s_w = tql.bitnet_quantize_pack_weights(torch.from_numpy(W).to(device))
+    xd = torch.from_numpy(x).to(device)
+    y = torch.empty((16, 512), dtype=torch.float32, device=device)
+    ws = torch.empty(tql.bitnet_linear_forward_workspace_bytes(16, 512, 256), dtype=torch.uint8,
+                     device=device)
+
+    def tiny_call(h):
+        rc = lib.bitnet_linear_forward(P(xd.data_ptr()), tql.BITNET_F32, None,
+                                       ctypes.c_float(1e-5), P(W_p.data_ptr()),
+                                       P(s_w.data_ptr()), 16, 512, 256, P(y.data_ptr()),
+                                       tql.BITNET_F32, P(ws.data_ptr()), ws.numel(), h)
+        if rc != 0:
+            raise RuntimeError(tql.bitnet_status_string(rc))
+
+    t = statistics.median(timed_graph_steps(torch, stream, [tiny_call], 50, 5, trials)) / 50
+    b = forward_bytes(16, 512, 256, 4, 4)
+    out.append({"config": "tiny", "problems": [[256, 512, 16]], "us_per_forward": round(1e3 * t, 2),
+                "gbs": round(b / (t * 1e-3) / 1e9, 1), "note": "fp32 in/out, L2-resident, "
+                "launch-bound (two launches of a 65 KB problem)"})
+
+    # decode configs: grouped steps on tiled weights
+    for name in ("decode_bitnet3b", "decode_llama3_8b"):
+        wl = DecodeWorkload(tql, workloads, name, None, 6, device, tiled_cache)
+        calls = [lambda h, st=st: grouped_call(lib, tql, st, tql.BITNET_PHASE_ALL, h)
+                 for st in wl.sets]
+        ms = statistics.median(timed_graph_steps(torch, stream, calls, steps, 3, trials)) / steps
+        mm_calls = [lambda h, st=st: grouped_call(lib, tql, st, tql.BITNET_PHASE_MATMUL, h)
+                    for st in wl.sets]
+        mm = statistics.median(timed_graph_steps(torch, stream, mm_calls, steps, 3, trials)) / steps
+        gb = sum(gemv_bytes(M, N, K) for _, K, N, M in wl.probs)
+        out.append({"config": name, "problems": [[K, N, M] for _, K, N, M in wl.probs],
+                    "step_us": round(1e3 * ms, 2),
+                    "gbs": round(wl.step_bytes() / (ms * 1e-3) / 1e9, 1),
+                    "tok_s": round(wl.tokens() / (ms * 1e-3), 1),
+                    "matmul_us": round(1e3 * mm, 2),
+                    "matmul_frac_of_hbm": round(gb / (mm * 1e-3) / 1e9 / hbm_peak, 4)})
+        del wl
+        torch.cuda.empty_cache()
+
+    # prefill: the tcgen05 kernel on tiled weights
+    def prefill(name, ms_list):
+        case = workloads.CASE_BY_NAME[name]
+        rows = []
+        for si, (K, N) in enumerate(case.shapes):
+            key = (name, si)
+            if key not in tiled_cache:
+                Wd = torch.from_numpy(workloads.weights(case, si)).to(device)
+                Wp, sw = tql.bitnet_quantize_pack_weights(Wd)
+                del Wd
+                tiled_cache[key] = (tql.bitnet_tile_weights(Wp), sw)
+            Wt, sw = tiled_cache[key]
+            for M in ms_list:
+                xh = workloads.activations(case, si, M)
+                xs = torch.from_numpy(xh.view(np.int16).copy()).view(torch.bfloat16).to(device)
+                yy = torch.empty((M, N), dtype=torch.bfloat16, device=device)
+                items = [(xs, None, 1e-5, Wt, sw, yy)]
+                arr, count = tql.grouped_problems(items)
+                nb = tql.bitnet_linear_forward_grouped_workspace_bytes(arr, count)
+                wsp = torch.empty(nb, dtype=torch.uint8, device=device)
+                st = {"items": items, "arr": arr, "count": count, "ws": wsp}
+                n_it = 4 if M >= 4096 else 10
+                f = statistics.median(timed_graph_steps(
+                    torch, stream, [lambda h: grouped_call(lib, tql, st, tql.BITNET_PHASE_ALL, h)],
+                    n_it, 2, trials)) / n_it
+                mm = statistics.median(timed_graph_steps(
+                    torch, stream,
+                    [lambda h: grouped_call(lib, tql, st, tql.BITNET_PHASE_MATMUL, h)],
+                    n_it, 2, trials)) / n_it
+                ops = 2.0 * M * N * K
+                tops = ops / (mm * 1e-3) / 1e12
+                rows.append({"K": K, "N": N, "M": M, "forward_us": round(1e3 * f, 2),
+                             "gemm_us": round(1e3 * mm, 2), "gemm_tops": round(tops, 1),
+                             "forward_tops": round(ops / (f * 1e-3) / 1e12, 1),
+                             "frac_of_measured_int8": round(tops / i8["tops"], 4),
+                             "frac_of_4500_spec": round(tops / 4500.0, 4)})
+                del xs, yy, wsp, st
+        return rows
+
+    pre = prefill("prefill_llama3_8b", (512, 2048, 8192))
+    out.append({"config": "prefill_llama3_8b", "shapes": pre,
+                "tops_mean": round(statistics.mean(r["gemm_tops"] for r in pre), 1),
+                "frac_of_measured_int8_mean": round(statistics.mean(
+                    r["frac_of_measured_int8"] for r in pre), 4)})
+    pre70 = prefill(HEADLINE, (1024, 4096))
+    out.append({"config": HEADLINE, "decode": {
+        "problems": [[K, N, M] for _, K, N, M in head.probs], "gbs": round(head_value, 1),
+        "tiled_gemv_us": round(1e3 * head_gt_ms, 2),
+        "tiled_gemv_frac_of_hbm": round(head_gt_b / (head_gt_ms * 1e-3) / 1e9 / hbm_peak, 4)},
+        "prefill": pre70,
+        "prefill_tops_mean": round(statistics.mean(r["gemm_tops"] for r in pre70), 1)})
+    return out
+
+
+def measure_e2e(args, tql, lib, torch, stream, device, head, world, barrier):
+    """The headline step through the public C-ABI call with host buffers:
+    every step uploads its six inputs from pinned host memory, makes the
+    grouped call and downloads its six outputs; uploads, calls and downloads
+    run on three streams ordered per rotation set by events, so step i's
+    upload overlaps step i-1's call and download.  Device-timed."""
+    P = ctypes.c_void_p
+    R = len(head.sets)
+    e2e_sets = []
+    for st in head.sets:
+        xs = [tuple(it[0].shape) for it in st["items"]]
+        ys = [tuple(it[5].shape) for it in st["items"]]
+
+        def packed(shapes):
+            offs, n = [], 0
+            for s in shapes:
+                offs.append(n)
+                n += -(-s[0] * s[1] // 64) * 64
+            return offs, n
+
+        xo, xn = packed(xs)
+        yo, yn = packed(ys)
+        dx = torch.empty(xn, dtype=torch.bfloat16, device=device)
+        dy = torch.empty(yn, dtype=torch.bfloat16, device=device)
+        hx = torch.empty(xn, dtype=torch.bfloat16).pin_memory()
+        hy = torch.empty(yn, dtype=torch.bfloat16).pin_memory()
+        items = []
+        for j, it in enumerate(st["items"]):
+            n = xs[j][0] * xs[j][1]
+            hx[xo[j]:xo[j] + n].view(xs[j]).copy_(it[0].cpu())
+            xv = dx[xo[j]:xo[j] + n].view(xs[j])
+            yv = dy[yo[j]:yo[j] + ys[j][0] * ys[j][1]].view(ys[j])
+            items.append((xv, None, it[2], it[3], it[4], yv))
+        arr, count = tql.grouped_problems(items)
+        e2e_sets.append({"dx": dx, "dy": dy, "hx": hx, "hy": hy, "arr": arr, "count": count,
+                         "ws": st["ws"], "items": items, "yo": yo})
+    h2d = sum(it[0].numel() * 2 for it in head.sets[0]["items"])
+    d2h = sum(it[5].numel() * 2 for it in head.sets[0]["items"])
+
+    cu = ctypes.CDLL("libcuda.so.1")
+    VP, U64, SZ = ctypes.c_void_p, ctypes.c_uint64, ctypes.c_size_t
+    h2d_copy, d2h_copy = cu.cuMemcpyHtoDAsync_v2, cu.cuMemcpyDtoHAsync_v2
+    h2d_copy.argtypes = [U64, VP, SZ, VP]
+    d2h_copy.argtypes = [VP, U64, SZ, VP]
+    ev_create, ev_record, ev_destroy = cu.cuEventCreate, cu.cuEventRecord, cu.cuEventDestroy_v2
+    ev_create.argtypes = [ctypes.POINTER(VP), ctypes.c_uint]
+    ev_record.argtypes = [VP, VP]
+    ev_destroy.argtypes = [VP]
+    wait_ev = cu.cuStreamWaitEvent
+    wait_ev.argtypes = [VP, VP, ctypes.c_uint]
+
+    def ok(rc, what):
+        if rc != 0:
+            raise RuntimeError(f"{what} returned CUDA driver error {rc}")
+
+    s_up, s_dn = torch.cuda.Stream(device), torch.cuda.Stream(device)
+    h_up, h_c, h_dn = VP(s_up.cuda_stream), VP(stream.cuda_stream), VP(s_dn.cuda_stream)
+    events = []
+
+    def new_event():
+        e = VP()
+        ok(ev_create(ctypes.byref(e), 2), "cuEventCreate")  # CU_EVENT_DISABLE_TIMING
+        events.append(e)
+        return e
+
+    up = [new_event() for _ in range(R)]
+    called = [new_event() for _ in range(R)]
+    down = [new_event() for _ in range(R)]
+    used = [False] * R
+    plan = []
+    for s in e2e_sets:
+        plan.append((U64(s["dx"].data_ptr()), VP(s["hx"].data_ptr()),
+                     SZ(s["dx"].numel() * 2), VP(s["hy"].data_ptr()), U64(s["dy"].data_ptr()),
+                     SZ(s["dy"].numel() * 2), s["count"], ctypes.cast(s["arr"], P),
+                     P(s["ws"].data_ptr()), s["ws"].numel()))
+    call = lib.bitnet_linear_forward_grouped
+
+    def step(r):
+        dxp, hxp, nx, hyp, dyp, ny, count, arr_p, ws_p, nb = plan[r]
+        if used[r]:
+            ok(wait_ev(h_up, called[r], 0), "cuStreamWaitEvent")
+        ok(h2d_copy(dxp, hxp, nx, h_up), "cuMemcpyHtoDAsync")
+        ok(ev_record(up[r], h_up), "cuEventRecord")
+        ok(wait_ev(h_c, up[r], 0), "cuStreamWaitEvent")
+        if used[r]:
+            ok(wait_ev(h_c, down[r], 0), "cuStreamWaitEvent")
+        rc = call(count, arr_p, ws_p, nb, tql.BITNET_PHASE_ALL, h_c)
+        if rc != 0:
+            raise RuntimeError(tql.bitnet_status_string(rc))
+        ok(ev_record(called[r], h_c), "cuEventRecord")
+        ok(wait_ev(h_dn, called[r], 0), "cuStreamWaitEvent")
+        ok(d2h_copy(hyp, dyp, ny, h_dn), "cuMemcpyDtoHAsync")
+        ok(ev_record(down[r], h_dn), "cuEventRecord")
+        used[r] = True
+
+    def join():
+        stream.wait_stream(s_up)
+        stream.wait_stream(s_dn)
+
+    times = []
+    try:
+        for i in range(args.warmup):
+            step(i % R)
+        join()
+        torch.cuda.synchronize()
+        barrier()
+        for _ in range(max(3, args.trials // 2)):
+            a0 = torch.cuda.Event(enable_timing=True)
+            a1 = torch.cuda.Event(enable_timing=True)
+            a0.record(stream)
+            s_up.wait_stream(stream)
+            s_dn.wait_stream(stream)
+            for i in range(args.steps):
+                step(i % R)
+            join()
+            a1.record(stream)
+            torch.cuda.synchronize()
+            times.append(a0.elapsed_time(a1))
+    finally:
+        torch.cuda.synchronize()
+        for e in events:
+            ev_destroy(e)
+    # the downloads hold what the device path computes for each set
+    for r, s in enumerate(e2e_sets):
+        if not used[r]:
+            continue
+        got = torch.cat([s["hy"][o:o + it[5].numel()] for o, it in zip(s["yo"], s["items"])])
+        want = torch.cat([it[5].reshape(-1).cpu() for it in head.sets[r]["items"]])
+        if not torch.equal(got.view(torch.int16), want.view(torch.int16)):
+            raise RuntimeError(f"end-to-end outputs of set {r} differ from the device path")
+    med = statistics.median(times)
+    e2e_ms = max_over_ranks(med, world, device)
+    return {"value": round(job_throughput(head.step_bytes(), args.steps, world, e2e_ms), 2),
+            "unit": "GB/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+            "ms_per_step": e2e_ms / args.steps,
+            "how": "per step: one pinned-host -> device copy of the six inputs, one "
+                   "bitnet_linear_forward_grouped call (C ABI, eager), one device -> "
+                   "pinned-host copy of the six outputs; uploads, calls and downloads on "
+                   "three streams ordered per rotation set by events (copies and events "
+                   "through the CUDA driver API); outputs checked against the device path; "
+                   f"device-timed, median of {len(times)} trials"}
+
+
+def measure_weight_pack(args, tql, workloads, torch, stream, device, hbm_peak):
+    """bitnet_quantize_pack_weights on the BitNet-3B-shaped fp32 matrices
+    (261 MB together, more than L2), cycled, outputs preallocated: the
+    absmean pass reads W, the quantize pass reads it again and writes the
     packed codes (the scale must be known before any code is decided)."""
-    import torch
-
-    import ternary_quantized_linear_b200 as tql
-    from ternary_quantized_linear_b200 import workloads
-
-    case = workloads.CASE_BY_NAME[WORKLOAD]
+    case = workloads.CASE_BY_NAME["decode_bitnet3b"]
     mats = []
     for si, (K, N) in enumerate(case.shapes):
         W = torch.from_numpy(workloads.weights(case, si)).to(device)
@@ -716,9 +774,9 @@ def measure_weight_pack(args, device, stream, hbm_peak):
         ws = torch.empty(nb, dtype=torch.uint8, device=device)
         mats.append((W, W_p, s_w, ws, N, K))
     n = len(mats)
-    reps = max(3, min(args.steps, 30))
+    reps = 10
     with torch.cuda.stream(stream):
-        for i in range(max(args.warmup, 3) * n):
+        for i in range(3 * n):
             W, W_p, s_w, ws, _, _ = mats[i % n]
             tql.bitnet_quantize_pack_weights(W, W_p, s_w, ws, stream=stream)
         stream.synchronize()
@@ -732,84 +790,30 @@ def measure_weight_pack(args, device, stream, hbm_peak):
     per = []
     tot_b, tot_ms = 0, 0.0
     for j, (W, W_p, _, _, N, K) in enumerate(mats):
-        ms = sum(ev[i][0].elapsed_time(ev[i][1]) for i in range(j, reps * n, n)) / reps
+        ms = statistics.median(ev[i][0].elapsed_time(ev[i][1]) for i in range(j, reps * n, n))
         b = 2 * 4 * N * K + N * K // 4
         tot_b += b
         tot_ms += ms
         per.append({"N": N, "K": K, "us": round(1e3 * ms, 2),
                     "gbs": round(b / (ms * 1e-3) / 1e9, 1)})
     gbs = tot_b / (tot_ms * 1e-3) / 1e9
-    return {"workload": f"{WORKLOAD} weights, fp32, cycled", "matrices": per,
+    return {"workload": "decode_bitnet3b weights, fp32, cycled", "matrices": per,
             "gbs": round(gbs, 1), "frac_of_hbm": round(gbs / hbm_peak, 4),
-            "bytes": "two reads of W (absmean, then quantize) + the packed write",
-            "how": "CUDA events around each call on the launching stream, "
-                   f"{reps} calls per matrix after warm-up"}
-
-
-def measure_prefill(args, device, stream, peaks, peak_src):
-    """Tensor-core path on the Llama-3-8B FFN shapes at M = 2048 (not the
-    headline number): TOPS of the GEMM kernel alone and of the whole forward."""
-    import numpy as np
-    import torch
-
-    import ternary_quantized_linear_b200 as tql
-    from ternary_quantized_linear_b200 import workloads
-
-    case = workloads.CASE_BY_NAME["prefill_llama3_8b"]
-    M = 2048
-    out = []
-    i8_peak = 2.0 * float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
-    for si, (K, N) in enumerate(case.shapes):
-        W = torch.from_numpy(workloads.weights(case, si)).to(device)
-        W_p, s_w = tql.bitnet_quantize_pack_weights(W)
-        del W
-        xh = workloads.activations(case, si, M)
-        R = 6
-        xs = [torch.from_numpy(xh.view(np.int16).copy()).view(torch.bfloat16).to(device)
-              for _ in range(R)]
-        wps = [W_p.clone() for _ in range(R)]
-        y = torch.empty((M, N), dtype=torch.bfloat16, device=device)
-        ws = torch.zeros(tql.bitnet_linear_forward_workspace_bytes(M, N, K), dtype=torch.uint8,
-                         device=device)
-        iters = 20
-        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(iters)]
-        with torch.cuda.stream(stream):
-            for i in range(3):
-                tql.bitnet_linear_forward(xs[i % R], None, 1e-5, wps[i % R], s_w, y=y,
-                                          workspace=ws, stream=stream)
-            for i in range(iters):
-                evs[i][0].record(stream)
-                tql.bitnet_linear_quantize_input(xs[i % R], None, 1e-5, N, ws, stream=stream)
-                evs[i][1].record(stream)
-                tql.bitnet_linear_matmul(wps[i % R], s_w, M, K, ws, y=y, stream=stream)
-                evs[i][2].record(stream)
-            stream.synchronize()
-        gemm_ms = statistics.median(e[1].elapsed_time(e[2]) for e in evs)
-        fwd_ms = statistics.median(e[0].elapsed_time(e[2]) for e in evs)
-        ops = 2.0 * M * N * K
-        out.append({"K": K, "N": N, "M": M, "gemm_us": round(1e3 * gemm_ms, 2),
-                    "gemm_tops": round(ops / (gemm_ms * 1e-3) / 1e12, 1),
-                    "forward_tops": round(ops / (fwd_ms * 1e-3) / 1e12, 1)})
-    tops = [o["gemm_tops"] for o in out]
-    return {"workload": "prefill_llama3_8b at M=2048 (K=4096->N=14336, K=14336->N=4096)",
-            "shapes": out, "gemm_tops_mean": round(statistics.mean(tops), 1),
-            "frac_of_int8_peak": round(statistics.mean(tops) / i8_peak, 4),
-            "int8_peak_tops": i8_peak,
-            "int8_peak_source": f"{peak_src} bf16 burst x 2 (dense int8 = 2x bf16 rate)",
-            "frac_of_4500_tops_spec": round(statistics.mean(tops) / 4500.0, 4)}
+            "bytes": "two reads of W (absmean, then quantize) + the packed write"}
 
 
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__)
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=200)
-    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--steps", type=int, default=30)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--trials", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--rotations", type=int, default=6)
+    ap.add_argument("--rotations", type=int, default=3)
     ap.add_argument("--cpu-budget", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
-    ap.add_argument("--no-prefill", action="store_true")
+    ap.add_argument("--no-configs", action="store_true")
     ap.add_argument("--no-weight-pack", action="store_true")
     args = ap.parse_args(argv)
     if args.warmup < 3 and args.impl == "ours":

@@ -92,6 +92,12 @@ typedef enum {
     BITNET_PATH_GEMM = 2   /* tcgen05 + TMA GEMM with TMEM accumulators */
 } bitnet_path;
 
+/* Layout of the packed weights a forward reads (see bitnet_tile_weights). */
+typedef enum {
+    BITNET_LAYOUT_ROWS = 0,   /* W_packed [N][K/4], the exported layout */
+    BITNET_LAYOUT_TILED = 1   /* 128-row x 256-k tiles, bitnet_tile_weights */
+} bitnet_layout;
+
 #define BITNET_MAX_K (1 << 20)
 /* Token rows of one call: 65535 tiles of 128 tokens (the tensor-core grid's
  * token dimension); weight rows: 2^24. */
@@ -103,6 +109,12 @@ BITNET_API const char *bitnet_status_string(int status);
 
 /* Library version as 10000*major + 100*minor + patch. */
 BITNET_API int bitnet_version(void);
+
+/* The CUDA runtime error code (cudaError_t) behind the last
+ * BITNET_ERR_CUDA a call of this thread returned, 0 if none since the last
+ * query; *name (may be NULL) receives the runtime's name for it.  Clears the
+ * record. */
+BITNET_API int bitnet_last_cuda_error(const char **name);
 
 /* ------------------------------------------------------------------------
  * bitnet_quantize_pack_weights -- absmean ternary quantization + packing.
@@ -154,6 +166,73 @@ BITNET_API bitnet_status bitnet_quantize_pack_weights_static(const float *W, int
                                                              int64_t K, uint8_t *W_packed,
                                                              float *s_w,
                                                              bitnet_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * bitnet_tile_weights -- rearrange packed weights into the tiled layout the
+ * matmul kernels stream fastest (an offline step, like the packing itself;
+ * first page, 主な発見: the packed weights are stored for the kernels, and
+ * 推論最適化とカスタムカーネル / タイル化行列乗算: the kernels read them
+ * tile by tile).  The codes are unchanged; only their order is:
+ *
+ *   RB = ceil(N/128) row blocks, KC = ceil(K/256) k chunks; tile (rb, c)
+ *   occupies bytes [(rb*KC + c) * 8192, +8192) of W_tiled.  Inside a tile,
+ *   row r (0..127) is 64 bytes = four 16-byte pieces, piece q holding the
+ *   packed bytes of weights k = 256c + 64q .. +63 of row 128*rb + r (i.e.
+ *   W_packed[(128*rb + r)*K/4 + 64c + 16q .. +16]) at byte
+ *   r*64 + 16*(q ^ ((r >> 1) & 3)).  Rows >= N and weights >= K are zero.
+ *
+ * With this layout a run of tiles of one row block is one contiguous range,
+ * which a copy engine moves in one operation.
+ *
+ *   W_packed  [N][K/4] bytes in (device).
+ *   W_tiled   bitnet_tiled_weights_bytes(N, K) bytes out (device, 16-byte
+ *             aligned), caller-owned.
+ * Shape rules as every entry point; returns 0 from the size query for an
+ * unsupported shape.  Queues one kernel on `stream`.
+ * ---------------------------------------------------------------------- */
+BITNET_API size_t bitnet_tiled_weights_bytes(int64_t N, int64_t K);
+BITNET_API bitnet_status bitnet_tile_weights(const uint8_t *W_packed, int64_t N, int64_t K,
+                                             uint8_t *W_tiled, bitnet_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * bitnet_tile_weights_pair -- the pair-tiled layout of two packed matrices
+ * of the same shape [N][K/4] (the gate and up projections of a SwiGLU, The
+ * Era of 1-bit LLMs review, 提案手法): unit (rb, c), at bytes
+ * [(rb*KC + c) * 16384, +16384), is tile (rb, c) of Wa (layout of
+ * bitnet_tile_weights) followed by tile (rb, c) of Wb.  Codes unchanged.
+ *   W_pair  bitnet_tiled_pair_weights_bytes(N, K) bytes out (16-byte aligned).
+ * ---------------------------------------------------------------------- */
+BITNET_API size_t bitnet_tiled_pair_weights_bytes(int64_t N, int64_t K);
+BITNET_API bitnet_status bitnet_tile_weights_pair(const uint8_t *Wa_packed,
+                                                  const uint8_t *Wb_packed, int64_t N, int64_t K,
+                                                  uint8_t *W_pair, bitnet_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * bitnet_swiglu_forward -- the feed-forward's gate and up BitLinear forwards
+ * of one input and the SwiGLU that joins them, y = silu(gate) * up with
+ * silu(z) = z / (1 + e^-z) (The Era of 1-bit LLMs review, 提案手法: SwiGLU in
+ * the LLaMA-like block; each forward as bitnet_linear_forward).  One
+ * activation-quant launch and one matmul launch that computes both
+ * projections of every output row and applies the activation in its
+ * epilogue: gate and up are bit-identical to two separate forwards (fp32),
+ * the activation is computed in fp32 (expf, then IEEE add, divide and
+ * multiply; within a few fp32 ulp of the exact value).
+ *
+ *   W_pair                 pair-tiled gate/up weights (bitnet_tile_weights_pair).
+ *   s_w_gate, s_w_up       their scales (device, one fp32 each).
+ *   M                      0 <= M <= 16 (decode); larger M returns
+ *                          BITNET_ERR_UNSUPPORTED_SHAPE.
+ *   y                      [M][N] out, fp32 or bf16.
+ *   workspace              >= bitnet_swiglu_forward_workspace_bytes(M, N, K),
+ *                          256-byte aligned, contents on entry irrelevant.
+ * ---------------------------------------------------------------------- */
+BITNET_API size_t bitnet_swiglu_forward_workspace_bytes(int64_t M, int64_t N, int64_t K);
+BITNET_API bitnet_status bitnet_swiglu_forward(const void *x, int x_dtype, const float *gamma,
+                                               float eps, const uint8_t *W_pair,
+                                               const float *s_w_gate, const float *s_w_up,
+                                               int64_t M, int64_t N, int64_t K, void *y,
+                                               int y_dtype, void *workspace,
+                                               size_t workspace_bytes, bitnet_stream_t stream);
 
 /* ------------------------------------------------------------------------
  * bitnet_rmsnorm_quant_act -- fused RMSNorm + per-token absmax int8 quant.
@@ -268,11 +347,12 @@ typedef struct {
     int x_dtype;              /* bitnet_dtype */
     const float *gamma;       /* [K] or NULL */
     float eps;
-    const uint8_t *W_packed;  /* [N][K/4] */
+    const uint8_t *W_packed;  /* [N][K/4] row-major, or the tiled layout (w_layout) */
     const float *s_w;         /* [1] */
     int64_t M, N, K;
     void *y;                  /* [M][N] */
     int y_dtype;              /* bitnet_dtype */
+    int w_layout;             /* bitnet_layout of W_packed (zero = row-major) */
 } bitnet_linear_problem;
 
 BITNET_API size_t bitnet_linear_forward_grouped_workspace_bytes(
@@ -299,6 +379,69 @@ BITNET_API bitnet_status bitnet_linear_forward_debug(
     const float *s_w, int64_t M, int64_t N, int64_t K, void *y, int y_dtype, void *workspace,
     size_t workspace_bytes, int8_t *x_q_out, float *s_x_out, int32_t *acc_out, int path,
     bitnet_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * Group-wise scales (bitnet.cpp article, グループ量子化と正規化: the weights
+ * and the activations are split into groups quantized independently, so
+ * that the groups need no communication).  Reading: G = K / group_k
+ * contiguous groups along K, group_k a multiple of 256 with G <= 512:
+ *   s_w[g]   = 1 / max(mean |W| over all rows and the group's columns, 1e-5)
+ *              (fp64 sum in the order of the per-tensor scale, applied to the
+ *              N x group_k block of group g)
+ *   t        = clamp(rint(W * s_w[g(k)]), -1, 1), packed as W_packed
+ *   x_n      = RMSNorm of the whole row (as bitnet_rmsnorm_quant_act)
+ *   s_x[m,g] = 127 / max(max over the group of |x_n|, 1e-5)
+ *   x_q      = clamp(rint(x_n * s_x[m,g(k)]), -128, 127)
+ *   acc_g    = sum over the group of x_q * t            (int32, exact)
+ *   y[m,n]   = sum_g (float)acc_g / (s_x[m,g] * s_w[g]): fp32 terms (product
+ *              rounded first, correctly rounded division) summed in fp64 in
+ *              increasing g and rounded once to fp32.
+ * With group_k = K this is the per-tensor forward bit for bit.
+ *
+ * bitnet_quantize_pack_weights_group_scales -- W [N][K] fp32 -> W_packed
+ *   [N][K/4], s_w [G] (device); workspace >= the size query (fp64 row sums).
+ * bitnet_linear_forward_group_scales -- the forward.  W_packed in either
+ *   layout (w_layout, a bitnet_layout); the tiled decode kernel serves tiled
+ *   weights with M <= 16, the tcgen05 kernel the rest, one K split per group;
+ *   both write the groups' integer sums and a last kernel forms y.
+ *   y          [M][N] fp32 or bf16, or NULL when acc_out is given.
+ *   x_q_out    [M][K] int8 natural order, s_x_out [M][G] fp32, acc_out
+ *              [G][M][N] int32 (the group sums): optional debug exports.
+ *   workspace  >= bitnet_linear_forward_group_scales_workspace_bytes, 256-byte
+ *              aligned, contents on entry irrelevant.
+ * Unsupported group_k -> BITNET_ERR_UNSUPPORTED_SHAPE.
+ * ---------------------------------------------------------------------- */
+BITNET_API size_t bitnet_quantize_pack_weights_group_scales_workspace_bytes(int64_t N,
+                                                                            int64_t K,
+                                                                            int64_t group_k);
+BITNET_API bitnet_status bitnet_quantize_pack_weights_group_scales(
+    const float *W, int64_t N, int64_t K, int64_t group_k, uint8_t *W_packed, float *s_w,
+    void *workspace, size_t workspace_bytes, bitnet_stream_t stream);
+BITNET_API size_t bitnet_linear_forward_group_scales_workspace_bytes(int64_t M, int64_t N,
+                                                                     int64_t K,
+                                                                     int64_t group_k);
+BITNET_API bitnet_status bitnet_linear_forward_group_scales(
+    const void *x, int x_dtype, const float *gamma, float eps, const uint8_t *W_packed,
+    int w_layout, const float *s_w, int64_t M, int64_t N, int64_t K, int64_t group_k, void *y,
+    int y_dtype, void *workspace, size_t workspace_bytes, int8_t *x_q_out, float *s_x_out,
+    int32_t *acc_out, bitnet_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * bitnet_linear_forward_ex -- one forward described by a problem record, so
+ * that it can read weights in either layout (problem->w_layout); otherwise
+ * as bitnet_linear_forward_debug: the same steps, the same bits, optional
+ * exports of x_q (natural order), s_x and the int32 accumulators, and a
+ * matmul path selector.  problem->y may be NULL when acc_out is given.
+ * With tiled weights the automatic path takes the tiled decode kernel for
+ * every M <= 16 and the tcgen05 kernel above.
+ *
+ *   workspace  >= bitnet_linear_forward_workspace_bytes(M, N, K).
+ * ---------------------------------------------------------------------- */
+BITNET_API bitnet_status bitnet_linear_forward_ex(const bitnet_linear_problem *problem,
+                                                  void *workspace, size_t workspace_bytes,
+                                                  int8_t *x_q_out, float *s_x_out,
+                                                  int32_t *acc_out, int path,
+                                                  bitnet_stream_t stream);
 
 /* ------------------------------------------------------------------------
  * bitnet_ternary_matmul_i32 -- debug: acc = x_q * t^T on the integer path
@@ -356,6 +499,19 @@ BITNET_API bitnet_status bitnet_selftest_bounded_wait(uint64_t limit_ns, bitnet_
  * ---------------------------------------------------------------------- */
 BITNET_API bitnet_status bitnet_selftest_divide(const float *a, const float *b, float *q,
                                                 int64_t n, bitnet_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * bitnet_selftest_mma_i8 -- measurement aid, not part of the forward: queues
+ * one kernel of `ctas` CTAs (one per SM for a whole-GPU figure), each
+ * issuing `iters` back-to-back int8 tensor-core MMAs of shape 128 x 256 x 32
+ * (tcgen05.mma kind::i8, A from shared memory, or from tensor memory like
+ * the forward's kernels when a_in_tmem != 0) on zero data.  Timing it with
+ * events on `stream` gives the dense int8 rate of the GPU as clocked:
+ * int8 operations = 2 * 128 * 256 * 32 * iters * ctas.  Touches no tensor.
+ *   iters  1 .. 1e8;  ctas  1 .. 65535.
+ * ---------------------------------------------------------------------- */
+BITNET_API bitnet_status bitnet_selftest_mma_i8(int64_t iters, int ctas, int a_in_tmem,
+                                                bitnet_stream_t stream);
 
 #ifdef __cplusplus
 }

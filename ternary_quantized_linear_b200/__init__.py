@@ -48,7 +48,18 @@ EXPORTED = (
     "bitnet_quantize_pack_weights_static",
     "bitnet_linear_forward_grouped_workspace_bytes", "bitnet_linear_forward_grouped",
     "bitnet_workspace_bytes", "bitnet_last_device_status",
+    "bitnet_tiled_weights_bytes", "bitnet_tile_weights", "bitnet_linear_forward_ex",
+    "bitnet_selftest_mma_i8",
+    "bitnet_tiled_pair_weights_bytes", "bitnet_tile_weights_pair",
+    "bitnet_swiglu_forward_workspace_bytes", "bitnet_swiglu_forward",
+    "bitnet_last_cuda_error",
+    "bitnet_quantize_pack_weights_group_scales_workspace_bytes",
+    "bitnet_quantize_pack_weights_group_scales",
+    "bitnet_linear_forward_group_scales_workspace_bytes", "bitnet_linear_forward_group_scales",
 )
+
+BITNET_LAYOUT_ROWS = 0
+BITNET_LAYOUT_TILED = 1
 
 BITNET_MAX_GROUP = 16
 BITNET_PHASE_QUANTIZE = 1
@@ -62,7 +73,7 @@ class LinearProblem(ctypes.Structure):
                 ("gamma", ctypes.c_void_p), ("eps", ctypes.c_float),
                 ("W_packed", ctypes.c_void_p), ("s_w", ctypes.c_void_p),
                 ("M", ctypes.c_int64), ("N", ctypes.c_int64), ("K", ctypes.c_int64),
-                ("y", ctypes.c_void_p), ("y_dtype", ctypes.c_int)]
+                ("y", ctypes.c_void_p), ("y_dtype", ctypes.c_int), ("w_layout", ctypes.c_int)]
 
 
 class BitnetError(RuntimeError):
@@ -109,6 +120,20 @@ def load_library(path: str = LIB_PATH):
             "bitnet_linear_forward_grouped": ([I, P, P, SZ, I, P], I),
             "bitnet_workspace_bytes": ([I64, I64, I64], SZ),
             "bitnet_last_device_status": ([P], I),
+            "bitnet_tiled_weights_bytes": ([I64, I64], SZ),
+            "bitnet_tile_weights": ([P, I64, I64, P, P], I),
+            "bitnet_linear_forward_ex": ([P, P, SZ, P, P, P, I, P], I),
+            "bitnet_selftest_mma_i8": ([I64, I, I, P], I),
+            "bitnet_tiled_pair_weights_bytes": ([I64, I64], SZ),
+            "bitnet_tile_weights_pair": ([P, P, I64, I64, P, P], I),
+            "bitnet_swiglu_forward_workspace_bytes": ([I64, I64, I64], SZ),
+            "bitnet_swiglu_forward": ([P, I, P, F, P, P, P, I64, I64, I64, P, I, P, SZ, P], I),
+            "bitnet_last_cuda_error": ([ctypes.POINTER(ctypes.c_char_p)], I),
+            "bitnet_quantize_pack_weights_group_scales_workspace_bytes": ([I64, I64, I64], SZ),
+            "bitnet_quantize_pack_weights_group_scales": ([P, I64, I64, I64, P, P, P, SZ, P], I),
+            "bitnet_linear_forward_group_scales_workspace_bytes": ([I64, I64, I64, I64], SZ),
+            "bitnet_linear_forward_group_scales": (
+                [P, I, P, F, P, I, P, I64, I64, I64, I64, P, I, P, SZ, P, P, P, P], I),
         }
         for name, (argtypes, restype) in sig.items():
             fn = getattr(lib, name)
@@ -120,7 +145,13 @@ def load_library(path: str = LIB_PATH):
 
 def _check(fn_name, code):
     if code != BITNET_OK:
-        msg = load_library().bitnet_status_string(code).decode()
+        lib = load_library()
+        msg = lib.bitnet_status_string(code).decode()
+        if code == BITNET_ERR_CUDA:
+            name = ctypes.c_char_p()
+            err = lib.bitnet_last_cuda_error(ctypes.byref(name))
+            if err:
+                msg += f" ({name.value.decode() if name.value else 'cudaError'} = {err})"
         raise BitnetError(fn_name, code, msg)
 
 
@@ -363,23 +394,245 @@ def bitnet_linear_matmul(W_packed, s_w, M, K, workspace, y_dtype=torch.bfloat16,
     return y
 
 
+class TiledWeights:
+    """Packed weights in the tiled layout (bitnet_tile_weights): the flat byte
+    buffer plus the matrix shape it holds."""
+
+    def __init__(self, data, N, K):
+        _expect(data, "tiled weights", torch.uint8,
+                numel=bitnet_tiled_weights_bytes(int(N), int(K)))
+        self.data, self.N, self.K = data, int(N), int(K)
+        self.shape = (self.N, self.K // 4)
+
+    @property
+    def device(self):
+        return self.data.device
+
+
+def bitnet_tiled_weights_bytes(N: int, K: int) -> int:
+    return int(load_library().bitnet_tiled_weights_bytes(int(N), int(K)))
+
+
+def bitnet_tile_weights(W_packed, out=None, stream=None):
+    """Row-major packed weights uint8 [N, K/4] -> TiledWeights (same codes,
+    in the tiled order the matmul kernels stream fastest)."""
+    N = _expect_packed(W_packed)
+    K = W_packed.shape[1] * 4
+    nb = bitnet_tiled_weights_bytes(N, K)
+    if nb == 0:
+        raise ValueError(f"unsupported shape N={N}, K={K}")
+    if out is not None:
+        _expect(out, "out", torch.uint8, numel=nb)
+    _need_cuda(W_packed, out)
+    if out is None:
+        out = torch.empty(nb, dtype=torch.uint8, device=W_packed.device)
+    _check("bitnet_tile_weights", load_library().bitnet_tile_weights(
+        _ptr(W_packed), N, K, _ptr(out), _stream(stream)))
+    return TiledWeights(out, N, K)
+
+
+class PairTiledWeights:
+    """The gate and up projections of a SwiGLU in the pair-tiled layout
+    (bitnet_tile_weights_pair): flat bytes plus the shape of each matrix."""
+
+    def __init__(self, data, N, K):
+        _expect(data, "pair-tiled weights", torch.uint8,
+                numel=bitnet_tiled_pair_weights_bytes(int(N), int(K)))
+        self.data, self.N, self.K = data, int(N), int(K)
+        self.shape = (self.N, self.K // 4)
+
+
+def bitnet_tiled_pair_weights_bytes(N: int, K: int) -> int:
+    return int(load_library().bitnet_tiled_pair_weights_bytes(int(N), int(K)))
+
+
+def bitnet_tile_weights_pair(W_gate, W_up, out=None, stream=None):
+    """Two row-major packed matrices of the same shape [N, K/4] -> their
+    pair-tiled layout (for bitnet_swiglu_forward)."""
+    N = _expect_packed(W_gate)
+    K = W_gate.shape[1] * 4
+    if tuple(W_up.shape) != tuple(W_gate.shape):
+        raise ValueError("W_gate and W_up must have the same shape")
+    _expect_packed(W_up, K)
+    nb = bitnet_tiled_pair_weights_bytes(N, K)
+    if nb == 0:
+        raise ValueError(f"unsupported shape N={N}, K={K}")
+    if out is not None:
+        _expect(out, "out", torch.uint8, numel=nb)
+    _need_cuda(W_gate, W_up, out)
+    if out is None:
+        out = torch.empty(nb, dtype=torch.uint8, device=W_gate.device)
+    _check("bitnet_tile_weights_pair", load_library().bitnet_tile_weights_pair(
+        _ptr(W_gate), _ptr(W_up), N, K, _ptr(out), _stream(stream)))
+    return PairTiledWeights(out, N, K)
+
+
+def bitnet_swiglu_forward(x, gamma, eps, W_pair, s_w_gate, s_w_up, y_dtype=torch.bfloat16,
+                          y=None, workspace=None, stream=None):
+    """silu(gate) * up of the two BitLinear forwards of x (M <= 16 tokens),
+    fused into one decode matmul launch.  W_pair: PairTiledWeights."""
+    M, K = _expect_x(x)
+    _expect_gamma(gamma, K)
+    if not isinstance(W_pair, PairTiledWeights) or W_pair.K != K:
+        raise ValueError("W_pair must be PairTiledWeights with the input's K")
+    N = W_pair.N
+    _expect_scale(s_w_gate)
+    _expect_scale(s_w_up)
+    if y is not None:
+        _expect_y(y, M, N)
+    nb = int(load_library().bitnet_swiglu_forward_workspace_bytes(M, N, K))
+    if workspace is not None:
+        _expect(workspace, "workspace", torch.uint8, numel=nb)
+    _need_cuda(x, gamma, W_pair.data, s_w_gate, s_w_up, y, workspace)
+    if y is None:
+        y = torch.empty((M, N), dtype=y_dtype, device=x.device)
+    if workspace is None:
+        workspace = _default_ws.get(nb, x.device, stream)
+    _check("bitnet_swiglu_forward", load_library().bitnet_swiglu_forward(
+        _ptr(x), _dtype_code(x.dtype), _ptr(gamma), float(eps), _ptr(W_pair.data),
+        _ptr(s_w_gate), _ptr(s_w_up), M, N, K, _ptr(y), _dtype_code(y.dtype), _ptr(workspace),
+        workspace.numel(), _stream(stream)))
+    return y
+
+
+def bitnet_quantize_pack_weights_group_scales(W, group_k, W_packed=None, s_w=None,
+                                              workspace=None, stream=None):
+    """W fp32 [N,K] -> (W_packed uint8 [N,K/4], s_w fp32 [K/group_k]): one
+    absmean scale per group of group_k consecutive input features."""
+    N, K = _expect_weights(W)
+    group_k = int(group_k)
+    if group_k <= 0 or K % group_k:
+        raise ValueError("group_k must divide K")
+    G = K // group_k
+    if W_packed is not None:
+        _expect(W_packed, "W_packed", torch.uint8, numel=N * (K // 4))
+    if s_w is not None:
+        _expect(s_w, "s_w", torch.float32, numel=G)
+    lib = load_library()
+    nb = int(lib.bitnet_quantize_pack_weights_group_scales_workspace_bytes(N, K, group_k))
+    if workspace is not None:
+        _expect(workspace, "workspace", torch.uint8, numel=nb)
+    _need_cuda(W, W_packed, s_w, workspace)
+    if W_packed is None:
+        W_packed = torch.empty((N, K // 4), dtype=torch.uint8, device=W.device)
+    if s_w is None:
+        s_w = torch.empty((G,), dtype=torch.float32, device=W.device)
+    if workspace is None:
+        workspace = torch.empty(max(nb, 256), dtype=torch.uint8, device=W.device)
+    _check("bitnet_quantize_pack_weights_group_scales",
+           lib.bitnet_quantize_pack_weights_group_scales(
+               _ptr(W), N, K, group_k, _ptr(W_packed), _ptr(s_w), _ptr(workspace),
+               workspace.numel(), _stream(stream)))
+    return W_packed, s_w
+
+
+def bitnet_linear_forward_group_scales(x, gamma, eps, W, s_w, group_k, y_dtype=torch.float32,
+                                       y=None, debug=False, workspace=None, stream=None):
+    """The forward with group-wise scales (W row-major [N, K/4] or
+    TiledWeights, s_w [K/group_k]).  With debug, also returns x_q (natural
+    order), s_x [M, G] and the per-group integer sums acc [G, M, N]."""
+    M, K = _expect_x(x)
+    _expect_gamma(gamma, K)
+    group_k = int(group_k)
+    if group_k <= 0 or K % group_k:
+        raise ValueError("group_k must divide K")
+    G = K // group_k
+    if not isinstance(W, TiledWeights):
+        _expect_packed(W, K)
+    N = W.shape[0]
+    _expect(s_w, "s_w", torch.float32, numel=G)
+    if y is not None:
+        _expect_y(y, M, N)
+    lib = load_library()
+    nb = int(lib.bitnet_linear_forward_group_scales_workspace_bytes(M, N, K, group_k))
+    if workspace is not None:
+        _expect(workspace, "workspace", torch.uint8, numel=nb)
+    _need_cuda(x, gamma, s_w, y, workspace)
+    wp, layout, _ = _weights_ptr_layout(W, K)
+    dev = x.device
+    if y is None:
+        y = torch.empty((M, N), dtype=y_dtype, device=dev)
+    x_q = torch.empty((M, K), dtype=torch.int8, device=dev) if debug else None
+    s_x = torch.empty((M, G), dtype=torch.float32, device=dev) if debug else None
+    acc = torch.empty((G, M, N), dtype=torch.int32, device=dev) if debug else None
+    if workspace is None:
+        workspace = _default_ws.get(nb, dev, stream)
+    _check("bitnet_linear_forward_group_scales", lib.bitnet_linear_forward_group_scales(
+        _ptr(x), _dtype_code(x.dtype), _ptr(gamma), float(eps), ctypes.c_void_p(wp), layout,
+        _ptr(s_w), M, N, K, group_k, _ptr(y), _dtype_code(y.dtype), _ptr(workspace),
+        workspace.numel(), _ptr(x_q), _ptr(s_x), _ptr(acc), _stream(stream)))
+    return {"y": y, "x_q": x_q, "s_x": s_x, "acc": acc}
+
+
+def _weights_ptr_layout(W, K):
+    """(pointer, layout code, N) of row-major packed weights or TiledWeights."""
+    if isinstance(W, TiledWeights):
+        if W.K != K:
+            raise ValueError(f"tiled weights hold K={W.K}, the input has K={K}")
+        _need_cuda(W.data)
+        return W.data.data_ptr(), BITNET_LAYOUT_TILED, W.N
+    N = _expect_packed(W, K)
+    _need_cuda(W)
+    return W.data_ptr(), BITNET_LAYOUT_ROWS, N
+
+
 def grouped_problems(items):
-    """items: iterable of (x, gamma, eps, W_packed, s_w, y) -> ctypes array of
-    LinearProblem (keep the tensors alive while it is used)."""
+    """items: iterable of (x, gamma, eps, W, s_w, y), W row-major packed
+    weights [N, K/4] or TiledWeights -> ctypes array of LinearProblem (keep
+    the tensors alive while it is used)."""
     items = list(items)
     arr = (LinearProblem * max(1, len(items)))()
-    for i, (x, gamma, eps, W_packed, s_w, y) in enumerate(items):
+    for i, (x, gamma, eps, W, s_w, y) in enumerate(items):
         M, K = _expect_x(x)
         _expect_gamma(gamma, K)
-        N = _expect_packed(W_packed, K)
+        if not isinstance(W, TiledWeights):
+            _expect_packed(W, K)
         _expect_scale(s_w)
-        _expect_y(y, M, N)
-        _need_cuda(x, gamma, W_packed, s_w, y)
+        _expect_y(y, M, W.shape[0])
+        _need_cuda(x, gamma, s_w, y)
+        wp, layout, N = _weights_ptr_layout(W, K)
         arr[i] = LinearProblem(x.data_ptr(), _dtype_code(x.dtype),
                                None if gamma is None else gamma.data_ptr(), float(eps),
-                               W_packed.data_ptr(), s_w.data_ptr(), M, N, K,
-                               y.data_ptr(), _dtype_code(y.dtype))
+                               wp, s_w.data_ptr(), M, N, K,
+                               y.data_ptr(), _dtype_code(y.dtype), layout)
     return arr, len(items)
+
+
+def bitnet_linear_forward_ex(x, gamma, eps, W, s_w, y_dtype=torch.float32, y=None,
+                             path=BITNET_PATH_AUTO, want_y=True, debug=True, workspace=None,
+                             stream=None):
+    """One forward on row-major or tiled weights (W: uint8 [N, K/4] or
+    TiledWeights).  With debug, also returns x_q (natural order), s_x and the
+    int32 accumulators."""
+    M, K = _expect_x(x)
+    _expect_gamma(gamma, K)
+    if not isinstance(W, TiledWeights):
+        _expect_packed(W, K)
+    N = W.shape[0]
+    _expect_scale(s_w)
+    _dtype_code(y_dtype)
+    if y is not None:
+        _expect_y(y, M, N)
+    if workspace is not None:
+        _expect(workspace, "workspace", torch.uint8,
+                numel=bitnet_linear_forward_workspace_bytes(M, N, K))
+    _need_cuda(x, gamma, s_w, y, workspace)
+    wp, layout, _ = _weights_ptr_layout(W, K)
+    dev = x.device
+    if y is None and want_y:
+        y = torch.empty((M, N), dtype=y_dtype, device=dev)
+    x_q = torch.empty((M, K), dtype=torch.int8, device=dev) if debug else None
+    s_x = torch.empty((M,), dtype=torch.float32, device=dev) if debug else None
+    acc = torch.empty((M, N), dtype=torch.int32, device=dev) if debug else None
+    ws = _ws_for(M, N, K, dev, workspace, stream)
+    prob = LinearProblem(x.data_ptr(), _dtype_code(x.dtype),
+                         None if gamma is None else gamma.data_ptr(), float(eps), wp,
+                         s_w.data_ptr(), M, N, K, None if y is None else y.data_ptr(),
+                         _dtype_code(y.dtype if y is not None else y_dtype), layout)
+    _check("bitnet_linear_forward_ex", load_library().bitnet_linear_forward_ex(
+        ctypes.byref(prob), _ptr(ws), ws.numel(), _ptr(x_q), _ptr(s_x), _ptr(acc), int(path),
+        _stream(stream)))
+    return {"y": y, "x_q": x_q, "s_x": s_x, "acc": acc}
 
 
 def bitnet_linear_forward_grouped_workspace_bytes(problems, count):
@@ -463,6 +716,14 @@ def bitnet_device_status(reset=True, stream=None):
 def bitnet_selftest_bounded_wait(limit_ns: int, stream=None):
     _check("bitnet_selftest_bounded_wait",
            load_library().bitnet_selftest_bounded_wait(int(limit_ns), _stream(stream)))
+
+
+def bitnet_selftest_mma_i8(iters, ctas, a_in_tmem=False, stream=None):
+    """Queue the int8 tensor-core rate kernel (see the header); returns the
+    int8 operation count it performs."""
+    _check("bitnet_selftest_mma_i8", load_library().bitnet_selftest_mma_i8(
+        int(iters), int(ctas), 1 if a_in_tmem else 0, _stream(stream)))
+    return 2 * 128 * 256 * 32 * int(iters) * int(ctas)
 
 
 def bitnet_selftest_divide(a, b, stream=None):

@@ -55,9 +55,12 @@ struct Chunk8 {
 // the warp must call this (valid or not).
 // perm: -1 keeps the block order; 0 / 1 applies x_block_pos with that
 // token parity.
+// cs: bytes from one 256-element chunk of the row to the next (256 for a
+// plain row; M * 256 for the decode-tiled layout, where chunk c of every
+// token row sits together).
 template <bool kInterleave>
 __device__ __forceinline__ void store_chunk8(int8_t* xq_row, int64_t k, Chunk8 c, bool valid,
-                                             int perm = -1) {
+                                             int perm = -1, int64_t cs = 256) {
   if (!kInterleave) {
     if (valid) *reinterpret_cast<uint2*>(xq_row + k) = make_uint2(c.lo, c.hi);
     return;
@@ -65,6 +68,7 @@ __device__ __forceinline__ void store_chunk8(int8_t* xq_row, int64_t k, Chunk8 c
   if (perm >= 0)
     k = (k & ~static_cast<int64_t>(255)) +
         16 * x_block_pos(static_cast<int>((k & 255) >> 4), perm) + (k & 15);
+  k = (k >> 8) * cs + (k & 255);
   const int h = static_cast<int>((k >> 3) & 1);   // which half of the 16-group
   // A = bytes (q0, q4, q1, q5), B = (q2, q6, q3, q7) of this half.
   const uint32_t A = __byte_perm(c.lo, c.hi, 0x5140);
@@ -233,7 +237,8 @@ __device__ __forceinline__ void quant_row(const void* __restrict__ x,
                                           const float* __restrict__ gamma, float eps, int64_t m,
                                           int64_t K, int8_t* __restrict__ x_q,
                                           float* __restrict__ s_x, int32_t* __restrict__ rowsum,
-                                          float* redf, int* redi, bool perm = false) {
+                                          float* redf, int* redi, bool perm = false,
+                                          int64_t M_tiled = 0) {
   const int tid = threadIdx.x;
   const int64_t nchunk = K >> 3;
   const int iters = static_cast<int>((nchunk + kActThreads - 1) / kActThreads);
@@ -300,15 +305,19 @@ __device__ __forceinline__ void quant_row(const void* __restrict__ x,
   // Pass 3: quantize, store, row sum (every lane runs every iteration: the
   // interleaved store exchanges bytes between lane pairs).
   int sum = 0;
-  int8_t* xq_row = x_q + row;
+  const bool tiled = M_tiled > 0;   // decode-tiled layout, as in quant_row_staged
+  int8_t* xq_row = tiled ? x_q + m * 256 : x_q + row;
+  const int64_t cs = tiled ? M_tiled * 256 : 256;
+  const int64_t nstore = tiled ? ((K + 255) >> 8) << 5 : nchunk;
+  const int store_iters = static_cast<int>((nstore + kActThreads - 1) / kActThreads);
 #pragma unroll
   for (int it = 0; it < (CACHE > 0 ? CN : 1); ++it) {
-    for (int it2 = it; it2 < (CACHE > 0 ? it + 1 : iters); ++it2) {
-      if (it2 >= iters) continue;  // uniform: iters is the same for the whole CTA
+    for (int it2 = it; it2 < (CACHE > 0 ? it + 1 : store_iters); ++it2) {
+      if (it2 >= store_iters) continue;  // uniform over the CTA
       const int64_t c = tid + static_cast<int64_t>(kActThreads) * it2;
-      const bool valid = c < nchunk;
+      const bool valid = c < nstore;
       int8_t q[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-      if (valid && !zero_row) {
+      if (c < nchunk && !zero_row) {
         float v[8], g[8];
         chunk(it2, c, v);
         load_gamma8(gamma, 8 * c, g);
@@ -319,7 +328,8 @@ __device__ __forceinline__ void quant_row(const void* __restrict__ x,
         }
       }
       Chunk8 ch{pack4(q[0], q[1], q[2], q[3]), pack4(q[4], q[5], q[6], q[7])};
-      store_chunk8<kInterleave>(xq_row, 8 * c, ch, valid, perm ? static_cast<int>(m & 1) : -1);
+      store_chunk8<kInterleave>(xq_row, 8 * c, ch, valid, perm ? static_cast<int>(m & 1) : -1,
+                                cs);
     }
   }
   sum = block_sum_i32(sum, redi);
@@ -347,7 +357,7 @@ __device__ bool quant_row_staged(const void* __restrict__ x, const float* __rest
                                  float eps, int64_t m, int64_t K, int8_t* __restrict__ x_q,
                                  float* __restrict__ s_x, int32_t* __restrict__ rowsum,
                                  float* redf, int* redi, uint8_t* stage, uint64_t* bar,
-                                 uint64_t wait_limit_ns, bool perm) {
+                                 uint64_t wait_limit_ns, bool perm, int64_t M_tiled = 0) {
   constexpr int ES = kBF16 ? 2 : 4;
   const int tid = threadIdx.x;
   const uint32_t xbytes = static_cast<uint32_t>(K * ES);
@@ -366,7 +376,6 @@ __device__ bool quant_row_staged(const void* __restrict__ x, const float* __rest
   if (!__syncthreads_and(landed ? 1 : 0)) return false;
 
   const int64_t nchunk = K >> 3;
-  const int iters = static_cast<int>((nchunk + kActThreads - 1) / kActThreads);
   auto chunk = [&](int64_t c, float (&v)[8]) {
     RawChunk<kBF16> r;
     const uint4* src = reinterpret_cast<const uint4*>(stage + c * 8 * ES);
@@ -428,15 +437,20 @@ __device__ bool quant_row_staged(const void* __restrict__ x, const float* __rest
   const float sx = __fdiv_rn(127.0f, amax);
 
   // Pass 3: quantize, store, row sum (every lane runs every iteration: the
-  // interleaved store exchanges bytes between lane pairs).
+  // interleaved store exchanges bytes between lane pairs).  In the
+  // decode-tiled layout (M_tiled > 0) the row is stored as 256-element
+  // chunks M_tiled * 256 bytes apart, its last chunk zero-padded past K.
   int sum = 0;
-  int8_t* xq_row = x_q + m * K;
+  const bool tiled = M_tiled > 0;
+  int8_t* xq_row = tiled ? x_q + m * 256 : x_q + m * K;
+  const int64_t cs = tiled ? M_tiled * 256 : 256;
+  const int64_t nstore = tiled ? ((K + 255) >> 8) << 5 : nchunk;   // 8-element chunks
+  const int store_iters = static_cast<int>((nstore + kActThreads - 1) / kActThreads);
 #pragma unroll 1
-  for (int it = 0; it < iters; ++it) {
+  for (int it = 0; it < store_iters; ++it) {
     const int64_t c = tid + static_cast<int64_t>(kActThreads) * it;
-    const bool valid = c < nchunk;
     int8_t q[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-    if (valid && !zero_row) {
+    if (c < nchunk && !zero_row) {
       float v[8], g[8];
       chunk(c, v);
       gam(c, g);
@@ -447,7 +461,8 @@ __device__ bool quant_row_staged(const void* __restrict__ x, const float* __rest
       }
     }
     Chunk8 ch{pack4(q[0], q[1], q[2], q[3]), pack4(q[4], q[5], q[6], q[7])};
-    store_chunk8<kInterleave>(xq_row, 8 * c, ch, valid, perm ? static_cast<int>(m & 1) : -1);
+    store_chunk8<kInterleave>(xq_row, 8 * c, ch, c < nstore, perm ? static_cast<int>(m & 1) : -1,
+                              cs);
   }
   sum = block_sum_i32(sum, redi);
   if (tid == 0) {
@@ -465,7 +480,8 @@ __global__ void __launch_bounds__(kActThreads)
 rmsnorm_quant_kernel(const void* __restrict__ x, const float* __restrict__ gamma, float eps,
                      int64_t M, int64_t K, int8_t* __restrict__ x_q, float* __restrict__ s_x,
                      int32_t* __restrict__ rowsum, uint4* __restrict__ zero16, int64_t n_zero16,
-                     int trigger_dependents, int* status, uint64_t wait_limit_ns, int perm) {
+                     int trigger_dependents, int* status, uint64_t wait_limit_ns, int perm,
+                     int tiled) {
   __shared__ float redf[kActThreads];
   __shared__ int redi[kActThreads / 32];
   __shared__ __align__(8) uint64_t bar;
@@ -478,13 +494,13 @@ rmsnorm_quant_kernel(const void* __restrict__ x, const float* __restrict__ gamma
   }
   if (STAGED) {
     if (!quant_row_staged<kBF16, kInterleave>(x, gamma, eps, blockIdx.x, K, x_q, s_x, rowsum,
-                                              redf, redi, stage, &bar, wait_limit_ns,
-                                              perm != 0) &&
+                                              redf, redi, stage, &bar, wait_limit_ns, perm != 0,
+                                              tiled ? M : 0) &&
         threadIdx.x == 0)
       record_failure(status, DEV_TIMEOUT_QUANT);
   } else {
     quant_row<kBF16, kInterleave, 0>(x, gamma, eps, blockIdx.x, K, x_q, s_x, rowsum, redf, redi,
-                                     perm != 0);
+                                     perm != 0, tiled ? M : 0);
   }
 }
 
@@ -502,6 +518,7 @@ struct QuantProblem {
   int M, K;
   int x_bf16;
   int perm;               // decode-matmul block order (x_block_pos)
+  int tiled;              // decode-tiled layout: x_q [ceil(K/256)][M][256]
   int block_begin;        // first block of this problem
   int zero_blocks;        // blocks after the M row blocks that clear zero16
 };
@@ -535,20 +552,21 @@ rmsnorm_quant_grouped_kernel(const __grid_constant__ QuantLaunch L) {
     return;
   }
   if (STAGED) {
+    const int64_t mt = q.tiled ? q.M : 0;
     const bool ok =
         q.x_bf16 ? quant_row_staged<true, true>(q.x, q.gamma, q.eps, local, q.K, q.xi, q.s_x,
                                                 q.rowsum, redf, redi, stage, &bar, L.wait_limit_ns,
-                                                q.perm != 0)
+                                                q.perm != 0, mt)
                  : quant_row_staged<false, true>(q.x, q.gamma, q.eps, local, q.K, q.xi, q.s_x,
                                                  q.rowsum, redf, redi, stage, &bar,
-                                                 L.wait_limit_ns, q.perm != 0);
+                                                 L.wait_limit_ns, q.perm != 0, mt);
     if (!ok && threadIdx.x == 0) record_failure(L.status, DEV_TIMEOUT_QUANT);
   } else if (q.x_bf16) {
     quant_row<true, true, 0>(q.x, q.gamma, q.eps, local, q.K, q.xi, q.s_x, q.rowsum, redf, redi,
-                             q.perm != 0);
+                             q.perm != 0, q.tiled ? q.M : 0);
   } else {
     quant_row<false, true, 0>(q.x, q.gamma, q.eps, local, q.K, q.xi, q.s_x, q.rowsum, redf, redi,
-                              q.perm != 0);
+                              q.perm != 0, q.tiled ? q.M : 0);
   }
 }
 

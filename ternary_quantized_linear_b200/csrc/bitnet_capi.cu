@@ -19,6 +19,10 @@
 #include "common.cuh"
 #include "gemm_tc.cuh"
 #include "gemv.cuh"
+#include "gemv_tiled.cuh"
+#include "group_quant.cuh"
+#include "peak.cuh"
+#include "tiled.cuh"
 #include "weight_quant.cuh"
 
 namespace bitnet {
@@ -36,9 +40,17 @@ size_t align256(size_t v) { return (v + 255) & ~static_cast<size_t>(255); }
 
 cudaStream_t as_stream(bitnet_stream_t s) { return reinterpret_cast<cudaStream_t>(s); }
 
-bitnet_status launch_status() {
-  return cudaGetLastError() == cudaSuccess ? BITNET_OK : BITNET_ERR_CUDA;
+// The last CUDA error a call of this thread met (0 = none since the last
+// query), for bitnet_last_cuda_error.
+thread_local int g_last_cuda_error = 0;
+
+bitnet_status cuda_status(cudaError_t e) {
+  if (e == cudaSuccess) return BITNET_OK;
+  g_last_cuda_error = static_cast<int>(e);
+  return BITNET_ERR_CUDA;
 }
+
+bitnet_status launch_status() { return cuda_status(cudaGetLastError()); }
 
 // ------------------------------------------------------------ per-device state
 
@@ -95,11 +107,22 @@ DeviceState* device_state() {
     ok = ok && set_smem(rmsnorm_quant_kernel<false, true, false>, 0);
     ok = ok && set_smem(rmsnorm_quant_kernel<false, false, false>, 0);
     ok = ok && set_smem(interleave_rowsum_kernel, 0);
-    ok = ok && set_smem(ternary_gemm_tc_kernel<16>, GemmCfg<16>::SMEM_DYN);
-    ok = ok && set_smem(ternary_gemm_tc_kernel<32>, GemmCfg<32>::SMEM_DYN);
-    ok = ok && set_smem(ternary_gemm_tc_kernel<64>, GemmCfg<64>::SMEM_DYN);
-    ok = ok && set_smem(ternary_gemm_tc_kernel<128>, GemmCfg<128>::SMEM_DYN);
-    ok = ok && set_smem(ternary_gemm_tc_kernel<256>, GemmCfg<256>::SMEM_DYN);
+    ok = ok && set_smem(ternary_gemm_tc_kernel<16, false>, GemmCfg<16>::SMEM_DYN);
+    ok = ok && set_smem(ternary_gemm_tc_kernel<32, false>, GemmCfg<32>::SMEM_DYN);
+    ok = ok && set_smem(ternary_gemm_tc_kernel<64, false>, GemmCfg<64>::SMEM_DYN);
+    ok = ok && set_smem(ternary_gemm_tc_kernel<128, false>, GemmCfg<128>::SMEM_DYN);
+    ok = ok && set_smem(ternary_gemm_tc_kernel<256, false>, GemmCfg<256>::SMEM_DYN);
+    ok = ok && set_smem(ternary_gemm_tc_kernel<16, true>, GemmCfg<16>::SMEM_DYN);
+    ok = ok && set_smem(ternary_gemm_tc_kernel<32, true>, GemmCfg<32>::SMEM_DYN);
+    ok = ok && set_smem(ternary_gemm_tc_kernel<64, true>, GemmCfg<64>::SMEM_DYN);
+    ok = ok && set_smem(ternary_gemm_tc_kernel<128, true>, GemmCfg<128>::SMEM_DYN);
+    ok = ok && set_smem(ternary_gemm_tc_kernel<256, true>, GemmCfg<256>::SMEM_DYN);
+    ok = ok && set_smem(mma_i8_peak_kernel<false>, kPeakSmem);
+    ok = ok && set_smem(mma_i8_peak_kernel<true>, kPeakSmem);
+    ok = ok && set_smem(ternary_gemv_tiled_kernel<1, false>, GtCfg<false>::SMEM_DYN);
+    ok = ok && set_smem(ternary_gemv_tiled_kernel<2, false>, GtCfg<false>::SMEM_DYN);
+    ok = ok && set_smem(ternary_gemv_tiled_kernel<1, true>, GtCfg<true>::SMEM_DYN);
+    ok = ok && set_smem(ternary_gemv_tiled_kernel<2, true>, GtCfg<true>::SMEM_DYN);
     st.ok = ok;
   });
   return st.ok ? &st : nullptr;
@@ -149,21 +172,38 @@ struct FwdWorkspace {
 };
 
 constexpr int64_t kGemvMaxM = 16;
+// Token counts up to this one are "decode-sized" for the tcgen05 kernel too:
+// it splits K across CTAs to fill the GPU and needs the partial-sum region.
+constexpr int64_t kSplitMaxM = 64;
 
+// Workspace of one forward.  The quantized input takes M * 256 * ceil(K/256)
+// bytes: row-major [M][K] for the tcgen05 kernel and the row-major decode
+// kernel, chunk-major [K/256][M][256] (zero-padded past K) for the tiled
+// decode kernel.  For M <= 16 the partial-sum region serves either decode
+// kernel: the row-major one accumulates [M][N] int32 split-K partials with
+// atomics, the tiled one stores [M][128] int32 partial slots, two per CTA
+// that touches the problem; the counters follow it.
 FwdWorkspace fwd_layout(int64_t M, int64_t N, int64_t K) {
   FwdWorkspace w{};
   size_t o = 0;
   w.xq = o;
-  o = align256(o + static_cast<size_t>(M * K));
+  o = align256(o + static_cast<size_t>(M * 256 * tiled_chunks(K)));
   w.sx = o;
   o = align256(o + 4 * static_cast<size_t>(M));
   w.rs = o;
   o = align256(o + 4 * static_cast<size_t>(M));
-  const bool gemv_capable = M <= kGemvMaxM;
+  const bool split_capable = M <= kSplitMaxM;
+  const int64_t tiles = tiled_row_blocks(N) * tiled_chunks(K);
+  const size_t slots =
+      M <= kGemvMaxM ? 2 * static_cast<size_t>(std::min<int64_t>(kGtMaxCtas, tiles)) : 0;
   w.acc = o;
-  o = align256(o + (gemv_capable ? 4 * static_cast<size_t>(M * N) : 0));
+  o = align256(o + (split_capable ? std::max(4 * static_cast<size_t>(M * N),
+                                             slots * kTileRows * 4 * static_cast<size_t>(M))
+                                  : 0));
   w.cnt = o;
-  o = align256(o + (gemv_capable ? 4 * static_cast<size_t>((N + 15) / 16) : 0));
+  o = align256(o + (split_capable ? 4 * static_cast<size_t>(std::max<int64_t>((N + 15) / 16,
+                                                                               tiled_row_blocks(N)))
+                                  : 0));
   w.total = o;
   return w;
 }
@@ -353,7 +393,7 @@ bitnet_status launch_gemv_group(const DeviceState& ds, GemvLaunch& L, long long 
   cfg.numAttrs = pdl ? 1 : 0;
   const cudaError_t e = nt == 2 ? cudaLaunchKernelEx(&cfg, ternary_gemv_kernel<2>, L)
                                 : cudaLaunchKernelEx(&cfg, ternary_gemv_kernel<1>, L);
-  return e == cudaSuccess ? BITNET_OK : BITNET_ERR_CUDA;
+  return cuda_status(e);
 }
 
 long long gemv_capacity(const DeviceState& ds, int M) {
@@ -382,6 +422,123 @@ bitnet_status launch_gemv(const DeviceState& ds, const uint8_t* Wp, const float*
   return launch_gemv_group(ds, L, G, pdl, early_weights, stream);
 }
 
+// ------------------------------------------------------ tiled decode GEMV
+
+// Relative time of one 8 KiB tile: two token tiles take about 1.2 times as
+// long as one (the same weights as the row-major kernel's cost model).
+long long gt_tile_cost(const GtProblem& P) { return P.M > 8 ? 6 : 5; }
+
+// Shape fields (M, N, K) of prob[0..count) must be set.  Lays the problems'
+// tiles end to end and splits them into `capacity` (at most the tile count)
+// contiguous ranges of equal cost; every range holds at least one tile.
+void plan_gt_launch(GtLaunch& L, long long capacity) {
+  long long T = 0, W = 0;
+  for (int i = 0; i < L.count; ++i) {
+    GtProblem& P = L.prob[i];
+    P.KC = static_cast<int>(tiled_chunks(P.K));
+    P.RB = static_cast<int>(tiled_row_blocks(P.N));
+    P.tile_base = T;
+    const long long tiles = static_cast<long long>(P.RB) * P.KC;
+    T += tiles;
+    W += tiles * gt_tile_cost(P);
+  }
+  long long G = std::max(1LL, std::min({capacity, T, static_cast<long long>(kGtMaxCtas)}));
+  L.ctas = static_cast<int>(G);
+  // tile_begin[b]: first tile whose cost prefix reaches b * W / G.
+  int p = 0;
+  long long pre = 0;  // cost of the tiles before problem p
+  for (long long b = 0; b <= G; ++b) {
+    const long long target = (b * W + G - 1) / G;
+    while (p + 1 < L.count &&
+           pre + (static_cast<long long>(L.prob[p].RB) * L.prob[p].KC) * gt_tile_cost(L.prob[p]) <
+               target) {
+      pre += static_cast<long long>(L.prob[p].RB) * L.prob[p].KC * gt_tile_cost(L.prob[p]);
+      ++p;
+    }
+    const long long c = gt_tile_cost(L.prob[p]);
+    long long t = L.prob[p].tile_base + (target - pre + c - 1) / c;
+    L.tile_begin[b] = std::min(t, T);
+  }
+  L.tile_begin[0] = 0;
+  L.tile_begin[G] = T;
+  for (long long b = 1; b < G; ++b)  // strictly increasing, room for the rest
+    L.tile_begin[b] = std::min(std::max(L.tile_begin[b], L.tile_begin[b - 1] + 1), T - (G - b));
+  for (int i = 0; i < L.count; ++i) {
+    GtProblem& P = L.prob[i];
+    int b = 0;
+    while (b + 1 < G && L.tile_begin[b + 1] <= P.tile_base) ++b;
+    P.cta_first = b;
+  }
+}
+
+bool fill_gt_problem(GtProblem& q, const uint8_t* Wt, uint8_t* xws, const FwdWorkspace& xL,
+                     uint8_t* ws, const FwdWorkspace& Lw, const float* s_x, const float* s_w,
+                     int64_t M, int64_t N, int64_t K, void* y, int y_dtype, int32_t* acc_out) {
+  q.Wt = Wt;
+  q.xd = xws + xL.xq;
+  q.rowsum = reinterpret_cast<const int32_t*>(xws + xL.rs);
+  q.s_x = s_x;
+  q.s_w = s_w;
+  q.y = y;
+  q.acc_out = acc_out;
+  q.part = reinterpret_cast<int32_t*>(ws + Lw.acc);
+  q.cnt = reinterpret_cast<unsigned*>(ws + Lw.cnt);
+  q.M = static_cast<int>(M);
+  q.N = static_cast<int>(N);
+  q.K = static_cast<int>(K);
+  q.y_bf16 = (y_dtype == BITNET_BF16) ? 1 : 0;
+  q.s_w2 = nullptr;
+  q.gc = 0;
+  q.G = 1;
+  q.gacc = nullptr;
+  return true;
+}
+
+int gt_tiles(const GtLaunch& L) {
+  for (int i = 0; i < L.count; ++i)
+    if (L.prob[i].M > 8) return 2;
+  return 1;
+}
+
+// pair: the fused SwiGLU variant (every problem of L has pair-tiled weights).
+bitnet_status launch_gt(const DeviceState& ds, GtLaunch& L, bool pdl, cudaStream_t stream,
+                        bool pair = false) {
+  L.use_pdl = pdl ? 1 : 0;
+  L.status = ds.status;
+  L.wait_limit_ns = kWaitLimitNs;
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(static_cast<unsigned>(L.ctas), 1, 1);
+  cfg.blockDim = dim3(kGtThreads, 1, 1);
+  cfg.dynamicSmemBytes = pair ? GtCfg<true>::SMEM_DYN : GtCfg<false>::SMEM_DYN;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  const int nt = gt_tiles(L);
+  cudaError_t e;
+  if (pair)
+    e = nt == 2 ? cudaLaunchKernelEx(&cfg, ternary_gemv_tiled_kernel<2, true>, L)
+                : cudaLaunchKernelEx(&cfg, ternary_gemv_tiled_kernel<1, true>, L);
+  else
+    e = nt == 2 ? cudaLaunchKernelEx(&cfg, ternary_gemv_tiled_kernel<2, false>, L)
+                : cudaLaunchKernelEx(&cfg, ternary_gemv_tiled_kernel<1, false>, L);
+  return cuda_status(e);
+}
+
+// One problem on tiled weights.
+bitnet_status launch_gt_single(const DeviceState& ds, const uint8_t* Wt, const float* s_x,
+                               const float* s_w, int64_t M, int64_t N, int64_t K, uint8_t* ws,
+                               const FwdWorkspace& Lw, void* y, int y_dtype, int32_t* acc_out,
+                               bool pdl, cudaStream_t stream) {
+  static thread_local GtLaunch L;  // ~6 KB: keep it off the stack
+  L.count = 1;
+  fill_gt_problem(L.prob[0], Wt, ws, Lw, ws, Lw, s_x, s_w, M, N, K, y, y_dtype, acc_out);
+  plan_gt_launch(L, ds.num_sms);
+  return launch_gt(ds, L, pdl, stream);
+}
+
 struct GemmPlan {
   int BN, rb, tb, ksplit, steps_per_split;
 };
@@ -402,7 +559,7 @@ GemmPlan plan_gemm(int64_t M, int64_t N, int64_t K, int num_sms) {
   const int kstep = 256;                      // GemmCfg<BN>::KSTEP
   const int steps = static_cast<int>((K + kstep - 1) / kstep);
   int ks = 1;
-  if (M <= kGemvMaxM) {
+  if (M <= kSplitMaxM) {
     // Resident slots: two CTAs per SM for small token tiles.  Split K so the
     // grid fills the slots without starting a partial second wave.
     const int slots = (small ? 2 : 1) * num_sms;
@@ -416,7 +573,7 @@ GemmPlan plan_gemm(int64_t M, int64_t N, int64_t K, int num_sms) {
 
 template <int BN>
 bitnet_status launch_gemm_bn(const CUtensorMap& tx, const CUtensorMap& tw, const GemmParams& p,
-                             const GemmPlan& pl, cudaStream_t stream) {
+                             const GemmPlan& pl, bool tiled_w, cudaStream_t stream) {
   cudaLaunchConfig_t cfg{};
   cfg.gridDim = dim3(static_cast<unsigned>(pl.rb), static_cast<unsigned>(pl.tb),
                      static_cast<unsigned>(pl.ksplit));
@@ -428,15 +585,17 @@ bitnet_status launch_gemm_bn(const CUtensorMap& tx, const CUtensorMap& tw, const
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = p.use_pdl ? 1 : 0;
-  return cudaLaunchKernelEx(&cfg, ternary_gemm_tc_kernel<BN>, tx, tw, p) == cudaSuccess
-             ? BITNET_OK
-             : BITNET_ERR_CUDA;
+  const cudaError_t e = tiled_w ? cudaLaunchKernelEx(&cfg, ternary_gemm_tc_kernel<BN, true>, tx, tw, p)
+                                : cudaLaunchKernelEx(&cfg, ternary_gemm_tc_kernel<BN, false>, tx, tw, p);
+  return cuda_status(e);
 }
 
+// Wp: row-major packed weights, or the tiled layout when tiled_w.
 bitnet_status launch_gemm(const DeviceState& ds, const uint8_t* Wp, const int8_t* xi,
                           const int32_t* rowsum, const float* s_x, const float* s_w, int64_t M,
                           int64_t N, int64_t K, uint8_t* ws, const FwdWorkspace& Lw, void* y,
-                          int y_dtype, int32_t* acc_out, bool pdl, cudaStream_t stream) {
+                          int y_dtype, int32_t* acc_out, bool pdl, cudaStream_t stream,
+                          bool tiled_w = false) {
   const GemmPlan pl = plan_gemm(M, N, K, ds.num_sms);
   CUtensorMap tx, tw;
   if (!make_tmap_u8(&tx, xi, static_cast<uint64_t>(K), static_cast<uint64_t>(M),
@@ -444,11 +603,15 @@ bitnet_status launch_gemm(const DeviceState& ds, const uint8_t* Wp, const int8_t
                     CU_TENSOR_MAP_SWIZZLE_128B))
     return BITNET_ERR_CUDA;
   // GemmCfg<BN>::WP_ROW = 64 bytes per row, swizzled so the unpack reads are
-  // bank-conflict free.
-  if (!make_tmap_u8(&tw, Wp, static_cast<uint64_t>(K / 4), static_cast<uint64_t>(N),
-                    static_cast<uint64_t>(K / 4), 64, 128, CU_TENSOR_MAP_SWIZZLE_64B))
+  // bank-conflict free (the tiled layout is stored in that order already).
+  if (tiled_w)
+    std::memset(&tw, 0, sizeof(tw));
+  else if (!make_tmap_u8(&tw, Wp, static_cast<uint64_t>(K / 4), static_cast<uint64_t>(N),
+                         static_cast<uint64_t>(K / 4), 64, 128, CU_TENSOR_MAP_SWIZZLE_64B))
     return BITNET_ERR_CUDA;
   GemmParams p{};
+  p.Wt = tiled_w ? Wp : nullptr;
+  p.KC = static_cast<int>(tiled_chunks(K));
   p.rowsum = rowsum;
   p.s_x = s_x;
   p.s_w = s_w;
@@ -466,18 +629,57 @@ bitnet_status launch_gemm(const DeviceState& ds, const uint8_t* Wp, const int8_t
   p.wait_limit_ns = kWaitLimitNs;
   p.use_pdl = pdl ? 1 : 0;
   switch (pl.BN) {
-    case 16: return launch_gemm_bn<16>(tx, tw, p, pl, stream);
-    case 32: return launch_gemm_bn<32>(tx, tw, p, pl, stream);
-    case 64: return launch_gemm_bn<64>(tx, tw, p, pl, stream);
-    case 128: return launch_gemm_bn<128>(tx, tw, p, pl, stream);
-    default: return launch_gemm_bn<256>(tx, tw, p, pl, stream);
+    case 16: return launch_gemm_bn<16>(tx, tw, p, pl, tiled_w, stream);
+    case 32: return launch_gemm_bn<32>(tx, tw, p, pl, tiled_w, stream);
+    case 64: return launch_gemm_bn<64>(tx, tw, p, pl, tiled_w, stream);
+    case 128: return launch_gemm_bn<128>(tx, tw, p, pl, tiled_w, stream);
+    default: return launch_gemm_bn<256>(tx, tw, p, pl, tiled_w, stream);
+  }
+}
+
+// The tcgen05 kernel in group mode: K split z = group z, each CTA writes its
+// group's integer sums (row sums of the group subtracted) to gacc [G][M][N].
+bitnet_status launch_gemm_groups(const DeviceState& ds, const uint8_t* Wp, const int8_t* xi,
+                                 const int32_t* rowsum, int64_t M, int64_t N, int64_t K,
+                                 int64_t G, int32_t* gacc, const GemmPlan& pl, bool tiled_w,
+                                 cudaStream_t stream) {
+  CUtensorMap tx, tw;
+  if (!make_tmap_u8(&tx, xi, static_cast<uint64_t>(K), static_cast<uint64_t>(M),
+                    static_cast<uint64_t>(K), 128, static_cast<uint32_t>(pl.BN),
+                    CU_TENSOR_MAP_SWIZZLE_128B))
+    return BITNET_ERR_CUDA;
+  if (tiled_w)
+    std::memset(&tw, 0, sizeof(tw));
+  else if (!make_tmap_u8(&tw, Wp, static_cast<uint64_t>(K / 4), static_cast<uint64_t>(N),
+                         static_cast<uint64_t>(K / 4), 64, 128, CU_TENSOR_MAP_SWIZZLE_64B))
+    return BITNET_ERR_CUDA;
+  GemmParams p{};
+  p.Wt = tiled_w ? Wp : nullptr;
+  p.KC = static_cast<int>(tiled_chunks(K));
+  p.rowsum = rowsum;
+  p.M = static_cast<int>(M);
+  p.N = static_cast<int>(N);
+  p.K = static_cast<int>(K);
+  p.ksplit = pl.ksplit;
+  p.steps_per_split = pl.steps_per_split;
+  p.status = ds.status;
+  p.wait_limit_ns = kWaitLimitNs;
+  p.use_pdl = 1;
+  p.gacc = gacc;
+  p.G = static_cast<int>(G);
+  switch (pl.BN) {
+    case 16: return launch_gemm_bn<16>(tx, tw, p, pl, tiled_w, stream);
+    case 32: return launch_gemm_bn<32>(tx, tw, p, pl, tiled_w, stream);
+    case 64: return launch_gemm_bn<64>(tx, tw, p, pl, tiled_w, stream);
+    case 128: return launch_gemm_bn<128>(tx, tw, p, pl, tiled_w, stream);
+    default: return launch_gemm_bn<256>(tx, tw, p, pl, tiled_w, stream);
   }
 }
 
 // Whether the matmul chosen for (path, M, N, K) accumulates split-K partials
 // in the workspace (which must then start at zero).
 bool needs_zeroed_partials(const DeviceState& ds, int path, int64_t M, int64_t N, int64_t K) {
-  if (M > kGemvMaxM) return false;
+  if (M > kSplitMaxM) return false;
   if (path == BITNET_PATH_GEMV) {
     static thread_local GemvLaunch L;
     const long long G = plan_gemv_single(ds, L, M, N, K);
@@ -494,7 +696,9 @@ int64_t zero_blocks(size_t bytes) {
 }
 
 // Layouts of the quantized activations a launch writes.
-enum XLayout { kXNatural = 0, kXInterleaved = 1, kXDecode = 2 };  // decode: + x_block_pos
+// kXDecode: interleaved + x_block_pos (row-major decode kernel);
+// kXDecodeTiled: the same, chunk-major [K/256][M][256] (tiled decode kernel).
+enum XLayout { kXNatural = 0, kXInterleaved = 1, kXDecode = 2, kXDecodeTiled = 3 };
 
 // zero/zero_bytes: a 16-byte aligned range (multiple of 16 bytes) cleared by
 // extra blocks of the same launch, or null/0.
@@ -503,7 +707,8 @@ bitnet_status launch_act_quant(const void* x, int x_dtype, const float* gamma, f
                                int layout, bool trigger, void* zero, size_t zero_bytes,
                                cudaStream_t stream) {
   const bool interleave = layout != kXNatural;
-  const int perm = layout == kXDecode ? 1 : 0;
+  const int perm = (layout == kXDecode || layout == kXDecodeTiled) ? 1 : 0;
+  const int tiled = layout == kXDecodeTiled ? 1 : 0;
   const int64_t zb = zero ? zero_blocks(zero_bytes) : 0;
   dim3 grid(static_cast<unsigned>(M + zb)), block(kActThreads);
   const int trig = trigger ? 1 : 0;
@@ -516,7 +721,7 @@ bitnet_status launch_act_quant(const void* x, int x_dtype, const float* gamma, f
   const size_t dyn = staged ? stage : 0;
 #define BITNET_QUANT(BF, IL, ST)                                                             \
   rmsnorm_quant_kernel<BF, IL, ST><<<grid, block, dyn, stream>>>(                           \
-      x, gamma, eps, M, K, x_q, s_x, rowsum, z, n16, trig, status, kWaitLimitNs, perm)
+      x, gamma, eps, M, K, x_q, s_x, rowsum, z, n16, trig, status, kWaitLimitNs, perm, tiled)
   if (bf16) {
     if (interleave) {
       if (staged) BITNET_QUANT(true, true, true); else BITNET_QUANT(true, true, false);
@@ -535,24 +740,53 @@ bitnet_status launch_act_quant(const void* x, int x_dtype, const float* gamma, f
 }
 
 // The split-K partials + counters of a layout (zero bytes when the layout
-// has no GEMV region).
+// has no partial-sum region).
 void* splitk_region(uint8_t* ws, const FwdWorkspace& L, size_t* bytes) {
   *bytes = L.total - L.acc;
   return *bytes ? ws + L.acc : nullptr;
 }
 
+// Only the arrival counters: the tiled decode kernel's partial slots are
+// written before they are read.
+void* counter_region(uint8_t* ws, const FwdWorkspace& L, size_t* bytes) {
+  *bytes = L.total - L.cnt;
+  return *bytes ? ws + L.cnt : nullptr;
+}
+
 // Matmul + fused dequant on already-prepared interleaved activations.
+// w_layout: BITNET_LAYOUT_ROWS or BITNET_LAYOUT_TILED (then the decode path
+// is the tiled decode kernel, whose activations are chunk-major).
 bitnet_status run_matmul(const DeviceState& ds, int path, const uint8_t* Wp, uint8_t* ws,
                          const FwdWorkspace& L, const float* s_x, const float* s_w, int64_t M,
                          int64_t N, int64_t K, void* y, int y_dtype, int32_t* acc_out, bool pdl,
-                         bool early_weights, cudaStream_t stream) {
-  if (path == BITNET_PATH_GEMV)
+                         bool early_weights, cudaStream_t stream, int w_layout = 0) {
+  const bool tiled = w_layout == BITNET_LAYOUT_TILED;
+  if (path == BITNET_PATH_GEMV) {
+    if (tiled)
+      return launch_gt_single(ds, Wp, s_x, s_w, M, N, K, ws, L, y, y_dtype, acc_out, pdl,
+                              stream);
     return launch_gemv(ds, Wp, s_x, s_w, M, N, K, ws, L, y, y_dtype, acc_out, pdl,
                        early_weights, stream);
+  }
   const int8_t* xi = reinterpret_cast<const int8_t*>(ws + L.xq);
   const int32_t* rs = reinterpret_cast<const int32_t*>(ws + L.rs);
   return launch_gemm(ds, Wp, xi, rs, s_x, s_w, M, N, K, ws, L, y, y_dtype, acc_out, pdl,
-                     stream);
+                     stream, tiled);
+}
+
+// The activation layout the chosen matmul reads.
+int x_layout_for(int path, int w_layout) {
+  if (path != BITNET_PATH_GEMV) return kXInterleaved;
+  return w_layout == BITNET_LAYOUT_TILED ? kXDecodeTiled : kXDecode;
+}
+
+// Which part of the workspace the quant launch clears for the chosen matmul.
+void* zero_region_for(const DeviceState& ds, int path, int w_layout, int64_t M, int64_t N,
+                      int64_t K, uint8_t* ws, const FwdWorkspace& L, size_t* bytes) {
+  *bytes = 0;
+  if (path == BITNET_PATH_GEMV && w_layout == BITNET_LAYOUT_TILED)
+    return counter_region(ws, L, bytes);
+  return needs_zeroed_partials(ds, path, M, N, K) ? splitk_region(ws, L, bytes) : nullptr;
 }
 
 // Decode GEMV (warp-level MMA) for M <= 16 unless the matrix is large: above
@@ -560,9 +794,12 @@ bitnet_status run_matmul(const DeviceState& ds, int path, const uint8_t* Wp, uin
 // B200), and for M > 16 it is the only path.
 constexpr int64_t kGemvAutoMaxBytes = int64_t(32) << 20;
 
-int resolve_path(int path, int64_t M, int64_t N = 0, int64_t K = 0) {
+// With tiled weights the decode kernel streams any size at full rate, so
+// it serves every M <= 16.
+int resolve_path(int path, int64_t M, int64_t N = 0, int64_t K = 0, int w_layout = 0) {
   if (path != BITNET_PATH_AUTO) return path;
   if (M > kGemvMaxM) return BITNET_PATH_GEMM;
+  if (w_layout == BITNET_LAYOUT_TILED) return BITNET_PATH_GEMV;
   return (N * (K / 4) <= kGemvAutoMaxBytes) ? BITNET_PATH_GEMV : BITNET_PATH_GEMM;
 }
 
@@ -570,7 +807,7 @@ bitnet_status forward_impl(const void* x, int x_dtype, const float* gamma, float
                            const uint8_t* W_packed, const float* s_w, int64_t M, int64_t N,
                            int64_t K, void* y, int y_dtype, void* workspace,
                            size_t workspace_bytes, int8_t* x_q_out, float* s_x_out,
-                           int32_t* acc_out, int path, cudaStream_t stream) {
+                           int32_t* acc_out, int path, cudaStream_t stream, int w_layout = 0) {
   bitnet_status st = check_shape(M, N, K);
   if (st != BITNET_OK) return st;
   if (M == 0) return BITNET_OK;  // empty batch: nothing to read or write
@@ -578,7 +815,9 @@ bitnet_status forward_impl(const void* x, int x_dtype, const float* gamma, float
     return BITNET_ERR_INVALID_ARG;
   if (y && !ok_dtype(y_dtype)) return BITNET_ERR_INVALID_ARG;
   if (path < BITNET_PATH_AUTO || path > BITNET_PATH_GEMM) return BITNET_ERR_INVALID_ARG;
-  path = resolve_path(path, M, N, K);
+  if (w_layout != BITNET_LAYOUT_ROWS && w_layout != BITNET_LAYOUT_TILED)
+    return BITNET_ERR_INVALID_ARG;
+  path = resolve_path(path, M, N, K, w_layout);
   if (path == BITNET_PATH_GEMV && M > kGemvMaxM) return BITNET_ERR_INVALID_ARG;
   if (!aligned(x, 16) || (gamma && !aligned(gamma, 16)) || !aligned(W_packed, 16) ||
       !aligned(s_w, 4) || (y && !aligned(y, 16)) || (x_q_out && !aligned(x_q_out, 16)) ||
@@ -601,23 +840,23 @@ bitnet_status forward_impl(const void* x, int x_dtype, const float* gamma, float
   const bool pdl = true;  // the matmul launch follows the quant launch directly
   float* sx = reinterpret_cast<float*>(ws + L.sx);
   size_t zbytes = 0;
-  void* zero = needs_zeroed_partials(*ds, path, M, N, K) ? splitk_region(ws, L, &zbytes)
-                                                          : nullptr;
+  void* zero = zero_region_for(*ds, path, w_layout, M, N, K, ws, L, &zbytes);
   st = launch_act_quant(x, x_dtype, gamma, eps, M, K, reinterpret_cast<int8_t*>(ws + L.xq), sx,
-                        reinterpret_cast<int32_t*>(ws + L.rs),
-                        path == BITNET_PATH_GEMV ? kXDecode : kXInterleaved, pdl, zero, zbytes,
-                        stream);
+                        reinterpret_cast<int32_t*>(ws + L.rs), x_layout_for(path, w_layout), pdl,
+                        zero, zbytes, stream);
   if (st != BITNET_OK) return st;
   // The activation-quant kernel just queued started after every earlier
   // write to W_packed, so the GEMV may fetch weights before waiting on it.
   return run_matmul(*ds, path, W_packed, ws, L, sx, s_w, M, N, K, y, y_dtype, acc_out, pdl,
-                    pdl, stream);
+                    pdl, stream, w_layout);
 }
 
 // Checks of one problem of a grouped call (the same rules as the forward).
 bitnet_status check_problem(const bitnet_linear_problem& q) {
   bitnet_status st = check_shape(q.M, q.N, q.K);
   if (st != BITNET_OK) return st;
+  if (q.w_layout != BITNET_LAYOUT_ROWS && q.w_layout != BITNET_LAYOUT_TILED)
+    return BITNET_ERR_INVALID_ARG;
   if (q.M == 0) return BITNET_OK;
   if (!q.x || !q.W_packed || !q.s_w || !q.y || !ok_dtype(q.x_dtype) || !ok_dtype(q.y_dtype) ||
       !(q.eps >= 0.0f) || q.eps > 3.0e38f)
@@ -646,9 +885,11 @@ struct DecodePlan {
   size_t ws_bytes = 0;
   bitnet_linear_problem probs[BITNET_MAX_GROUP];
   QuantLaunch QL;
-  GemvLaunch GL;
+  GemvLaunch GL;    // decode problems on row-major weights
+  GtLaunch TL;      // decode problems on tiled weights
   long long G = 0;
-  int n = 0;        // decode problems
+  int n = 0;        // decode problems (both layouts)
+  int nrow = 0;     // ... on row-major weights
   int qblocks = 0;  // blocks of the quant launch
   uint32_t stage = 0;
 };
@@ -661,7 +902,7 @@ bool same_problem(const bitnet_linear_problem& a, const bitnet_linear_problem& b
   return a.x == b.x && a.x_dtype == b.x_dtype && a.gamma == b.gamma &&
          std::memcmp(&a.eps, &b.eps, sizeof(float)) == 0 && a.W_packed == b.W_packed &&
          a.s_w == b.s_w && a.M == b.M && a.N == b.N && a.K == b.K && a.y == b.y &&
-         a.y_dtype == b.y_dtype;
+         a.y_dtype == b.y_dtype && a.w_layout == b.w_layout;
 }
 
 // Whether problems a and b quantize the same activations identically.
@@ -705,30 +946,45 @@ bool build_decode_plan(const DeviceState& ds, int count, const bitnet_linear_pro
                        uint8_t* base, DecodePlan& plan) {
   QuantLaunch& QL = plan.QL;
   GemvLaunch& GL = plan.GL;
+  GtLaunch& TL = plan.TL;
   QL = QuantLaunch{};
   GL.count = 0;
-  // First pass: the matmul plan (it decides which partial regions need
-  // zeroing by the quant launch).
-  int n = 0, mmax = 0;
+  TL.count = 0;
+  // First pass: the matmul plans (the row-major one decides which partial
+  // regions need zeroing by the quant launch).
+  int nr = 0, nt = 0, mmax = 0;
   for (int i = 0; i < count; ++i) {
     const bitnet_linear_problem& q = problems[i];
     if (q.M == 0 || q.M > kGemvMaxM) continue;
-    GL.prob[n].M = static_cast<int>(q.M);
-    GL.prob[n].N = static_cast<int>(q.N);
-    GL.prob[n].K = static_cast<int>(q.K);
+    if (q.w_layout == BITNET_LAYOUT_TILED) {
+      TL.prob[nt].M = static_cast<int>(q.M);
+      TL.prob[nt].N = static_cast<int>(q.N);
+      TL.prob[nt].K = static_cast<int>(q.K);
+      ++nt;
+      continue;
+    }
+    GL.prob[nr].M = static_cast<int>(q.M);
+    GL.prob[nr].N = static_cast<int>(q.N);
+    GL.prob[nr].K = static_cast<int>(q.K);
     mmax = std::max(mmax, static_cast<int>(q.M));
-    ++n;
+    ++nr;
   }
-  GL.count = n;
-  plan.n = n;
-  plan.G = n > 0 ? plan_gemv_launch(GL, gemv_capacity(ds, mmax)) : 0;
+  GL.count = nr;
+  TL.count = nt;
+  plan.nrow = nr;
+  plan.n = nr + nt;
+  plan.G = nr > 0 ? plan_gemv_launch(GL, gemv_capacity(ds, mmax)) : 0;
+  if (nt > 0) plan_gt_launch(TL, ds.num_sms);
   int qblocks = 0, qn = 0;
   uint32_t stage = 0;
   size_t off = 0;
   int src[BITNET_MAX_GROUP];            // problem index of each decode problem
   uint8_t* qws[BITNET_MAX_GROUP];       // its quantized-activation workspace
   FwdWorkspace qL[BITNET_MAX_GROUP];
-  n = 0;
+  bool tl[BITNET_MAX_GROUP];
+  int n = 0;
+  nr = 0;
+  nt = 0;
   for (int i = 0; i < count; ++i) {
     const bitnet_linear_problem& q = problems[i];
     if (q.M == 0) continue;
@@ -736,43 +992,59 @@ bool build_decode_plan(const DeviceState& ds, int count, const bitnet_linear_pro
     uint8_t* ws = base + off;
     off += L.total;
     if (q.M > kGemvMaxM) continue;
-    const bool shared_rows = gemv_problem_shared(GL, n, plan.G);
+    const bool tiled = q.w_layout == BITNET_LAYOUT_TILED;
+    // Region the quant launch clears: the tiled kernel's arrival counters,
+    // or the row-major kernel's split-K partials when its CTAs share rows.
+    const bool shared_rows = !tiled && gemv_problem_shared(GL, nr, plan.G);
+    size_t zbytes = 0;
+    void* zero = tiled ? counter_region(ws, L, &zbytes)
+                       : (shared_rows ? splitk_region(ws, L, &zbytes) : nullptr);
     int owner = -1;
     if (!shared_rows)
       for (int j = 0; j < n && owner < 0; ++j)
-        if (same_input(problems[src[j]], q)) owner = j;
+        if (tl[j] == tiled && same_input(problems[src[j]], q)) owner = j;
     src[n] = i;
+    tl[n] = tiled;
+    QuantProblem& qp = QL.prob[qn++];
+    qp = QuantProblem{};
+    qp.zero16 = static_cast<uint4*>(zero);
+    qp.n_zero16 = zero ? static_cast<int64_t>(zbytes / 16) : 0;
+    qp.zero_blocks = static_cast<int>(zero ? zero_blocks(zbytes) : 0);
+    qp.block_begin = qblocks;
     if (owner >= 0) {
-      // Reuse that problem's quantization.
+      // Reuse that problem's quantization; this entry only clears.
       qws[n] = qws[owner];
       qL[n] = qL[owner];
+      qp.M = 0;
+      if (!zero) --qn;
     } else {
       qws[n] = ws;
       qL[n] = L;
-      size_t zbytes = 0;
-      void* zero = shared_rows ? splitk_region(ws, L, &zbytes) : nullptr;
-      QuantProblem& qp = QL.prob[qn++];
       qp.x = q.x;
       qp.gamma = q.gamma;
       qp.xi = reinterpret_cast<int8_t*>(ws + L.xq);
       qp.s_x = reinterpret_cast<float*>(ws + L.sx);
       qp.rowsum = reinterpret_cast<int32_t*>(ws + L.rs);
-      qp.zero16 = static_cast<uint4*>(zero);
-      qp.n_zero16 = zero ? static_cast<int64_t>(zbytes / 16) : 0;
       qp.eps = q.eps;
       qp.M = static_cast<int>(q.M);
       qp.K = static_cast<int>(q.K);
       qp.x_bf16 = (q.x_dtype == BITNET_BF16) ? 1 : 0;
       qp.perm = 1;  // decode matmul
-      qp.block_begin = qblocks;
-      qp.zero_blocks = static_cast<int>(zero ? zero_blocks(zbytes) : 0);
-      qblocks += qp.M + qp.zero_blocks;
+      qp.tiled = tiled ? 1 : 0;
       stage = std::max(stage, quant_stage_bytes(q.K, qp.x_bf16 != 0, q.gamma != nullptr));
     }
+    if (owner < 0 || zero) qblocks += qp.M + qp.zero_blocks;
     const float* sx = reinterpret_cast<const float*>(qws[n] + qL[n].sx);
-    if (!fill_gemv_problem(GL.maps[n], GL.prob[n], q.W_packed, qws[n], qL[n], ws, L, sx, q.s_w,
-                           q.M, q.N, q.K, q.y, q.y_dtype, nullptr))
-      return false;
+    if (tiled) {
+      fill_gt_problem(TL.prob[nt], q.W_packed, qws[n], qL[n], ws, L, sx, q.s_w, q.M, q.N, q.K,
+                      q.y, q.y_dtype, nullptr);
+      ++nt;
+    } else {
+      if (!fill_gemv_problem(GL.maps[nr], GL.prob[nr], q.W_packed, qws[n], qL[n], ws, L, sx,
+                             q.s_w, q.M, q.N, q.K, q.y, q.y_dtype, nullptr))
+        return false;
+      ++nr;
+    }
     ++n;
   }
   QL.count = qn;
@@ -827,10 +1099,17 @@ bitnet_status forward_grouped_impl(int count, const bitnet_linear_problem* probl
       const bitnet_status st = launch_status();
       if (st != BITNET_OK) return st;
     }
-    if (do_matmul) {
+    if (do_matmul && plan->nrow > 0) {
       // When the quant grid was just queued it started after every earlier
       // write to the weights, so the loads may begin before waiting on it.
       const bitnet_status st = launch_gemv_group(*ds, GL, plan->G, true, do_quant, stream);
+      if (st != BITNET_OK) return st;
+    }
+    if (do_matmul && plan->TL.count > 0) {
+      // Only a kernel of this library lets a dependent grid start early (the
+      // quant grid above), and it writes no weights: the tiled kernel's
+      // weight copies never need to wait.
+      const bitnet_status st = launch_gt(*ds, plan->TL, true, stream);
       if (st != BITNET_OK) return st;
     }
   }
@@ -846,7 +1125,8 @@ bitnet_status forward_grouped_impl(int count, const bitnet_linear_problem* probl
     if (q.M <= kGemvMaxM) continue;
     const bitnet_status st =
         forward_impl(q.x, q.x_dtype, q.gamma, q.eps, q.W_packed, q.s_w, q.M, q.N, q.K, q.y,
-                     q.y_dtype, ws, L.total, nullptr, nullptr, nullptr, BITNET_PATH_GEMM, stream);
+                     q.y_dtype, ws, L.total, nullptr, nullptr, nullptr, BITNET_PATH_GEMM, stream,
+                     q.w_layout);
     if (st != BITNET_OK) return st;
   }
   return BITNET_OK;
@@ -876,7 +1156,14 @@ BITNET_API const char* bitnet_status_string(int status) {
   }
 }
 
-BITNET_API int bitnet_version(void) { return 100; }
+BITNET_API int bitnet_version(void) { return 200; }
+
+BITNET_API int bitnet_last_cuda_error(const char** name) {
+  const int e = g_last_cuda_error;
+  g_last_cuda_error = 0;
+  if (name) *name = cudaGetErrorName(static_cast<cudaError_t>(e));
+  return e;
+}
 
 BITNET_API size_t bitnet_quantize_pack_weights_workspace_bytes(int64_t N, int64_t K) {
   (void)K;
@@ -983,6 +1270,303 @@ BITNET_API bitnet_status bitnet_linear_matmul(const uint8_t* W_packed, const flo
   return run_matmul(*ds, path, W_packed, ws, L, reinterpret_cast<const float*>(ws + L.sx), s_w,
                     M, N, K, y, y_dtype, nullptr, path == BITNET_PATH_GEMV, false,
                     as_stream(stream));
+}
+
+BITNET_API size_t bitnet_tiled_weights_bytes(int64_t N, int64_t K) {
+  if (N < 1 || K < 64 || N > BITNET_MAX_N || K > BITNET_MAX_K || K % 64 != 0) return 0;
+  return static_cast<size_t>(tiled_row_blocks(N) * tiled_chunks(K)) * kTileBytes;
+}
+
+BITNET_API bitnet_status bitnet_tile_weights(const uint8_t* W_packed, int64_t N, int64_t K,
+                                             uint8_t* W_tiled, bitnet_stream_t stream) {
+  bitnet_status st = check_shape(0, N, K);
+  if (st != BITNET_OK) return st;
+  if (!W_packed || !W_tiled) return BITNET_ERR_INVALID_ARG;
+  if (!aligned(W_packed, 16) || !aligned(W_tiled, 16)) return BITNET_ERR_MISALIGNED;
+  DeviceState* ds = device_state();
+  if (!ds) return BITNET_ERR_CUDA;
+  const int64_t npieces = tiled_row_blocks(N) * tiled_chunks(K) * (kTileBytes / 16);
+  const int64_t blocks = std::min<int64_t>((npieces + 255) / 256, 16LL * ds->num_sms);
+  tile_weights_kernel<<<static_cast<unsigned>(blocks), 256, 0, as_stream(stream)>>>(
+      W_packed, N, K, W_tiled, npieces);
+  return launch_status();
+}
+
+BITNET_API size_t bitnet_tiled_pair_weights_bytes(int64_t N, int64_t K) {
+  return 2 * bitnet_tiled_weights_bytes(N, K);
+}
+
+BITNET_API bitnet_status bitnet_tile_weights_pair(const uint8_t* Wa_packed,
+                                                  const uint8_t* Wb_packed, int64_t N, int64_t K,
+                                                  uint8_t* W_pair, bitnet_stream_t stream) {
+  bitnet_status st = check_shape(0, N, K);
+  if (st != BITNET_OK) return st;
+  if (!Wa_packed || !Wb_packed || !W_pair) return BITNET_ERR_INVALID_ARG;
+  if (!aligned(Wa_packed, 16) || !aligned(Wb_packed, 16) || !aligned(W_pair, 16))
+    return BITNET_ERR_MISALIGNED;
+  DeviceState* ds = device_state();
+  if (!ds) return BITNET_ERR_CUDA;
+  const int64_t npieces = tiled_row_blocks(N) * tiled_chunks(K) * (kTileBytes / 16);
+  const int64_t blocks = std::min<int64_t>((npieces + 255) / 256, 16LL * ds->num_sms);
+  tile_pair_weights_kernel<<<static_cast<unsigned>(blocks), 256, 0, as_stream(stream)>>>(
+      Wa_packed, Wb_packed, N, K, W_pair, npieces);
+  return launch_status();
+}
+
+namespace {
+// Workspace of the fused SwiGLU decode forward: the quantized input, its
+// scales and row sums, partial slots of 256 table rows, the counters.
+FwdWorkspace swiglu_layout(int64_t M, int64_t N, int64_t K) {
+  FwdWorkspace w{};
+  size_t o = 0;
+  w.xq = o;
+  o = align256(o + static_cast<size_t>(M * 256 * tiled_chunks(K)));
+  w.sx = o;
+  o = align256(o + 4 * static_cast<size_t>(M));
+  w.rs = o;
+  o = align256(o + 4 * static_cast<size_t>(M));
+  const int64_t units = tiled_row_blocks(N) * tiled_chunks(K);
+  w.acc = o;
+  o = align256(o + 2 * static_cast<size_t>(std::min<int64_t>(kGtMaxCtas, units)) *
+                       GtCfg<true>::TAB_ROWS * 4 * static_cast<size_t>(M));
+  w.cnt = o;
+  o = align256(o + 4 * static_cast<size_t>(tiled_row_blocks(N)));
+  w.total = o;
+  return w;
+}
+}  // namespace
+
+BITNET_API size_t bitnet_swiglu_forward_workspace_bytes(int64_t M, int64_t N, int64_t K) {
+  if (M < 0 || N < 0 || K < 0) return 0;
+  return swiglu_layout(M, N, K).total;
+}
+
+BITNET_API bitnet_status bitnet_swiglu_forward(const void* x, int x_dtype, const float* gamma,
+                                               float eps, const uint8_t* W_pair,
+                                               const float* s_w_gate, const float* s_w_up,
+                                               int64_t M, int64_t N, int64_t K, void* y,
+                                               int y_dtype, void* workspace,
+                                               size_t workspace_bytes, bitnet_stream_t stream) {
+  bitnet_status st = check_shape(M, N, K);
+  if (st != BITNET_OK) return st;
+  if (M == 0) return BITNET_OK;
+  if (M > kGemvMaxM) return BITNET_ERR_UNSUPPORTED_SHAPE;
+  if (!x || !W_pair || !s_w_gate || !s_w_up || !y || !ok_dtype(x_dtype) || !ok_dtype(y_dtype) ||
+      !(eps >= 0.0f) || eps > 3.0e38f)
+    return BITNET_ERR_INVALID_ARG;
+  if (!aligned(x, 16) || (gamma && !aligned(gamma, 16)) || !aligned(W_pair, 16) ||
+      !aligned(s_w_gate, 4) || !aligned(s_w_up, 4) || !aligned(y, 16))
+    return BITNET_ERR_MISALIGNED;
+  const FwdWorkspace L = swiglu_layout(M, N, K);
+  if (!workspace || workspace_bytes < L.total) return BITNET_ERR_WORKSPACE;
+  if (!aligned(workspace, 256)) return BITNET_ERR_MISALIGNED;
+  DeviceState* ds = device_state();
+  if (!ds) return BITNET_ERR_CUDA;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  cudaStream_t s = as_stream(stream);
+  size_t zbytes = 0;
+  void* zero = counter_region(ws, L, &zbytes);
+  float* sx = reinterpret_cast<float*>(ws + L.sx);
+  st = launch_act_quant(x, x_dtype, gamma, eps, M, K, reinterpret_cast<int8_t*>(ws + L.xq), sx,
+                        reinterpret_cast<int32_t*>(ws + L.rs), kXDecodeTiled, true, zero, zbytes,
+                        s);
+  if (st != BITNET_OK) return st;
+  static thread_local GtLaunch GL;
+  GL.count = 1;
+  fill_gt_problem(GL.prob[0], W_pair, ws, L, ws, L, sx, s_w_gate, M, N, K, y, y_dtype, nullptr);
+  GL.prob[0].s_w2 = s_w_up;
+  plan_gt_launch(GL, ds->num_sms);
+  return launch_gt(*ds, GL, true, s, true);
+}
+
+// ------------------------------------------------------ group-wise scales
+
+namespace {
+
+bitnet_status check_groups(int64_t K, int64_t group_k) {
+  if (group_k < 256 || group_k % 256 != 0 || K % group_k != 0 || K / group_k > kGroupMaxG)
+    return BITNET_ERR_UNSUPPORTED_SHAPE;
+  return BITNET_OK;
+}
+
+struct GsWorkspace {
+  size_t xq, sx, rs, gacc, part, cnt, total;
+};
+
+// x_q | s_x [M][G] | group row sums [M][G] | group sums [G][M][N] | tiled
+// decode kernel's partial slots and counters (M <= 16).
+GsWorkspace gs_layout(int64_t M, int64_t N, int64_t K, int64_t group_k) {
+  GsWorkspace w{};
+  const int64_t G = K / group_k;
+  size_t o = 0;
+  w.xq = o;
+  o = align256(o + static_cast<size_t>(M * 256 * tiled_chunks(K)));
+  w.sx = o;
+  o = align256(o + 4 * static_cast<size_t>(M * G));
+  w.rs = o;
+  o = align256(o + 4 * static_cast<size_t>(M * G));
+  w.gacc = o;
+  o = align256(o + 4 * static_cast<size_t>(G * M * N));
+  const int64_t tiles = tiled_row_blocks(N) * tiled_chunks(K);
+  w.part = o;
+  if (M <= kGemvMaxM)
+    o = align256(o + 2 * static_cast<size_t>(std::min<int64_t>(kGtMaxCtas, tiles)) *
+                         kTileRows * 4 * static_cast<size_t>(M));
+  w.cnt = o;
+  if (M <= kGemvMaxM) o = align256(o + 4 * static_cast<size_t>(tiled_row_blocks(N) * G));
+  w.total = o;
+  return w;
+}
+
+}  // namespace
+
+BITNET_API size_t bitnet_quantize_pack_weights_group_scales_workspace_bytes(int64_t N,
+                                                                            int64_t K,
+                                                                            int64_t group_k) {
+  if (N <= 0 || K <= 0 || group_k <= 0 || K % group_k != 0) return 0;
+  return align256(8 * static_cast<size_t>(N * (K / group_k)));
+}
+
+BITNET_API bitnet_status bitnet_quantize_pack_weights_group_scales(
+    const float* W, int64_t N, int64_t K, int64_t group_k, uint8_t* W_packed, float* s_w,
+    void* workspace, size_t workspace_bytes, bitnet_stream_t stream) {
+  bitnet_status st = check_shape(0, N, K);
+  if (st != BITNET_OK) return st;
+  st = check_groups(K, group_k);
+  if (st != BITNET_OK) return st;
+  if (!W || !W_packed || !s_w) return BITNET_ERR_INVALID_ARG;
+  if (!aligned(W, 16) || !aligned(W_packed, 16) || !aligned(s_w, 4)) return BITNET_ERR_MISALIGNED;
+  if (!workspace ||
+      workspace_bytes < bitnet_quantize_pack_weights_group_scales_workspace_bytes(N, K, group_k))
+    return BITNET_ERR_WORKSPACE;
+  if (!aligned(workspace, 256)) return BITNET_ERR_MISALIGNED;
+  DeviceState* ds = device_state();
+  if (!ds) return BITNET_ERR_CUDA;
+  cudaStream_t s = as_stream(stream);
+  const int64_t G = K / group_k;
+  double* R = static_cast<double*>(workspace);
+  group_row_abs_sum_kernel<<<static_cast<unsigned>(N), kWqThreads, 0, s>>>(W, K, group_k, R);
+  group_abs_total_kernel<<<static_cast<unsigned>(G), kWqThreads, 0, s>>>(R, N, G, group_k, s_w);
+  const int64_t nwords = N * K / 16;
+  const int64_t blocks = std::min<int64_t>((nwords + kWqThreads - 1) / kWqThreads,
+                                           static_cast<int64_t>(ds->num_sms) * 16);
+  group_pack_kernel<<<static_cast<unsigned>(blocks), kWqThreads, 0, s>>>(
+      W, nwords, K, group_k, s_w, reinterpret_cast<uint32_t*>(W_packed));
+  return launch_status();
+}
+
+BITNET_API size_t bitnet_linear_forward_group_scales_workspace_bytes(int64_t M, int64_t N,
+                                                                     int64_t K,
+                                                                     int64_t group_k) {
+  if (M < 0 || N < 0 || K <= 0 || group_k <= 0 || K % group_k != 0) return 0;
+  return gs_layout(M, N, K, group_k).total;
+}
+
+BITNET_API bitnet_status bitnet_linear_forward_group_scales(
+    const void* x, int x_dtype, const float* gamma, float eps, const uint8_t* W_packed,
+    int w_layout, const float* s_w, int64_t M, int64_t N, int64_t K, int64_t group_k, void* y,
+    int y_dtype, void* workspace, size_t workspace_bytes, int8_t* x_q_out, float* s_x_out,
+    int32_t* acc_out, bitnet_stream_t stream) {
+  bitnet_status st = check_shape(M, N, K);
+  if (st != BITNET_OK) return st;
+  st = check_groups(K, group_k);
+  if (st != BITNET_OK) return st;
+  if (M == 0) return BITNET_OK;
+  if (!x || !W_packed || !s_w || (!y && !acc_out) || !ok_dtype(x_dtype) || !(eps >= 0.0f) ||
+      eps > 3.0e38f || (y && !ok_dtype(y_dtype)))
+    return BITNET_ERR_INVALID_ARG;
+  if (w_layout != BITNET_LAYOUT_ROWS && w_layout != BITNET_LAYOUT_TILED)
+    return BITNET_ERR_INVALID_ARG;
+  if (!aligned(x, 16) || (gamma && !aligned(gamma, 16)) || !aligned(W_packed, 16) ||
+      !aligned(s_w, 4) || (y && !aligned(y, 16)) || (x_q_out && !aligned(x_q_out, 16)) ||
+      (s_x_out && !aligned(s_x_out, 4)) || (acc_out && !aligned(acc_out, 16)))
+    return BITNET_ERR_MISALIGNED;
+  const GsWorkspace L = gs_layout(M, N, K, group_k);
+  if (!workspace || workspace_bytes < L.total) return BITNET_ERR_WORKSPACE;
+  if (!aligned(workspace, 256)) return BITNET_ERR_MISALIGNED;
+  DeviceState* ds = device_state();
+  if (!ds) return BITNET_ERR_CUDA;
+  cudaStream_t s = as_stream(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  const int64_t G = K / group_k;
+  const bool tiled_decode = w_layout == BITNET_LAYOUT_TILED && M <= kGemvMaxM;
+  int8_t* xq = reinterpret_cast<int8_t*>(ws + L.xq);
+  float* sx = reinterpret_cast<float*>(ws + L.sx);
+  int32_t* rs = reinterpret_cast<int32_t*>(ws + L.rs);
+  int32_t* gacc = acc_out ? acc_out : reinterpret_cast<int32_t*>(ws + L.gacc);
+  const bool bf16 = x_dtype == BITNET_BF16;
+  if (x_q_out || s_x_out) {   // debug export: natural order, same arithmetic
+    float* sx_dbg = s_x_out ? s_x_out : sx;
+    int8_t* xq_dbg = x_q_out ? x_q_out : xq;
+    if (bf16)
+      group_rmsnorm_quant_kernel<true><<<static_cast<unsigned>(M), kActThreads, 0, s>>>(
+          x, gamma, eps, M, K, group_k, xq_dbg, sx_dbg, nullptr, 0, 0, 1, nullptr, 0, 0);
+    else
+      group_rmsnorm_quant_kernel<false><<<static_cast<unsigned>(M), kActThreads, 0, s>>>(
+          x, gamma, eps, M, K, group_k, xq_dbg, sx_dbg, nullptr, 0, 0, 1, nullptr, 0, 0);
+    st = launch_status();
+    if (st != BITNET_OK) return st;
+  }
+  size_t zbytes = tiled_decode ? L.total - L.cnt : 0;
+  uint4* zero = zbytes ? reinterpret_cast<uint4*>(ws + L.cnt) : nullptr;
+  const int64_t zb = zero ? zero_blocks(zbytes) : 0;
+  const dim3 qgrid(static_cast<unsigned>(M + zb));
+  if (bf16)
+    group_rmsnorm_quant_kernel<true><<<qgrid, kActThreads, 0, s>>>(
+        x, gamma, eps, M, K, group_k, xq, sx, rs, tiled_decode ? 1 : 0, tiled_decode ? 1 : 0, 0,
+        zero, zero ? static_cast<int64_t>(zbytes / 16) : 0, 1);
+  else
+    group_rmsnorm_quant_kernel<false><<<qgrid, kActThreads, 0, s>>>(
+        x, gamma, eps, M, K, group_k, xq, sx, rs, tiled_decode ? 1 : 0, tiled_decode ? 1 : 0, 0,
+        zero, zero ? static_cast<int64_t>(zbytes / 16) : 0, 1);
+  st = launch_status();
+  if (st != BITNET_OK) return st;
+  if (tiled_decode) {
+    static thread_local GtLaunch GL;
+    GL.count = 1;
+    GtProblem& q = GL.prob[0];
+    FwdWorkspace FL{};
+    FL.xq = L.xq;
+    FL.sx = L.sx;
+    FL.rs = L.rs;
+    FL.acc = L.part;
+    FL.cnt = L.cnt;
+    FL.total = L.total;
+    fill_gt_problem(q, W_packed, ws, FL, ws, FL, sx, s_w, M, N, K, nullptr, BITNET_F32, nullptr);
+    q.gc = static_cast<int>(group_k / 256);
+    q.G = static_cast<int>(G);
+    q.gacc = gacc;
+    plan_gt_launch(GL, ds->num_sms);
+    st = launch_gt(*ds, GL, true, s);
+  } else {
+    // tcgen05: one K split per group, each CTA writes its group's sums
+    GemmPlan pl = plan_gemm(M, N, K, ds->num_sms);
+    pl.steps_per_split = static_cast<int>(group_k / 256);
+    pl.ksplit = static_cast<int>(G);
+    st = launch_gemm_groups(*ds, W_packed, xq, rs, M, N, K, G, gacc, pl,
+                            w_layout == BITNET_LAYOUT_TILED, s);
+  }
+  if (st != BITNET_OK) return st;
+  if (y) {
+    const int64_t blocks = std::min<int64_t>((M * N + 255) / 256, 16LL * ds->num_sms);
+    group_combine_kernel<<<static_cast<unsigned>(blocks), 256, 0, s>>>(
+        gacc, sx, s_w, M, N, G, y, y_dtype == BITNET_BF16 ? 1 : 0);
+    st = launch_status();
+  }
+  return st;
+}
+
+BITNET_API bitnet_status bitnet_linear_forward_ex(const bitnet_linear_problem* problem,
+                                                  void* workspace, size_t workspace_bytes,
+                                                  int8_t* x_q_out, float* s_x_out,
+                                                  int32_t* acc_out, int path,
+                                                  bitnet_stream_t stream) {
+  if (!problem) return BITNET_ERR_INVALID_ARG;
+  const bitnet_linear_problem& q = *problem;
+  if (!q.y && !acc_out && q.M != 0) return BITNET_ERR_INVALID_ARG;
+  return forward_impl(q.x, q.x_dtype, q.gamma, q.eps, q.W_packed, q.s_w, q.M, q.N, q.K, q.y,
+                      q.y_dtype, workspace, workspace_bytes, x_q_out, s_x_out, acc_out, path,
+                      as_stream(stream), q.w_layout);
 }
 
 BITNET_API size_t bitnet_linear_forward_grouped_workspace_bytes(
@@ -1107,6 +1691,20 @@ extern "C" BITNET_API bitnet_status bitnet_selftest_divide(const float* a, const
   const int64_t blocks = std::min<int64_t>((n + 255) / 256, 4 * ds->num_sms);
   divide_selftest_kernel<<<static_cast<unsigned>(blocks), 256, 0, as_stream(stream)>>>(a, b, q,
                                                                                         n);
+  return launch_status();
+}
+
+extern "C" BITNET_API bitnet_status bitnet_selftest_mma_i8(int64_t iters, int ctas, int a_in_tmem,
+                                                          bitnet_stream_t stream) {
+  if (iters < 1 || iters > 100000000LL || ctas < 1 || ctas > 65535) return BITNET_ERR_INVALID_ARG;
+  DeviceState* ds = device_state();
+  if (!ds) return BITNET_ERR_CUDA;
+  if (a_in_tmem)
+    mma_i8_peak_kernel<true><<<ctas, 128, kPeakSmem, as_stream(stream)>>>(iters, ds->status,
+                                                                          kWaitLimitNs);
+  else
+    mma_i8_peak_kernel<false><<<ctas, 128, kPeakSmem, as_stream(stream)>>>(iters, ds->status,
+                                                                           kWaitLimitNs);
   return launch_status();
 }
 

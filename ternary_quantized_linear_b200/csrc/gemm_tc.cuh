@@ -10,10 +10,16 @@
 //
 // A CTA computes a 128 (weight rows, TMEM lanes) x BN (tokens) tile of
 // acc^T over a range of K, in 256-k steps:
-//   warp 0      TMA producer: per step the packed weight tile (128 rows x
-//               KSTEP/4 bytes) and the activation tile (BN rows of KSTEP int8
-//               as 128-byte swizzle atoms = the MMA's canonical K-major
-//               layout) into a STAGES-deep shared-memory ring;
+//   warp 0      weight producer: per step the packed weight tile (128 rows x
+//               KSTEP/4 bytes) into a STAGES-deep shared-memory ring, by a
+//               2-D tensor copy from the row-major layout or, with the tiled
+//               layout (tiled.cuh), by one 1-D bulk copy of the tile, which
+//               arrives already in the swizzled order the unpack reads;
+//   warps 2, 3  activation producers: one 128-byte swizzle atom each of the
+//               activation tile (BN rows of KSTEP int8 = the MMA's canonical
+//               K-major layout).  A thread can start a bulk copy only every
+//               few hundred nanoseconds, so the three copies of a step are
+//               issued by three threads;
 //   warp 1      allocates TMEM; one thread issues KSTEP/32 MMAs (K = 32 each)
 //               per step reading A from TMEM and B from shared memory;
 //   warps 4-11  unpack: each thread expands 16 packed bytes of its weight
@@ -45,6 +51,8 @@
 namespace bitnet {
 
 struct GemmParams {
+  const uint8_t* Wt;      // tiled weights (tiled.cuh), when the kernel reads that layout
+  int KC;                 // k chunks of the tiled layout
   const int32_t* rowsum;  // [M]
   const float* s_x;       // [M] (null: no dequant)
   const float* s_w;       // [1]
@@ -59,6 +67,11 @@ struct GemmParams {
   int* status;            // device status word
   uint64_t wait_limit_ns;
   int use_pdl;            // wait for the preceding grid before touching its outputs
+  // Group-wise scales (group_quant.cuh): the K split z is group z, rowsum
+  // is [M][G], and each CTA writes its group's integer sums to gacc
+  // [G][M][N] (no atomics, no dequant).  Null: per-tensor scales.
+  int32_t* gacc;
+  int G;
 };
 
 template <int BN>
@@ -96,7 +109,7 @@ struct GemmCfg {
   static constexpr int OFF_X = 0;
   static constexpr int OFF_WP = OFF_X + STAGES * X_BYTES;
   static constexpr int OFF_BAR = OFF_WP + STAGES * WP_BYTES;
-  static constexpr int NBAR = 2 * STAGES + A_STAGES + 1;  // full/done, aready, accfull
+  static constexpr int NBAR = 3 * STAGES + A_STAGES + 1;  // fullw/fullx/done, aready, accfull
   static constexpr int OFF_MISC = OFF_BAR + 8 * NBAR;
   static constexpr int OFF_TAB = (OFF_MISC + 16 + 15) & ~15;  // epilogue table: one int4 per token
   static constexpr int BYTES = OFF_TAB + 16 * BN;
@@ -178,7 +191,7 @@ __device__ __forceinline__ void gemm_store(const GemmParams& p, int4 e, int m, i
   }
 }
 
-template <int BN>
+template <int BN, bool kTiledW>
 __global__ void __launch_bounds__(GemmCfg<BN>::THREADS, GemmCfg<BN>::MIN_BLOCKS)
 ternary_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x,
                        const __grid_constant__ CUtensorMap tmap_w, const GemmParams p) {
@@ -188,14 +201,16 @@ ternary_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x,
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   uint8_t* xs = smem + C::OFF_X;
   uint8_t* wps = smem + C::OFF_WP;
-  // full[s]: both tiles of a step landed (TMA transaction bytes).
+  // fullw[s]: the step's weight tile landed; fullx[s]: its activation tile
+  //          (both atoms) landed (TMA transaction bytes).
   // done[s]: the step's MMAs completed (one tcgen05.commit) -- which also
   //          means the unpack warps had finished reading its weight tile,
   //          since the MMAs waited for them; it frees the shared-memory stage
-  //          for the producer and, A_STAGES steps later, the TMEM A stage.
+  //          for the producers and, A_STAGES steps later, the TMEM A stage.
   // aready[a]: the unpack warps stored TMEM A stage a.
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
-  uint64_t* done = full + C::STAGES;
+  uint64_t* fullw = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
+  uint64_t* fullx = fullw + C::STAGES;
+  uint64_t* done = fullx + C::STAGES;
   uint64_t* aready = done + C::STAGES;
   uint64_t* accfull = aready + C::A_STAGES;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
@@ -214,7 +229,8 @@ ternary_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x,
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::STAGES; ++s) {
-      mbar_init(&full[s], 1);
+      mbar_init(&fullw[s], 1);
+      mbar_init(&fullx[s], C::ATOMS);             // one producer per activation atom
       mbar_init(&done[s], 1);                     // MMA commit
     }
     for (int a = 0; a < C::A_STAGES; ++a) mbar_init(&aready[a], C::UNPACK_WARPS);
@@ -224,7 +240,7 @@ ternary_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x,
   }
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&tmap_x);
-    tma_prefetch_desc(&tmap_w);
+    if (!kTiledW) tma_prefetch_desc(&tmap_w);
   }
   if (warp == 1) {
     tmem_alloc(tmem_slot, C::TMEM_COLS);
@@ -238,34 +254,49 @@ ternary_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x,
   // sums, scales) are read only after this point.
   if (p.use_pdl) pdl_wait_prior_grid();
 
-  if (warp == 0) {
+  if (warp == 0 || warp == 2 || warp == 3) {
     if (lane == 0) {
-      // ------------------------------------------------------------ producer
-      int issued = 0;
-      for (int j = 0; j < nk; ++j) {
-        const int s = j % C::STAGES;
-        const uint32_t use = static_cast<uint32_t>(j / C::STAGES);
-        if (j >= C::STAGES && !mbar_wait_bounded(&done[s], (use - 1u) & 1u, abort_flag, limit)) {
-          gemm_fail(abort_flag, p.status, DEV_TIMEOUT_PRODUCER);
-          break;
-        }
-        const int kb = kb0 + j;
-        mbar_arrive_expect_tx(&full[s], C::X_BYTES + C::WP_BYTES);
-#pragma unroll
-        for (int at = 0; at < C::ATOMS; ++at)
-          tma_load_2d(xs + s * C::X_BYTES + at * C::X_ATOM, &tmap_x, kb * C::KSTEP + 128 * at, m0,
-                      &full[s]);
-        tma_load_2d(wps + s * C::WP_BYTES, &tmap_w, kb * C::WP_ROW, n0, &full[s]);
-        issued = j + 1;
-      }
-      if (*abort_flag) {
-        // Let the copies already in flight land before the CTA exits.
-        const int first = issued > C::STAGES ? issued - C::STAGES : 0;
-        for (int j = first; j < issued; ++j) {
+      // ----------------------------------------------------------- producers
+      // warp 0: weights; warp 2 + a: activation atom a.
+      const int atom = warp - 2;
+      const bool wprod = warp == 0;
+      uint64_t* full = wprod ? fullw : fullx;
+      if (wprod || atom < C::ATOMS) {
+        int issued = 0;
+        for (int j = 0; j < nk; ++j) {
           const int s = j % C::STAGES;
-          if (!mbar_wait_bounded(&full[s], static_cast<uint32_t>(j / C::STAGES) & 1u, nullptr,
-                                 limit))
-            record_failure(p.status, DEV_TIMEOUT_DRAIN);
+          const uint32_t use = static_cast<uint32_t>(j / C::STAGES);
+          if (j >= C::STAGES &&
+              !mbar_wait_bounded(&done[s], (use - 1u) & 1u, abort_flag, limit)) {
+            gemm_fail(abort_flag, p.status, DEV_TIMEOUT_PRODUCER);
+            break;
+          }
+          const int kb = kb0 + j;
+          if (wprod) {
+            mbar_arrive_expect_tx(&full[s], C::WP_BYTES);
+            if (kTiledW)
+              bulk_load(wps + s * C::WP_BYTES,
+                        p.Wt + (static_cast<int64_t>(blockIdx.x) * p.KC + kb) * C::WP_BYTES,
+                        C::WP_BYTES, &full[s]);
+            else
+              tma_load_2d(wps + s * C::WP_BYTES, &tmap_w, kb * C::WP_ROW, n0, &full[s]);
+          } else {
+            mbar_arrive_expect_tx(&full[s], C::X_ATOM);
+            tma_load_2d(xs + s * C::X_BYTES + atom * C::X_ATOM, &tmap_x,
+                        kb * C::KSTEP + 128 * atom, m0, &full[s]);
+          }
+          issued = j + 1;
+        }
+        if (*abort_flag) {
+          // Let this producer's copies in flight land before the CTA exits
+          // (the activation barrier completes only when both atoms land).
+          const int first = issued > C::STAGES ? issued - C::STAGES : 0;
+          for (int j = first; j < issued; ++j) {
+            const int s = j % C::STAGES;
+            if (!mbar_wait_bounded(&full[s], static_cast<uint32_t>(j / C::STAGES) & 1u, nullptr,
+                                   limit))
+              record_failure(p.status, DEV_TIMEOUT_DRAIN);
+          }
         }
       }
     }
@@ -276,12 +307,10 @@ ternary_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x,
       const uint32_t d_tmem = tmem_base + C::D_COL;
       for (int j = 0; j < nk; ++j) {
         const int s = j % C::STAGES, a = j % C::A_STAGES;
-        // aready implies full[s] already completed (the unpack warps waited
-        // on it); the MMA thread still observes full[s] itself so the copy
-        // engine's writes are ordered before its own tensor-core reads.
+        // The unpacked weights (aready) and the activation tile (fullx).
         if (!mbar_wait_bounded(&aready[a], static_cast<uint32_t>(j / C::A_STAGES) & 1u,
                                abort_flag, limit) ||
-            !mbar_wait_bounded(&full[s], static_cast<uint32_t>(j / C::STAGES) & 1u, abort_flag,
+            !mbar_wait_bounded(&fullx[s], static_cast<uint32_t>(j / C::STAGES) & 1u, abort_flag,
                                limit)) {
           gemm_fail(abort_flag, p.status, DEV_TIMEOUT_MMA);
           break;
@@ -319,7 +348,7 @@ ternary_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x,
         int rs = 0;
         float d = 1.0f;
         if (m < p.M) {
-          rs = p.rowsum[m];
+          rs = p.gacc ? p.rowsum[m * p.G + blockIdx.z] : p.rowsum[m];
           if (p.y) d = __fmul_rn(p.s_x[m], swv);
         }
         tab[c] = make_int4(rs, __float_as_int(d), __float_as_int(__frcp_rn(d)), 0);
@@ -331,7 +360,7 @@ ternary_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x,
       // A stage a was last used by step j - A_STAGES; its MMAs completed when
       // done[] of that step's shared-memory stage did.
       const int jp = j - C::A_STAGES;
-      if (!warp_wait(&full[s], static_cast<uint32_t>(j / C::STAGES) & 1u, abort_flag, limit) ||
+      if (!warp_wait(&fullw[s], static_cast<uint32_t>(j / C::STAGES) & 1u, abort_flag, limit) ||
           (jp >= 0 && !warp_wait(&done[jp % C::STAGES],
                                  static_cast<uint32_t>(jp / C::STAGES) & 1u, abort_flag, limit))) {
         gemm_fail(abort_flag, p.status, DEV_TIMEOUT_UNPACK);
@@ -375,7 +404,7 @@ ternary_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x,
     constexpr int kHalf = BN >= 32 ? BN / 2 : BN;
     if (write && (BN >= 32 || h == 0)) {
       const int n = n0 + i;
-      const bool split = p.ksplit > 1;
+      const bool split = p.ksplit > 1 && !p.gacc;
       for (int c0 = h * kHalf; c0 < (h + 1) * kHalf; c0 += 16) {
         if (m0 + c0 >= p.M) break;  // uniform across the warp
         uint32_t r[16];
@@ -386,7 +415,10 @@ ternary_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x,
           for (int jj = 0; jj < 16; ++jj) {
             const int m = m0 + c0 + jj;
             if (m < p.M) {
-              if (split)
+              if (p.gacc)
+                p.gacc[(static_cast<int64_t>(blockIdx.z) * p.M + m) * p.N + n] =
+                    static_cast<int>(r[jj]) - tab[c0 + jj].x;
+              else if (split)
                 atomicAdd(p.ws_acc + static_cast<int64_t>(m) * p.N + n, static_cast<int>(r[jj]));
               else
                 gemm_store(p, tab[c0 + jj], m, n, static_cast<int>(r[jj]));
@@ -405,7 +437,7 @@ ternary_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x,
   }
 
   // Split-K: the last CTA of this output tile finishes (no waiting).
-  if (p.ksplit > 1) {
+  if (p.ksplit > 1 && !p.gacc) {
     const int ok = __syncthreads_and(*abort_flag == 0 ? 1 : 0);
     if (!ok) return;
     const int tile = blockIdx.y * gridDim.x + blockIdx.x;

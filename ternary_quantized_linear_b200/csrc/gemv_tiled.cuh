@@ -1,0 +1,605 @@
+// gemv_tiled.cuh -- decode-path ternary matmul (M <= 16 tokens) plus fused
+// dequant on weights in the tiled layout (tiled.cuh), for one problem or a
+// group of independent problems in a single launch.
+//
+// Method: "LLM を 1.58 ビットにファインチューニング：BitNet による極端な量子化",
+// sections 計算パラダイム (integer accumulation), 推論最適化とカスタムカーネル
+// (weights unpacked on the fly inside the matmul), タイル化行列乗算 (tiles
+// staged in fast on-chip memory so global memory is read once) and
+// 量子化の仕組み (rescale by both scales).
+//
+// The decode matmul is bound by HBM: the packed weights are the traffic.
+// On B200 a thread can start a bulk copy only every few hundred nanoseconds
+// whatever its size, so the copies must be large: with the tiled layout the
+// weights of consecutive tiles are contiguous and move as one copy.
+//   * The problems' tiles (128 rows x 256 k, 8 KiB) are laid end to end,
+//     problem by problem, row block by row block; CTA b owns the contiguous
+//     tile range [tile_begin[b], tile_begin[b+1]) (cost-balanced by the
+//     host).  A "segment" is the part of one row block (with group-wise
+//     scales: of one group of a row block) inside that range.
+//   * Eight warps, one CTA per SM (up to 255 registers a thread).  A ring of
+//     shared-memory stages, each up to 32 KiB of weights of one segment plus
+//     the activations of the same k chunks: lane 0 of warp 0 copies the
+//     first half of a stage's weights, lane 0 of warp 1 the second half and
+//     the activations (the quantized input is stored chunk-major,
+//     [K/256][M][256 bytes], so those chunks are contiguous), one bulk copy
+//     each, refilling a stage once every warp has read it.  Weight copies
+//     start at once; activation copies wait for the preceding
+//     activation-quant grid (programmatic dependent launch).
+//   * Every warp takes rows 64 (w & 1) .. +63 of tile w >> 1 of a stage
+//     (64 rows x 256 k), unpacks the codes in registers (mask and shift; the
+//     activations are k-interleaved so a code word pairs with a plain
+//     activation word; the codes of k = 4i+2 and 4i+3 are kept times 16 in a
+//     second accumulator set, which saves two shifts per word) and issues
+//     mma.sync m16n8k32 s8 in swap-AB form (weight rows = MMA M, tokens = N,
+//     one or two n8 tiles) into register accumulators that live for the
+//     whole segment.  Tokens past M read some valid token's bytes: they only
+//     feed accumulator columns that are never stored.
+//   * At the end of a segment the warps add their accumulators into a
+//     shared 128 x 16 table (two tables, alternating) and, after a bounded
+//     barrier, finish it: y = (acc - rowsum) / (s_x * s_w) for a whole row
+//     block (constants fetched while the segment streams).  A part of a row
+//     block (the first and last segment of a CTA's range may be parts) goes
+//     to a per-CTA workspace slot with plain stores; a second, small kernel
+//     (gemv_tiled_fixup_kernel) sums the slots once the grid is done -- the
+//     kernel boundary orders the stores, so no fence, counter or waiting is
+//     needed in the streaming kernel.
+//   * Every wait is bounded; on a timeout the kernel records the failure,
+//     raises a CTA abort flag, lets the copies in flight land and exits
+//     without writing results.
+#pragma once
+
+#include "common.cuh"
+#include "gemv.cuh"
+#include "tiled.cuh"
+
+namespace bitnet {
+
+constexpr int kGtMmaWarps = 8;
+constexpr int kGtMmaThreads = 32 * kGtMmaWarps;
+constexpr int kGtThreads = kGtMmaThreads + 64;  // + weight producer warp + activation producer warp
+constexpr int kGtMaxCtas = 296;
+constexpr int kGtMaxGroup = 16;
+constexpr int kGtWBytes = 4 * kTileBytes;   // 32 KiB of weights per stage
+
+// Shape of the kernel's work unit.  Plain: a unit is one 128-row tile, four
+// per stage.  Pair (the fused SwiGLU): a unit is the gate tile and the up
+// tile of the same rows and k chunk (pair-tiled layout, 16 KiB), two per
+// stage; the table then holds 256 rows (gate rows 0-127, up rows 128-255).
+template <bool kPair>
+struct GtCfg {
+  static constexpr int UNIT_BYTES = kPair ? 2 * kTileBytes : kTileBytes;
+  static constexpr int UNITS = kGtWBytes / UNIT_BYTES;         // units (= k chunks) per stage
+  static constexpr int TAB_ROWS = kPair ? 2 * kTileRows : kTileRows;
+  static constexpr int STAGES = kPair ? 3 : 4;                 // the pair's larger table
+  static constexpr int X_BYTES = UNITS * 16 * 256;             // up to 16 tokens per chunk
+  static constexpr int STAGE_BYTES = kGtWBytes + X_BYTES;
+  static constexpr int SMEM_DYN = STAGES * STAGE_BYTES + 1024;  // + alignment slack
+};
+
+struct GtProblem {
+  const uint8_t* Wt;      // tiled weights
+  const uint8_t* xd;      // quantized activations, chunk-major [KC][M][256] (decode block order)
+  const int32_t* rowsum;  // [M]
+  const float* s_x;       // [M] (null: no dequant)
+  const float* s_w;       // [1] (null: no dequant); the gate's scale for a pair
+  const float* s_w2;      // [1] the up projection's scale (pair only)
+  void* y;                // [M][N] fp32 or bf16, may be null
+  int32_t* acc_out;       // [M][N] debug accumulators, may be null
+  int32_t* part;          // partial slots, 2 per contributing CTA, [M][table rows] int32
+  unsigned* cnt;          // [RB] arrival counters, zero on entry
+  long long tile_base;    // first tile of this problem in the launch
+  int M, N, K, KC, RB;
+  int y_bf16;
+  int cta_first;          // first CTA whose range holds a tile of this problem
+  // Group-wise scales (group_quant.cuh): gc = k chunks per group (0: one
+  // per-tensor group).  Segments then end at group boundaries, rowsum is
+  // [M][G], and instead of y the kernel writes every group's integer sums
+  // to gacc [G][M][N].
+  int gc, G;
+  int32_t* gacc;
+};
+
+struct GtLaunch {
+  GtProblem prob[kGtMaxGroup];
+  long long tile_begin[kGtMaxCtas + 1];  // CTA b owns [tile_begin[b], tile_begin[b+1])
+  int count;
+  int ctas;
+  int use_pdl;
+  int* status;
+  uint64_t wait_limit_ns;
+};
+
+// The segment that starts at tile t of a CTA range ending at t1.
+struct GtSeg {
+  int p, rb, c, nt;       // problem, row block, first chunk, tiles
+  long long t;            // first tile
+};
+
+__device__ __forceinline__ GtSeg gt_segment(const GtProblem* prob, int count, long long t,
+                                            long long t1) {
+  int p = 0;
+  while (p + 1 < count && t >= prob[p + 1].tile_base) ++p;
+  const GtProblem& P = prob[p];
+  const long long local = t - P.tile_base;
+  GtSeg s;
+  s.p = p;
+  s.rb = static_cast<int>(local / P.KC);
+  s.c = static_cast<int>(local - static_cast<long long>(s.rb) * P.KC);
+  long long end = P.tile_base + static_cast<long long>(s.rb + 1) * P.KC;
+  if (P.gc > 0) {   // a segment never crosses a group boundary
+    const long long gend = P.tile_base + static_cast<long long>(s.rb) * P.KC +
+                           (s.c / P.gc + 1) * static_cast<long long>(P.gc);
+    if (gend < end) end = gend;
+  }
+  s.nt = static_cast<int>((t1 < end ? t1 : end) - t);
+  s.t = t;
+  return s;
+}
+
+// Group of a segment (0 without groups), its first tile and its tile count:
+// the unit whose sums a whole segment completes and partial ones share.
+struct GtSpan {
+  int grp;
+  long long first;
+  int len;
+};
+
+__device__ __forceinline__ GtSpan gt_span(const GtProblem& P, const GtSeg& sg) {
+  GtSpan sp;
+  const long long rb0 = P.tile_base + static_cast<long long>(sg.rb) * P.KC;
+  if (P.gc > 0) {
+    sp.grp = sg.c / P.gc;
+    sp.first = rb0 + static_cast<long long>(sp.grp) * P.gc;
+    sp.len = P.gc;
+  } else {
+    sp.grp = 0;
+    sp.first = rb0;
+    sp.len = P.KC;
+  }
+  return sp;
+}
+
+// CTA whose range holds tile t (tile_begin is increasing).
+__device__ __forceinline__ int gt_cta_of(const long long* tb, int ctas, long long t) {
+  int lo = 0, hi = ctas - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (tb[mid] <= t) lo = mid; else hi = mid - 1;
+  }
+  return lo;
+}
+
+// Per-token constants of a segment's finish: row sum, divisor s_x * s_w and
+// RN(1 / divisor) (for a pair also those of the second scale).
+struct GtTok {
+  int rs;
+  float d, rd, d2, rd2;
+};
+
+__device__ __forceinline__ void gt_write(const GtProblem& P, int64_t o, float yv) {
+  if (P.y_bf16)
+    reinterpret_cast<__nv_bfloat16*>(P.y)[o] = __float2bfloat16_rn(yv);
+  else
+    reinterpret_cast<float*>(P.y)[o] = yv;
+}
+
+// Output n of token m from the integer sum of codes x (t + 1):
+// y = (acc - rowsum) / (s_x * s_w) with the token's constants from tk (with
+// group-wise scales: the group's integer sum, for the combining kernel).
+__device__ __forceinline__ void gt_store(const GtProblem& P, const GtTok& tk, int m, int n,
+                                         int acc_codes, int grp) {
+  const int acc = acc_codes - tk.rs;
+  const int64_t o = static_cast<int64_t>(m) * P.N + n;
+  if (P.gacc) {
+    P.gacc[static_cast<int64_t>(grp) * P.M * P.N + o] = acc;
+    return;
+  }
+  if (P.acc_out) P.acc_out[o] = acc;
+  if (P.y) gt_write(P, o, div_rn_by_recip(__int2float_rn(acc), tk.d, tk.rd));
+}
+
+// The fused SwiGLU output: silu(gate) * up with silu(z) = z / (1 + e^-z),
+// gate and up the two BitLinear outputs (fp32, bit-identical to separate
+// forwards), the activation in rounded fp32 steps (expf, then IEEE add,
+// divide, multiply).
+__device__ __forceinline__ void gt_store_pair(const GtProblem& P, const GtTok& tk, int m, int n,
+                                              int gate_codes, int up_codes) {
+  const float g = div_rn_by_recip(__int2float_rn(gate_codes - tk.rs), tk.d, tk.rd);
+  const float u = div_rn_by_recip(__int2float_rn(up_codes - tk.rs), tk.d2, tk.rd2);
+  const float sg = __fdiv_rn(g, __fadd_rn(1.0f, expf(-g)));
+  gt_write(P, static_cast<int64_t>(m) * P.N + n, __fmul_rn(sg, u));
+}
+
+// The token constants of token m of problem P for group grp (global loads).
+__device__ __forceinline__ GtTok gt_token(const GtProblem& P, int m, bool pair, int grp) {
+  GtTok tk;
+  tk.rs = P.gc > 0 ? P.rowsum[m * P.G + grp] : P.rowsum[m];
+  tk.d = P.s_w ? __fmul_rn(P.s_x[m], P.s_w[0]) : 1.0f;
+  tk.rd = __frcp_rn(tk.d);
+  tk.d2 = (pair && P.s_w2) ? __fmul_rn(P.s_x[m], P.s_w2[0]) : 1.0f;
+  tk.rd2 = __frcp_rn(tk.d2);
+  return tk;
+}
+
+// Barrier among the MMA warps on an mbarrier (count = kGtMmaWarps), so that
+// it can give up: lane 0 of each warp arrives, every lane waits on the
+// phase.  Returns false on a timeout or abort (warp-uniform).
+__device__ __forceinline__ bool gt_mma_sync(uint64_t* bar, uint32_t& phase,
+                                            const volatile int* abort_flag, uint64_t limit) {
+  __syncwarp();
+  if ((threadIdx.x & 31) == 0) mbar_arrive(bar);
+  const bool ok = mbar_wait_bounded(bar, phase, abort_flag, limit);
+  phase ^= 1u;
+  return __all_sync(0xFFFFFFFFu, ok);
+}
+
+// The MMAs of one 64-row x 256-k unit for TILES token tiles, one
+// accumulator set: the four code words of a packed word P are
+// (P >> 2r) & 0x03030303 for r = 0..3 (k = 4i + r of its 16-k group), paired
+// with the matching word of the k-interleaved activations.  Row groups
+// innermost, so consecutive MMAs feed independent accumulators.
+template <int NT, int TILES>
+__device__ __forceinline__ void gt_mma_unit(int (&acc)[4][NT][4], const GemvBuf<NT>& b) {
+#pragma unroll
+  for (int w = 0; w < 4; ++w) {
+#pragma unroll
+    for (int half = 0; half < 2; ++half) {
+      uint32_t a[4][4];  // [rg][a0 a1 a2 a3]
+#pragma unroll
+      for (int rg = 0; rg < 4; ++rg) {
+        const uint32_t Pa = word_of(b.wa[rg], w) >> (4 * half);
+        const uint32_t Pb = word_of(b.wb[rg], w) >> (4 * half);
+        a[rg][0] = Pa & kCodeMask;
+        a[rg][1] = Pb & kCodeMask;
+        a[rg][2] = (Pa >> 2) & kCodeMask;
+        a[rg][3] = (Pb >> 2) & kCodeMask;
+      }
+#pragma unroll
+      for (int nt = 0; nt < TILES; ++nt)
+#pragma unroll
+        for (int rg = 0; rg < 4; ++rg)
+          mma_m16n8k32_s8(acc[rg][nt], a[rg][0], a[rg][1], a[rg][2], a[rg][3],
+                          word_of(b.x[nt][w], 2 * half), word_of(b.x[nt][w], 2 * half + 1));
+    }
+  }
+}
+
+// Add a warp's accumulators into the segment's shared table and clear them.
+template <int NT, int TILES>
+__device__ __forceinline__ void gt_flush(int (&acc)[4][NT][4], int* red, int M, int g, int t) {
+#pragma unroll
+  for (int rg = 0; rg < 4; ++rg) {
+#pragma unroll
+    for (int nt = 0; nt < TILES; ++nt) {
+      const int r0 = 16 * rg + g, c0 = 8 * nt + 2 * t;
+      if (c0 < M) {
+        atomicAdd(&red[r0 * 16 + c0], acc[rg][nt][0]);
+        atomicAdd(&red[(r0 + 8) * 16 + c0], acc[rg][nt][2]);
+      }
+      if (c0 + 1 < M) {
+        atomicAdd(&red[r0 * 16 + c0 + 1], acc[rg][nt][1]);
+        atomicAdd(&red[(r0 + 8) * 16 + c0 + 1], acc[rg][nt][3]);
+      }
+#pragma unroll
+      for (int e = 0; e < 4; ++e) acc[rg][nt][e] = 0;
+    }
+  }
+}
+
+// One CTA of 320 threads (ten warps) per SM.  The register file is split
+// between the SM's four sub-partitions and two of them hold three warps, so
+// the launch bound caps a thread at about 170 registers.
+template <int NT, bool kPair>
+__global__ void __launch_bounds__(kGtThreads, 1)
+ternary_gemv_tiled_kernel(const __grid_constant__ GtLaunch L) {
+  using C = GtCfg<kPair>;
+  constexpr int S = C::STAGES;
+  constexpr int UNITS = C::UNITS;
+  constexpr int kTabRows = C::TAB_ROWS;
+  extern __shared__ uint8_t gt_smem_raw[];
+  uint8_t* ring = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(gt_smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  __shared__ int acc_tab[2][kTabRows * 16];        // [row][token] sums of a segment
+  __shared__ GtTok tok[2][16];                     // token constants of a segment
+  __shared__ GtTok tok_part[2][16];                // ... of the CTA's partial segments
+  __shared__ __align__(8) uint64_t full_w[S], full_x[S], empty[S];
+  __shared__ __align__(8) uint64_t seg_bar;
+  __shared__ volatile int abort_flag;
+  __shared__ int part_last[2];                     // last contributor of partial segment k?
+
+  // The problem table and the CTA ranges stay in kernel-parameter space:
+  // every access below uses an index that is the same for all threads of a
+  // warp, which that space serves as one broadcast.
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int count = L.count, ctas = L.ctas;
+  const uint64_t limit = L.wait_limit_ns;
+  const long long* stb = L.tile_begin;
+  if (tid == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(&full_w[s], 1);
+      mbar_init(&full_x[s], 1);
+      mbar_init(&empty[s], kGtMmaWarps);
+    }
+    mbar_init(&seg_bar, kGtMmaWarps);
+    abort_flag = 0;
+    fence_mbarrier_init();
+  }
+  __syncthreads();
+  const long long t0 = stb[blockIdx.x], t1 = stb[blockIdx.x + 1];
+  const GtProblem* prob = L.prob;
+
+  if (warp >= kGtMmaWarps) {
+    // ------------------------------------------------------------ producers
+    // A thread can start a bulk copy only every few hundred nanoseconds, so
+    // each stage's weights are split between the two producer threads:
+    // warp 8 copies the first half of the stage's units (full_w), warp 9 the
+    // second half and the activations (full_x).  Weights never depend on the
+    // preceding grid; warp 9 copies the weights of the first S stages, then
+    // waits for that grid (programmatic dependent launch) before copying any
+    // activations.
+    if (lane != 0) return;
+    const bool wprod = warp == kGtMmaWarps;
+    uint64_t* full = wprod ? full_w : full_x;
+    bool failed = false;
+    int j = 0;          // stage being issued
+    int pre = 0;        // warp 9: stages whose weight half went out before the wait
+    auto issue = [&](const GtSeg& sg, const GtProblem& P, int off, int jj, bool weights,
+                     bool acts, bool arrive) {
+      const int n = min(UNITS, sg.nt - off);
+      const int n1 = (n + 1) >> 1;                 // units of warp 8
+      const int s = jj % S;
+      uint8_t* st = ring + s * C::STAGE_BYTES;
+      const long long c = sg.c + off;
+      const uint8_t* wsrc = P.Wt + (static_cast<long long>(sg.rb) * P.KC + c) * C::UNIT_BYTES;
+      if (wprod) {
+        mbar_arrive_expect_tx(&full[s], static_cast<uint32_t>(n1 * C::UNIT_BYTES));
+        bulk_load(st, wsrc, static_cast<uint32_t>(n1 * C::UNIT_BYTES), &full[s]);
+        return;
+      }
+      const uint32_t wb = static_cast<uint32_t>((n - n1) * C::UNIT_BYTES);
+      const uint32_t xb = static_cast<uint32_t>(n * P.M * 256);
+      if (arrive) mbar_arrive_expect_tx(&full[s], wb + xb);
+      if (weights && wb)
+        bulk_load(st + n1 * C::UNIT_BYTES, wsrc + n1 * C::UNIT_BYTES, wb, &full[s]);
+      if (acts) bulk_load(st + kGtWBytes, P.xd + c * P.M * 256, xb, &full[s]);
+    };
+    if (!wprod) {
+      for (long long t = t0; t < t1 && pre < S;) {
+        const GtSeg sg = gt_segment(prob, count, t, t1);
+        const GtProblem& P = prob[sg.p];
+        for (int off = 0; off < sg.nt && pre < S; off += UNITS, ++pre)
+          issue(sg, P, off, pre, true, false, true);
+        t += sg.nt;
+      }
+      if (L.use_pdl) pdl_wait_prior_grid();
+    }
+    for (long long t = t0; t < t1 && !failed;) {
+      const GtSeg sg = gt_segment(prob, count, t, t1);
+      const GtProblem& P = prob[sg.p];
+      for (int off = 0; off < sg.nt; off += UNITS, ++j) {
+        const int s = j % S;
+        if (j >= S &&
+            !mbar_wait_bounded(&empty[s], static_cast<uint32_t>(j / S - 1) & 1u, &abort_flag,
+                               limit)) {
+          abort_flag = 1;
+          record_failure(L.status, DEV_TIMEOUT_PRODUCER);
+          failed = true;
+          break;
+        }
+        if (wprod || j >= pre)
+          issue(sg, P, off, j, true, !wprod, true);
+        else
+          issue(sg, P, off, j, false, true, false);   // weights already out
+      }
+      t += sg.nt;
+    }
+    if (abort_flag) {
+      // Let this producer's copies in flight land before the CTA exits.
+      for (int q = (j > S ? j - S : 0); q < max(j, pre); ++q)
+        if (!mbar_wait_bounded(&full[q % S], static_cast<uint32_t>(q / S) & 1u, nullptr, limit))
+          record_failure(L.status, DEV_TIMEOUT_DRAIN);
+    }
+    return;
+  }
+
+  // --------------------------------------------------------------- MMA warps
+  for (int i = tid; i < 2 * kTabRows * 16; i += kGtMmaThreads) (&acc_tab[0][0])[i] = 0;
+  // The token constants come from the quant grid.
+  if (L.use_pdl) pdl_wait_prior_grid();
+  const int g = lane >> 2, t = lane & 3;
+  // Unit u of each stage, sub-tile sub (pair: 0 = gate, 1 = up), half h.
+  const int u = kPair ? warp >> 2 : warp >> 1;
+  const int sub = kPair ? (warp >> 1) & 1 : 0;
+  const int h = warp & 1;
+  const int tab_row0 = sub * kTileRows + 64 * h;   // this warp's first table row
+  int acc[4][NT][4];
+#pragma unroll
+  for (int rg = 0; rg < 4; ++rg)
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) acc[rg][nt][e] = 0;
+  GemvBuf<NT> buf;
+  int j = 0, segi = 0, npart = 0;
+  uint32_t seg_phase = 0;
+  bool ok = gt_mma_sync(&seg_bar, seg_phase, &abort_flag, limit);   // tables cleared
+  GtSeg parts[2];
+  unsigned part_prev = 0u;         // thread 0: counter values before its arrivals
+  for (long long tt = t0; tt < t1 && ok; ++segi) {
+    const GtSeg sg = gt_segment(prob, count, tt, t1);
+    const GtProblem& P = prob[sg.p];
+    const int M = P.M;
+    const bool two = NT == 2 && M > 8;
+    // Warp 0 fetches the segment's token constants now; they are stored
+    // after the stage loop, which hides the loads' latency.
+    const GtSpan span = gt_span(P, sg);
+    GtTok tk{};
+    if (warp == 0 && lane < M) tk = gt_token(P, lane, kPair, span.grp);
+    bool any = false;
+    for (int off = 0; off < sg.nt; off += UNITS, ++j) {
+      const int n = min(UNITS, sg.nt - off);
+      const int s = j % S;
+      const uint32_t par = static_cast<uint32_t>(j / S) & 1u;
+      const bool got = mbar_wait_bounded(&full_w[s], par, &abort_flag, limit) &&
+                       mbar_wait_bounded(&full_x[s], par, &abort_flag, limit);
+      if (!__all_sync(0xFFFFFFFFu, got)) {
+        abort_flag = 1;
+        if (lane == 0) record_failure(L.status, DEV_TIMEOUT_GEMV);
+        ok = false;
+        break;
+      }
+      if (u < n) {
+        const uint8_t* ws =
+            ring + s * C::STAGE_BYTES + u * C::UNIT_BYTES + sub * kTileBytes + h * (64 * 64);
+        // Rows 64h + 16rg + g and +8 of the tile; piece t, swizzled by row.
+#pragma unroll
+        for (int rg = 0; rg < 4; ++rg) {
+          const int r = 16 * rg + g;           // (64h + r) >> 1 has the same low bits
+          const int sw = 16 * (t ^ ((r >> 1) & 3));
+          buf.wa[rg] = *reinterpret_cast<const uint4*>(ws + r * 64 + sw);
+          buf.wb[rg] = *reinterpret_cast<const uint4*>(ws + (r + 8) * 64 + sw);
+        }
+        const uint8_t* xs = ring + s * C::STAGE_BYTES + kGtWBytes + u * M * 256;
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+          if (nt == 0 || two) {
+            const int m = min(8 * nt + g, M - 1);   // tokens past M: any valid bytes
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+              buf.x[nt][q] = *reinterpret_cast<const uint4*>(
+                  xs + m * 256 + 16 * x_block_pos(4 * t + q, m & 1));
+          }
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[s]);
+      if (u < n) {
+        any = true;
+        if (two)
+          gt_mma_unit<NT, NT>(acc, buf);
+        else
+          gt_mma_unit<NT, 1>(acc, buf);
+      }
+    }
+    if (!ok) break;
+    const bool whole = sg.t == span.first && sg.nt == span.len;
+    const int kpart = (sg.t == t0) ? 0 : 1;       // a part is the CTA's first or last segment
+    if (warp == 0 && lane < M) {
+      if (whole) tok[segi & 1][lane] = tk; else tok_part[kpart][lane] = tk;
+    }
+    int* tab = acc_tab[segi & 1];
+    if (any) {
+      if (two)
+        gt_flush<NT, NT>(acc, tab + tab_row0 * 16, M, g, t);
+      else
+        gt_flush<NT, 1>(acc, tab + tab_row0 * 16, M, g, t);
+    }
+    if (!gt_mma_sync(&seg_bar, seg_phase, &abort_flag, limit)) {
+      ok = false;
+      break;
+    }
+    // ------------------------------------------------------- finish segment
+    // Every thread clears the table entries it reads, right after reading
+    // them (entries of tokens >= M are never written): the table is clean
+    // for its reuse two segments later, which the next segment's barrier
+    // orders after these writes.
+    const int n0 = sg.rb * kTileRows;
+    if (whole) {
+      for (int idx = tid; idx < kTileRows * M; idx += kGtMmaThreads) {
+        const int r = idx & (kTileRows - 1), m = idx >> 7;
+        const int v = tab[r * 16 + m];
+        tab[r * 16 + m] = 0;
+        if (kPair) {
+          const int v2 = tab[(kTileRows + r) * 16 + m];
+          tab[(kTileRows + r) * 16 + m] = 0;
+          if (n0 + r < P.N) gt_store_pair(P, tok[segi & 1][m], m, n0 + r, v, v2);
+        } else if (n0 + r < P.N) {
+          gt_store(P, tok[segi & 1][m], m, n0 + r, v, span.grp);
+        }
+      }
+    } else {
+      // Part of a row block: publish the partial sums in this CTA's slot
+      // and count the arrival; whether this CTA arrived last (and so
+      // finishes the row block) is looked at only after its last segment,
+      // so no thread waits for the counter here.
+      const int b = blockIdx.x;
+      int32_t* slot =
+          P.part + static_cast<int64_t>(2 * (b - P.cta_first) + kpart) * kTabRows * M;
+      for (int idx = tid; idx < kTabRows * M; idx += kGtMmaThreads) {
+        const int r = idx % kTabRows, m = idx / kTabRows;
+        slot[m * kTabRows + r] = tab[r * 16 + m];
+        tab[r * 16 + m] = 0;
+      }
+      if (!gt_mma_sync(&seg_bar, seg_phase, &abort_flag, limit)) {
+        ok = false;
+        break;
+      }
+      if (tid == 0) {
+        // The barrier made every thread's slot stores visible to this one;
+        // its fence orders them (cumulatively) before the counter update.
+        __threadfence();
+        part_prev |= atomicAdd(P.cnt + sg.rb * (P.gc > 0 ? P.G : 1) + span.grp, 1u)
+                     << (16 * kpart);
+      }
+      parts[kpart] = sg;
+      npart |= 1 << kpart;
+    }
+    tt += sg.nt;
+  }
+  if (!ok) {
+    if (lane == 0) record_failure(L.status, DEV_TIMEOUT_GEMV);
+    return;
+  }
+  if (npart == 0) return;   // uniform over the MMA warps
+  // Finish the row blocks this CTA arrived last on.
+  if (tid == 0) {
+    for (int k = 0; k < 2; ++k) {
+      int last = 0;
+      if (npart & (1 << k)) {
+        const GtSeg& sg = parts[k];
+        const GtSpan sp = gt_span(prob[sg.p], sg);
+        const int c_first = gt_cta_of(stb, ctas, sp.first);
+        const int c_last = gt_cta_of(stb, ctas, sp.first + sp.len - 1);
+        last = ((part_prev >> (16 * k)) & 0xFFFFu) == static_cast<unsigned>(c_last - c_first);
+      }
+      part_last[k] = last;
+    }
+    __threadfence();   // the other contributors' slots are read below
+  }
+  if (!gt_mma_sync(&seg_bar, seg_phase, &abort_flag, limit)) {
+    if (lane == 0) record_failure(L.status, DEV_TIMEOUT_GEMV);
+    return;
+  }
+  for (int k = 0; k < 2; ++k) {
+    if (!(npart & (1 << k)) || !part_last[k]) continue;
+    const GtSeg& sg = parts[k];
+    const GtProblem& P = prob[sg.p];
+    const int M = P.M;
+    const int n0 = sg.rb * kTileRows;
+    const GtSpan sp = gt_span(P, sg);
+    const long long r_first = sp.first;
+    const int c_first = gt_cta_of(stb, ctas, r_first);
+    const int c_last = gt_cta_of(stb, ctas, r_first + sp.len - 1);
+    for (int idx = tid; idx < kTileRows * M; idx += kGtMmaThreads) {
+      const int r = idx & (kTileRows - 1), m = idx >> 7;
+      int v = 0, v2 = 0;
+      for (int cb = c_first; cb <= c_last; ++cb) {
+        const int sd = (stb[cb] >= r_first) ? 0 : 1;
+        const int32_t* sl =
+            P.part + static_cast<int64_t>(2 * (cb - P.cta_first) + sd) * kTabRows * M;
+        v += __ldcg(sl + m * kTabRows + r);
+        if (kPair) v2 += __ldcg(sl + m * kTabRows + kTileRows + r);
+      }
+      if (n0 + r < P.N) {
+        if (kPair)
+          gt_store_pair(P, tok_part[k][m], m, n0 + r, v, v2);
+        else
+          gt_store(P, tok_part[k][m], m, n0 + r, v, sp.grp);
+      }
+    }
+    if (tid == 0) P.cnt[sg.rb * (P.gc > 0 ? P.G : 1) + sp.grp] = 0u;  // ready for the next call
+  }
+}
+
+}  // namespace bitnet

@@ -65,12 +65,14 @@ def test_single_rank_identity():
 
 
 def test_step_accounting():
-    case, probs = bench.problems()
-    assert len(probs) == 9
-    assert bench.step_tokens(probs) == 3 * (1 + 4 + 16)
-    # packed weights dominate: 3 x (3200*3200 + 2*3200*8640)/4 bytes per step
-    w = 3 * (3200 * 3200 + 2 * 3200 * 8640) // 4
-    assert w < bench.step_bytes(probs) < 1.05 * w
+    # the headline step: both 70B-shaped layers at M = 1, 16 and 64
+    case, probs = bench.case_problems(bench.HEADLINE, bench.HEADLINE_MS)
+    assert len(probs) == 6
+    assert sum(p[3] for p in probs) == 2 * (1 + 16 + 64)
+    # packed weights dominate: 3 x 2 x 8192*28672/4 bytes per step
+    w = 3 * 2 * 8192 * 28672 // 4
+    step = sum(bench.forward_bytes(M, N, K) for _, K, N, M in probs)
+    assert w < step < 1.06 * w   # + activations, x_q round trip and outputs
 
 
 def test_reference_arm_prints_json_line():
