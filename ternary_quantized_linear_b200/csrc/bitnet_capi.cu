@@ -119,10 +119,10 @@ DeviceState* device_state() {
     ok = ok && set_smem(ternary_gemm_tc_kernel<256, true>, GemmCfg<256>::SMEM_DYN);
     ok = ok && set_smem(mma_i8_peak_kernel<false>, kPeakSmem);
     ok = ok && set_smem(mma_i8_peak_kernel<true>, kPeakSmem);
-    ok = ok && set_smem(ternary_gemv_tiled_kernel<1, false>, GtCfg<false>::SMEM_DYN);
-    ok = ok && set_smem(ternary_gemv_tiled_kernel<2, false>, GtCfg<false>::SMEM_DYN);
-    ok = ok && set_smem(ternary_gemv_tiled_kernel<1, true>, GtCfg<true>::SMEM_DYN);
-    ok = ok && set_smem(ternary_gemv_tiled_kernel<2, true>, GtCfg<true>::SMEM_DYN);
+    ok = ok && set_smem(ternary_gemv_tiled_kernel<1, false>, GtCfg<false, 1>::SMEM_DYN);
+    ok = ok && set_smem(ternary_gemv_tiled_kernel<2, false>, GtCfg<false, 2>::SMEM_DYN);
+    ok = ok && set_smem(ternary_gemv_tiled_kernel<1, true>, GtCfg<true, 1>::SMEM_DYN);
+    ok = ok && set_smem(ternary_gemv_tiled_kernel<2, true>, GtCfg<true, 2>::SMEM_DYN);
     st.ok = ok;
   });
   return st.ok ? &st : nullptr;
@@ -482,7 +482,6 @@ bool fill_gt_problem(GtProblem& q, const uint8_t* Wt, uint8_t* xws, const FwdWor
   q.y = y;
   q.acc_out = acc_out;
   q.part = reinterpret_cast<int32_t*>(ws + Lw.acc);
-  q.cnt = reinterpret_cast<unsigned*>(ws + Lw.cnt);
   q.M = static_cast<int>(M);
   q.N = static_cast<int>(N);
   q.K = static_cast<int>(K);
@@ -500,7 +499,24 @@ int gt_tiles(const GtLaunch& L) {
   return 1;
 }
 
+// Whether a row block (with group-wise scales: a row-block group) of L is
+// split between CTAs: then the fixup kernel has to add the parts.  A CTA
+// range that starts where no such span starts splits one.
+bool gt_needs_fixup(const GtLaunch& L) {
+  int p = 0;
+  for (int b = 1; b < L.ctas; ++b) {
+    const long long t = L.tile_begin[b];
+    while (p + 1 < L.count && t >= L.prob[p + 1].tile_base) ++p;
+    const GtProblem& P = L.prob[p];
+    const long long c = (t - P.tile_base) % P.KC;
+    if (c % (P.gc > 0 ? P.gc : P.KC) != 0) return true;
+  }
+  return false;
+}
+
 // pair: the fused SwiGLU variant (every problem of L has pair-tiled weights).
+// The streaming kernel, then (when a span is split) the fixup kernel as its
+// programmatic dependent.
 bitnet_status launch_gt(const DeviceState& ds, GtLaunch& L, bool pdl, cudaStream_t stream,
                         bool pair = false) {
   L.use_pdl = pdl ? 1 : 0;
@@ -509,14 +525,15 @@ bitnet_status launch_gt(const DeviceState& ds, GtLaunch& L, bool pdl, cudaStream
   cudaLaunchConfig_t cfg{};
   cfg.gridDim = dim3(static_cast<unsigned>(L.ctas), 1, 1);
   cfg.blockDim = dim3(kGtThreads, 1, 1);
-  cfg.dynamicSmemBytes = pair ? GtCfg<true>::SMEM_DYN : GtCfg<false>::SMEM_DYN;
+  const int nt = gt_tiles(L);
+  cfg.dynamicSmemBytes = pair ? (nt == 2 ? GtCfg<true, 2>::SMEM_DYN : GtCfg<true, 1>::SMEM_DYN)
+                              : (nt == 2 ? GtCfg<false, 2>::SMEM_DYN : GtCfg<false, 1>::SMEM_DYN);
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = pdl ? 1 : 0;
-  const int nt = gt_tiles(L);
   cudaError_t e;
   if (pair)
     e = nt == 2 ? cudaLaunchKernelEx(&cfg, ternary_gemv_tiled_kernel<2, true>, L)
@@ -524,6 +541,16 @@ bitnet_status launch_gt(const DeviceState& ds, GtLaunch& L, bool pdl, cudaStream
   else
     e = nt == 2 ? cudaLaunchKernelEx(&cfg, ternary_gemv_tiled_kernel<2, false>, L)
                 : cudaLaunchKernelEx(&cfg, ternary_gemv_tiled_kernel<1, false>, L);
+  if (e != cudaSuccess || !gt_needs_fixup(L)) return cuda_status(e);
+  int mmax = 1;
+  for (int i = 0; i < L.count; ++i) mmax = std::max(mmax, L.prob[i].M);
+  cfg.gridDim = dim3(static_cast<unsigned>(L.ctas),
+                     static_cast<unsigned>((mmax + kGtFixTokens - 1) / kGtFixTokens), 1);
+  cfg.blockDim = dim3(kTileRows * kGtFixTokens, 1, 1);
+  cfg.dynamicSmemBytes = 0;
+  cfg.numAttrs = 1;
+  e = pair ? cudaLaunchKernelEx(&cfg, gemv_tiled_fixup_kernel<true>, L)
+           : cudaLaunchKernelEx(&cfg, gemv_tiled_fixup_kernel<false>, L);
   return cuda_status(e);
 }
 
@@ -1328,7 +1355,7 @@ FwdWorkspace swiglu_layout(int64_t M, int64_t N, int64_t K) {
   const int64_t units = tiled_row_blocks(N) * tiled_chunks(K);
   w.acc = o;
   o = align256(o + 2 * static_cast<size_t>(std::min<int64_t>(kGtMaxCtas, units)) *
-                       GtCfg<true>::TAB_ROWS * 4 * static_cast<size_t>(M));
+                       GtCfg<true, 1>::TAB_ROWS * 4 * static_cast<size_t>(M));
   w.cnt = o;
   o = align256(o + 4 * static_cast<size_t>(tiled_row_blocks(N)));
   w.total = o;

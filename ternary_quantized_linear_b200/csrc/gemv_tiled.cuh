@@ -17,20 +17,21 @@
 //     tile range [tile_begin[b], tile_begin[b+1]) (cost-balanced by the
 //     host).  A "segment" is the part of one row block (with group-wise
 //     scales: of one group of a row block) inside that range.
-//   * Eight warps, one CTA per SM (up to 255 registers a thread).  A ring of
+//   * Eight MMA warps and three producer warps, one CTA per SM.  A ring of
 //     shared-memory stages, each up to 32 KiB of weights of one segment plus
-//     the activations of the same k chunks: lane 0 of warp 0 copies the
-//     first half of a stage's weights, lane 0 of warp 1 the second half and
-//     the activations (the quantized input is stored chunk-major,
-//     [K/256][M][256 bytes], so those chunks are contiguous), one bulk copy
-//     each, refilling a stage once every warp has read it.  Weight copies
+//     the activations of the same k chunks.  One lane of each producer warp
+//     issues one bulk copy per stage: the first half of the stage's weights,
+//     the second half, and the activations (the quantized input is stored
+//     chunk-major, [K/256][M][256 bytes], so those chunks are contiguous).
+//     A stage is refilled once every MMA warp has read it.  Weight copies
 //     start at once; activation copies wait for the preceding
 //     activation-quant grid (programmatic dependent launch).
 //   * Every warp takes rows 64 (w & 1) .. +63 of tile w >> 1 of a stage
 //     (64 rows x 256 k), unpacks the codes in registers (mask and shift; the
 //     activations are k-interleaved so a code word pairs with a plain
-//     activation word; the codes of k = 4i+2 and 4i+3 are kept times 16 in a
-//     second accumulator set, which saves two shifts per word) and issues
+//     activation word; with one token tile the codes of k = 4i+2 and 4i+3
+//     are kept times 16 in a second accumulator set, which saves two shifts
+//     per word) and issues
 //     mma.sync m16n8k32 s8 in swap-AB form (weight rows = MMA M, tokens = N,
 //     one or two n8 tiles) into register accumulators that live for the
 //     whole segment.  Tokens past M read some valid token's bytes: they only
@@ -57,7 +58,7 @@ namespace bitnet {
 
 constexpr int kGtMmaWarps = 8;
 constexpr int kGtMmaThreads = 32 * kGtMmaWarps;
-constexpr int kGtThreads = kGtMmaThreads + 64;  // + weight producer warp + activation producer warp
+constexpr int kGtThreads = kGtMmaThreads + 96;  // + two weight producer warps + one activation producer
 constexpr int kGtMaxCtas = 296;
 constexpr int kGtMaxGroup = 16;
 constexpr int kGtWBytes = 4 * kTileBytes;   // 32 KiB of weights per stage
@@ -66,13 +67,15 @@ constexpr int kGtWBytes = 4 * kTileBytes;   // 32 KiB of weights per stage
 // per stage.  Pair (the fused SwiGLU): a unit is the gate tile and the up
 // tile of the same rows and k chunk (pair-tiled layout, 16 KiB), two per
 // stage; the table then holds 256 rows (gate rows 0-127, up rows 128-255).
-template <bool kPair>
+// NT token tiles of 8: a stage holds the activations of up to 8 NT tokens;
+// with one token tile the stages are smaller and the ring one deeper.
+template <bool kPair, int NT>
 struct GtCfg {
   static constexpr int UNIT_BYTES = kPair ? 2 * kTileBytes : kTileBytes;
   static constexpr int UNITS = kGtWBytes / UNIT_BYTES;         // units (= k chunks) per stage
   static constexpr int TAB_ROWS = kPair ? 2 * kTileRows : kTileRows;
-  static constexpr int STAGES = kPair ? 3 : 4;                 // the pair's larger table
-  static constexpr int X_BYTES = UNITS * 16 * 256;             // up to 16 tokens per chunk
+  static constexpr int STAGES = NT == 1 ? 5 : 4;
+  static constexpr int X_BYTES = UNITS * 8 * NT * 256;
   static constexpr int STAGE_BYTES = kGtWBytes + X_BYTES;
   static constexpr int SMEM_DYN = STAGES * STAGE_BYTES + 1024;  // + alignment slack
 };
@@ -87,7 +90,6 @@ struct GtProblem {
   void* y;                // [M][N] fp32 or bf16, may be null
   int32_t* acc_out;       // [M][N] debug accumulators, may be null
   int32_t* part;          // partial slots, 2 per contributing CTA, [M][table rows] int32
-  unsigned* cnt;          // [RB] arrival counters, zero on entry
   long long tile_base;    // first tile of this problem in the launch
   int M, N, K, KC, RB;
   int y_bf16;
@@ -265,35 +267,47 @@ __device__ __forceinline__ void gt_mma_unit(int (&acc)[4][NT][4], const GemvBuf<
   }
 }
 
-// Add a warp's accumulators into the segment's shared table and clear them.
-template <int NT, int TILES>
-__device__ __forceinline__ void gt_flush(int (&acc)[4][NT][4], int* red, int M, int g, int t) {
+// Add a warp's accumulators into the segment's shared table and clear them
+// (kHi: acc16 holds the times-16 sums of gemv_mma_unit, divided exactly).
+template <int NT, int TILES, bool kHi>
+__device__ __forceinline__ void gt_flush(int (&acc)[4][NT][4], int (&acc16)[4][NT][4], int* red,
+                                         int M, int g, int t) {
 #pragma unroll
   for (int rg = 0; rg < 4; ++rg) {
 #pragma unroll
     for (int nt = 0; nt < TILES; ++nt) {
       const int r0 = 16 * rg + g, c0 = 8 * nt + 2 * t;
+      int v[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) v[e] = kHi ? acc[rg][nt][e] + (acc16[rg][nt][e] >> 4) : acc[rg][nt][e];
       if (c0 < M) {
-        atomicAdd(&red[r0 * 16 + c0], acc[rg][nt][0]);
-        atomicAdd(&red[(r0 + 8) * 16 + c0], acc[rg][nt][2]);
+        atomicAdd(&red[r0 * 16 + c0], v[0]);
+        atomicAdd(&red[(r0 + 8) * 16 + c0], v[2]);
       }
       if (c0 + 1 < M) {
-        atomicAdd(&red[r0 * 16 + c0 + 1], acc[rg][nt][1]);
-        atomicAdd(&red[(r0 + 8) * 16 + c0 + 1], acc[rg][nt][3]);
+        atomicAdd(&red[r0 * 16 + c0 + 1], v[1]);
+        atomicAdd(&red[(r0 + 8) * 16 + c0 + 1], v[3]);
       }
 #pragma unroll
-      for (int e = 0; e < 4; ++e) acc[rg][nt][e] = 0;
+      for (int e = 0; e < 4; ++e) {
+        acc[rg][nt][e] = 0;
+        if (kHi) acc16[rg][nt][e] = 0;
+      }
     }
   }
 }
 
-// One CTA of 320 threads (ten warps) per SM.  The register file is split
-// between the SM's four sub-partitions and two of them hold three warps, so
-// the launch bound caps a thread at about 170 registers.
+// One CTA of 352 threads (eleven warps) per SM.  The register file is split
+// between the SM's four sub-partitions and three of them hold three warps,
+// so the launch bound caps a thread at about 170 registers.
 template <int NT, bool kPair>
 __global__ void __launch_bounds__(kGtThreads, 1)
 ternary_gemv_tiled_kernel(const __grid_constant__ GtLaunch L) {
-  using C = GtCfg<kPair>;
+  using C = GtCfg<kPair, NT>;
+  // One token tile: the unpack with a second, times-16 accumulator set
+  // (gemv_mma_unit, 5 ALU operations per MMA instead of 7); two token tiles
+  // would not leave the registers for it.
+  constexpr bool kHi = NT == 1;
   constexpr int S = C::STAGES;
   constexpr int UNITS = C::UNITS;
   constexpr int kTabRows = C::TAB_ROWS;
@@ -302,23 +316,24 @@ ternary_gemv_tiled_kernel(const __grid_constant__ GtLaunch L) {
       (reinterpret_cast<uintptr_t>(gt_smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   __shared__ int acc_tab[2][kTabRows * 16];        // [row][token] sums of a segment
   __shared__ GtTok tok[2][16];                     // token constants of a segment
-  __shared__ GtTok tok_part[2][16];                // ... of the CTA's partial segments
-  __shared__ __align__(8) uint64_t full_w[S], full_x[S], empty[S];
+  // full[s]: stage s has landed (three arrivals, one per producer thread,
+  // plus the bytes of its copies).  empty[s]: every MMA warp has read it.
+  __shared__ __align__(8) uint64_t full[S], empty[S];
   __shared__ __align__(8) uint64_t seg_bar;
   __shared__ volatile int abort_flag;
-  __shared__ int part_last[2];                     // last contributor of partial segment k?
 
+  // The dependent grid (the fixup of partial row blocks) only ever waits for
+  // this grid to complete, so it may be scheduled at once.
+  pdl_launch_dependents();
   // The problem table and the CTA ranges stay in kernel-parameter space:
   // every access below uses an index that is the same for all threads of a
   // warp, which that space serves as one broadcast.
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int count = L.count, ctas = L.ctas;
+  const int count = L.count;
   const uint64_t limit = L.wait_limit_ns;
-  const long long* stb = L.tile_begin;
   if (tid == 0) {
     for (int s = 0; s < S; ++s) {
-      mbar_init(&full_w[s], 1);
-      mbar_init(&full_x[s], 1);
+      mbar_init(&full[s], 3);
       mbar_init(&empty[s], kGtMmaWarps);
     }
     mbar_init(&seg_bar, kGtMmaWarps);
@@ -326,78 +341,60 @@ ternary_gemv_tiled_kernel(const __grid_constant__ GtLaunch L) {
     fence_mbarrier_init();
   }
   __syncthreads();
-  const long long t0 = stb[blockIdx.x], t1 = stb[blockIdx.x + 1];
+  const long long t0 = L.tile_begin[blockIdx.x], t1 = L.tile_begin[blockIdx.x + 1];
   const GtProblem* prob = L.prob;
 
   if (warp >= kGtMmaWarps) {
     // ------------------------------------------------------------ producers
-    // A thread can start a bulk copy only every few hundred nanoseconds, so
-    // each stage's weights are split between the two producer threads:
-    // warp 8 copies the first half of the stage's units (full_w), warp 9 the
-    // second half and the activations (full_x).  Weights never depend on the
-    // preceding grid; warp 9 copies the weights of the first S stages, then
-    // waits for that grid (programmatic dependent launch) before copying any
-    // activations.
+    // A thread starts a bulk copy only every few hundred nanoseconds, so
+    // every producer thread issues one copy per stage: role 0 the first half
+    // of the stage's units, role 1 the second half, role 2 the activations.
+    // Weights never depend on the preceding grid; the activations do, so
+    // role 2 waits for that grid (programmatic dependent launch) first.
     if (lane != 0) return;
-    const bool wprod = warp == kGtMmaWarps;
-    uint64_t* full = wprod ? full_w : full_x;
+    const int role = warp - kGtMmaWarps;
+    if (role == 2 && L.use_pdl) pdl_wait_prior_grid();
+    uint64_t* fb = full;
     bool failed = false;
     int j = 0;          // stage being issued
-    int pre = 0;        // warp 9: stages whose weight half went out before the wait
-    auto issue = [&](const GtSeg& sg, const GtProblem& P, int off, int jj, bool weights,
-                     bool acts, bool arrive) {
-      const int n = min(UNITS, sg.nt - off);
-      const int n1 = (n + 1) >> 1;                 // units of warp 8
-      const int s = jj % S;
-      uint8_t* st = ring + s * C::STAGE_BYTES;
-      const long long c = sg.c + off;
-      const uint8_t* wsrc = P.Wt + (static_cast<long long>(sg.rb) * P.KC + c) * C::UNIT_BYTES;
-      if (wprod) {
-        mbar_arrive_expect_tx(&full[s], static_cast<uint32_t>(n1 * C::UNIT_BYTES));
-        bulk_load(st, wsrc, static_cast<uint32_t>(n1 * C::UNIT_BYTES), &full[s]);
-        return;
-      }
-      const uint32_t wb = static_cast<uint32_t>((n - n1) * C::UNIT_BYTES);
-      const uint32_t xb = static_cast<uint32_t>(n * P.M * 256);
-      if (arrive) mbar_arrive_expect_tx(&full[s], wb + xb);
-      if (weights && wb)
-        bulk_load(st + n1 * C::UNIT_BYTES, wsrc + n1 * C::UNIT_BYTES, wb, &full[s]);
-      if (acts) bulk_load(st + kGtWBytes, P.xd + c * P.M * 256, xb, &full[s]);
-    };
-    if (!wprod) {
-      for (long long t = t0; t < t1 && pre < S;) {
-        const GtSeg sg = gt_segment(prob, count, t, t1);
-        const GtProblem& P = prob[sg.p];
-        for (int off = 0; off < sg.nt && pre < S; off += UNITS, ++pre)
-          issue(sg, P, off, pre, true, false, true);
-        t += sg.nt;
-      }
-      if (L.use_pdl) pdl_wait_prior_grid();
-    }
     for (long long t = t0; t < t1 && !failed;) {
       const GtSeg sg = gt_segment(prob, count, t, t1);
       const GtProblem& P = prob[sg.p];
       for (int off = 0; off < sg.nt; off += UNITS, ++j) {
         const int s = j % S;
-        if (j >= S &&
-            !mbar_wait_bounded(&empty[s], static_cast<uint32_t>(j / S - 1) & 1u, &abort_flag,
-                               limit)) {
+        if (j >= S && !mbar_wait_bounded_sleep(&empty[s], static_cast<uint32_t>(j / S - 1) & 1u,
+                                               &abort_flag, limit)) {
           abort_flag = 1;
           record_failure(L.status, DEV_TIMEOUT_PRODUCER);
           failed = true;
           break;
         }
-        if (wprod || j >= pre)
-          issue(sg, P, off, j, true, !wprod, true);
-        else
-          issue(sg, P, off, j, false, true, false);   // weights already out
+        const int n = min(UNITS, sg.nt - off);
+        const int n1 = (n + 1) >> 1;               // units of role 0
+        uint8_t* st = ring + s * C::STAGE_BYTES;
+        const long long c = sg.c + off;
+        const uint8_t* wsrc = P.Wt + (static_cast<long long>(sg.rb) * P.KC + c) * C::UNIT_BYTES;
+        if (role == 0) {
+          const uint32_t b = static_cast<uint32_t>(n1 * C::UNIT_BYTES);
+          mbar_arrive_expect_tx(&fb[s], b);
+          bulk_load(st, wsrc, b, &fb[s]);
+        } else if (role == 1) {
+          const uint32_t b = static_cast<uint32_t>((n - n1) * C::UNIT_BYTES);
+          mbar_arrive_expect_tx(&fb[s], b);
+          if (b) bulk_load(st + n1 * C::UNIT_BYTES, wsrc + n1 * C::UNIT_BYTES, b, &fb[s]);
+        } else {
+          const uint32_t b = static_cast<uint32_t>(n * P.M * 256);
+          mbar_arrive_expect_tx(&fb[s], b);
+          bulk_load(st + kGtWBytes, P.xd + c * P.M * 256, b, &fb[s]);
+        }
       }
       t += sg.nt;
     }
     if (abort_flag) {
-      // Let this producer's copies in flight land before the CTA exits.
-      for (int q = (j > S ? j - S : 0); q < max(j, pre); ++q)
-        if (!mbar_wait_bounded(&full[q % S], static_cast<uint32_t>(q / S) & 1u, nullptr, limit))
+      // Let this thread's copies in flight land before the CTA exits (the
+      // wait gives up at the limit if another producer stopped arriving).
+      for (int q = (j > S ? j - S : 0); q < j; ++q)
+        if (!mbar_wait_bounded(&fb[q % S], static_cast<uint32_t>(q / S) & 1u, nullptr, limit))
           record_failure(L.status, DEV_TIMEOUT_DRAIN);
     }
     return;
@@ -413,36 +410,44 @@ ternary_gemv_tiled_kernel(const __grid_constant__ GtLaunch L) {
   const int sub = kPair ? (warp >> 1) & 1 : 0;
   const int h = warp & 1;
   const int tab_row0 = sub * kTileRows + 64 * h;   // this warp's first table row
-  int acc[4][NT][4];
+  int acc[4][NT][4], acc16[4][NT][4];
 #pragma unroll
   for (int rg = 0; rg < 4; ++rg)
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-      for (int e = 0; e < 4; ++e) acc[rg][nt][e] = 0;
+      for (int e = 0; e < 4; ++e) {
+        acc[rg][nt][e] = 0;
+        acc16[rg][nt][e] = 0;
+      }
   GemvBuf<NT> buf;
-  int j = 0, segi = 0, npart = 0;
+  int j = 0, segi = 0;
+  GtTok tk{};
+  int tk_p = -1, tk_grp = -1;
   uint32_t seg_phase = 0;
   bool ok = gt_mma_sync(&seg_bar, seg_phase, &abort_flag, limit);   // tables cleared
-  GtSeg parts[2];
-  unsigned part_prev = 0u;         // thread 0: counter values before its arrivals
   for (long long tt = t0; tt < t1 && ok; ++segi) {
     const GtSeg sg = gt_segment(prob, count, tt, t1);
     const GtProblem& P = prob[sg.p];
     const int M = P.M;
     const bool two = NT == 2 && M > 8;
-    // Warp 0 fetches the segment's token constants now; they are stored
-    // after the stage loop, which hides the loads' latency.
     const GtSpan span = gt_span(P, sg);
-    GtTok tk{};
-    if (warp == 0 && lane < M) tk = gt_token(P, lane, kPair, span.grp);
+    const bool whole = sg.t == span.first && sg.nt == span.len;
+    // Warp 0 keeps the token constants of the current (problem, group) in
+    // registers and fetches them only when that changes: a fetch stalls the
+    // warp for a global-memory round trip, and every other warp would wait
+    // for it at the next stage release.
+    if (warp == 0 && (sg.p != tk_p || span.grp != tk_grp)) {
+      if (lane < M) tk = gt_token(P, lane, kPair, span.grp);
+      tk_p = sg.p;
+      tk_grp = span.grp;
+    }
     bool any = false;
     for (int off = 0; off < sg.nt; off += UNITS, ++j) {
       const int n = min(UNITS, sg.nt - off);
       const int s = j % S;
       const uint32_t par = static_cast<uint32_t>(j / S) & 1u;
-      const bool got = mbar_wait_bounded(&full_w[s], par, &abort_flag, limit) &&
-                       mbar_wait_bounded(&full_x[s], par, &abort_flag, limit);
+      const bool got = mbar_wait_bounded_sleep(&full[s], par, &abort_flag, limit);
       if (!__all_sync(0xFFFFFFFFu, got)) {
         abort_flag = 1;
         if (lane == 0) record_failure(L.status, DEV_TIMEOUT_GEMV);
@@ -476,24 +481,22 @@ ternary_gemv_tiled_kernel(const __grid_constant__ GtLaunch L) {
       if (lane == 0) mbar_arrive(&empty[s]);
       if (u < n) {
         any = true;
-        if (two)
+        if (kHi)
+          gemv_mma_unit<NT, 1>(acc, acc16, buf);
+        else if (two)
           gt_mma_unit<NT, NT>(acc, buf);
         else
           gt_mma_unit<NT, 1>(acc, buf);
       }
     }
     if (!ok) break;
-    const bool whole = sg.t == span.first && sg.nt == span.len;
-    const int kpart = (sg.t == t0) ? 0 : 1;       // a part is the CTA's first or last segment
-    if (warp == 0 && lane < M) {
-      if (whole) tok[segi & 1][lane] = tk; else tok_part[kpart][lane] = tk;
-    }
+    if (whole && warp == 0 && lane < M) tok[segi & 1][lane] = tk;
     int* tab = acc_tab[segi & 1];
     if (any) {
       if (two)
-        gt_flush<NT, NT>(acc, tab + tab_row0 * 16, M, g, t);
+        gt_flush<NT, NT, kHi>(acc, acc16, tab + tab_row0 * 16, M, g, t);
       else
-        gt_flush<NT, 1>(acc, tab + tab_row0 * 16, M, g, t);
+        gt_flush<NT, 1, kHi>(acc, acc16, tab + tab_row0 * 16, M, g, t);
     }
     if (!gt_mma_sync(&seg_bar, seg_phase, &abort_flag, limit)) {
       ok = false;
@@ -519,87 +522,65 @@ ternary_gemv_tiled_kernel(const __grid_constant__ GtLaunch L) {
         }
       }
     } else {
-      // Part of a row block: publish the partial sums in this CTA's slot
-      // and count the arrival; whether this CTA arrived last (and so
-      // finishes the row block) is looked at only after its last segment,
-      // so no thread waits for the counter here.
-      const int b = blockIdx.x;
-      int32_t* slot =
-          P.part + static_cast<int64_t>(2 * (b - P.cta_first) + kpart) * kTabRows * M;
+      // Part of a row block (the CTA's first or last segment): its sums go
+      // to this CTA's slot; gemv_tiled_fixup_kernel adds the slots up.
+      const int kpart = (sg.t == t0) ? 0 : 1;
+      int32_t* slot = P.part + static_cast<int64_t>(2 * (static_cast<int>(blockIdx.x) -
+                                                         P.cta_first) + kpart) *
+                                   kTabRows * M;
       for (int idx = tid; idx < kTabRows * M; idx += kGtMmaThreads) {
         const int r = idx % kTabRows, m = idx / kTabRows;
         slot[m * kTabRows + r] = tab[r * 16 + m];
         tab[r * 16 + m] = 0;
       }
-      if (!gt_mma_sync(&seg_bar, seg_phase, &abort_flag, limit)) {
-        ok = false;
-        break;
-      }
-      if (tid == 0) {
-        // The barrier made every thread's slot stores visible to this one;
-        // its fence orders them (cumulatively) before the counter update.
-        __threadfence();
-        part_prev |= atomicAdd(P.cnt + sg.rb * (P.gc > 0 ? P.G : 1) + span.grp, 1u)
-                     << (16 * kpart);
-      }
-      parts[kpart] = sg;
-      npart |= 1 << kpart;
     }
     tt += sg.nt;
   }
-  if (!ok) {
-    if (lane == 0) record_failure(L.status, DEV_TIMEOUT_GEMV);
-    return;
+  if (!ok && lane == 0) record_failure(L.status, DEV_TIMEOUT_GEMV);
+}
+
+// Finish of the row blocks (with group-wise scales: row-block groups) that
+// several CTAs of ternary_gemv_tiled_kernel share.  Such a span is finished
+// by the CTAs of column blockIdx.x, the CTA of the streaming kernel whose
+// range holds the span's first tile: that CTA's last span, when it starts
+// inside the CTA's range and ends past it.  The contributors are the CTAs
+// whose ranges meet the span; each left its sums in its slot 0 (its range
+// starts inside the span) or slot 1 (the finishing CTA, whose range starts
+// before the span).  One thread per output (row r = threadIdx.x % 128,
+// token kGtFixTokens * blockIdx.y + threadIdx.x / 128), so every load of a
+// thread is independent of the others and they overlap.  Launched right
+// after the streaming kernel as its programmatic dependent: the wait below
+// returns once that grid has completed and its stores are visible.
+constexpr int kGtFixTokens = 4;
+template <bool kPair>
+__global__ void __launch_bounds__(kTileRows * kGtFixTokens)
+gemv_tiled_fixup_kernel(const __grid_constant__ GtLaunch L) {
+  constexpr int kTabRows = GtCfg<kPair, 1>::TAB_ROWS;
+  pdl_wait_prior_grid();
+  const long long* stb = L.tile_begin;
+  const long long t0 = stb[blockIdx.x], t1 = stb[blockIdx.x + 1];
+  const GtSeg sg = gt_segment(L.prob, L.count, t1 - 1, t1);
+  const GtProblem& P = L.prob[sg.p];
+  const GtSpan sp = gt_span(P, sg);
+  if (sp.first < t0 || sp.first + sp.len <= t1) return;
+  const int r = threadIdx.x % kTileRows;
+  const int m = kGtFixTokens * blockIdx.y + threadIdx.x / kTileRows;
+  const int n = sg.rb * kTileRows + r;
+  if (m >= P.M || n >= P.N) return;
+  const int c_last = gt_cta_of(stb, L.ctas, sp.first + sp.len - 1);
+  const GtTok tk = gt_token(P, m, kPair, sp.grp);
+  int v = 0, v2 = 0;
+  for (int cb = blockIdx.x; cb <= c_last; ++cb) {
+    const int sd = (stb[cb] >= sp.first) ? 0 : 1;
+    const int32_t* sl =
+        P.part + static_cast<int64_t>(2 * (cb - P.cta_first) + sd) * kTabRows * P.M;
+    v += __ldcg(sl + m * kTabRows + r);
+    if (kPair) v2 += __ldcg(sl + m * kTabRows + kTileRows + r);
   }
-  if (npart == 0) return;   // uniform over the MMA warps
-  // Finish the row blocks this CTA arrived last on.
-  if (tid == 0) {
-    for (int k = 0; k < 2; ++k) {
-      int last = 0;
-      if (npart & (1 << k)) {
-        const GtSeg& sg = parts[k];
-        const GtSpan sp = gt_span(prob[sg.p], sg);
-        const int c_first = gt_cta_of(stb, ctas, sp.first);
-        const int c_last = gt_cta_of(stb, ctas, sp.first + sp.len - 1);
-        last = ((part_prev >> (16 * k)) & 0xFFFFu) == static_cast<unsigned>(c_last - c_first);
-      }
-      part_last[k] = last;
-    }
-    __threadfence();   // the other contributors' slots are read below
-  }
-  if (!gt_mma_sync(&seg_bar, seg_phase, &abort_flag, limit)) {
-    if (lane == 0) record_failure(L.status, DEV_TIMEOUT_GEMV);
-    return;
-  }
-  for (int k = 0; k < 2; ++k) {
-    if (!(npart & (1 << k)) || !part_last[k]) continue;
-    const GtSeg& sg = parts[k];
-    const GtProblem& P = prob[sg.p];
-    const int M = P.M;
-    const int n0 = sg.rb * kTileRows;
-    const GtSpan sp = gt_span(P, sg);
-    const long long r_first = sp.first;
-    const int c_first = gt_cta_of(stb, ctas, r_first);
-    const int c_last = gt_cta_of(stb, ctas, r_first + sp.len - 1);
-    for (int idx = tid; idx < kTileRows * M; idx += kGtMmaThreads) {
-      const int r = idx & (kTileRows - 1), m = idx >> 7;
-      int v = 0, v2 = 0;
-      for (int cb = c_first; cb <= c_last; ++cb) {
-        const int sd = (stb[cb] >= r_first) ? 0 : 1;
-        const int32_t* sl =
-            P.part + static_cast<int64_t>(2 * (cb - P.cta_first) + sd) * kTabRows * M;
-        v += __ldcg(sl + m * kTabRows + r);
-        if (kPair) v2 += __ldcg(sl + m * kTabRows + kTileRows + r);
-      }
-      if (n0 + r < P.N) {
-        if (kPair)
-          gt_store_pair(P, tok_part[k][m], m, n0 + r, v, v2);
-        else
-          gt_store(P, tok_part[k][m], m, n0 + r, v, sp.grp);
-      }
-    }
-    if (tid == 0) P.cnt[sg.rb * (P.gc > 0 ? P.G : 1) + sp.grp] = 0u;  // ready for the next call
-  }
+  if (kPair)
+    gt_store_pair(P, tk, m, n, v, v2);
+  else
+    gt_store(P, tk, m, n, v, sp.grp);
 }
 
 }  // namespace bitnet

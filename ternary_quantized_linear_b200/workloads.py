@@ -144,3 +144,26 @@ def all_problems(case: Case):
     for si, (K, N) in enumerate(case.shapes):
         for M in case.ms:
             yield si, K, N, M
+
+
+def group_scaled_weights(N: int, K: int, group_k: int, seed: int = 0) -> np.ndarray:
+    """W [N, K] fp32 whose column groups of group_k have different spreads:
+    group g ~ N(0, (0.02 * 2^u_g)^2), u_g ~ U(-1.5, 1.5) (so per-group scales
+    differ by up to 8x).  PCG64(77, seed, N, K, group_k)."""
+    rng = _rng(77, seed, N, K, group_k)
+    u = rng.uniform(-1.5, 1.5, size=(K // group_k,)).astype(np.float32)
+    W = rng.standard_normal((N, K), dtype=np.float32)
+    W *= np.repeat(np.float32(0.02) * np.exp2(u), group_k)[None, :]
+    return W.astype(np.float32)
+
+
+def group_scaled_activations(M: int, K: int, group_k: int, seed: int = 0) -> np.ndarray:
+    """x [M, K] as bf16 bit patterns: N(0,1) with each column group scaled by
+    2^v_g, v_g ~ U(-2, 2), and 0.1% x20 outlier channels.  PCG64(78, seed, M, K, group_k)."""
+    rng = _rng(78, seed, M, K, group_k)
+    v = rng.uniform(-2.0, 2.0, size=(K // group_k,)).astype(np.float32)
+    x = rng.standard_normal((M, K), dtype=np.float32)
+    x *= np.repeat(np.exp2(v), group_k)[None, :]
+    ch = rng.choice(K, size=max(1, int(round(0.001 * K))), replace=False)
+    x[:, ch] *= np.float32(20.0)
+    return _to_bf16_bits(x)
