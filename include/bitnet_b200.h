@@ -427,6 +427,82 @@ BITNET_API bitnet_status bitnet_linear_forward_group_scales(
     int32_t *acc_out, bitnet_stream_t stream);
 
 /* ------------------------------------------------------------------------
+ * Quantization warm-up for fine-tuning ("LLM を 1.58 ビットにファインチューニ
+ * ング：BitNet による極端な量子化", section 動的ウォームアップ量子化: lambda =
+ * min(step / total_steps, 1) scales the difference between the full-precision
+ * and the quantized values; the straight-through estimator of the same page
+ * for the backward).  Reading: the blend applies to both operands the page
+ * quantizes, in rounded fp32 steps, each rounded to bf16 for the tensor cores:
+ *   W_lam = W + lambda * (t / s_w - W)         t, s_w as bitnet_quantize_pack_weights
+ *   x_lam = x_n + lambda * (x_q / s_x - x_n)   x_n, x_q, s_x as bitnet_rmsnorm_quant_act
+ *   y     = x_lam W_lam^T                       bf16 operands, fp32 accumulation
+ * lambda = 0 is the plain bf16 layer on the normalised input; lambda = 1 is
+ * the fake-quantized layer (y = the dequantized ternary forward up to the
+ * bf16 rounding of x_q / s_x and t / s_w and fp32 summation order).
+ * Shapes: N and K multiples of 8, 0 <= lambda <= 1.
+ *
+ * bitnet_warmup_quantize_weights -- W [N][K] fp32 (device, 16-byte aligned)
+ *   -> W_lam [N][K] bf16 and s_w [1] fp32; workspace >= the size query.
+ * bitnet_warmup_forward -- x [M][K] (fp32 or bf16), gamma [K] or NULL,
+ *   W_lam from the call above -> y [M][N] (y_dtype).  x_lam [M][K] bf16 is
+ *   written to x_lam when it is non-NULL (kept for the backward), else to the
+ *   workspace (>= bitnet_warmup_forward_workspace_bytes, 256-byte aligned).
+ * bitnet_warmup_backward -- the straight-through backward of y = x_lam
+ *   W_lam^T given dy [M][N] bf16: dx [M][K] fp32 = dy W_lam (the gradient
+ *   of x_n; the RMSNorm's own backward is not part of this layer) and dW
+ *   [N][K] fp32 = dy^T x_lam (the gradient of W, the quantizer passing it
+ *   through).  Either output may be NULL.  workspace >= the size query
+ *   (transposed bf16 copies).
+ * All calls queue work on `stream` and return at once; device buffers only.
+ * ---------------------------------------------------------------------- */
+BITNET_API size_t bitnet_warmup_quantize_weights_workspace_bytes(int64_t N, int64_t K);
+BITNET_API bitnet_status bitnet_warmup_quantize_weights(const float *W, int64_t N, int64_t K,
+                                                        float lambda, void *W_lam, float *s_w,
+                                                        void *workspace, size_t workspace_bytes,
+                                                        bitnet_stream_t stream);
+BITNET_API size_t bitnet_warmup_forward_workspace_bytes(int64_t M, int64_t N, int64_t K);
+BITNET_API bitnet_status bitnet_warmup_forward(const void *x, int x_dtype, const float *gamma,
+                                               float eps, const void *W_lam, int64_t M,
+                                               int64_t N, int64_t K, float lambda, void *y,
+                                               int y_dtype, void *x_lam, void *workspace,
+                                               size_t workspace_bytes, bitnet_stream_t stream);
+BITNET_API size_t bitnet_warmup_backward_workspace_bytes(int64_t M, int64_t N, int64_t K);
+BITNET_API bitnet_status bitnet_warmup_backward(const void *dy, const void *x_lam,
+                                                const void *W_lam, int64_t M, int64_t N,
+                                                int64_t K, float *dx, float *dW, void *workspace,
+                                                size_t workspace_bytes, bitnet_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * BitDelta ("【論文要約】BitDelta: Your Fine-Tune May Only Be Worth One Bit",
+ * Eq. 1-4: Delta = W_fine - W_base is stored as its sign and one scale per
+ * matrix, alpha = mean |Delta|; Eq. 6 and Fig. 4: a shared base matrix
+ * serves B tenants at once, each token through base + its tenant's delta).
+ * Readings: Sign(0) = -1; bit j (least significant first) of word w of row n
+ * is the sign of Delta[n][32 w + j] (1 = +1); alpha is the fp64 sum of |Delta|
+ * in the fixed order of the weight scale divided by N K, rounded to fp32.
+ *
+ * bitnet_bitdelta_compress -- W_base, W_fine [N][K] bf16 (device, 16-byte
+ *   aligned), K a multiple of 32 -> signs [N][K/32] uint32 and alpha [1]
+ *   fp32; workspace >= the size query (fp64 row sums).
+ * bitnet_bitdelta_forward -- B <= 8 tenants, one token each: x [B][K] bf16,
+ *   W_base [N][K] bf16, signs [B][N][K/32] (tenant after tenant), alpha [B]
+ *   -> y [B][N] (y_dtype) with
+ *     y[b][n] = sum_k x[b][k] W_base[n][k] + alpha[b] sum_k x[b][k] s_b[n][k]
+ *   (bf16 products, fp32 sums on the tensor cores, the delta's sum scaled
+ *   by alpha with one fused multiply-add).  B == 0 queues nothing.
+ * ---------------------------------------------------------------------- */
+BITNET_API size_t bitnet_bitdelta_compress_workspace_bytes(int64_t N, int64_t K);
+BITNET_API bitnet_status bitnet_bitdelta_compress(const void *W_base, const void *W_fine,
+                                                  int64_t N, int64_t K, uint32_t *signs,
+                                                  float *alpha, void *workspace,
+                                                  size_t workspace_bytes,
+                                                  bitnet_stream_t stream);
+BITNET_API bitnet_status bitnet_bitdelta_forward(const void *x, const void *W_base,
+                                                 const uint32_t *signs, const float *alpha,
+                                                 int64_t B, int64_t N, int64_t K, void *y,
+                                                 int y_dtype, bitnet_stream_t stream);
+
+/* ------------------------------------------------------------------------
  * bitnet_linear_forward_ex -- one forward described by a problem record, so
  * that it can read weights in either layout (problem->w_layout); otherwise
  * as bitnet_linear_forward_debug: the same steps, the same bits, optional

@@ -183,7 +183,9 @@ def _load_variants():
     lib.oracle_group_quantize_pack.argtypes = [P, I64, I64, I64, P, P]
     lib.oracle_group_rmsnorm_quant_act.argtypes = [P, ctypes.c_int, P, F, I64, I64, I64, P, P]
     lib.oracle_group_matmul_dequant.argtypes = [P, P, P, P, I64, I64, I64, I64, P, I64, P, P, P]
-    for name in ("oracle_swiglu", "oracle_warmup_forward", "oracle_bitdelta_compress",
+    lib.oracle_warmup_weights.argtypes = [P, I64, I64, F, P, P]
+    for name in ("oracle_swiglu", "oracle_warmup_forward", "oracle_warmup_weights",
+                 "oracle_bitdelta_compress",
                  "oracle_bitdelta_forward", "oracle_group_weight_scale",
                  "oracle_group_quantize_pack", "oracle_group_rmsnorm_quant_act",
                  "oracle_group_matmul_dequant"):
@@ -238,6 +240,28 @@ def warmup_forward(x, gamma, eps, W, lam, cols=None):
         _ptr(x), is_bf16, _ptr(g), float(eps), _ptr(W), M, N, K, float(np.float32(lam)),
         _ptr(c), nc, _ptr(xl), _ptr(y), _ptr(yb), _ptr(ad)), "warmup_forward")
     return {"y": y, "y_b": yb, "absdot": ad, "x_lam": xl}
+
+
+def warmup_weights(W, lam):
+    """(W_lam fp32 [N,K], s_w): the weight operand of the warm-up forward."""
+    W = np.ascontiguousarray(W, dtype=np.float32)
+    N, K = W.shape
+    out = np.empty((N, K), np.float32)
+    s = np.empty((1,), np.float32)
+    _check(_load_variants().oracle_warmup_weights(_ptr(W), N, K, float(np.float32(lam)),
+                                                  _ptr(out), _ptr(s)), "warmup_weights")
+    return out, np.float32(s[0])
+
+
+def warmup_backward(dy_bits, x_lam_bits, W_lam_bits):
+    """Straight-through backward of y = x_lam W_lam^T (the warm-up page's
+    estimator: the quantizers pass the gradient through unchanged), on bf16
+    operands given as bit patterns: dx = dy W_lam, dW = dy^T x_lam, each a
+    plain matrix product of the exactly widened values summed in fp64."""
+    dy = bf16_bits_to_f32(dy_bits).astype(np.float64)
+    xl = bf16_bits_to_f32(x_lam_bits).astype(np.float64)
+    wl = bf16_bits_to_f32(W_lam_bits).astype(np.float64)
+    return dy @ wl, dy.T @ xl
 
 
 def bitdelta_compress(W_base_bits, W_fine_bits):
@@ -323,6 +347,7 @@ def group_linear_forward(x, gamma, eps, W_p, s_w, K, group_k, cols=None):
     return {"x_q": x_q, "s_x": s_x, "acc": acc, "y": y, "y_bf16": yb}
 
 
-__all__ += ["swiglu", "swiglu_forward", "warmup_lambda", "warmup_forward",
+__all__ += ["swiglu", "swiglu_forward", "warmup_lambda", "warmup_forward", "warmup_weights",
+            "warmup_backward",
             "bitdelta_compress", "bitdelta_forward", "group_weight_scale",
             "group_quantize_pack", "group_rmsnorm_quant_act", "group_linear_forward"]

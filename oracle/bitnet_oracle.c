@@ -492,6 +492,30 @@ int oracle_warmup_forward(const void *x, int x_is_bf16, const float *gamma,
     return e;
 }
 
+/*
+ * The weight operand of the warm-up forward on its own: W_lam [N][K] fp32 as
+ * oracle_warmup_forward forms it per column (t and s_w of the per-tensor
+ * weight quantization; t / s_w correctly rounded, then the three rounded
+ * fp32 steps of the blend).  s_w_out may be NULL.
+ */
+int oracle_warmup_weights(const float *W, int64_t N, int64_t K, float lambda,
+                          float *W_lam, float *s_w_out) {
+    if (!W || !W_lam || N <= 0 || K <= 0 || !(lambda >= 0.0f) || lambda > 1.0f)
+        return ORACLE_ERR_ARG;
+    float s_w;
+    int e = oracle_weight_scale(W, N, K, &s_w, NULL);
+    if (e) return e;
+    for (int64_t i = 0; i < N * K; ++i) {
+        float w = W[i];
+        float wt = (float)ternary_of(w, s_w) / s_w;
+        float d = wt - w;
+        float l = lambda * d;
+        W_lam[i] = w + l;
+    }
+    if (s_w_out) *s_w_out = s_w;
+    return ORACLE_OK;
+}
+
 /* -------------------------------------------- BitDelta: 1-bit deltas */
 
 /*

@@ -56,6 +56,11 @@ EXPORTED = (
     "bitnet_quantize_pack_weights_group_scales_workspace_bytes",
     "bitnet_quantize_pack_weights_group_scales",
     "bitnet_linear_forward_group_scales_workspace_bytes", "bitnet_linear_forward_group_scales",
+    "bitnet_warmup_quantize_weights_workspace_bytes", "bitnet_warmup_quantize_weights",
+    "bitnet_warmup_forward_workspace_bytes", "bitnet_warmup_forward",
+    "bitnet_warmup_backward_workspace_bytes", "bitnet_warmup_backward",
+    "bitnet_bitdelta_compress_workspace_bytes", "bitnet_bitdelta_compress",
+    "bitnet_bitdelta_forward",
 )
 
 BITNET_LAYOUT_ROWS = 0
@@ -134,6 +139,15 @@ def load_library(path: str = LIB_PATH):
             "bitnet_linear_forward_group_scales_workspace_bytes": ([I64, I64, I64, I64], SZ),
             "bitnet_linear_forward_group_scales": (
                 [P, I, P, F, P, I, P, I64, I64, I64, I64, P, I, P, SZ, P, P, P, P], I),
+            "bitnet_warmup_quantize_weights_workspace_bytes": ([I64, I64], SZ),
+            "bitnet_warmup_quantize_weights": ([P, I64, I64, F, P, P, P, SZ, P], I),
+            "bitnet_warmup_forward_workspace_bytes": ([I64, I64, I64], SZ),
+            "bitnet_warmup_forward": ([P, I, P, F, P, I64, I64, I64, F, P, I, P, P, SZ, P], I),
+            "bitnet_warmup_backward_workspace_bytes": ([I64, I64, I64], SZ),
+            "bitnet_warmup_backward": ([P, P, P, I64, I64, I64, P, P, P, SZ, P], I),
+            "bitnet_bitdelta_compress_workspace_bytes": ([I64, I64], SZ),
+            "bitnet_bitdelta_compress": ([P, P, I64, I64, P, P, P, SZ, P], I),
+            "bitnet_bitdelta_forward": ([P, P, P, P, I64, I64, I64, P, I, P], I),
         }
         for name, (argtypes, restype) in sig.items():
             fn = getattr(lib, name)
@@ -562,6 +576,144 @@ def bitnet_linear_forward_group_scales(x, gamma, eps, W, s_w, group_k, y_dtype=t
         _ptr(s_w), M, N, K, group_k, _ptr(y), _dtype_code(y.dtype), _ptr(workspace),
         workspace.numel(), _ptr(x_q), _ptr(s_x), _ptr(acc), _stream(stream)))
     return {"y": y, "x_q": x_q, "s_x": s_x, "acc": acc}
+
+
+def _check_lambda(lam):
+    lam = float(lam)
+    if not (0.0 <= lam <= 1.0):
+        raise ValueError("lambda must be in [0, 1]")
+    return lam
+
+
+def bitnet_warmup_quantize_weights(W, lam, W_lam=None, s_w=None, workspace=None, stream=None):
+    """W fp32 [N,K] -> (W_lam bf16 [N,K], s_w fp32 [1]): the warm-up blend
+    W + lam (t / s_w - W) of the weights, rounded to bf16."""
+    N, K = _expect_weights(W)
+    lam = _check_lambda(lam)
+    if W_lam is not None:
+        _expect(W_lam, "W_lam", torch.bfloat16, shape=(N, K))
+    if s_w is not None:
+        _expect(s_w, "s_w", torch.float32, numel=1)
+    lib = load_library()
+    nb = int(lib.bitnet_warmup_quantize_weights_workspace_bytes(N, K))
+    if workspace is not None:
+        _expect(workspace, "workspace", torch.uint8, numel=nb)
+    _need_cuda(W, W_lam, s_w, workspace)
+    if W_lam is None:
+        W_lam = torch.empty((N, K), dtype=torch.bfloat16, device=W.device)
+    if s_w is None:
+        s_w = torch.empty((1,), dtype=torch.float32, device=W.device)
+    if workspace is None:
+        workspace = torch.empty(max(nb, 256), dtype=torch.uint8, device=W.device)
+    _check("bitnet_warmup_quantize_weights", lib.bitnet_warmup_quantize_weights(
+        _ptr(W), N, K, ctypes.c_float(lam), _ptr(W_lam), _ptr(s_w), _ptr(workspace),
+        workspace.numel(), _stream(stream)))
+    return W_lam, s_w
+
+
+def bitnet_warmup_forward(x, gamma, eps, W_lam, lam, y_dtype=torch.float32, y=None,
+                          keep_x_lam=False, stream=None):
+    """y = x_lam W_lam^T with x_lam = x_n + lam (x_q / s_x - x_n) (bf16 tensor
+    cores, fp32 sums).  Returns y, or (y, x_lam bf16 [M,K]) with keep_x_lam."""
+    M, K = _expect_x(x)
+    _expect_gamma(gamma, K)
+    lam = _check_lambda(lam)
+    _expect(W_lam, "W_lam", torch.bfloat16)
+    if W_lam.dim() != 2 or W_lam.shape[1] != K:
+        raise ValueError(f"W_lam must be [N, {K}]")
+    N = W_lam.shape[0]
+    if y is not None:
+        _expect_y(y, M, N)
+    lib = load_library()
+    _need_cuda(x, gamma, W_lam, y)
+    dev = x.device
+    if y is None:
+        y = torch.empty((M, N), dtype=y_dtype, device=dev)
+    x_lam = torch.empty((M, K), dtype=torch.bfloat16, device=dev) if keep_x_lam else None
+    ws = None
+    if x_lam is None:
+        nb = int(lib.bitnet_warmup_forward_workspace_bytes(M, N, K))
+        ws = torch.empty(max(nb, 256), dtype=torch.uint8, device=dev)
+    _check("bitnet_warmup_forward", lib.bitnet_warmup_forward(
+        _ptr(x), _dtype_code(x.dtype), _ptr(gamma), float(eps), _ptr(W_lam), M, N, K,
+        ctypes.c_float(lam), _ptr(y), _dtype_code(y.dtype), _ptr(x_lam), _ptr(ws),
+        0 if ws is None else ws.numel(), _stream(stream)))
+    return (y, x_lam) if keep_x_lam else y
+
+
+def bitnet_warmup_backward(dy, x_lam, W_lam, need_dx=True, need_dW=True, stream=None):
+    """Straight-through backward of y = x_lam W_lam^T: (dx fp32 [M,K] = dy
+    W_lam, dW fp32 [N,K] = dy^T x_lam); either may be skipped (None)."""
+    _expect(dy, "dy", torch.bfloat16)
+    _expect(x_lam, "x_lam", torch.bfloat16)
+    _expect(W_lam, "W_lam", torch.bfloat16)
+    M, N = dy.shape
+    K = x_lam.shape[1]
+    if x_lam.shape != (M, K) or W_lam.shape != (N, K):
+        raise ValueError("shapes: dy [M,N], x_lam [M,K], W_lam [N,K]")
+    lib = load_library()
+    _need_cuda(dy, x_lam, W_lam)
+    dev = dy.device
+    dx = torch.empty((M, K), dtype=torch.float32, device=dev) if need_dx else None
+    dW = torch.empty((N, K), dtype=torch.float32, device=dev) if need_dW else None
+    nb = int(lib.bitnet_warmup_backward_workspace_bytes(M, N, K))
+    ws = torch.empty(max(nb, 256), dtype=torch.uint8, device=dev)
+    _check("bitnet_warmup_backward", lib.bitnet_warmup_backward(
+        _ptr(dy), _ptr(x_lam), _ptr(W_lam), M, N, K, _ptr(dx), _ptr(dW), _ptr(ws), ws.numel(),
+        _stream(stream)))
+    return dx, dW
+
+
+def bitnet_bitdelta_compress(W_base, W_fine, signs=None, alpha=None, stream=None):
+    """W_base, W_fine bf16 [N,K] -> (signs int32 [N, K/32] (the bit patterns of
+    the uint32 words), alpha fp32 [1])."""
+    _expect(W_base, "W_base", torch.bfloat16)
+    _expect(W_fine, "W_fine", torch.bfloat16)
+    if W_base.dim() != 2 or W_fine.shape != W_base.shape:
+        raise ValueError("W_base and W_fine must both be [N, K]")
+    N, K = W_base.shape
+    if K % 32:
+        raise ValueError("K must be a multiple of 32")
+    if signs is not None:
+        _expect(signs, "signs", torch.int32, numel=N * (K // 32))
+    if alpha is not None:
+        _expect(alpha, "alpha", torch.float32, numel=1)
+    lib = load_library()
+    _need_cuda(W_base, W_fine, signs, alpha)
+    dev = W_base.device
+    if signs is None:
+        signs = torch.empty((N, K // 32), dtype=torch.int32, device=dev)
+    if alpha is None:
+        alpha = torch.empty((1,), dtype=torch.float32, device=dev)
+    nb = int(lib.bitnet_bitdelta_compress_workspace_bytes(N, K))
+    ws = torch.empty(max(nb, 256), dtype=torch.uint8, device=dev)
+    _check("bitnet_bitdelta_compress", lib.bitnet_bitdelta_compress(
+        _ptr(W_base), _ptr(W_fine), N, K, _ptr(signs), _ptr(alpha), _ptr(ws), ws.numel(),
+        _stream(stream)))
+    return signs, alpha
+
+
+def bitnet_bitdelta_forward(x, W_base, signs, alpha, y_dtype=torch.float32, y=None, stream=None):
+    """B <= 8 tenants, one token each: x bf16 [B,K], W_base bf16 [N,K], signs
+    int32 [B, N, K/32], alpha fp32 [B] -> y [B,N] = x W_base^T + alpha_b x Sign_b^T."""
+    _expect(x, "x", torch.bfloat16)
+    _expect(W_base, "W_base", torch.bfloat16)
+    _expect(signs, "signs", torch.int32)
+    _expect(alpha, "alpha", torch.float32)
+    B, K = x.shape
+    N = W_base.shape[0]
+    if W_base.shape != (N, K) or signs.numel() != B * N * (K // 32) or alpha.numel() != B:
+        raise ValueError("shapes: x [B,K], W_base [N,K], signs [B,N,K/32], alpha [B]")
+    if y is not None:
+        _expect_y(y, B, N)
+    lib = load_library()
+    _need_cuda(x, W_base, signs, alpha, y)
+    if y is None:
+        y = torch.empty((B, N), dtype=y_dtype, device=x.device)
+    _check("bitnet_bitdelta_forward", lib.bitnet_bitdelta_forward(
+        _ptr(x), _ptr(W_base), _ptr(signs), _ptr(alpha), B, N, K, _ptr(y),
+        _dtype_code(y.dtype), _stream(stream)))
+    return y
 
 
 def _weights_ptr_layout(W, K):

@@ -16,6 +16,7 @@
 #include <vector>
 
 #include "act_quant.cuh"
+#include "bitdelta.cuh"
 #include "common.cuh"
 #include "gemm_tc.cuh"
 #include "gemv.cuh"
@@ -23,6 +24,7 @@
 #include "group_quant.cuh"
 #include "peak.cuh"
 #include "tiled.cuh"
+#include "warmup.cuh"
 #include "weight_quant.cuh"
 
 namespace bitnet {
@@ -1677,6 +1679,267 @@ BITNET_API bitnet_status bitnet_device_status(bitnet_stream_t stream, int reset,
     if (cudaStreamSynchronize(s) != cudaSuccess) return BITNET_ERR_CUDA;
   }
   return v == 0 ? BITNET_OK : BITNET_ERR_TIMEOUT;
+}
+
+// ------------------------------------------------ lambda-warmup fake quant
+
+}  // extern "C"
+
+namespace {
+
+// 2-D bf16 tensor [rows][inner] (row stride in bytes), boxes of 64 x
+// box_rows elements, 128-byte swizzle (the tcgen05 K-major canonical layout);
+// out-of-range elements read as zero.
+bool make_tmap_bf16(CUtensorMap* map, const void* base, uint64_t inner, uint64_t rows,
+                    uint64_t row_stride, uint32_t box_rows) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {inner, rows};
+  cuuint64_t strides[1] = {row_stride};
+  cuuint32_t box[2] = {64, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
+             box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+         CUDA_SUCCESS;
+}
+
+template <int BN>
+bitnet_status launch_wg_bn(const CUtensorMap& ta, const CUtensorMap& tb, const WgParams& p,
+                           cudaStream_t s) {
+  static std::once_flag once;
+  static bool ok = false;
+  std::call_once(once, []() {
+    ok = cudaFuncSetAttribute(bf16_gemm_nt_kernel<BN>,
+                              cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              WgCfg<BN>::SMEM_DYN) == cudaSuccess;
+  });
+  if (!ok) return BITNET_ERR_CUDA;
+  const dim3 grid(static_cast<unsigned>((p.N + 127) / 128),
+                  static_cast<unsigned>((p.M + BN - 1) / BN));
+  bf16_gemm_nt_kernel<BN><<<grid, WgCfg<BN>::THREADS, WgCfg<BN>::SMEM_DYN, s>>>(ta, tb, p);
+  return launch_status();
+}
+
+// y[m][n] (row stride ldy) = sum_k B[m][k] A[n][k]; A [N][K], B [M][K] bf16
+// with row strides lda, ldb elements (multiples of 8).
+bitnet_status launch_bf16_gemm_nt(const DeviceState& ds, const void* A, int64_t lda,
+                                  const void* B, int64_t ldb, int64_t M, int64_t N, int64_t K,
+                                  void* y, int64_t ldy, int y_dtype, cudaStream_t s) {
+  if (M == 0 || N == 0) return BITNET_OK;
+  const int BN = M <= 64 ? 64 : (M <= 128 ? 128 : 256);
+  CUtensorMap ta, tb;
+  if (!make_tmap_bf16(&ta, A, static_cast<uint64_t>(K), static_cast<uint64_t>(N),
+                      static_cast<uint64_t>(2 * lda), 128) ||
+      !make_tmap_bf16(&tb, B, static_cast<uint64_t>(K), static_cast<uint64_t>(M),
+                      static_cast<uint64_t>(2 * ldb), static_cast<uint32_t>(BN)))
+    return BITNET_ERR_CUDA;
+  WgParams p{};
+  p.M = static_cast<int>(M);
+  p.N = static_cast<int>(N);
+  p.K = static_cast<int>(K);
+  p.y = y;
+  p.ldy = ldy;
+  p.y_bf16 = y_dtype == BITNET_BF16 ? 1 : 0;
+  p.status = ds.status;
+  p.wait_limit_ns = kWaitLimitNs;
+  p.use_pdl = 0;
+  if (BN == 64) return launch_wg_bn<64>(ta, tb, p, s);
+  if (BN == 128) return launch_wg_bn<128>(ta, tb, p, s);
+  return launch_wg_bn<256>(ta, tb, p, s);
+}
+
+bitnet_status check_warmup_shape(int64_t M, int64_t N, int64_t K, float lambda) {
+  if (M < 0 || N < 0 || K < 0 || !(lambda >= 0.0f) || lambda > 1.0f)
+    return BITNET_ERR_INVALID_ARG;
+  if (N < 1 || K < 8 || K % 8 != 0 || N % 8 != 0 || N > BITNET_MAX_N || K > BITNET_MAX_K ||
+      M > BITNET_MAX_M)
+    return BITNET_ERR_UNSUPPORTED_SHAPE;
+  return BITNET_OK;
+}
+
+int64_t round8(int64_t v) { return (v + 7) / 8 * 8; }
+
+}  // namespace
+
+extern "C" {
+
+BITNET_API size_t bitnet_warmup_quantize_weights_workspace_bytes(int64_t N, int64_t K) {
+  return bitnet_quantize_pack_weights_workspace_bytes(N, K);
+}
+
+BITNET_API bitnet_status bitnet_warmup_quantize_weights(const float* W, int64_t N, int64_t K,
+                                                        float lambda, void* W_lam, float* s_w,
+                                                        void* workspace, size_t workspace_bytes,
+                                                        bitnet_stream_t stream) {
+  bitnet_status st = check_warmup_shape(0, N, K, lambda);
+  if (st != BITNET_OK) return st;
+  if (!W || !W_lam || !s_w) return BITNET_ERR_INVALID_ARG;
+  if (!aligned(W, 16) || !aligned(W_lam, 16) || !aligned(s_w, 4)) return BITNET_ERR_MISALIGNED;
+  if (!workspace || workspace_bytes < bitnet_warmup_quantize_weights_workspace_bytes(N, K))
+    return BITNET_ERR_WORKSPACE;
+  if (!aligned(workspace, 256)) return BITNET_ERR_MISALIGNED;
+  DeviceState* ds = device_state();
+  if (!ds) return BITNET_ERR_CUDA;
+  cudaStream_t s = as_stream(stream);
+  double* R = static_cast<double*>(workspace);
+  row_abs_sum_kernel<<<static_cast<unsigned>(N), kWqThreads, 0, s>>>(W, K, R);
+  abs_total_kernel<<<1, kWqThreads, 0, s>>>(R, N, K, s_w);
+  const int64_t n4 = N * K / 4;
+  const int64_t blocks = std::min<int64_t>((n4 + 255) / 256, 16LL * ds->num_sms);
+  warmup_weights_kernel<<<static_cast<unsigned>(blocks), 256, 0, s>>>(
+      W, n4, s_w, lambda, static_cast<__nv_bfloat16*>(W_lam));
+  return launch_status();
+}
+
+BITNET_API size_t bitnet_warmup_forward_workspace_bytes(int64_t M, int64_t N, int64_t K) {
+  (void)N;
+  if (M < 0 || K < 0) return 0;
+  return align256(2 * static_cast<size_t>(M * K));
+}
+
+BITNET_API bitnet_status bitnet_warmup_forward(const void* x, int x_dtype, const float* gamma,
+                                               float eps, const void* W_lam, int64_t M,
+                                               int64_t N, int64_t K, float lambda, void* y,
+                                               int y_dtype, void* x_lam, void* workspace,
+                                               size_t workspace_bytes, bitnet_stream_t stream) {
+  bitnet_status st = check_warmup_shape(M, N, K, lambda);
+  if (st != BITNET_OK) return st;
+  if (M == 0) return BITNET_OK;
+  if (!x || !W_lam || !y || !ok_dtype(x_dtype) || !ok_dtype(y_dtype) || !(eps >= 0.0f) ||
+      eps > 3.0e38f)
+    return BITNET_ERR_INVALID_ARG;
+  if (!aligned(x, 16) || (gamma && !aligned(gamma, 16)) || !aligned(W_lam, 16) ||
+      !aligned(y, 4) || (x_lam && !aligned(x_lam, 16)))
+    return BITNET_ERR_MISALIGNED;
+  if (!x_lam && (!workspace || workspace_bytes < bitnet_warmup_forward_workspace_bytes(M, N, K)))
+    return BITNET_ERR_WORKSPACE;
+  if (!x_lam && !aligned(workspace, 256)) return BITNET_ERR_MISALIGNED;
+  DeviceState* ds = device_state();
+  if (!ds) return BITNET_ERR_CUDA;
+  cudaStream_t s = as_stream(stream);
+  __nv_bfloat16* xl = static_cast<__nv_bfloat16*>(x_lam ? x_lam : workspace);
+  if (x_dtype == BITNET_BF16)
+    warmup_act_kernel<true><<<static_cast<unsigned>(M), kActThreads, 0, s>>>(x, gamma, eps, K,
+                                                                             lambda, xl);
+  else
+    warmup_act_kernel<false><<<static_cast<unsigned>(M), kActThreads, 0, s>>>(x, gamma, eps, K,
+                                                                              lambda, xl);
+  st = launch_status();
+  if (st != BITNET_OK) return st;
+  return launch_bf16_gemm_nt(*ds, W_lam, K, xl, K, M, N, K, y, N, y_dtype, s);
+}
+
+BITNET_API size_t bitnet_warmup_backward_workspace_bytes(int64_t M, int64_t N, int64_t K) {
+  if (M < 0 || N < 0 || K < 0) return 0;
+  const int64_t Mp = round8(M);
+  return align256(2 * static_cast<size_t>(K * N)) + align256(2 * static_cast<size_t>(N * Mp)) +
+         align256(2 * static_cast<size_t>(K * Mp));
+}
+
+BITNET_API bitnet_status bitnet_warmup_backward(const void* dy, const void* x_lam,
+                                                const void* W_lam, int64_t M, int64_t N,
+                                                int64_t K, float* dx, float* dW, void* workspace,
+                                                size_t workspace_bytes, bitnet_stream_t stream) {
+  bitnet_status st = check_warmup_shape(M, N, K, 0.0f);
+  if (st != BITNET_OK) return st;
+  if (!dy || (dx && !W_lam) || (dW && !x_lam)) return BITNET_ERR_INVALID_ARG;
+  if (!aligned(dy, 16) || (x_lam && !aligned(x_lam, 16)) || (W_lam && !aligned(W_lam, 16)) ||
+      (dx && !aligned(dx, 4)) || (dW && !aligned(dW, 4)))
+    return BITNET_ERR_MISALIGNED;
+  if (!workspace || workspace_bytes < bitnet_warmup_backward_workspace_bytes(M, N, K))
+    return BITNET_ERR_WORKSPACE;
+  if (!aligned(workspace, 256)) return BITNET_ERR_MISALIGNED;
+  DeviceState* ds = device_state();
+  if (!ds) return BITNET_ERR_CUDA;
+  cudaStream_t s = as_stream(stream);
+  if (dW && M == 0) {
+    if (cudaMemsetAsync(dW, 0, 4 * static_cast<size_t>(N * K), s) != cudaSuccess)
+      return BITNET_ERR_CUDA;
+  }
+  if (M == 0) return BITNET_OK;
+  const int64_t Mp = round8(M);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  __nv_bfloat16* WT = reinterpret_cast<__nv_bfloat16*>(ws);                    // [K][N]
+  uint8_t* p1 = ws + align256(2 * static_cast<size_t>(K * N));
+  __nv_bfloat16* dyT = reinterpret_cast<__nv_bfloat16*>(p1);                   // [N][Mp]
+  __nv_bfloat16* xT = reinterpret_cast<__nv_bfloat16*>(p1 + align256(2 * static_cast<size_t>(N * Mp)));  // [K][Mp]
+  const __nv_bfloat16* dyb = static_cast<const __nv_bfloat16*>(dy);
+  auto transpose = [&](const __nv_bfloat16* src, int64_t R, int64_t C, __nv_bfloat16* dst,
+                       int64_t ldd) {
+    const dim3 grid(static_cast<unsigned>((C + 31) / 32), static_cast<unsigned>((ldd + 31) / 32));
+    transpose_bf16_kernel<<<grid, 256, 0, s>>>(src, R, C, dst, ldd);
+    return launch_status();
+  };
+  if (dx) {
+    // dx [M][K] = dy [M][N] . W_lam [N][K]: B = dy (K-major over n), A = W_lam^T.
+    st = transpose(static_cast<const __nv_bfloat16*>(W_lam), N, K, WT, N);
+    if (st != BITNET_OK) return st;
+    st = launch_bf16_gemm_nt(*ds, WT, N, dyb, N, M, K, N, dx, K, BITNET_F32, s);
+    if (st != BITNET_OK) return st;
+  }
+  if (dW) {
+    // dW [N][K] = dy^T [N][M] . x_lam [M][K]: B = dy^T, A = x_lam^T (zero-padded to Mp).
+    st = transpose(dyb, M, N, dyT, Mp);
+    if (st != BITNET_OK) return st;
+    st = transpose(static_cast<const __nv_bfloat16*>(x_lam), M, K, xT, Mp);
+    if (st != BITNET_OK) return st;
+    st = launch_bf16_gemm_nt(*ds, xT, Mp, dyT, Mp, N, K, Mp, dW, K, BITNET_F32, s);
+    if (st != BITNET_OK) return st;
+  }
+  return BITNET_OK;
+}
+
+// ------------------------------------------------------ BitDelta 1-bit deltas
+
+BITNET_API size_t bitnet_bitdelta_compress_workspace_bytes(int64_t N, int64_t K) {
+  (void)K;
+  return N > 0 ? align256(8 * static_cast<size_t>(N)) : 0;
+}
+
+BITNET_API bitnet_status bitnet_bitdelta_compress(const void* W_base, const void* W_fine,
+                                                  int64_t N, int64_t K, uint32_t* signs,
+                                                  float* alpha, void* workspace,
+                                                  size_t workspace_bytes,
+                                                  bitnet_stream_t stream) {
+  if (N < 0 || K < 0) return BITNET_ERR_INVALID_ARG;
+  if (N < 1 || K < 32 || K % 32 != 0 || N > BITNET_MAX_N || K > BITNET_MAX_K)
+    return BITNET_ERR_UNSUPPORTED_SHAPE;
+  if (!W_base || !W_fine || !signs || !alpha) return BITNET_ERR_INVALID_ARG;
+  if (!aligned(W_base, 16) || !aligned(W_fine, 16) || !aligned(signs, 4) || !aligned(alpha, 4))
+    return BITNET_ERR_MISALIGNED;
+  if (!workspace || workspace_bytes < bitnet_bitdelta_compress_workspace_bytes(N, K))
+    return BITNET_ERR_WORKSPACE;
+  if (!aligned(workspace, 256)) return BITNET_ERR_MISALIGNED;
+  if (!device_state()) return BITNET_ERR_CUDA;
+  cudaStream_t s = as_stream(stream);
+  double* R = static_cast<double*>(workspace);
+  bitdelta_row_kernel<<<static_cast<unsigned>(N), kWqThreads, 0, s>>>(
+      static_cast<const __nv_bfloat16*>(W_base), static_cast<const __nv_bfloat16*>(W_fine), K,
+      signs, R);
+  bitdelta_alpha_kernel<<<1, kWqThreads, 0, s>>>(R, N, K, alpha);
+  return launch_status();
+}
+
+BITNET_API bitnet_status bitnet_bitdelta_forward(const void* x, const void* W_base,
+                                                 const uint32_t* signs, const float* alpha,
+                                                 int64_t B, int64_t N, int64_t K, void* y,
+                                                 int y_dtype, bitnet_stream_t stream) {
+  if (B < 0 || N < 0 || K < 0) return BITNET_ERR_INVALID_ARG;
+  if (B > kBdMaxTenants || N < 1 || K < 32 || K % 32 != 0 || N > BITNET_MAX_N ||
+      K > BITNET_MAX_K || (N + 15) / 16 > 0x7FFFFFFFLL)
+    return BITNET_ERR_UNSUPPORTED_SHAPE;
+  if (B == 0) return BITNET_OK;
+  if (!x || !W_base || !signs || !alpha || !y || !ok_dtype(y_dtype)) return BITNET_ERR_INVALID_ARG;
+  if (!aligned(x, 16) || !aligned(W_base, 16) || !aligned(signs, 4) || !aligned(alpha, 4) ||
+      !aligned(y, 4))
+    return BITNET_ERR_MISALIGNED;
+  if (!device_state()) return BITNET_ERR_CUDA;
+  bitdelta_forward_kernel<<<static_cast<unsigned>((N + 15) / 16), 32 * kBdWarps, 0,
+                            as_stream(stream)>>>(
+      static_cast<const __nv_bfloat16*>(x), static_cast<const __nv_bfloat16*>(W_base), signs,
+      alpha, static_cast<int>(B), N, K, y, y_dtype == BITNET_BF16 ? 1 : 0);
+  return launch_status();
 }
 
 }  // extern "C"

@@ -167,3 +167,36 @@ def group_scaled_activations(M: int, K: int, group_k: int, seed: int = 0) -> np.
     ch = rng.choice(K, size=max(1, int(round(0.001 * K))), replace=False)
     x[:, ch] *= np.float32(20.0)
     return _to_bf16_bits(x)
+
+
+def bitdelta_inputs(N: int, K: int, B: int, seed: int = 0):
+    """BitDelta serving inputs, all bf16 bit patterns: W_base [N,K] ~ N(0, 0.02^2);
+    B fine-tuned copies W_fine[b] = W_base + d, d ~ N(0, 0.002^2) (a fine-tune
+    that moves each weight by about a tenth of its spread) with 5% of the
+    entries left exactly equal to the base (zero deltas); one decode token
+    per tenant x [B,K] ~ N(0,1).  PCG64(79, seed, N, K, B)."""
+    rng = _rng(79, seed, N, K, B)
+    base32 = (rng.standard_normal((N, K), dtype=np.float32) * np.float32(0.02)).astype(np.float32)
+    base = _to_bf16_bits(base32)
+    base_f = (base.astype(np.uint32) << 16).view(np.float32)
+    fine = []
+    for _ in range(B):
+        d = (rng.standard_normal((N, K), dtype=np.float32) * np.float32(0.002)).astype(np.float32)
+        d[rng.random((N, K)) < 0.05] = 0.0
+        f = _to_bf16_bits(base_f + d)
+        fine.append(f)
+    x = _to_bf16_bits(rng.standard_normal((B, K), dtype=np.float32))
+    return base, fine, x
+
+
+def warmup_inputs(M: int, N: int, K: int, seed: int = 0, f32: bool = False):
+    """Fine-tuning inputs: W [N,K] fp32 ~ N(0, 0.02^2), x [M,K] ~ N(0,1) with
+    0.1% x20 outlier channels (bf16 bits unless f32), upstream gradient
+    dy [M,N] ~ N(0, 1) as bf16 bits.  PCG64(80, seed, M, N, K)."""
+    rng = _rng(80, seed, M, N, K)
+    W = (rng.standard_normal((N, K), dtype=np.float32) * np.float32(0.02)).astype(np.float32)
+    x = rng.standard_normal((M, K), dtype=np.float32)
+    ch = rng.choice(K, size=max(1, int(round(0.001 * K))), replace=False)
+    x[:, ch] *= np.float32(20.0)
+    dy = _to_bf16_bits(rng.standard_normal((M, N), dtype=np.float32))
+    return W, (x if f32 else _to_bf16_bits(x)), dy

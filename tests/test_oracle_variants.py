@@ -283,3 +283,71 @@ def test_group_forward_matches_the_fake_quant_identity():
                (T[:, sl] / float(s[g])).T
     rel = np.abs(r["y"] - ref) / np.maximum(np.abs(ref), 1e-30)
     assert rel.max() <= 1e-6
+
+
+# ----------------------------------------------- warm-up weights and backward
+
+def test_warmup_weights_endpoints_and_agreement_with_the_forward():
+    rng = np.random.default_rng(21)
+    W = (rng.standard_normal((24, 256)) * 0.02).astype(np.float32)
+    w0, s0 = oracle.warmup_weights(W, 0.0)
+    assert np.array_equal(w0.view(np.uint32), W.view(np.uint32))          # lambda = 0: W itself
+    s_w, _ = oracle.weight_scale(W)
+    assert np.float32(s0) == np.float32(s_w)
+    # lambda = 1: every entry is a ternary level -1/s_w, 0 or 1/s_w, up to the
+    # rounding of w + (t/s_w - w) (one fp32 subtraction, one addition)
+    w1, _ = oracle.warmup_weights(W, 1.0)
+    lev = np.float32(1.0) / np.float32(s_w)
+    nearest = np.array([-lev, 0.0, lev], np.float32)
+    dist = np.abs(w1[..., None] - nearest).min(-1)
+    assert np.all(dist <= 4 * np.spacing(np.maximum(np.abs(W), lev)))
+    # intermediate lambda: between W and its level, entry by entry
+    wh, _ = oracle.warmup_weights(W, 0.5)
+    lo = np.minimum(W, w1) - 4 * np.spacing(lev)
+    hi = np.maximum(W, w1) + 4 * np.spacing(lev)
+    assert np.all((wh >= lo) & (wh <= hi))
+    # the forward's own W_lam: y(lambda) recomputed from the exported operands
+    x = workloads._to_bf16_bits(rng.standard_normal((3, 256)).astype(np.float32))
+    r = oracle.warmup_forward(x, None, 1e-5, W, 0.5)
+    ref = r["x_lam"].astype(np.float64) @ wh.astype(np.float64).T
+    assert np.allclose(r["y"], ref, rtol=0, atol=1e-12 * np.abs(ref).max())
+
+
+def _brute_bilinear(dy, xl, wl):
+    """sum_{m,n} dy[m,n] sum_k xl[m,k] wl[n,k] by explicit loops (Fractions)."""
+    M, N = dy.shape
+    K = xl.shape[1]
+    tot = Fraction(0)
+    for m in range(M):
+        for n in range(N):
+            s = Fraction(0)
+            for k in range(K):
+                s += Fraction(float(xl[m, k])) * Fraction(float(wl[n, k]))
+            tot += Fraction(float(dy[m, n])) * s
+    return tot
+
+
+def test_warmup_backward_is_the_derivative_of_the_bilinear_forward():
+    # Small integers as bf16: every product and sum is exact.  The gradient
+    # of f(X, W) = <dy, X W^T> in a direction E must equal the central
+    # difference (exact for a bilinear f), and Euler's identity
+    # <dy, y> = <dx, X> = <dW, W> must hold.
+    rng = np.random.default_rng(22)
+    M, N, K = 3, 4, 5
+    to_bits = lambda a: workloads._to_bf16_bits(a.astype(np.float32))
+    dy = to_bits(rng.integers(-3, 4, (M, N)))
+    xl = to_bits(rng.integers(-4, 5, (M, K)))
+    wl = to_bits(rng.integers(-2, 3, (N, K)))
+    dx, dW = oracle.warmup_backward(dy, xl, wl)
+    f = lambda X, Wm: _brute_bilinear(oracle.bf16_bits_to_f32(dy), X, Wm)
+    X = oracle.bf16_bits_to_f32(xl)
+    Wm = oracle.bf16_bits_to_f32(wl)
+    E = rng.integers(-2, 3, (N, K)).astype(np.float32)
+    Ex = rng.integers(-2, 3, (M, K)).astype(np.float32)
+    dW_dir = (f(X, Wm + E) - f(X, Wm - E)) / 2
+    dx_dir = (f(X + Ex, Wm) - f(X - Ex, Wm)) / 2
+    assert Fraction(float((dW * E).sum())) == dW_dir
+    assert Fraction(float((dx * Ex).sum())) == dx_dir
+    y_dot = f(X, Wm)
+    assert Fraction(float((dx * X).sum())) == y_dot
+    assert Fraction(float((dW * Wm).sum())) == y_dot
