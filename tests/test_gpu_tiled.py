@@ -338,3 +338,20 @@ def test_concatenated_qkv_weights_in_one_buffer():
     torch.cuda.synchronize()
     for it, ref in zip(items, refs):
         _check_y(it[5], ref["y"], ref["y_bf16"])
+
+
+# The tcgen05 kernel on tiled weights for 16 < M <= 64 (split-K token tiles
+# of 32 and 64): odd row-block counts, long K split over many CTAs, many
+# short row blocks.
+STREAM = [(17, 128, 256), (20, 300, 1088), (32, 4096, 4096), (33, 1000, 16384),
+          (40, 129, 8192), (64, 4096, 4096), (64, 200, 65536), (48, 40000, 256)]
+
+
+@pytest.mark.parametrize("M,N,K", STREAM)
+def test_tcgen05_small_batch_tiled_shapes(M, N, K):
+    rng = np.random.default_rng(M * 104729 + N * 131 + K)
+    W = (rng.standard_normal((N, K)) * 0.02).astype(np.float32)
+    x = workloads._to_bf16_bits(rng.standard_normal((M, K)).astype(np.float32))
+    cols = None if N <= 4096 else sample_columns(N, 512, seed=N + M)
+    exact = _forward_tiled_and_check(x, W, M, N, K, tql.BITNET_PATH_GEMM, cols=cols)
+    assert min(exact) >= 0.0
