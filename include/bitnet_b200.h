@@ -560,13 +560,13 @@ BITNET_API bitnet_status bitnet_selftest_bounded_wait(uint64_t limit_ns, bitnet_
 
 /* ------------------------------------------------------------------------
  * bitnet_selftest_divide -- q[i] = a[i] / b[i] through the division the
- * decode epilogue uses for y = acc / (s_x * s_w): the correctly rounded
+ * dequant epilogues use for y = acc / (s_x * s_w): the correctly rounded
  * reciprocal of b and two fused residual corrections (Markstein's method),
- * which rounds to nearest even exactly like an IEEE binary32 division for
- * finite a and normal b > 0 whose quotient is zero or normal; outside that
- * range (subnormal or huge divisors, quotients near overflow) the kernel
- * falls back to the IEEE division itself.  Lets a test check that the
- * result always equals a host IEEE division.
+ * which rounds to nearest even exactly like an IEEE binary32 division when
+ * 2^-95 <= |b| <= 2^100 and a is 0 or 1 <= |a| <= 2^31 (every numerator the
+ * dequant produces is an integer in that range, so the epilogues check only
+ * the divisor, once per token); any other pair takes the IEEE division.
+ * Lets a test check that the result always equals a host IEEE division.
  *
  *   a, b, q   device fp32 arrays of n elements (16-byte aligned), caller-owned.
  *   n         >= 0.

@@ -130,15 +130,17 @@ __device__ __forceinline__ uint32_t spread_byte(uint32_t inv_word, int i) {
 
 // Grid: ceil(N/16) CTAs of kBdWarps warps; CTA r owns rows 16r..16r+15,
 // warp w the words [w*nw/kBdWarps, (w+1)*nw/kBdWarps) of K, taken four at a
-// time.  Lane (g, t) owns word 4U + t of such a group for rows g and g+8:
-// its 32 weights of each row (four 16-byte loads), the 32 activations of
-// every token at the same k, and each tenant's sign word of the two rows.
-// Eight m16n8k16 MMAs consume a group: MMA h takes k = 32 (4U + t) + 4h +
-// {0,1} as the MMA's k positions 2t, 2t+1 and + {2,3} as 2t+8, 2t+9 (any
-// assignment works as long as both operands use it).  The tokens (the MMA's
-// N = 8 = the tenants) read x at the same k; the base MMA multiplies
-// W_base, tenant b's MMA its signs as bf16 +-1, keeping column b.  The
-// warps' partial sums meet in shared memory, added in warp order.
+// time (128 k).  For quarter q of such a group (word 4U + q), lane (g, t)
+// holds k = 32 (4U + q) + 8 t .. +7 of rows g and g+8 (one 16-byte load
+// each; the four lanes of a row read 64 contiguous bytes), the same k of
+// every token, and bits 8t..8t+7 of each tenant's sign word (the four words
+// of a group come in one 16-byte load per row and tenant).  Two m16n8k16
+// MMAs consume a quarter: MMA h takes k + 4h + {0,1} as the MMA's k
+// positions 2t, 2t+1 and k + 4h + {2,3} as 2t+8, 2t+9 (any assignment works
+// as long as both operands use it).  The tokens (the MMA's N = 8 = the
+// tenants) read x at the same k; the base MMA multiplies W_base, tenant b's
+// MMA its signs as bf16 +-1, keeping column b.  The warps' partial sums meet
+// in shared memory, added in warp order.
 __global__ void __launch_bounds__(32 * kBdWarps)
 bitdelta_forward_kernel(const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* __restrict__ Wb,
                         const uint32_t* __restrict__ signs, const float* __restrict__ alpha,
@@ -147,14 +149,19 @@ bitdelta_forward_kernel(const __nv_bfloat16* __restrict__ x, const __nv_bfloat16
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = lane >> 2, t = lane & 3;
   const int64_t nw = K >> 5;
-  const int64_t w0 = nw * warp / kBdWarps, w1 = nw * (warp + 1) / kBdWarps;
+  // Warp ranges start on 4-word boundaries, so every group but the last
+  // is four whole words.
+  const int64_t w0 = (nw * warp / kBdWarps) & ~static_cast<int64_t>(3);
+  const int64_t w1 = warp == kBdWarps - 1 ? nw : (nw * (warp + 1) / kBdWarps) & ~static_cast<int64_t>(3);
+  // 16-byte sign loads need 16-byte aligned rows and tenants.
+  const bool vec_ok = (reinterpret_cast<uintptr_t>(signs) & 15) == 0 && (nw & 3) == 0;
   const int64_t r0 = static_cast<int64_t>(blockIdx.x) * 16;
   const int64_t ra = r0 + g, rb = r0 + g + 8;
   const bool va = ra < N, vb = rb < N;
   const bool vx = g < B;
-  const uint8_t* pa = reinterpret_cast<const uint8_t*>(Wb + (va ? ra : 0) * K);
-  const uint8_t* pb = reinterpret_cast<const uint8_t*>(Wb + (vb ? rb : 0) * K);
-  const uint8_t* px = reinterpret_cast<const uint8_t*>(x + (vx ? g : 0) * K);
+  const uint8_t* pa = reinterpret_cast<const uint8_t*>(Wb + (va ? ra : 0) * K) + 16 * t;
+  const uint8_t* pb = reinterpret_cast<const uint8_t*>(Wb + (vb ? rb : 0) * K) + 16 * t;
+  const uint8_t* px = reinterpret_cast<const uint8_t*>(x + (vx ? g : 0) * K) + 16 * t;
   const uint32_t* sa = signs + (va ? ra : 0) * nw;
   const uint32_t* sb = signs + (vb ? rb : 0) * nw;
   const int64_t tstride = N * nw;   // words from one tenant's signs to the next
@@ -166,31 +173,48 @@ bitdelta_forward_kernel(const __nv_bfloat16* __restrict__ x, const __nv_bfloat16
     for (int e = 0; e < 4; ++e) dl[b][e] = 0.f;
 
   for (int64_t u0 = w0; u0 < w1; u0 += 4) {
-    const int64_t u = u0 + t;          // this lane's word
-    const bool in = u < w1;
+    const bool full = vec_ok && u0 + 4 <= w1;   // u0 is a multiple of 4
     uint4 wa[4], wbv[4], xv[4];
-    uint32_t s_a[kBdMaxTenants], s_b[kBdMaxTenants];
+    uint4 s_a[kBdMaxTenants], s_b[kBdMaxTenants];
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
-      wa[q] = (in && va) ? ldg_stream_u4(pa + 64 * u + 16 * q) : make_uint4(0u, 0u, 0u, 0u);
-      wbv[q] = (in && vb) ? ldg_stream_u4(pb + 64 * u + 16 * q) : make_uint4(0u, 0u, 0u, 0u);
-      xv[q] = (in && vx) ? __ldg(reinterpret_cast<const uint4*>(px + 64 * u) + q)
+      const int64_t u = u0 + q;
+      const bool in = u < w1;
+      wa[q] = (in && va) ? ldg_stream_u4(pa + 64 * u) : make_uint4(0u, 0u, 0u, 0u);
+      wbv[q] = (in && vb) ? ldg_stream_u4(pb + 64 * u) : make_uint4(0u, 0u, 0u, 0u);
+      xv[q] = (in && vx) ? __ldg(reinterpret_cast<const uint4*>(px + 64 * u))
                          : make_uint4(0u, 0u, 0u, 0u);
     }
 #pragma unroll
     for (int b = 0; b < kBdMaxTenants; ++b) {
-      const bool tb = in && b < B;
-      s_a[b] = (tb && va) ? ~ldg_stream_u32(sa + b * tstride + u) : 0u;
-      s_b[b] = (tb && vb) ? ~ldg_stream_u32(sb + b * tstride + u) : 0u;
+      const bool tb = b < B;
+      if (full) {
+        s_a[b] = (tb && va) ? __ldg(reinterpret_cast<const uint4*>(sa + b * tstride + u0))
+                            : make_uint4(0u, 0u, 0u, 0u);
+        s_b[b] = (tb && vb) ? __ldg(reinterpret_cast<const uint4*>(sb + b * tstride + u0))
+                            : make_uint4(0u, 0u, 0u, 0u);
+      } else {
+        uint32_t ea[4], eb[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const bool in = tb && u0 + q < w1;
+          ea[q] = (in && va) ? __ldg(sa + b * tstride + u0 + q) : 0u;
+          eb[q] = (in && vb) ? __ldg(sb + b * tstride + u0 + q) : 0u;
+        }
+        s_a[b] = make_uint4(ea[0], ea[1], ea[2], ea[3]);
+        s_b[b] = make_uint4(eb[0], eb[1], eb[2], eb[3]);
+      }
     }
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {      // 16-byte quarter q = MMAs 2q, 2q+1 = sign byte q
+    for (int q = 0; q < 4; ++q) {
       mma_m16n8k16_bf16(base, wa[q].x, wbv[q].x, wa[q].y, wbv[q].y, xv[q].x, xv[q].y);
       mma_m16n8k16_bf16(base, wa[q].z, wbv[q].z, wa[q].w, wbv[q].w, xv[q].z, xv[q].w);
 #pragma unroll
       for (int b = 0; b < kBdMaxTenants; ++b) {
         if (b < B) {   // uniform across the CTA
-          const uint32_t ga = spread_byte(s_a[b], q), gb = spread_byte(s_b[b], q);
+          const uint32_t wda = q == 0 ? s_a[b].x : q == 1 ? s_a[b].y : q == 2 ? s_a[b].z : s_a[b].w;
+          const uint32_t wdb = q == 0 ? s_b[b].x : q == 1 ? s_b[b].y : q == 2 ? s_b[b].z : s_b[b].w;
+          const uint32_t ga = spread_byte(~wda, t), gb = spread_byte(~wdb, t);
           mma_m16n8k16_bf16(dl[b], sign_pair(ga, 0), sign_pair(gb, 0), sign_pair(ga, 2),
                             sign_pair(gb, 2), xv[q].x, xv[q].y);
           mma_m16n8k16_bf16(dl[b], sign_pair(ga, 4), sign_pair(gb, 4), sign_pair(ga, 6),

@@ -1965,7 +1965,14 @@ __global__ void divide_selftest_kernel(const float* __restrict__ a, const float*
                                        float* __restrict__ q, int64_t n) {
   for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n;
        i += static_cast<int64_t>(gridDim.x) * blockDim.x)
-    q[i] = div_rn_by_recip(a[i], b[i], __frcp_rn(b[i]));
+  {
+    // The epilogue's division for numerators it can see (integer-valued or
+    // not, |a| in {0} U [1, 2^31]); any other numerator takes the IEEE
+    // division, so the result is always RN(a / b).
+    const float av = fabsf(a[i]);
+    const bool in_range = a[i] == 0.0f || (av >= 1.0f && av <= 0x1p31f);
+    q[i] = in_range ? div_rn_int(a[i], b[i], recip_for_div(b[i])) : __fdiv_rn(a[i], b[i]);
+  }
 }
 }  // namespace
 }  // namespace bitnet

@@ -281,28 +281,45 @@ __device__ __forceinline__ void named_barrier_sync(int id, int count) {
 
 // ------------------------------------------------------------ division
 
-// a / b rounded to nearest even (binary32), for finite a and normal b > 0
-// whose quotient is zero or normal, given y = RN(1 / b): Markstein's method
-// (P. Markstein, "Computation of elementary functions on the IBM RISC
-// System/6000 processor", IBM J. Res. Dev. 34(1), 1990): with y within half
-// an ulp of 1/b and q within one ulp of a/b, the residual a - b q is exact
-// under a fused multiply-add and RN(q + (a - b q) y) = RN(a / b).  One
-// correction brings RN(a y) within one ulp; the second rounds correctly.
+// a / b rounded to nearest even (binary32) through y = RN(1 / b):
+// Markstein's method (P. Markstein, "Computation of elementary functions on
+// the IBM RISC System/6000 processor", IBM J. Res. Dev. 34(1), 1990): with y
+// within half an ulp of 1/b and q within one ulp of a/b, the residual
+// a - b q is exact under a fused multiply-add and RN(q + (a - b q) y) =
+// RN(a / b).  One correction brings RN(a y) within one ulp; the second
+// rounds correctly.  That holds for finite a and b whose quotient and
+// numerator are zero or stay well inside the normal range.
 //
-// Outside that range (a divisor that is subnormal, zero or above 2^126, a
-// quotient or numerator near overflow or underflow -- reachable only with
-// extreme gains or weight magnitudes) the function returns the IEEE
-// division itself, so the result is always RN(a / b).
-__device__ __forceinline__ float div_rn_by_recip(float a, float b, float y) {
+// The dequant divides integers (|a| <= 2^31) by s_x * s_w.  For a divisor
+// with 2^-95 <= |b| <= 2^100 every such quotient lies in [2^-100, 2^126],
+// so the divisor alone decides: recip_for_div(b) returns RN(1 / b) for such
+// divisors and 0 otherwise, computed once per token, and div_rn_int takes
+// the IEEE division for a zero reciprocal (reachable only with extreme
+// gains or weight magnitudes).  No test per output: an extra range check
+// there cost the tensor-core prefill kernel a fifth of its throughput.
+__device__ __forceinline__ float recip_for_div(float b) {
+  const float ab = fabsf(b);
+  return (ab >= 0x1p-95f && ab <= 0x1p100f) ? __frcp_rn(b) : 0.0f;
+}
+
+// Kept out of line: an inlined IEEE division in an unrolled epilogue
+// multiplies the kernel's code size.
+__device__ __noinline__ float div_rn_out_of_range(float a, float b) { return __fdiv_rn(a, b); }
+
+// RN(a / b) for an integer-valued a with |a| <= 2^31 and y = recip_for_div(b)
+// known to be non-zero (a kernel that checked all its divisors beforehand).
+__device__ __forceinline__ float div_rn_int_fast(float a, float b, float y) {
   float q = __fmul_rn(a, y);
-  const float ab = fabsf(b), aq = fabsf(q), aa = fabsf(a);
-  if (!(ab >= 0x1p-126f && ab <= 0x1p126f) ||
-      (a != 0.0f && !(aq >= 0x1p-100f && aq <= 0x1p126f && aa >= 0x1p-100f && aa <= 0x1p126f)))
-    return __fdiv_rn(a, b);
   float r = __fmaf_rn(-q, b, a);
   q = __fmaf_rn(r, y, q);
   r = __fmaf_rn(-q, b, a);
   return __fmaf_rn(r, y, q);
+}
+
+// RN(a / b) for an integer-valued a with |a| <= 2^31, y = recip_for_div(b).
+__device__ __forceinline__ float div_rn_int(float a, float b, float y) {
+  if (y == 0.0f) return div_rn_out_of_range(a, b);
+  return div_rn_int_fast(a, b, y);
 }
 
 // ------------------------------------------------- decode activation order

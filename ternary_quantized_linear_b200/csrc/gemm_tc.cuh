@@ -10,16 +10,13 @@
 //
 // A CTA computes a 128 (weight rows, TMEM lanes) x BN (tokens) tile of
 // acc^T over a range of K, in 256-k steps:
-//   warp 0      weight producer: per step the packed weight tile (128 rows x
-//               KSTEP/4 bytes) into a STAGES-deep shared-memory ring, by a
-//               2-D tensor copy from the row-major layout or, with the tiled
-//               layout (tiled.cuh), by one 1-D bulk copy of the tile, which
-//               arrives already in the swizzled order the unpack reads;
-//   warps 2, 3  activation producers: one 128-byte swizzle atom each of the
-//               activation tile (BN rows of KSTEP int8 = the MMA's canonical
-//               K-major layout).  A thread can start a bulk copy only every
-//               few hundred nanoseconds, so the three copies of a step are
-//               issued by three threads;
+//   warp 0      producer: per step the packed weight tile (128 rows x
+//               KSTEP/4 bytes) -- a 2-D tensor copy from the row-major layout
+//               or, with the tiled layout (tiled.cuh), one 1-D bulk copy of
+//               the tile, which arrives already in the swizzled order the
+//               unpack reads -- and the activation tile (BN rows of KSTEP
+//               int8 as 128-byte swizzle atoms = the MMA's canonical K-major
+//               layout) into a STAGES-deep shared-memory ring;
 //   warp 1      allocates TMEM; one thread issues KSTEP/32 MMAs (K = 32 each)
 //               per step reading A from TMEM and B from shared memory;
 //   warps 4-11  unpack: each thread expands 16 packed bytes of its weight
@@ -177,13 +174,16 @@ __device__ __forceinline__ void tc_mma_i8_ts(uint32_t d_tmem, uint32_t a_tmem, u
 
 // One output: e = the tile's epilogue entry of token m, {row sum, divisor
 // s_x * s_w, RN(1 / divisor)} (the last two as float bits).
+// kFast: every divisor of the tile passed recip_for_div (no per-output test).
+template <bool kFast = false>
 __device__ __forceinline__ void gemm_store(const GemmParams& p, int4 e, int m, int n, int acc_codes) {
   const int acc = acc_codes - e.x;
   const int64_t o = static_cast<int64_t>(m) * p.N + n;
   if (p.acc_out) p.acc_out[o] = acc;
   if (p.y) {
     const float yv =
-        div_rn_by_recip(__int2float_rn(acc), __int_as_float(e.y), __int_as_float(e.z));
+        kFast ? div_rn_int_fast(__int2float_rn(acc), __int_as_float(e.y), __int_as_float(e.z))
+              : div_rn_int(__int2float_rn(acc), __int_as_float(e.y), __int_as_float(e.z));
     if (p.y_bf16)
       reinterpret_cast<__nv_bfloat16*>(p.y)[o] = __float2bfloat16_rn(yv);
     else
@@ -216,6 +216,7 @@ ternary_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x,
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
   int* is_last = reinterpret_cast<int*>(smem + C::OFF_MISC + 8);
+  int* all_fast = reinterpret_cast<int*>(smem + C::OFF_MISC + 12);   // every divisor in range
   int4* tab = reinterpret_cast<int4*>(smem + C::OFF_TAB);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -230,12 +231,13 @@ ternary_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x,
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::STAGES; ++s) {
       mbar_init(&fullw[s], 1);
-      mbar_init(&fullx[s], C::ATOMS);             // one producer per activation atom
+      mbar_init(&fullx[s], 1);
       mbar_init(&done[s], 1);                     // MMA commit
     }
     for (int a = 0; a < C::A_STAGES; ++a) mbar_init(&aready[a], C::UNPACK_WARPS);
     mbar_init(accfull, 1);
     *abort_flag = 0;
+    *all_fast = 1;
     fence_mbarrier_init();
   }
   if (warp == 0 && lane == 0) {
@@ -254,49 +256,44 @@ ternary_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x,
   // sums, scales) are read only after this point.
   if (p.use_pdl) pdl_wait_prior_grid();
 
-  if (warp == 0 || warp == 2 || warp == 3) {
+  if (warp == 0) {
     if (lane == 0) {
-      // ----------------------------------------------------------- producers
-      // warp 0: weights; warp 2 + a: activation atom a.
-      const int atom = warp - 2;
-      const bool wprod = warp == 0;
-      uint64_t* full = wprod ? fullw : fullx;
-      if (wprod || atom < C::ATOMS) {
-        int issued = 0;
-        for (int j = 0; j < nk; ++j) {
-          const int s = j % C::STAGES;
-          const uint32_t use = static_cast<uint32_t>(j / C::STAGES);
-          if (j >= C::STAGES &&
-              !mbar_wait_bounded(&done[s], (use - 1u) & 1u, abort_flag, limit)) {
-            gemm_fail(abort_flag, p.status, DEV_TIMEOUT_PRODUCER);
-            break;
-          }
-          const int kb = kb0 + j;
-          if (wprod) {
-            mbar_arrive_expect_tx(&full[s], C::WP_BYTES);
-            if (kTiledW)
-              bulk_load(wps + s * C::WP_BYTES,
-                        p.Wt + (static_cast<int64_t>(blockIdx.x) * p.KC + kb) * C::WP_BYTES,
-                        C::WP_BYTES, &full[s]);
-            else
-              tma_load_2d(wps + s * C::WP_BYTES, &tmap_w, kb * C::WP_ROW, n0, &full[s]);
-          } else {
-            mbar_arrive_expect_tx(&full[s], C::X_ATOM);
-            tma_load_2d(xs + s * C::X_BYTES + atom * C::X_ATOM, &tmap_x,
-                        kb * C::KSTEP + 128 * atom, m0, &full[s]);
-          }
-          issued = j + 1;
+      // ------------------------------------------------------------ producer
+      // One thread issues the step's three copies (the weight tile, then the
+      // two activation atoms): splitting them over three threads measured
+      // slower on prefill.
+      int issued = 0;
+      for (int j = 0; j < nk; ++j) {
+        const int s = j % C::STAGES;
+        const uint32_t use = static_cast<uint32_t>(j / C::STAGES);
+        if (j >= C::STAGES && !mbar_wait_bounded(&done[s], (use - 1u) & 1u, abort_flag, limit)) {
+          gemm_fail(abort_flag, p.status, DEV_TIMEOUT_PRODUCER);
+          break;
         }
-        if (*abort_flag) {
-          // Let this producer's copies in flight land before the CTA exits
-          // (the activation barrier completes only when both atoms land).
-          const int first = issued > C::STAGES ? issued - C::STAGES : 0;
-          for (int j = first; j < issued; ++j) {
-            const int s = j % C::STAGES;
-            if (!mbar_wait_bounded(&full[s], static_cast<uint32_t>(j / C::STAGES) & 1u, nullptr,
-                                   limit))
-              record_failure(p.status, DEV_TIMEOUT_DRAIN);
-          }
+        const int kb = kb0 + j;
+        mbar_arrive_expect_tx(&fullw[s], C::WP_BYTES);
+        if (kTiledW)
+          bulk_load(wps + s * C::WP_BYTES,
+                    p.Wt + (static_cast<int64_t>(blockIdx.x) * p.KC + kb) * C::WP_BYTES,
+                    C::WP_BYTES, &fullw[s]);
+        else
+          tma_load_2d(wps + s * C::WP_BYTES, &tmap_w, kb * C::WP_ROW, n0, &fullw[s]);
+        mbar_arrive_expect_tx(&fullx[s], C::X_BYTES);
+#pragma unroll
+        for (int at = 0; at < C::ATOMS; ++at)
+          tma_load_2d(xs + s * C::X_BYTES + at * C::X_ATOM, &tmap_x, kb * C::KSTEP + 128 * at, m0,
+                      &fullx[s]);
+        issued = j + 1;
+      }
+      if (*abort_flag) {
+        // Let the copies already in flight land before the CTA exits.
+        const int first = issued > C::STAGES ? issued - C::STAGES : 0;
+        for (int j = first; j < issued; ++j) {
+          const int s = j % C::STAGES;
+          const uint32_t par = static_cast<uint32_t>(j / C::STAGES) & 1u;
+          if (!mbar_wait_bounded(&fullw[s], par, nullptr, limit) ||
+              !mbar_wait_bounded(&fullx[s], par, nullptr, limit))
+            record_failure(p.status, DEV_TIMEOUT_DRAIN);
         }
       }
     }
@@ -351,7 +348,9 @@ ternary_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x,
           rs = p.gacc ? p.rowsum[m * p.G + blockIdx.z] : p.rowsum[m];
           if (p.y) d = __fmul_rn(p.s_x[m], swv);
         }
-        tab[c] = make_int4(rs, __float_as_int(d), __float_as_int(__frcp_rn(d)), 0);
+        const float y = recip_for_div(d);
+        if (y == 0.0f) atomicAnd(all_fast, 0);
+        tab[c] = make_int4(rs, __float_as_int(d), __float_as_int(y), 0);
       }
       named_barrier_sync(1, 32 * C::UNPACK_WARPS);
     }
@@ -405,12 +404,21 @@ ternary_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x,
     if (write && (BN >= 32 || h == 0)) {
       const int n = n0 + i;
       const bool split = p.ksplit > 1 && !p.gacc;
+      // The common case -- a plain tile whose divisors all passed -- runs a
+      // loop with no per-output test.
+      const bool fast = !split && !p.gacc && *all_fast != 0;
       for (int c0 = h * kHalf; c0 < (h + 1) * kHalf; c0 += 16) {
         if (m0 + c0 >= p.M) break;  // uniform across the warp
         uint32_t r[16];
         tmem_ld_32x32b_x16(tmem_base + lane_addr + C::D_COL + c0, r);
         tmem_ld_wait();
-        if (n < p.N) {
+        if (n < p.N && fast) {
+#pragma unroll
+          for (int jj = 0; jj < 16; ++jj) {
+            const int m = m0 + c0 + jj;
+            if (m < p.M) gemm_store<true>(p, tab[c0 + jj], m, n, static_cast<int>(r[jj]));
+          }
+        } else if (n < p.N) {
 #pragma unroll
           for (int jj = 0; jj < 16; ++jj) {
             const int m = m0 + c0 + jj;

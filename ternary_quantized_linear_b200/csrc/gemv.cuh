@@ -246,7 +246,7 @@ __device__ __forceinline__ void gemv_finish(const GemvProblem& p, float d, float
   const int64_t o = static_cast<int64_t>(m) * p.N + n;
   if (p.acc_out) p.acc_out[o] = acc;
   if (p.y) {
-    const float yv = div_rn_by_recip(__int2float_rn(acc), d, rd);
+    const float yv = div_rn_int(__int2float_rn(acc), d, rd);
     if (p.y_bf16)
       reinterpret_cast<__nv_bfloat16*>(p.y)[o] = __float2bfloat16_rn(yv);
     else
@@ -418,7 +418,7 @@ ternary_gemv_kernel(const __grid_constant__ GemvLaunch L) {
       seg_rs[warp][lane] = P.rowsum[lane];
       const float d = (P.y && P.s_x && P.s_w) ? __fmul_rn(P.s_x[lane], P.s_w[0]) : 1.0f;
       seg_d[warp][lane] = d;
-      seg_rd[warp][lane] = __frcp_rn(d);
+      seg_rd[warp][lane] = recip_for_div(d);
     }
   }
   if (lane == 0) {

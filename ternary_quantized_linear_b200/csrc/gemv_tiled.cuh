@@ -198,7 +198,7 @@ __device__ __forceinline__ void gt_store(const GtProblem& P, const GtTok& tk, in
     return;
   }
   if (P.acc_out) P.acc_out[o] = acc;
-  if (P.y) gt_write(P, o, div_rn_by_recip(__int2float_rn(acc), tk.d, tk.rd));
+  if (P.y) gt_write(P, o, div_rn_int(__int2float_rn(acc), tk.d, tk.rd));
 }
 
 // The fused SwiGLU output: silu(gate) * up with silu(z) = z / (1 + e^-z),
@@ -207,8 +207,8 @@ __device__ __forceinline__ void gt_store(const GtProblem& P, const GtTok& tk, in
 // divide, multiply).
 __device__ __forceinline__ void gt_store_pair(const GtProblem& P, const GtTok& tk, int m, int n,
                                               int gate_codes, int up_codes) {
-  const float g = div_rn_by_recip(__int2float_rn(gate_codes - tk.rs), tk.d, tk.rd);
-  const float u = div_rn_by_recip(__int2float_rn(up_codes - tk.rs), tk.d2, tk.rd2);
+  const float g = div_rn_int(__int2float_rn(gate_codes - tk.rs), tk.d, tk.rd);
+  const float u = div_rn_int(__int2float_rn(up_codes - tk.rs), tk.d2, tk.rd2);
   const float sg = __fdiv_rn(g, __fadd_rn(1.0f, expf(-g)));
   gt_write(P, static_cast<int64_t>(m) * P.N + n, __fmul_rn(sg, u));
 }
@@ -218,9 +218,9 @@ __device__ __forceinline__ GtTok gt_token(const GtProblem& P, int m, bool pair, 
   GtTok tk;
   tk.rs = P.gc > 0 ? P.rowsum[m * P.G + grp] : P.rowsum[m];
   tk.d = P.s_w ? __fmul_rn(P.s_x[m], P.s_w[0]) : 1.0f;
-  tk.rd = __frcp_rn(tk.d);
+  tk.rd = recip_for_div(tk.d);
   tk.d2 = (pair && P.s_w2) ? __fmul_rn(P.s_x[m], P.s_w2[0]) : 1.0f;
-  tk.rd2 = __frcp_rn(tk.d2);
+  tk.rd2 = recip_for_div(tk.d2);
   return tk;
 }
 

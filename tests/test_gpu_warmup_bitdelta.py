@@ -170,3 +170,21 @@ def test_bitdelta_forward_bf16_output():
 def test_warmup_and_bitdelta_leave_no_device_failure():
     code, _ = tql.bitnet_device_status(reset=False)
     assert code == 0
+
+
+def test_bitdelta_forward_odd_word_count_and_unaligned_signs():
+    """K/32 not a multiple of 4 and a sign buffer that is only 4-byte
+    aligned: the kernel falls back from its 16-byte sign loads."""
+    N, K, B = 96, 1056, 3
+    base, fine, x = workloads.bitdelta_inputs(N, K, B, seed=6)
+    bd = _bits_to_dev(base)
+    buf = torch.empty(B * N * (K // 32) + 1, dtype=torch.int32, device="cuda")
+    signs = buf[1:].view(B, N, K // 32)
+    alpha = torch.empty((B,), dtype=torch.float32, device="cuda")
+    for b in range(B):
+        tql.bitnet_bitdelta_compress(bd, _bits_to_dev(fine[b]), signs=signs[b], alpha=alpha[b:b + 1])
+    y = tql.bitnet_bitdelta_forward(_bits_to_dev(x), bd, signs, alpha)
+    torch.cuda.synchronize()
+    ref, absdot = oracle.bitdelta_forward(x, base, signs.cpu().numpy().view(np.uint32),
+                                          alpha.cpu().numpy())
+    assert np.all(np.abs(y.cpu().numpy() - ref) <= _bound(K, absdot))
