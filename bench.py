@@ -44,7 +44,8 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # (the tiled decode matmul over the step's four M <= 16 forwards) from an
 # ncu capture (summary under profiles/), valid only for the kernel source it
 # was measured on (sha256 of csrc/gemv_tiled.cuh); reported as null otherwise.
-GT_TRAFFIC = {"src_sha256": None, "bytes_per_launch": None}
+GT_TRAFFIC = {"src_sha256": "76a40f2c8551b68637af97d415d022845aac5f12f3f0d4c2926d15b1981b2fa2",
+              "bytes_per_launch": 235552768 + 5115392}
 
 
 # ------------------------------------------------------------------ helpers
@@ -371,10 +372,12 @@ def run_ours(args):
     value = job_throughput(sb, args.steps, world, max_ms)
     trial_gbs = sorted(sb * args.steps / (t * 1e-3) / 1e9 for t in trial_ms)
     ms_per_step = max_ms / args.steps
-    # kernel launches per step: the grouped decode quant + the tiled decode
-    # matmul for the four M <= 16 forwards; quant + tcgen05 for each M = 64
+    # kernel launches per step: the grouped decode quant, the tiled decode
+    # matmul for the four M <= 16 forwards and its fixup of split row blocks
+    # (these shapes split some); a quant and a tcgen05 launch for each M = 64
+    # forward (the launch list under profiles/ shows the same count)
     n_big = sum(1 for p in head.probs if p[3] > 16)
-    launches_per_step = 2 + 2 * n_big
+    launches_per_step = 3 + 2 * n_big
 
     # ---- roofline: the tiled decode matmul of the four M <= 16 forwards
     # (the dominant kernel: 4 x 58.7 MB of the step's 6 x 58.7 MB), timed
@@ -802,6 +805,34 @@ def measure_weight_pack(args, tql, workloads, torch, stream, device, hbm_peak):
             "bytes": "two reads of W (absmean, then quantize) + the packed write"}
 
 
+def profile_kernel(args):
+    """A small driver for an ncu capture of the roofline kernel: one rotation
+    set of the headline's M <= 16 forwards (four forwards, each with its own
+    copy of the tiled weights, 235 MB -- more than L2), two full grouped
+    calls, then `--steps` calls of the matmul phase alone.  Prints one status
+    line; no timing (numbers under a profiler are not bench values)."""
+    import torch
+    import ternary_quantized_linear_b200 as tql
+    from ternary_quantized_linear_b200 import build as tql_build
+    from ternary_quantized_linear_b200 import workloads
+    tql_build.build()
+    lib = tql.load_library()
+    device = torch.device("cuda", 0)
+    small = tuple(m for m in HEADLINE_MS if m <= 16)
+    wl = DecodeWorkload(tql, workloads, HEADLINE, small, 1, device, {})
+    st = wl.sets[0]
+    h = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    for _ in range(2):
+        grouped_call(lib, tql, st, tql.BITNET_PHASE_ALL, h)
+    for _ in range(args.steps):
+        grouped_call(lib, tql, st, tql.BITNET_PHASE_MATMUL, h)
+    torch.cuda.synchronize()
+    code, detail = tql.bitnet_device_status(reset=False)
+    print(json.dumps({"profile_kernel": "done", "problems": [[K, N, M] for _, K, N, M in wl.probs],
+                      "weight_bytes": wl.weight_bytes, "device_status": [int(code), int(detail)]}))
+    return 0 if code == 0 else 1
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__)
     ap.add_argument("--gpus", type=int, default=1)
@@ -815,7 +846,11 @@ def main(argv=None):
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-configs", action="store_true")
     ap.add_argument("--no-weight-pack", action="store_true")
+    ap.add_argument("--profile-kernel", action="store_true",
+                    help="only run the roofline kernel's launches (a driver for ncu)")
     args = ap.parse_args(argv)
+    if args.profile_kernel:
+        return profile_kernel(args)
     if args.warmup < 3 and args.impl == "ours":
         args.warmup = 3
     if args.impl == "reference":
