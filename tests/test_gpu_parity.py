@@ -197,7 +197,8 @@ def test_large_cases_sampled(ci, si, M):
     K, N = case.shapes[si]
     x = workloads.activations(case, si, M)
     W = workloads.weights(case, si)
-    cols = None if M <= 16 else sample_columns(N, 96, seed=M + 7 * si)
+    # 1024 sampled columns (plus tile edges) up to 2048 tokens, 256 beyond
+    cols = None if M <= 16 else sample_columns(N, 1024 if M <= 2048 else 256, seed=M + 7 * si)
     _forward_and_check(x, W, M, N, K, tql.BITNET_PATH_AUTO, cols=cols,
                        y_dtypes=(torch.bfloat16,))
 

@@ -146,7 +146,7 @@ def test_tiled_large_cases_sampled(ci, si, M):
     K, N = case.shapes[si]
     x = workloads.activations(case, si, M)
     W = workloads.weights(case, si)
-    cols = None if M <= 16 else sample_columns(N, 256, seed=M + 7 * si)
+    cols = None if M <= 16 else sample_columns(N, 1024 if M <= 2048 else 256, seed=M + 7 * si)
     _forward_tiled_and_check(x, W, M, N, K, tql.BITNET_PATH_AUTO, cols=cols,
                              y_dtypes=(torch.bfloat16,))
 
