@@ -372,12 +372,13 @@ def run_ours(args):
     value = job_throughput(sb, args.steps, world, max_ms)
     trial_gbs = sorted(sb * args.steps / (t * 1e-3) / 1e9 for t in trial_ms)
     ms_per_step = max_ms / args.steps
-    # kernel launches per step: the grouped decode quant, the tiled decode
-    # matmul for the four M <= 16 forwards and its fixup of split row blocks
-    # (these shapes split some); a quant and a tcgen05 launch for each M = 64
-    # forward (the launch list under profiles/ shows the same count)
+    # kernel launches per step: one activation-quant launch for all six
+    # forwards, the tiled decode matmul for the four M <= 16 forwards and its
+    # fixup of split row blocks (these shapes split some), and a tcgen05
+    # launch for each M = 64 forward (the launch list under profiles/ shows
+    # the same count)
     n_big = sum(1 for p in head.probs if p[3] > 16)
-    launches_per_step = 3 + 2 * n_big
+    launches_per_step = 3 + n_big
 
     # ---- roofline: the tiled decode matmul of the four M <= 16 forwards
     # (the dominant kernel: 4 x 58.7 MB of the step's 6 x 58.7 MB), timed

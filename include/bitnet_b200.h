@@ -313,16 +313,17 @@ BITNET_API bitnet_status bitnet_linear_matmul(const uint8_t *W_packed, const flo
  * one call (each one the forward of the first page's 量子化の仕組み, as
  * bitnet_linear_forward; the projections of one LLaMA-like block, The Era of
  * 1-bit LLMs review, 提案手法, are the typical group): the result is exactly
- * that of calling bitnet_linear_forward on each problem in order, but the decode problems (M <= 16) share one
- * activation-quant launch and one matmul launch, so their weight streams
- * overlap instead of paying one launch latency each.  Typical use: the
- * projections of one decode step (q, k, v, o, gate, up, down).  Decode
- * problems with the same x, x_dtype, gamma, eps, M and K (q/k/v, gate/up)
- * share one activation quantization.  The host-side plan of a call is
+ * that of calling bitnet_linear_forward on each problem in order, but every
+ * problem's activation quantization is one launch and the decode problems
+ * (M <= 16) share one matmul launch, so their weight streams overlap instead
+ * of paying one launch latency each.  Typical use: the projections of one
+ * decode step (q, k, v, o, gate, up, down).  Problems with the same x,
+ * x_dtype, gamma, eps, M and K (q/k/v, gate/up) that use the same matmul
+ * kind share one activation quantization.  The host-side plan of a call is
  * cached per thread (a few entries, keyed by every field of every problem
  * and the workspace), so a decode loop that repeats the same call plans it
- * once.  Problems with M > 16 run afterwards on the tcgen05 kernel, one at a
- * time.
+ * once.  The matmuls of problems with M > 16 run afterwards on the tcgen05
+ * kernel, one at a time.
  *
  *   count      0 <= count <= BITNET_MAX_GROUP.
  *   problems   host array of `count` problem descriptions (each field as in
@@ -331,11 +332,11 @@ BITNET_API bitnet_status bitnet_linear_matmul(const uint8_t *W_packed, const flo
  *   workspace  >= bitnet_linear_forward_grouped_workspace_bytes(count,
  *              problems), 256-byte aligned, contents on entry irrelevant.
  *   phases     BITNET_PHASE_ALL, or one phase at a time: BITNET_PHASE_QUANTIZE
- *              (activation quant of the decode problems into the workspace)
- *              then, later on the same stream with the same problems and
- *              workspace, BITNET_PHASE_MATMUL (their matmuls, then every
- *              M > 16 problem in full).  Splitting lets a caller time the
- *              phases or reuse one quantization; the results are identical.
+ *              (activation quant of every problem into the workspace) then,
+ *              later on the same stream with the same problems and
+ *              workspace, BITNET_PHASE_MATMUL (every matmul).  Splitting
+ *              lets a caller time the phases or reuse one quantization; the
+ *              results are identical.
  * Any invalid problem rejects the whole call before anything is queued.
  * ---------------------------------------------------------------------- */
 #define BITNET_MAX_GROUP 16

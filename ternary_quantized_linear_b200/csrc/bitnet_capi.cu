@@ -921,6 +921,14 @@ struct DecodePlan {
   int nrow = 0;     // ... on row-major weights
   int qblocks = 0;  // blocks of the quant launch
   uint32_t stage = 0;
+  // Larger problems (the tcgen05 kernel): quantized by the same grouped
+  // launch, multiplied one after another.
+  int nbig = 0;
+  int big_src[BITNET_MAX_GROUP];
+  uint8_t* big_q[BITNET_MAX_GROUP];       // workspace holding its quantized input
+  FwdWorkspace big_qL[BITNET_MAX_GROUP];
+  uint8_t* big_ws[BITNET_MAX_GROUP];      // its own workspace (split-K partials)
+  FwdWorkspace big_L[BITNET_MAX_GROUP];
 };
 
 constexpr int kPlanCacheSize = 8;
@@ -1007,11 +1015,11 @@ bool build_decode_plan(const DeviceState& ds, int count, const bitnet_linear_pro
   int qblocks = 0, qn = 0;
   uint32_t stage = 0;
   size_t off = 0;
-  int src[BITNET_MAX_GROUP];            // problem index of each decode problem
+  int src[BITNET_MAX_GROUP];            // problem index of each entry
   uint8_t* qws[BITNET_MAX_GROUP];       // its quantized-activation workspace
   FwdWorkspace qL[BITNET_MAX_GROUP];
-  bool tl[BITNET_MAX_GROUP];
-  int n = 0;
+  int kind[BITNET_MAX_GROUP];           // 0 row-major decode, 1 tiled decode, 2 tcgen05
+  int n = 0, nb = 0;
   nr = 0;
   nt = 0;
   for (int i = 0; i < count; ++i) {
@@ -1020,20 +1028,23 @@ bool build_decode_plan(const DeviceState& ds, int count, const bitnet_linear_pro
     const FwdWorkspace L = fwd_layout(q.M, q.N, q.K);
     uint8_t* ws = base + off;
     off += L.total;
-    if (q.M > kGemvMaxM) continue;
     const bool tiled = q.w_layout == BITNET_LAYOUT_TILED;
+    const int kd = q.M > kGemvMaxM ? 2 : (tiled ? 1 : 0);
     // Region the quant launch clears: the tiled kernel's arrival counters,
-    // or the row-major kernel's split-K partials when its CTAs share rows.
-    const bool shared_rows = !tiled && gemv_problem_shared(GL, nr, plan.G);
+    // the row-major kernel's split-K partials when its CTAs share rows, or
+    // the tcgen05 kernel's split-K partials.
+    const bool shared_rows = kd == 0 && gemv_problem_shared(GL, nr, plan.G);
     size_t zbytes = 0;
-    void* zero = tiled ? counter_region(ws, L, &zbytes)
-                       : (shared_rows ? splitk_region(ws, L, &zbytes) : nullptr);
+    void* zero = kd == 2 ? zero_region_for(ds, BITNET_PATH_GEMM, q.w_layout, q.M, q.N, q.K, ws,
+                                           L, &zbytes)
+                 : kd == 1 ? counter_region(ws, L, &zbytes)
+                           : (shared_rows ? splitk_region(ws, L, &zbytes) : nullptr);
     int owner = -1;
     if (!shared_rows)
       for (int j = 0; j < n && owner < 0; ++j)
-        if (tl[j] == tiled && same_input(problems[src[j]], q)) owner = j;
+        if (kind[j] == kd && same_input(problems[src[j]], q)) owner = j;
     src[n] = i;
-    tl[n] = tiled;
+    kind[n] = kd;
     QuantProblem& qp = QL.prob[qn++];
     qp = QuantProblem{};
     qp.zero16 = static_cast<uint4*>(zero);
@@ -1058,13 +1069,20 @@ bool build_decode_plan(const DeviceState& ds, int count, const bitnet_linear_pro
       qp.M = static_cast<int>(q.M);
       qp.K = static_cast<int>(q.K);
       qp.x_bf16 = (q.x_dtype == BITNET_BF16) ? 1 : 0;
-      qp.perm = 1;  // decode matmul
-      qp.tiled = tiled ? 1 : 0;
+      qp.perm = kd == 2 ? 0 : 1;  // the decode matmuls' block order
+      qp.tiled = kd == 1 ? 1 : 0;
       stage = std::max(stage, quant_stage_bytes(q.K, qp.x_bf16 != 0, q.gamma != nullptr));
     }
     if (owner < 0 || zero) qblocks += qp.M + qp.zero_blocks;
     const float* sx = reinterpret_cast<const float*>(qws[n] + qL[n].sx);
-    if (tiled) {
+    if (kd == 2) {
+      plan.big_src[nb] = i;
+      plan.big_q[nb] = qws[n];
+      plan.big_qL[nb] = qL[n];
+      plan.big_ws[nb] = ws;
+      plan.big_L[nb] = L;
+      ++nb;
+    } else if (tiled) {
       fill_gt_problem(TL.prob[nt], q.W_packed, qws[n], qL[n], ws, L, sx, q.s_w, q.M, q.N, q.K,
                       q.y, q.y_dtype, nullptr);
       ++nt;
@@ -1077,6 +1095,7 @@ bool build_decode_plan(const DeviceState& ds, int count, const bitnet_linear_pro
     ++n;
   }
   QL.count = qn;
+  plan.nbig = nb;
   plan.qblocks = qblocks;
   plan.stage = stage;
   plan.valid = true;
@@ -1113,7 +1132,7 @@ bitnet_status forward_grouped_impl(int count, const bitnet_linear_problem* probl
       return BITNET_ERR_CUDA;
     }
   }
-  if (plan->n > 0) {
+  {
     QuantLaunch& QL = plan->QL;
     GemvLaunch& GL = plan->GL;
     QL.trigger_dependents = do_matmul ? 1 : 0;
@@ -1143,19 +1162,18 @@ bitnet_status forward_grouped_impl(int count, const bitnet_linear_problem* probl
     }
   }
   if (!do_matmul) return BITNET_OK;
-  // Larger problems: the tcgen05 kernel, one after another.
-  size_t off = 0;
-  for (int i = 0; i < count; ++i) {
-    const bitnet_linear_problem& q = problems[i];
-    if (q.M == 0) continue;
-    const FwdWorkspace L = fwd_layout(q.M, q.N, q.K);
-    uint8_t* ws = base + off;
-    off += L.total;
-    if (q.M <= kGemvMaxM) continue;
-    const bitnet_status st =
-        forward_impl(q.x, q.x_dtype, q.gamma, q.eps, q.W_packed, q.s_w, q.M, q.N, q.K, q.y,
-                     q.y_dtype, ws, L.total, nullptr, nullptr, nullptr, BITNET_PATH_GEMM, stream,
-                     q.w_layout);
+  // Larger problems: the tcgen05 kernel, one after another, on the inputs
+  // the grouped launch quantized (each launch waits for the grid before it
+  // -- which itself waited for the quant grid -- before reading them).
+  for (int b = 0; b < plan->nbig; ++b) {
+    const bitnet_linear_problem& q = problems[plan->big_src[b]];
+    const uint8_t* qw = plan->big_q[b];
+    const FwdWorkspace& qL = plan->big_qL[b];
+    const bitnet_status st = launch_gemm(
+        *ds, q.W_packed, reinterpret_cast<const int8_t*>(qw + qL.xq),
+        reinterpret_cast<const int32_t*>(qw + qL.rs), reinterpret_cast<const float*>(qw + qL.sx),
+        q.s_w, q.M, q.N, q.K, plan->big_ws[b], plan->big_L[b], q.y, q.y_dtype, nullptr, true,
+        stream, q.w_layout == BITNET_LAYOUT_TILED);
     if (st != BITNET_OK) return st;
   }
   return BITNET_OK;

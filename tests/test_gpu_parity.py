@@ -502,3 +502,40 @@ def test_division_outside_the_fast_range_is_ieee():
     got = q.cpu().numpy()
     same = (got.view(np.uint32) == ref.view(np.uint32)) | (np.isnan(got) & np.isnan(ref))
     assert same.all(), (a[~same], b[~same], got[~same], ref[~same])
+
+
+@pytest.mark.parametrize("split", [False, True])
+def test_grouped_tensor_core_problems_share_the_quant_launch(split):
+    # Larger problems are quantized by the grouped launch too: two M = 64
+    # problems on one input (split-K partials, one shared quantization), an
+    # M = 300 problem, and a decode problem; every output must equal the
+    # single-call forward bit for bit and the oracle within the usual bar.
+    rng = np.random.default_rng(404)
+    K = 1024
+    x64 = workloads._to_bf16_bits(rng.standard_normal((64, K)).astype(np.float32))
+    x300 = workloads._to_bf16_bits(rng.standard_normal((300, K)).astype(np.float32))
+    x1 = workloads._to_bf16_bits(rng.standard_normal((1, K)).astype(np.float32))
+    d64, d300, d1 = x_to_device(x64), x_to_device(x300), x_to_device(x1)
+    specs = [(x64, d64, 640), (x64, d64, 200), (x300, d300, 384), (x1, d1, 520)]
+    items, meta = [], []
+    for xh, xd, N in specs:
+        W = (rng.standard_normal((N, K)) * 0.02).astype(np.float32)
+        W_p, s_w = _dev_weights(W)
+        y = torch.empty((xh.shape[0], N), dtype=torch.bfloat16, device="cuda")
+        items.append((xd, None, workloads.DEFAULT_EPS, W_p, s_w, y))
+        meta.append((xh, W, N))
+    if split:
+        ws = torch.empty(1 << 26, dtype=torch.uint8, device="cuda")
+        ws.fill_(0x5A)
+        tql.bitnet_linear_forward_grouped(items, workspace=ws, phases=tql.BITNET_PHASE_QUANTIZE)
+        tql.bitnet_linear_forward_grouped(items, workspace=ws, phases=tql.BITNET_PHASE_MATMUL)
+    else:
+        tql.bitnet_linear_forward_grouped(items)
+    torch.cuda.synchronize()
+    for (xd, g, eps, W_p, s_w, y), (xh, W, N) in zip(items, meta):
+        y1 = tql.bitnet_linear_forward(xd, g, eps, W_p, s_w, y_dtype=torch.bfloat16)
+        torch.cuda.synchronize()
+        assert torch.equal(y.view(torch.int16), y1.view(torch.int16))
+        ref_p, ref_s = oracle_weights(W)
+        ref = oracle.linear_forward(xh, None, eps, ref_p, ref_s, K)
+        _check_y(y, ref["y"], ref["y_bf16"])
