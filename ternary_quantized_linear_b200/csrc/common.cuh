@@ -273,6 +273,14 @@ __device__ __forceinline__ void mma_m16n8k32_s8(int (&d)[4], uint32_t a0, uint32
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
+// d = c + the dot product of the four unsigned bytes of a with the four
+// signed bytes of b (exact, 32-bit wrap-around never reached by the callers).
+__device__ __forceinline__ int dp4a_us(uint32_t a, uint32_t b, int c) {
+  int d;
+  asm("dp4a.u32.s32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+  return d;
+}
+
 // Barrier `id` (1..15) over `count` threads (a multiple of 32): lets a
 // subset of a CTA's warps synchronise without the others.
 __device__ __forceinline__ void named_barrier_sync(int id, int count) {

@@ -35,7 +35,11 @@
 //     mma.sync m16n8k32 s8 in swap-AB form (weight rows = MMA M, tokens = N,
 //     one or two n8 tiles) into register accumulators that live for the
 //     whole segment.  Tokens past M read some valid token's bytes: they only
-//     feed accumulator columns that are never stored.
+//     feed accumulator columns that are never stored.  The legacy int8 MMA
+//     retires about one m16n8k32 per 8 cycles per SM on this GPU, which is
+//     what bounds the kernel once two token tiles are needed; a single token
+//     (M = 1) would waste seven eighths of every MMA, so its segments run on
+//     dp4a instead (gt_dp4a_unit) and stay bound by the weight stream.
 //   * At the end of a segment the warps add their accumulators into a
 //     shared 128 x 16 table (two tables, alternating) and, after a bounded
 //     barrier, finish it: y = (acc - rowsum) / (s_x * s_w) for a whole row
@@ -267,6 +271,61 @@ __device__ __forceinline__ void gt_mma_unit(int (&acc)[4][NT][4], const GemvBuf<
   }
 }
 
+// One 64-row x 256-k unit for a single token, on the integer dot-product
+// units instead of the tensor cores (an mma.sync costs the same for one
+// token as for eight, and its rate bounds this kernel).  Byte i of
+// P & (3 << 2r) is the code of k = 4i + r times 4^r, so one dp4a of it with
+// activation word r adds 4^r times that word's four products; each row keeps
+// its four scales apart (row g in A[rg][0][r], row g + 8 in B[rg][kB][r])
+// until gt_flush_one divides them out exactly.
+template <int NT, int kB>
+__device__ __forceinline__ void gt_dp4a_unit(int (&A)[4][NT][4], int (&B)[4][NT][4],
+                                             const GemvBuf<NT>& b) {
+#pragma unroll
+  for (int w = 0; w < 4; ++w) {
+    uint32_t x[4];
+#pragma unroll
+    for (int r = 0; r < 4; ++r) x[r] = word_of(b.x[0][w], r);
+#pragma unroll
+    for (int rg = 0; rg < 4; ++rg) {
+      const uint32_t Pa = word_of(b.wa[rg], w), Pb = word_of(b.wb[rg], w);
+#pragma unroll
+      for (int r = 0; r < 4; ++r) {
+        const uint32_t m = kCodeMask << (2 * r);
+        A[rg][0][r] = dp4a_us(Pa & m, x[r], A[rg][0][r]);
+        B[rg][kB][r] = dp4a_us(Pb & m, x[r], B[rg][kB][r]);
+      }
+    }
+  }
+}
+
+// Flush of gt_dp4a_unit's sums (the single token, column 0 of the table):
+// the four scales of a row divided out (exact: each sum is a multiple of its
+// 4^r), the four lanes t of a row added by shuffles, one shared-memory add
+// per row; the accumulators cleared.
+template <int NT, int kB>
+__device__ __forceinline__ void gt_flush_one(int (&A)[4][NT][4], int (&B)[4][NT][4], int* red,
+                                             int g, int t) {
+#pragma unroll
+  for (int rg = 0; rg < 4; ++rg) {
+    int va = A[rg][0][0] + (A[rg][0][1] >> 2) + (A[rg][0][2] >> 4) + (A[rg][0][3] >> 6);
+    int vb = B[rg][kB][0] + (B[rg][kB][1] >> 2) + (B[rg][kB][2] >> 4) + (B[rg][kB][3] >> 6);
+    va += __shfl_xor_sync(0xFFFFFFFFu, va, 1);
+    vb += __shfl_xor_sync(0xFFFFFFFFu, vb, 1);
+    va += __shfl_xor_sync(0xFFFFFFFFu, va, 2);
+    vb += __shfl_xor_sync(0xFFFFFFFFu, vb, 2);
+    if (t == 0) {
+      atomicAdd(&red[(16 * rg + g) * 16], va);
+      atomicAdd(&red[(16 * rg + g + 8) * 16], vb);
+    }
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+      A[rg][0][r] = 0;
+      B[rg][kB][r] = 0;
+    }
+  }
+}
+
 // Add a warp's accumulators into the segment's shared table and clear them
 // (kHi: acc16 holds the times-16 sums of gemv_mma_unit, divided exactly).
 template <int NT, int TILES, bool kHi>
@@ -431,6 +490,7 @@ ternary_gemv_tiled_kernel(const __grid_constant__ GtLaunch L) {
     const GtProblem& P = prob[sg.p];
     const int M = P.M;
     const bool two = NT == 2 && M > 8;
+    const bool one = M == 1;   // dp4a instead of mma.sync
     const GtSpan span = gt_span(P, sg);
     const bool whole = sg.t == span.first && sg.nt == span.len;
     // Warp 0 keeps the token constants of the current (problem, group) in
@@ -481,19 +541,30 @@ ternary_gemv_tiled_kernel(const __grid_constant__ GtLaunch L) {
       if (lane == 0) mbar_arrive(&empty[s]);
       if (u < n) {
         any = true;
-        if (kHi)
+        if (one) {
+          if constexpr (NT == 2)
+            gt_dp4a_unit<NT, 1>(acc, acc, buf);
+          else
+            gt_dp4a_unit<NT, 0>(acc, acc16, buf);
+        } else if (kHi) {
           gemv_mma_unit<NT, 1>(acc, acc16, buf);
-        else if (two)
+        } else if (two) {
           gt_mma_unit<NT, NT>(acc, buf);
-        else
+        } else {
           gt_mma_unit<NT, 1>(acc, buf);
+        }
       }
     }
     if (!ok) break;
     if (whole && warp == 0 && lane < M) tok[segi & 1][lane] = tk;
     int* tab = acc_tab[segi & 1];
     if (any) {
-      if (two)
+      if (one) {
+        if constexpr (NT == 2)
+          gt_flush_one<NT, 1>(acc, acc, tab + tab_row0 * 16, g, t);
+        else
+          gt_flush_one<NT, 0>(acc, acc16, tab + tab_row0 * 16, g, t);
+      } else if (two)
         gt_flush<NT, NT, kHi>(acc, acc16, tab + tab_row0 * 16, M, g, t);
       else
         gt_flush<NT, 1, kHi>(acc, acc16, tab + tab_row0 * 16, M, g, t);
