@@ -44,8 +44,8 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # (the tiled decode matmul over the step's four M <= 16 forwards) from an
 # ncu capture (summary under profiles/), valid only for the kernel source it
 # was measured on (sha256 of csrc/gemv_tiled.cuh); reported as null otherwise.
-GT_TRAFFIC = {"src_sha256": "76a40f2c8551b68637af97d415d022845aac5f12f3f0d4c2926d15b1981b2fa2",
-              "bytes_per_launch": 235552768 + 5115392}
+GT_TRAFFIC = {"src_sha256": "bb301936c005a44543591601ed7d4b47cc9790fd15227512e5d5bff9186c5db6",
+              "bytes_per_launch": 235698688 + 4319232}
 
 
 # ------------------------------------------------------------------ helpers
