@@ -213,6 +213,45 @@ def test_tiled_grouped_mixed_layouts_and_shared_input(M):
             _check_y(it[5], ref["y"], ref["y_bf16"], cols)
 
 
+# Tiled problems of one token tile (M <= 8) and of two (M > 8) in one grouped
+# call: one launch of the two-tile kernel in which single-token segments run
+# on dp4a, 2..8-token segments on one MMA token tile and the rest on two.
+# Ragged N and K, one-tile problems, both y dtypes.
+MIXED_TILES = [
+    [(1, 4096, 4096), (16, 4096, 4096), (1, 14336, 4096), (12, 4096, 1024)],
+    [(16, 256, 128), (1, 8192, 4096)],
+    [(9, 768, 300), (3, 1280, 1000), (1, 256, 130), (16, 2304, 520), (5, 512, 64)],
+]
+
+
+@pytest.mark.parametrize("ci", range(len(MIXED_TILES)))
+def test_tiled_grouped_one_and_two_token_tiles(ci):
+    rng = np.random.default_rng(31 + ci)
+    items, refs = [], []
+    for j, (M, K, N) in enumerate(MIXED_TILES[ci]):
+        xh = workloads._to_bf16_bits(rng.standard_normal((M, K)).astype(np.float32))
+        W = (rng.standard_normal((N, K)) * 0.02).astype(np.float32)
+        _, s_w, Wt = _weights_both(W)
+        ref_p, ref_s = oracle_weights(W)
+        ydt = torch.float32 if j % 2 else torch.bfloat16
+        y = torch.empty((M, N), dtype=ydt, device="cuda")
+        items.append((x_to_device(xh), None, workloads.DEFAULT_EPS, Wt, s_w, y))
+        refs.append(oracle.linear_forward(xh, None, workloads.DEFAULT_EPS, ref_p, ref_s, K))
+    arr, count = tql.grouped_problems(items)
+    nb = tql.bitnet_linear_forward_grouped_workspace_bytes(arr, count)
+    ws = torch.empty(nb, dtype=torch.uint8, device="cuda")
+    ws.fill_(0xA5)   # contents on entry must not matter
+    for _ in range(2):
+        for it in items:
+            it[5].fill_(0)
+        tql.bitnet_linear_forward_grouped(items, workspace=ws)
+        torch.cuda.synchronize()
+        for it, ref in zip(items, refs):
+            _check_y(it[5], ref["y"], ref["y_bf16"])
+    code, detail = tql.bitnet_device_status(reset=False)
+    assert code == 0, (code, detail)
+
+
 def test_tiled_workspace_garbage_on_entry():
     # Partial slots and counters: a workspace full of garbage must not
     # change the result (the counters are cleared by the quant launch).
