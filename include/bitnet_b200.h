@@ -88,7 +88,8 @@ typedef enum { BITNET_F32 = 0, BITNET_BF16 = 1 } bitnet_dtype;
 /* Matmul path selection for the debug entry point (results never depend on it). */
 typedef enum {
     BITNET_PATH_AUTO = 0,  /* decode GEMV for M <= 16 and <= 32 MB of packed weights, else tcgen05 */
-    BITNET_PATH_GEMV = 1,  /* tensor-core (mma.sync) streaming GEMV; needs M <= 16 */
+    BITNET_PATH_GEMV = 1,  /* streaming decode matmul (mma.sync; dp4a for M = 1 on tiled
+                              weights); needs M <= 16 */
     BITNET_PATH_GEMM = 2   /* tcgen05 + TMA GEMM with TMEM accumulators */
 } bitnet_path;
 
